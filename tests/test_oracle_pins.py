@@ -1,0 +1,338 @@
+"""Pins of the FP64 oracle to things other than itself (CPU only).
+
+Each test checks the oracle against a value printed on the pages (fixtures under
+tests/golden/, each citing its page and section), a closed form, a brute-force
+enumeration, or an invariant of the mathematics -- chosen so that a dropped term, a
+wrong sign, a swapped operand or a transposed weight fails at least one of them.
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from golden_io import floats, lines
+
+RNG = np.random.default_rng(1234)
+
+
+# ------------------------------------------------------------------ RMSNorm forms (a8)
+def _norm_rows():
+    for s in lines("norm_examples.txt"):
+        name, v, w, cen, ins, dec = [p.strip() for p in s.split("|")]
+        yield name, np.array(floats(v)), np.array(floats(w)), np.array(floats(cen)), \
+            np.array(floats(ins)), int(dec)
+
+
+@pytest.mark.parametrize("row", list(_norm_rows()), ids=lambda r: r[0])
+def test_rmsnorm_worked_examples(row):
+    name, v, w, cen, ins, dec = row
+    # one unit in the last printed place: the deep dive prints 1/4.301 = 0.23250 as 0.233
+    tol = 10.0 ** (-dec) + 1e-12
+    np.testing.assert_allclose(oracle.centred_rmsnorm(v, w, 0.0), cen, rtol=0, atol=tol)
+    np.testing.assert_allclose(oracle.input_scaled_rmsnorm(v, w, 0.0), ins, rtol=0, atol=tol)
+
+
+def test_rmsnorm_rms_printed_in_deep_dive():
+    rms = lambda a: math.sqrt(float(np.mean(a * a)))
+    # deep dive §5.3 example also prints the RMS of both outputs: 1.92 and 1.00
+    v, w = np.array([3.0, 1.0]), np.array([1.0, 0.0])
+    assert abs(rms(oracle.centred_rmsnorm(v, w, 0.0)) - 1.92) < 0.005
+    assert abs(rms(oracle.input_scaled_rmsnorm(v, w, 0.0)) - 1.00) < 0.005
+
+
+@pytest.mark.parametrize("row", list(lines("norm_rms_examples.txt")))
+def test_rmsnorm_epsilon_output_rms(row):
+    eps, in_rms, out_rms, dec = floats(row)
+    v = np.full(64, in_rms) * np.where(np.arange(64) % 2 == 0, 1.0, -1.0)
+    got = oracle.centred_rmsnorm(v, np.zeros(64), eps)
+    assert abs(math.sqrt(np.mean(got ** 2)) - out_rms) <= 0.5 * 10 ** (-int(dec))
+    # closed form sqrt(ms/(ms+eps)) for any row
+    y = RNG.normal(size=(5, 33)) * 1e-3
+    ms = np.mean(y * y, axis=1)
+    n = oracle.centred_rmsnorm(y, np.zeros(33), eps)
+    np.testing.assert_allclose(np.sqrt(np.mean(n * n, axis=1)), np.sqrt(ms / (ms + eps)), rtol=1e-13)
+
+
+def test_rmsnorm_unit_row_rms_equals_gain_rms():
+    # all |y_i| equal: rms(N(y)) = rms(1+gamma) * sqrt(ms/(ms+eps))
+    L, eps = 128, 1e-6
+    gamma = RNG.normal(size=L) * math.sqrt(0.1)
+    y = 0.37 * np.where(RNG.random(L) < 0.5, -1.0, 1.0)
+    n = oracle.centred_rmsnorm(y, gamma, eps)
+    expect = math.sqrt(np.mean((1 + gamma) ** 2)) * math.sqrt(0.37 ** 2 / (0.37 ** 2 + eps))
+    assert abs(math.sqrt(np.mean(n * n)) - expect) < 1e-13
+
+
+def test_input_scaled_norm_has_unit_rms_for_any_gain():
+    v = RNG.normal(size=(4, 64))
+    w = RNG.normal(size=64)
+    n = oracle.input_scaled_rmsnorm(v, w, 0.0)
+    np.testing.assert_allclose(np.sqrt(np.mean(n * n, axis=1)), 1.0, rtol=1e-14)
+
+
+def test_norm_is_scale_invariant_at_eps0():
+    v = RNG.normal(size=(3, 40))
+    g = RNG.normal(size=40) * 0.3
+    np.testing.assert_allclose(oracle.centred_rmsnorm(7.5 * v, g, 0.0), oracle.centred_rmsnorm(v, g, 0.0),
+                               rtol=1e-13)
+
+
+# ------------------------------------------------------------------ combine (a9)
+def test_norm_before_mix_counter_example():
+    rows = {s.split()[0]: floats(" ".join(s.split()[1:])) for s in lines("norm_before_mix.txt")
+            if not s.startswith("output")}
+    outs = np.array([floats(" ".join(s.split()[1:])) for s in lines("norm_before_mix.txt")
+                     if s.startswith("output")])
+    w = np.array(rows["weights"])
+    n = oracle.centred_rmsnorm(outs, np.zeros(2), 0.0)            # per expert
+    c = oracle.combine(n[None], w[None])[0]
+    np.testing.assert_allclose(c, rows["per_expert_then_mix"], rtol=1e-15)
+    wrong = oracle.centred_rmsnorm(w @ outs, np.zeros(2), 0.0)
+    np.testing.assert_allclose(wrong, rows["mix_then_normalise"], rtol=1e-15)
+    assert np.abs(c - wrong).max() > 0.5
+
+
+def test_combine_rms_bound_and_equality():
+    # gamma = 0, eps = 0: every normalised row has RMS 1, weights sum to 1 => rms(c) <= 1,
+    # equality iff all k rows are parallel.
+    n = oracle.centred_rmsnorm(RNG.normal(size=(6, 4, 32)), np.zeros(32), 0.0)
+    g = RNG.random((6, 4))
+    g /= g.sum(1, keepdims=True)
+    c = oracle.combine(n, g)
+    assert np.all(np.sqrt(np.mean(c * c, axis=1)) <= 1.0 + 1e-14)
+    same = np.repeat(n[:, :1], 4, axis=1)
+    c2 = oracle.combine(same, g)
+    np.testing.assert_allclose(np.sqrt(np.mean(c2 * c2, axis=1)), 1.0, rtol=1e-14)
+
+
+def test_combine_weights_follow_slots():
+    n = np.zeros((1, 3, 2))
+    n[0, 0] = [1, 0]
+    n[0, 1] = [0, 1]
+    n[0, 2] = [1, 1]
+    c = oracle.combine(n, np.array([[0.5, 0.3, 0.2]]))
+    np.testing.assert_allclose(c[0], [0.7, 0.5], rtol=1e-15)
+
+
+# ------------------------------------------------------------------ router (a1, a2)
+def test_topk_brute_force_small():
+    for E, k in [(8, 2), (16, 4), (9, 9), (12, 1)]:
+        for _ in range(30):
+            keys = RNG.normal(size=(1, E))
+            idx = oracle.select_topk(keys, k)[0]
+            best = max(itertools.combinations(range(E), k), key=lambda s: sum(keys[0, list(s)]))
+            assert set(idx.tolist()) == set(best)
+            # routing order: key descending
+            assert np.all(np.diff(keys[0, idx]) <= 0)
+
+
+def test_topk_ties_go_to_lower_index():
+    keys = np.array([[0.5, 1.0, 0.5, 1.0, 0.5, 0.2]])
+    assert oracle.select_topk(keys, 2)[0].tolist() == [1, 3]
+    assert oracle.select_topk(keys, 3)[0].tolist() == [1, 3, 0]
+    assert oracle.select_topk(keys, 5)[0].tolist() == [1, 3, 0, 2, 4]
+    # brute force over ties: the lexicographically smallest index set among the maxima
+    keys = np.round(RNG.normal(size=(1, 10)) * 2) / 2
+    for k in range(1, 10):
+        sel = oracle.select_topk(keys, k)[0]
+        sets = list(itertools.combinations(range(10), k))
+        vals = [sum(keys[0, list(s)]) for s in sets]
+        best = max(vals)
+        cands = sorted(tuple(sorted(s)) for s, v in zip(sets, vals) if abs(v - best) < 1e-12)
+        # lower index wins each tie: the candidate with the smallest indices at equal keys
+        ref = sorted(range(10), key=lambda e: (-keys[0, e], e))[:k]
+        assert tuple(sorted(ref)) in cands
+        assert sel.tolist() == ref
+
+
+def test_softmax_weights_are_renormalised_full_softmax():
+    logits = RNG.normal(size=(5, 16)) * 3
+    idx = oracle.select_topk(logits, 4)
+    g = oracle.softmax_weights(logits, idx)
+    full = np.exp(logits) / np.exp(logits).sum(1, keepdims=True)
+    sel = np.take_along_axis(full, idx, 1)
+    np.testing.assert_allclose(g, sel / sel.sum(1, keepdims=True), rtol=1e-13)
+    np.testing.assert_allclose(g.sum(1), 1.0, rtol=1e-15)
+    # k = 1 gives weight exactly 1
+    assert np.all(oracle.softmax_weights(logits, oracle.select_topk(logits, 1)) == 1.0)
+
+
+def test_router_renormalisation_example():
+    rows = {s.split()[0]: floats(" ".join(s.split()[1:])) for s in lines("router_examples.txt")
+            if not s.startswith("bias_case")}
+    s = np.array(rows["scores"])
+    assert abs(s.sum() - 4.00) < 1e-12
+    scale = 1 / math.sqrt(32)
+    logits = np.log(s / (1 - s)) / scale                       # sigmoid^-1 of the scores
+    g = oracle.sigmoid_weights(logits[None], np.arange(8)[None], scale, 1.0)[0]
+    np.testing.assert_allclose(g, rows["weights"], atol=0.005 + 1e-12)
+    assert abs(g.sum() - 1.0) < 1e-14
+
+
+def test_router_selection_only_bias_example():
+    cases = {int(s.split()[1]): floats(" ".join(s.split()[2:]))
+             for s in lines("router_examples.txt") if s.startswith("bias_case")}
+    E, k, scale = 256, 8, 1 / math.sqrt(32)
+    logits = np.full(E, -20.0)
+    winners = [3, 40, 77, 120, 150, 200, 250]
+    logits[winners] = 12.0
+    bias = np.zeros(E)
+    for e, (logit, scaled, s_pr, b, key_pr) in cases.items():
+        logits[e] = logit
+        bias[e] = b
+        s = 1 / (1 + math.exp(-scale * logit))
+        assert abs(s - s_pr) < 0.005
+        assert abs(s + b - key_pr) < 0.005
+        if not math.isnan(scaled):
+            assert abs(scale * logit - scaled) < 0.005
+    idx, g, keys = oracle.route(logits[None], k, bias, "sigmoid", scale, 1.0)
+    assert 90 in idx[0] and 17 not in idx[0]
+    # the weight of expert 90 comes from its raw score, not from score + bias
+    s_sel = 1 / (1 + np.exp(-scale * logits[idx[0]]))
+    j = list(idx[0]).index(90)
+    assert abs(g[0, j] - s_sel[j] / (s_sel.sum() + 1e-15)) < 1e-15
+    assert abs(s_sel[j] - 0.40) < 0.005
+    # without the bias, expert 17 would have taken the slot
+    idx0, _, _ = oracle.route(logits[None], k, None, "sigmoid", scale, 1.0)
+    assert 17 in idx0[0] and 90 not in idx0[0]
+
+
+def test_softmax_mode_bias_selects_but_does_not_weight():
+    logits = np.array([[1.0, 0.9, 0.0, -1.0]])
+    bias = np.array([0.0, 0.0, 2.0, 0.0])
+    idx, g, _ = oracle.route(logits, 2, bias)
+    assert idx[0].tolist() == [2, 0]
+    e = np.exp(np.array([0.0, 1.0]))
+    np.testing.assert_allclose(g[0], e / e.sum(), rtol=1e-15)
+
+
+def test_topk_alternatives():
+    keys = np.array([3.0, 2.0, 1.0, 1.0 + 5e-5, 0.0])
+    alts = oracle.topk_alternatives(keys, 3, 1e-4)
+    assert sorted(alts) == [(0, 1, 2), (0, 1, 3)]
+    assert oracle.topk_alternatives(keys, 2, 1e-4) == [(0, 1)]
+
+
+# ------------------------------------------------------------------ linear maps (a1, a4, a6, a7, a10)
+@pytest.mark.parametrize("fn,out_dim,in_dim", [
+    (oracle.router_logits, 6, 10), (oracle.pooler, 5, 10), (oracle.unpooler, 10, 5)])
+def test_linear_layers_use_out_by_in_storage(fn, out_dim, in_dim):
+    # weights are stored [out, in] (a bias-free linear layer; the deep dive §4.3 gives
+    # gate_up_proj as [256, 8192, 4096] = [experts, out, in]); a one-hot weight W[i, j] = 1
+    # must carry input coordinate j to output coordinate i.
+    W = np.zeros((out_dim, in_dim))
+    W[2, 3] = 1.0
+    x = np.zeros((1, in_dim))
+    x[0, 3] = 5.0
+    out = fn(x, W)
+    expect = np.zeros((1, out_dim))
+    expect[0, 2] = 5.0
+    np.testing.assert_array_equal(out, expect)
+
+
+def test_expert_swiglu_values_and_orientation():
+    L = I = 4
+    Wg, Wu, Wd = np.zeros((I, L)), np.zeros((I, L)), np.zeros((L, I))
+    Wg[1, 0] = 1.0          # gate unit 1 reads z[0]
+    Wu[1, 0] = 3.0          # up unit 1 reads 3 z[0]
+    Wd[2, 1] = 1.0          # output 2 reads hidden unit 1
+    z = np.array([[2.0, 0, 0, 0]])
+    y = oracle.expert_ffn(z, Wg, Wu, Wd)
+    # E(z) = W_down(SiLU(W_gate z) * W_up z): a = 2, u = 6, h = SiLU(2) * 6 (closed form)
+    silu2 = 2.0 / (1.0 + math.exp(-2.0))
+    expect = np.zeros((1, L))
+    expect[0, 2] = silu2 * 6.0
+    np.testing.assert_allclose(y, expect, rtol=1e-15, atol=0)
+    # SiLU goes on the gate, not the up projection
+    assert abs(y[0, 2] - 2.0 * (6.0 / (1 + math.exp(-6.0)))) > 1.0
+
+
+def test_silu_closed_forms():
+    assert oracle.silu(np.array([0.0]))[0] == 0.0
+    assert abs(oracle.silu(np.array([1.0]))[0] - 1.0 / (1.0 + math.exp(-1.0))) < 1e-16
+    assert abs(oracle.silu(np.array([-40.0]))[0]) < 1e-15
+    assert abs(oracle.silu(np.array([40.0]))[0] - 40.0) < 1e-12
+
+
+# ------------------------------------------------------------------ whole block
+def _random_block(T=7, D=24, L=16, I=12, E=5, seed=0):
+    r = np.random.default_rng(seed)
+    return dict(x=r.normal(size=(T, D)), W_router=r.normal(size=(E, D)) / math.sqrt(D),
+                W_pool=r.normal(size=(L, D)) / math.sqrt(D),
+                W_gate=r.normal(size=(E, I, L)) / math.sqrt(L), W_up=r.normal(size=(E, I, L)) / math.sqrt(L),
+                W_down=r.normal(size=(E, L, I)) / math.sqrt(I), gamma=r.normal(size=(E, L)) * 0.3,
+                W_unpool=r.normal(size=(D, L)) / math.sqrt(L))
+
+
+def _fwd(b, k, eps=1e-6, **kw):
+    return oracle.latent_moe_forward(b["x"], b["W_router"], b["W_pool"], (b["W_gate"], b["W_up"], b["W_down"]),
+                                     b["gamma"], b["W_unpool"], k, eps, **kw)
+
+
+def test_all_experts_identical_k_equals_E_is_one_dense_expert():
+    b = _random_block()
+    E = b["W_gate"].shape[0]
+    for name in ("W_gate", "W_up", "W_down", "gamma"):
+        b[name] = np.repeat(b[name][:1], E, axis=0)
+    got = _fwd(b, k=E)["out"]
+    z = b["x"] @ b["W_pool"].T
+    a, u = z @ b["W_gate"][0].T, z @ b["W_up"][0].T
+    y = (a / (1 + np.exp(-a)) * u) @ b["W_down"][0].T
+    n = y / np.sqrt(np.mean(y * y, 1, keepdims=True) + 1e-6) * (1 + b["gamma"][0])
+    np.testing.assert_allclose(got, n @ b["W_unpool"].T, rtol=1e-12, atol=1e-12)
+
+
+def test_token_permutation_equivariance():
+    b = _random_block(T=11)
+    ref = _fwd(b, k=2)
+    perm = np.random.default_rng(5).permutation(11)
+    b2 = dict(b, x=b["x"][perm])
+    got = _fwd(b2, k=2)
+    np.testing.assert_allclose(got["out"], ref["out"][perm], rtol=1e-13, atol=1e-13)
+    np.testing.assert_array_equal(got["idx"], ref["idx"][perm])
+
+
+def test_down_projection_scale_cancels_in_norm():
+    b = _random_block()
+    ref = _fwd(b, k=3, eps=0.0)["out"]
+    b2 = dict(b, W_down=b["W_down"] * np.array([0.5, 2.0, 3.0, 10.0, 0.1])[:, None, None])
+    np.testing.assert_allclose(_fwd(b2, k=3, eps=0.0)["out"], ref, rtol=1e-11, atol=1e-12)
+
+
+def test_per_expert_gain_is_taken_from_the_selected_expert():
+    b = _random_block(T=3, E=4)
+    res = _fwd(b, k=2)
+    t, j = 1, 1
+    e = int(res["idx"][t, j])
+    y = res["y"][t, j]
+    np.testing.assert_allclose(res["n"][t, j], y / math.sqrt(np.mean(y * y) + 1e-6) * (1 + b["gamma"][e]),
+                               rtol=1e-14)
+    # shared gain = broadcast of one [L] vector (pages' post_expert_norm)
+    shared = oracle.latent_moe_forward(b["x"], b["W_router"], b["W_pool"], (b["W_gate"], b["W_up"], b["W_down"]),
+                                       b["gamma"][0], b["W_unpool"], 2, 1e-6)
+    np.testing.assert_allclose(shared["n"][t, j], y / math.sqrt(np.mean(y * y) + 1e-6) * (1 + b["gamma"][0]),
+                               rtol=1e-14)
+
+
+def test_callable_expert_source_matches_arrays():
+    b = _random_block()
+    ref = _fwd(b, k=2)["out"]
+    got = oracle.latent_moe_forward(b["x"], b["W_router"], b["W_pool"],
+                                    lambda e: (b["W_gate"][e], b["W_up"][e], b["W_down"][e]),
+                                    b["gamma"], b["W_unpool"], 2, 1e-6)["out"]
+    np.testing.assert_array_equal(got, ref)
+
+
+# ------------------------------------------------------------------ accounting
+def test_parameter_and_flop_accounting():
+    a = {s.split()[0]: float(s.split()[1]) for s in lines("accounting.txt")}
+    D, L, I, E, k = (int(a[n]) for n in "D L I E k".split())
+    assert oracle.expert_param_count(L, I) == a["params_per_expert"]
+    assert E * oracle.expert_param_count(L, I) == a["params_all_experts"]
+    assert E * D + 2 * D * L + 2 * L == a["params_router_proj_norms"]
+    flops = oracle.moe_flops_per_token(D, L, I, E, k)
+    # 2 x active parameters, less the two 4096-entry norm gains the FLOP count leaves out
+    assert flops == 2 * (a["params_active_per_token"] - 2 * L)
+    assert round(flops / 1e6, 1) == a["moe_mflops_per_token_printed"]
