@@ -1,0 +1,166 @@
+/*
+ * muse_moe.h -- C ABI of the latent mixture-of-experts block (forward pass) on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * The block (Muse Spark Open deep dive, §4.3, block equation; §4.2 router):
+ *
+ *   l   = W_router x                     router logits over E experts, full width D
+ *   S,g = top-k of l (+ bias), weights    softmax over the E logits renormalised on S
+ *   z   = W_pool x                        shared pooler D -> L
+ *   y_j = W_down[e] (SiLU(W_gate[e] z) * W_up[e] z),   e = S_j   (SwiGLU L -> I -> L)
+ *   n_j = y_j / sqrt(mean(y_j^2) + eps) * (1 + gamma[e])          per-expert RMSNorm
+ *   c   = sum_j g_j n_j                   weighted combine, after each norm
+ *   out = W_unpool c                      shared unpooler L -> D
+ *
+ * Readings fixed by this library where the pages leave a step open: softmax router
+ * (the released model's sigmoid router is MUSE_ROUTER_SIGMOID), top-k ordered by key
+ * descending with ties to the lower expert index, per-expert centred gain (the released
+ * model's single input-scaled gain is MUSE_NORM_INPUT_SCALED with gamma_shared = 1).
+ *
+ * Layouts (row-major, every weight stored [out, in], the K dimension contiguous):
+ *   x        [T, D]        W_router [E, D]       W_pool   [L, D]
+ *   W_gate   [E, I, L]     W_up     [E, I, L]    W_down   [E, L, I]
+ *   gamma    [E, L] (or [L] when gamma_shared)    W_unpool [D, L]     out [T, D]
+ * Every tensor has the dtype cfg->dtype (float32 or bfloat16). Accumulation is FP32.
+ *
+ * Ownership: the caller owns every buffer, including the device workspace. The library
+ * allocates no device memory, keeps no per-call state, and enqueues all work on the
+ * given stream without synchronising (except muse_latent_moe_last_device_status).
+ * Errors: every function returns a muse_status. Arguments are validated before any
+ * launch; a failed validation launches nothing. Device-side waits are bounded: a wait
+ * that runs out records MUSE_ERR_TIMEOUT in the workspace's status word instead of
+ * hanging, readable with muse_latent_moe_last_device_status.
+ */
+#ifndef MUSE_MOE_H_
+#define MUSE_MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MUSE_API __attribute__((visibility("default")))
+#else
+#define MUSE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum muse_status {
+  MUSE_OK = 0,
+  MUSE_ERR_INVALID_ARG = 1,   /* null / misaligned pointer, inconsistent sizes */
+  MUSE_ERR_UNSUPPORTED = 2,   /* shape or mode this build does not implement */
+  MUSE_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required */
+  MUSE_ERR_CUDA = 4,          /* a CUDA runtime / driver call failed */
+  MUSE_ERR_TIMEOUT = 5,       /* a bounded device-side wait ran out */
+  MUSE_ERR_DEVICE = 6         /* a device-side check failed (e.g. a bad index) */
+} muse_status;
+
+typedef enum muse_dtype { MUSE_F32 = 0, MUSE_BF16 = 1 } muse_dtype;
+
+typedef enum muse_router_mode {
+  MUSE_ROUTER_SOFTMAX = 0,    /* key = l + b; g = softmax(l) renormalised on S        */
+  MUSE_ROUTER_SIGMOID = 1     /* released router (deep dive §4.2): s = sigmoid(scale*l),
+                                 key = s + b, g = rsf * s / (sum_S s + 1e-15)          */
+} muse_router_mode;
+
+typedef enum muse_norm_mode {
+  MUSE_NORM_CENTRED = 0,      /* y / sqrt(mean(y^2)+eps) * (1+gamma)                   */
+  MUSE_NORM_INPUT_SCALED = 1  /* u / sqrt(mean(u^2)+eps), u = y * (1+gamma)           */
+} muse_norm_mode;
+
+/* Block configuration. Zero-initialise, then set the sizes; muse_moe_config_init
+ * fills the defaults (softmax router, centred per-expert norm, eps 1e-6). */
+typedef struct muse_moe_config {
+  int64_t T;                  /* tokens, >= 1                                         */
+  int64_t D;                  /* hidden width; multiple of 128                        */
+  int64_t L;                  /* latent width; multiple of 128                        */
+  int64_t I;                  /* expert intermediate width; multiple of 128           */
+  int64_t E;                  /* experts, 1..1024                                     */
+  int32_t top_k;              /* 1..min(E, 32)                                        */
+  int32_t dtype;              /* muse_dtype of x, weights, gamma, out                 */
+  float eps;                  /* per-expert RMSNorm epsilon                           */
+  int32_t router_mode;        /* muse_router_mode                                     */
+  float router_logit_scale;   /* multiplies l before the sigmoid (sigmoid mode only)  */
+  float routed_scaling;       /* multiplies g (sigmoid mode only)                     */
+  const float* router_bias;   /* device [E] float32 selection-only bias, or NULL      */
+  int32_t norm_mode;          /* muse_norm_mode                                       */
+  int32_t gamma_shared;       /* 0: gamma is [E, L]; 1: one [L] gain for all experts  */
+  const void* pre_norm_gain;  /* optional device [L] gain offsets of a centred RMSNorm
+                                 on z before dispatch (pages' pre_expert_norm), or NULL */
+  float pre_norm_eps;         /* epsilon of that norm (pages: 1e-5)                   */
+  void* workspace;            /* device, 256-byte aligned, caller-owned               */
+  size_t workspace_bytes;
+  int32_t* topk_idx_out;      /* optional device [T, k] int32: selected experts       */
+  float* topk_w_out;          /* optional device [T, k] float32: their weights        */
+} muse_moe_config;
+
+/* Byte offsets of the intermediates inside the workspace after a forward call, for
+ * inspection by tests. Rows of the expert-ordered buffers are grouped by expert, each
+ * expert's group padded to a multiple of 16 rows; inv maps assignment t*k+j to its row. */
+typedef struct muse_moe_workspace_layout {
+  size_t status;        /* uint32[2]: status code, detail                            */
+  size_t expert_count;  /* int32 [E]     tokens routed to each expert                 */
+  size_t expert_offset; /* int32 [E+1]   first padded row of each expert              */
+  size_t logits;        /* float [T, E]  router logits                                */
+  size_t topk_idx;      /* int32 [T, k]  selected experts, key descending            */
+  size_t topk_w;        /* float [T, k]  routing weights                             */
+  size_t inv;           /* int32 [T*k]   row of assignment t*k+j                      */
+  size_t row_token;     /* int32 [R]     token of each row, -1 for padding            */
+  size_t z;             /* act   [T, L]  pooler output                                */
+  size_t zp;            /* act   [R, L]  z gathered into expert order                 */
+  size_t h;             /* act   [R, I]  SiLU(gate) * up                              */
+  size_t y;             /* act   [R, L]  expert outputs before the norm               */
+  size_t ss;            /* float [R, L/32] partial sums of y^2 per 32 columns         */
+  size_t c;             /* act   [T, L]  combined latent                              */
+  size_t total;         /* bytes required                                             */
+  int64_t rows;         /* R: upper bound of padded rows                              */
+} muse_moe_workspace_layout;
+
+/* Fills defaults: router softmax, scale 1, rsf 1, norm centred per expert, eps 1e-6. */
+MUSE_API void muse_moe_config_init(muse_moe_config* cfg);
+
+/* Workspace bytes for cfg's sizes (cfg->workspace is not read). */
+MUSE_API muse_status muse_latent_moe_workspace_size(const muse_moe_config* cfg, size_t* bytes);
+
+/* Offsets of each intermediate in the workspace for cfg's sizes. */
+MUSE_API muse_status muse_latent_moe_workspace_layout(const muse_moe_config* cfg,
+                                             muse_moe_workspace_layout* layout);
+
+/* Forward pass of the block on device buffers (layouts above); enqueued on `stream`
+ * (a cudaStream_t, NULL = legacy default stream). Pointers must be device memory,
+ * 16-byte aligned; `out` must not alias an input. Returns without synchronising. */
+MUSE_API muse_status muse_latent_moe_forward(const muse_moe_config* cfg, const void* x,
+                                    const void* W_router, const void* W_pool,
+                                    const void* W_gate, const void* W_up, const void* W_down,
+                                    const void* gamma, const void* W_unpool, void* out,
+                                    void* stream);
+
+/* Same, with x and out in HOST memory (pinned for asynchronous copies): copies x into
+ * the device buffer x_dev, runs the forward into out_dev, copies out_dev back to
+ * out_host, all on `stream`. x_dev / out_dev are caller-owned device buffers. The
+ * caller synchronises the stream before reading out_host. */
+MUSE_API muse_status muse_latent_moe_forward_host_io(const muse_moe_config* cfg, const void* x_host,
+                                            void* x_dev, const void* W_router,
+                                            const void* W_pool, const void* W_gate,
+                                            const void* W_up, const void* W_down,
+                                            const void* gamma, const void* W_unpool,
+                                            void* out_dev, void* out_host, void* stream);
+
+/* Synchronises `stream` and returns the status word the last forward on this
+ * workspace recorded on the device (MUSE_OK, MUSE_ERR_TIMEOUT or MUSE_ERR_DEVICE);
+ * *detail (may be NULL) receives the kernel-specific detail code. */
+MUSE_API muse_status muse_latent_moe_last_device_status(const muse_moe_config* cfg, void* stream,
+                                               uint32_t* detail);
+
+/* Static string for a status code. */
+MUSE_API const char* muse_status_string(muse_status s);
+
+/* Number of kernel launches one forward call makes for cfg's sizes (for accounting). */
+MUSE_API int32_t muse_latent_moe_launch_count(const muse_moe_config* cfg);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MUSE_MOE_H_ */

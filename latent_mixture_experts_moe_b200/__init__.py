@@ -1,0 +1,201 @@
+"""Python binding of libmuse_moe.so, the B200 (sm_100a) latent-MoE block forward pass.
+
+Argument marshalling only: every step of the block runs in the library's CUDA kernels.
+PyTorch tensors are accepted as containers of device memory (their data pointers are
+passed through the C ABI declared in include/muse_moe.h); nothing here computes.
+If the compiled library is missing, importing works but every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Optional
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libmuse_moe.so")
+
+MUSE_F32, MUSE_BF16 = 0, 1
+ROUTER_SOFTMAX, ROUTER_SIGMOID = 0, 1
+NORM_CENTRED, NORM_INPUT_SCALED = 0, 1
+
+STATUS = {0: "MUSE_OK", 1: "MUSE_ERR_INVALID_ARG", 2: "MUSE_ERR_UNSUPPORTED", 3: "MUSE_ERR_WORKSPACE",
+          4: "MUSE_ERR_CUDA", 5: "MUSE_ERR_TIMEOUT", 6: "MUSE_ERR_DEVICE"}
+
+# every extern "C" entry point of include/muse_moe.h
+EXPORTS = ("muse_moe_config_init", "muse_latent_moe_workspace_size", "muse_latent_moe_workspace_layout",
+           "muse_latent_moe_forward", "muse_latent_moe_forward_host_io", "muse_latent_moe_last_device_status",
+           "muse_status_string", "muse_latent_moe_launch_count")
+
+
+class MuseError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {STATUS.get(code, code)} ({status_string(code)})")
+
+
+class Config(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("D", ctypes.c_int64), ("L", ctypes.c_int64), ("I", ctypes.c_int64),
+                ("E", ctypes.c_int64), ("top_k", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("eps", ctypes.c_float), ("router_mode", ctypes.c_int32), ("router_logit_scale", ctypes.c_float),
+                ("routed_scaling", ctypes.c_float), ("router_bias", ctypes.c_void_p),
+                ("norm_mode", ctypes.c_int32), ("gamma_shared", ctypes.c_int32),
+                ("pre_norm_gain", ctypes.c_void_p), ("pre_norm_eps", ctypes.c_float),
+                ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+                ("topk_idx_out", ctypes.c_void_p), ("topk_w_out", ctypes.c_void_p)]
+
+
+class WorkspaceLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in ("status", "expert_count", "expert_offset", "logits", "topk_idx",
+                                              "topk_w", "inv", "row_token", "z", "zp", "h", "y", "ss", "c",
+                                              "total")] + [("rows", ctypes.c_int64)]
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library; raises if it has not been built (no fallback exists)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with python -m latent_mixture_experts_moe_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, cp = ctypes.c_void_p, ctypes.POINTER(Config)
+        L.muse_moe_config_init.argtypes = [cp]
+        L.muse_moe_config_init.restype = None
+        L.muse_latent_moe_workspace_size.argtypes = [cp, ctypes.POINTER(ctypes.c_size_t)]
+        L.muse_latent_moe_workspace_size.restype = ctypes.c_int
+        L.muse_latent_moe_workspace_layout.argtypes = [cp, ctypes.POINTER(WorkspaceLayout)]
+        L.muse_latent_moe_workspace_layout.restype = ctypes.c_int
+        L.muse_latent_moe_forward.argtypes = [cp] + [vp] * 10
+        L.muse_latent_moe_forward.restype = ctypes.c_int
+        L.muse_latent_moe_forward_host_io.argtypes = [cp] + [vp] * 12
+        L.muse_latent_moe_forward_host_io.restype = ctypes.c_int
+        L.muse_latent_moe_last_device_status.argtypes = [cp, vp, ctypes.POINTER(ctypes.c_uint32)]
+        L.muse_latent_moe_last_device_status.restype = ctypes.c_int
+        L.muse_status_string.argtypes = [ctypes.c_int]
+        L.muse_status_string.restype = ctypes.c_char_p
+        L.muse_latent_moe_launch_count.argtypes = [cp]
+        L.muse_latent_moe_launch_count.restype = ctypes.c_int32
+        _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().muse_status_string(code).decode()
+
+
+def _check(code: int, where: str) -> None:
+    if code != 0:
+        raise MuseError(code, where)
+
+
+def make_config(T: int, D: int, L: int, I: int, E: int, k: int, dtype: str = "bf16", eps: float = 1e-6,
+                router_mode: int = ROUTER_SOFTMAX, router_logit_scale: float = 1.0, routed_scaling: float = 1.0,
+                norm_mode: int = NORM_CENTRED, gamma_shared: bool = False) -> Config:
+    c = Config()
+    lib().muse_moe_config_init(ctypes.byref(c))
+    c.T, c.D, c.L, c.I, c.E, c.top_k = T, D, L, I, E, k
+    c.dtype = {"f32": MUSE_F32, "bf16": MUSE_BF16}[dtype]
+    c.eps = eps
+    c.router_mode, c.router_logit_scale, c.routed_scaling = router_mode, router_logit_scale, routed_scaling
+    c.norm_mode, c.gamma_shared = norm_mode, int(gamma_shared)
+    return c
+
+
+def workspace_size(cfg: Config) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().muse_latent_moe_workspace_size(ctypes.byref(cfg), ctypes.byref(n)), "workspace_size")
+    return int(n.value)
+
+
+def workspace_layout(cfg: Config) -> Dict[str, int]:
+    lay = WorkspaceLayout()
+    _check(lib().muse_latent_moe_workspace_layout(ctypes.byref(cfg), ctypes.byref(lay)), "workspace_layout")
+    return {name: int(getattr(lay, name)) for name, _ in WorkspaceLayout._fields_}
+
+
+def launch_count(cfg: Config) -> int:
+    return int(lib().muse_latent_moe_launch_count(ctypes.byref(cfg)))
+
+
+def _ptr(t) -> int:
+    if t is None:
+        return 0
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return int(t.data_ptr())
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        import torch
+        return int(torch.cuda.current_stream().cuda_stream)
+    return int(getattr(stream, "cuda_stream", stream))
+
+
+def forward(cfg: Config, x, W_router, W_pool, W_gate, W_up, W_down, gamma, W_unpool, out, stream=None) -> None:
+    """Enqueue one forward pass; cfg.workspace must point to workspace_size(cfg) bytes."""
+    code = lib().muse_latent_moe_forward(ctypes.byref(cfg), _ptr(x), _ptr(W_router), _ptr(W_pool), _ptr(W_gate),
+                                         _ptr(W_up), _ptr(W_down), _ptr(gamma), _ptr(W_unpool), _ptr(out),
+                                         _stream_handle(stream))
+    _check(code, "muse_latent_moe_forward")
+
+
+def forward_host_io(cfg: Config, x_host, x_dev, W_router, W_pool, W_gate, W_up, W_down, gamma, W_unpool,
+                    out_dev, out_host, stream=None) -> None:
+    code = lib().muse_latent_moe_forward_host_io(ctypes.byref(cfg), _ptr(x_host), _ptr(x_dev), _ptr(W_router),
+                                                 _ptr(W_pool), _ptr(W_gate), _ptr(W_up), _ptr(W_down),
+                                                 _ptr(gamma), _ptr(W_unpool), _ptr(out_dev), _ptr(out_host),
+                                                 _stream_handle(stream))
+    _check(code, "muse_latent_moe_forward_host_io")
+
+
+def last_device_status(cfg: Config, stream=None):
+    detail = ctypes.c_uint32(0)
+    code = lib().muse_latent_moe_last_device_status(ctypes.byref(cfg), _stream_handle(stream), ctypes.byref(detail))
+    return int(code), int(detail.value)
+
+
+class LatentMoE:
+    """Holds the block's device weights and a workspace; calling it runs the forward.
+
+    weights: dict with W_router, W_pool, W_gate, W_up, W_down, gamma, W_unpool (torch
+    CUDA tensors in the layouts of include/muse_moe.h); router_bias optional.
+    """
+
+    def __init__(self, weights: Dict, T_max: int, k: int, eps: float = 1e-6, **modes):
+        import torch
+        self.w = weights
+        E, D = weights["W_router"].shape
+        _, I, L = weights["W_gate"].shape
+        self.dtype = {torch.float32: "f32", torch.bfloat16: "bf16"}[weights["W_router"].dtype]
+        self.dims = dict(D=int(D), L=int(L), I=int(I), E=int(E), k=k, eps=eps)
+        self.modes = modes
+        cfg = self.config(T_max)
+        self.workspace = torch.empty(workspace_size(cfg), dtype=torch.uint8, device=weights["W_router"].device)
+        self.T_max = T_max
+
+    def config(self, T: int, workspace=None) -> Config:
+        d = self.dims
+        c = make_config(T, d["D"], d["L"], d["I"], d["E"], d["k"], self.dtype, d["eps"], **self.modes)
+        if self.w.get("router_bias") is not None:
+            c.router_bias = _ptr(self.w["router_bias"])
+        if workspace is not None:
+            c.workspace = _ptr(workspace)
+            c.workspace_bytes = workspace.numel()
+        return c
+
+    def __call__(self, x, out=None, stream=None, topk_idx=None, topk_w=None):
+        import torch
+        T = x.shape[0]
+        if T > self.T_max:
+            raise ValueError(f"T={T} exceeds T_max={self.T_max}")
+        cfg = self.config(T, self.workspace)
+        cfg.topk_idx_out, cfg.topk_w_out = _ptr(topk_idx), _ptr(topk_w)
+        if out is None:
+            out = torch.empty((T, self.dims["D"]), dtype=x.dtype, device=x.device)
+        w = self.w
+        forward(cfg, x, w["W_router"], w["W_pool"], w["W_gate"], w["W_up"], w["W_down"], w["gamma"],
+                w["W_unpool"], out, stream)
+        return out

@@ -1,0 +1,422 @@
+// muse_moe.cu -- C ABI of the latent-MoE block forward pass (see include/muse_moe.h).
+//
+// One forward call validates its arguments, carves the caller's workspace and enqueues
+// eleven kernels on the caller's stream:
+//   router logits (tcgen05 GEMM; FP32 FMA for float32 inputs) -> top-k + weights ->
+//   expert histogram -> padded offsets + tile lists -> stable row assignment ->
+//   pooler (tcgen05 GEMM) -> gather into expert order -> gate/up grouped GEMM with
+//   SiLU(gate)*up epilogue -> down grouped GEMM with sum-of-squares epilogue ->
+//   per-expert RMSNorm + weighted combine -> unpooler (tcgen05 GEMM).
+// No host synchronisation, no device allocation, no host read of routing results.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/muse_moe.h"
+#include "gemm_umma.cuh"
+#include "route_kernels.cuh"
+
+using namespace muse;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// ---------------------------------------------------------------------- tile sizing
+// tokens per grouped-GEMM tile: small tiles when experts see few tokens (decode)
+int grouped_bn(const muse_moe_config& c) { return (c.T * c.top_k) <= 32 * c.E ? 32 : 256; }
+int dense_bn(const muse_moe_config& c) { return c.T <= 32 ? 32 : 256; }
+
+struct Layout {
+  muse_moe_workspace_layout pub;
+  size_t tiles_gu, tiles_dn, ntiles;  // int4 lists and two int counters
+  int64_t max_tiles_gu, max_tiles_dn;
+};
+
+size_t act_size(const muse_moe_config& c) { return c.dtype == MUSE_BF16 ? 2 : 4; }
+
+Layout make_layout(const muse_moe_config& c) {
+  Layout l{};
+  const int64_t T = c.T, E = c.E, k = c.top_k;
+  const int64_t assign = T * k;
+  const int64_t rows = align_up(static_cast<size_t>(assign + 15 * std::min<int64_t>(E, assign)), 16);
+  const int bn = grouped_bn(c);
+  const int64_t chunks = cdiv(assign, bn) + std::min<int64_t>(E, assign);
+  l.max_tiles_gu = chunks * (c.I / 128);
+  l.max_tiles_dn = chunks * (c.L / 128);
+  const size_t as = act_size(c);
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align_up(o + bytes, kAlign);
+    return at;
+  };
+  l.pub.status = take(16);
+  l.pub.expert_count = take(sizeof(int32_t) * E);
+  l.pub.expert_offset = take(sizeof(int32_t) * (E + 1));
+  l.ntiles = take(sizeof(int32_t) * 2);
+  l.pub.logits = take(sizeof(float) * T * E);
+  l.pub.topk_idx = take(sizeof(int32_t) * assign);
+  l.pub.topk_w = take(sizeof(float) * assign);
+  l.pub.inv = take(sizeof(int32_t) * assign);
+  l.pub.row_token = take(sizeof(int32_t) * rows);
+  l.tiles_gu = take(sizeof(int4) * l.max_tiles_gu);
+  l.tiles_dn = take(sizeof(int4) * l.max_tiles_dn);
+  l.pub.z = take(as * T * c.L);
+  l.pub.zp = take(as * rows * c.L);
+  l.pub.h = take(as * rows * c.I);
+  l.pub.y = take(as * rows * c.L);
+  l.pub.ss = take(sizeof(float) * rows * (c.L / 32));
+  l.pub.c = take(as * T * c.L);
+  l.pub.total = o;
+  l.pub.rows = rows;
+  return l;
+}
+
+muse_status validate_sizes(const muse_moe_config* c) {
+  if (c == nullptr) return MUSE_ERR_INVALID_ARG;
+  if (c->T < 1 || c->D < 1 || c->L < 1 || c->I < 1 || c->E < 1) return MUSE_ERR_INVALID_ARG;
+  if (c->top_k < 1 || c->top_k > c->E) return MUSE_ERR_INVALID_ARG;
+  if (c->dtype != MUSE_F32 && c->dtype != MUSE_BF16) return MUSE_ERR_INVALID_ARG;
+  if (!(c->eps >= 0.0f)) return MUSE_ERR_INVALID_ARG;
+  if (c->router_mode != MUSE_ROUTER_SOFTMAX && c->router_mode != MUSE_ROUTER_SIGMOID) return MUSE_ERR_INVALID_ARG;
+  if (c->norm_mode != MUSE_NORM_CENTRED && c->norm_mode != MUSE_NORM_INPUT_SCALED) return MUSE_ERR_INVALID_ARG;
+  if (c->top_k > 32 || c->E > 1024) return MUSE_ERR_UNSUPPORTED;
+  if (c->D % 128 || c->L % 128 || c->I % 128) return MUSE_ERR_UNSUPPORTED;
+  if (c->L > 8192 || c->D > 65536 || c->I > 65536) return MUSE_ERR_UNSUPPORTED;
+  // 32-bit row / coordinate arithmetic inside the kernels
+  if (c->T * c->top_k + 16 * c->E > (int64_t(1) << 30) || c->E * std::max(c->I, c->L) > (int64_t(1) << 31) - 1)
+    return MUSE_ERR_UNSUPPORTED;
+  if (c->T > (int64_t(1) << 24)) return MUSE_ERR_UNSUPPORTED;
+  return MUSE_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------------------------- tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// K-major 2-D map over rows x K elements, box = box_rows x 128 bytes, 128-byte swizzle;
+// rows beyond the tensor read as zeros.
+bool make_map(CUtensorMap* m, const void* base, bool bf16, int64_t K, int64_t rows, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const uint32_t es = bf16 ? 2 : 4;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * es};
+  cuuint32_t box[2] = {128u / es, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+                        const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+// ---------------------------------------------------------------------- GEMM launch
+template <typename TIn, typename TOut, int BN, int EPI>
+cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b, const GemmArgs& args,
+                        int grid, cudaStream_t st) {
+  auto kern = k_umma_gemm<TIn, TOut, BN, EPI>;
+  const size_t smem = GemmShape<BN, EPI>::kSmemBytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  kern<<<grid, 192, smem, st>>>(a, a2, b, args);
+  return cudaGetLastError();
+}
+
+template <typename TIn, typename TOut, int EPI>
+cudaError_t launch_gemm_bn(int bn, const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b,
+                           const GemmArgs& args, int grid, cudaStream_t st) {
+  if (bn == 32) return launch_gemm<TIn, TOut, 32, EPI>(a, a2, b, args, grid, st);
+  return launch_gemm<TIn, TOut, 256, EPI>(a, a2, b, args, grid, st);
+}
+
+GemmArgs base_args(uint32_t* status) {
+  GemmArgs g{};
+  g.status = status;
+  return g;
+}
+
+// dense C[T, M] = X[T, K] W[M, K]^T
+template <typename TIn, typename TOut>
+muse_status dense_gemm(const void* W, int64_t M, const void* X, int64_t T, int64_t K, void* out, int bn,
+                       uint32_t* status, cudaStream_t st) {
+  CUtensorMap ma, mb;
+  const bool bf = sizeof(TIn) == 2;
+  if (!make_map(&ma, W, bf, K, M, 128) || !make_map(&mb, X, bf, K, T, 16)) return MUSE_ERR_CUDA;
+  GemmArgs g = base_args(status);
+  g.m_tiles = static_cast<int>(cdiv(M, 128));
+  g.num_tiles = static_cast<int>(g.m_tiles * cdiv(T, bn));
+  g.rows_per_group = 0;
+  g.m_valid = static_cast<int>(M);
+  g.T = static_cast<int>(T);
+  g.k_blocks = static_cast<int>(cdiv(K * sizeof(TIn), 128));
+  g.out = out;
+  g.ld_out = M;
+  const int grid = std::min(g.num_tiles, sm_count());
+  return launch_gemm_bn<TIn, TOut, EPI_STORE>(bn, ma, ma, mb, g, grid, st) == cudaSuccess ? MUSE_OK
+                                                                                          : MUSE_ERR_CUDA;
+}
+
+#define MUSE_CK(x)                                 \
+  do {                                             \
+    if ((x) != cudaSuccess) return MUSE_ERR_CUDA;  \
+  } while (0)
+
+template <typename T>
+muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void* x, const void* W_router,
+                         const void* W_pool, const void* W_gate, const void* W_up, const void* W_down,
+                         const void* gamma, const void* W_unpool, void* out, cudaStream_t st) {
+  uint8_t* ws = static_cast<uint8_t*>(c.workspace);
+  auto at = [&](size_t off) { return ws + off; };
+  uint32_t* status = reinterpret_cast<uint32_t*>(at(lay.pub.status));
+  int* counts = reinterpret_cast<int*>(at(lay.pub.expert_count));
+  int* offsets = reinterpret_cast<int*>(at(lay.pub.expert_offset));
+  int* ntiles = reinterpret_cast<int*>(at(lay.ntiles));
+  float* logits = reinterpret_cast<float*>(at(lay.pub.logits));
+  int* topk_idx = reinterpret_cast<int*>(at(lay.pub.topk_idx));
+  float* topk_w = reinterpret_cast<float*>(at(lay.pub.topk_w));
+  int* inv = reinterpret_cast<int*>(at(lay.pub.inv));
+  int* row_token = reinterpret_cast<int*>(at(lay.pub.row_token));
+  int4* tiles_gu = reinterpret_cast<int4*>(at(lay.tiles_gu));
+  int4* tiles_dn = reinterpret_cast<int4*>(at(lay.tiles_dn));
+  T* z = reinterpret_cast<T*>(at(lay.pub.z));
+  T* zp = reinterpret_cast<T*>(at(lay.pub.zp));
+  T* h = reinterpret_cast<T*>(at(lay.pub.h));
+  T* y = reinterpret_cast<T*>(at(lay.pub.y));
+  float* ss = reinterpret_cast<float*>(at(lay.pub.ss));
+  T* cbuf = reinterpret_cast<T*>(at(lay.pub.c));
+  const bool bf = sizeof(T) == 2;
+  const int64_t Tn = c.T, D = c.D, L = c.L, I = c.I, E = c.E, k = c.top_k;
+  const int64_t assign = Tn * k;
+  const int nsm = sm_count();
+  const int bn_d = dense_bn(c), bn_g = grouped_bn(c);
+
+  MUSE_CK(cudaMemsetAsync(status, 0, 16, st));
+  MUSE_CK(cudaMemsetAsync(counts, 0, sizeof(int) * E, st));
+
+  // (a1) router logits
+  if (bf) {
+    muse_status s = dense_gemm<T, float>(W_router, E, x, Tn, D, logits, bn_d, status, st);
+    if (s != MUSE_OK) return s;
+  } else {
+    k_router_logits_f32<<<static_cast<unsigned>(Tn), 256, 0, st>>>(reinterpret_cast<const float*>(x),
+                                                                  reinterpret_cast<const float*>(W_router),
+                                                                  static_cast<int>(D), static_cast<int>(E), logits);
+    MUSE_CK(cudaGetLastError());
+  }
+  // (a2) top-k and weights
+  k_topk<<<static_cast<unsigned>(cdiv(Tn * 32, 256)), 256, 0, st>>>(
+      logits, static_cast<int>(Tn), static_cast<int>(E), static_cast<int>(k), c.router_bias, c.router_mode,
+      c.router_logit_scale, c.routed_scaling, topk_idx, topk_w, c.topk_idx_out, c.topk_w_out);
+  MUSE_CK(cudaGetLastError());
+  // (a3) permutation
+  {
+    const int grid = static_cast<int>(std::min<int64_t>(cdiv(assign, 256), 4 * nsm));
+    k_expert_hist<<<grid, 256, sizeof(int) * E, st>>>(topk_idx, static_cast<int>(assign), static_cast<int>(E),
+                                                      counts, status);
+    MUSE_CK(cudaGetLastError());
+    const int threads = static_cast<int>(align_up(static_cast<size_t>(E), 32));
+    k_build_tiles<<<1, threads, 0, st>>>(counts, static_cast<int>(E), bn_g, static_cast<int>(I / 128),
+                                         static_cast<int>(L / 128), offsets, tiles_gu, ntiles, tiles_dn, ntiles + 1,
+                                         row_token);
+    MUSE_CK(cudaGetLastError());
+    k_assign_rows<<<static_cast<unsigned>(E), 1024, 0, st>>>(topk_idx, static_cast<int>(assign), static_cast<int>(k),
+                                                            counts, offsets, inv, row_token);
+    MUSE_CK(cudaGetLastError());
+  }
+  // (a4) pooler
+  {
+    muse_status s = dense_gemm<T, T>(W_pool, L, x, Tn, D, z, bn_d, status, st);
+    if (s != MUSE_OK) return s;
+  }
+  // (a5) gather into expert order
+  {
+    const int vpr = static_cast<int>(L * sizeof(T) / 16);
+    k_gather_rows<<<4 * nsm, 256, 0, st>>>(row_token, offsets + E, reinterpret_cast<const uint4*>(z),
+                                           reinterpret_cast<uint4*>(zp), vpr);
+    MUSE_CK(cudaGetLastError());
+  }
+  const int64_t R = lay.pub.rows;
+  // (a6) gate/up + SwiGLU
+  {
+    CUtensorMap mg, mu, mb;
+    if (!make_map(&mg, W_gate, bf, L, E * I, 128) || !make_map(&mu, W_up, bf, L, E * I, 128) ||
+        !make_map(&mb, zp, bf, L, R, 16))
+      return MUSE_ERR_CUDA;
+    GemmArgs g = base_args(status);
+    g.tiles = tiles_gu;
+    g.num_tiles_dev = ntiles;
+    g.rows_per_group = static_cast<int>(I);
+    g.m_valid = static_cast<int>(I);
+    g.k_blocks = static_cast<int>(L * sizeof(T) / 128);
+    g.out = h;
+    g.ld_out = I;
+    MUSE_CK((launch_gemm_bn<T, T, EPI_SWIGLU>(bn_g, mg, mu, mb, g, nsm, st)));
+  }
+  // (a7) down projection + sum-of-squares partials
+  {
+    CUtensorMap md, mb;
+    if (!make_map(&md, W_down, bf, I, E * L, 128) || !make_map(&mb, h, bf, I, R, 16)) return MUSE_ERR_CUDA;
+    GemmArgs g = base_args(status);
+    g.tiles = tiles_dn;
+    g.num_tiles_dev = ntiles + 1;
+    g.rows_per_group = static_cast<int>(L);
+    g.m_valid = static_cast<int>(L);
+    g.k_blocks = static_cast<int>(I * sizeof(T) / 128);
+    g.out = y;
+    g.ld_out = L;
+    g.ss = ss;
+    g.ss_ld = static_cast<int>(L / 32);
+    if (c.norm_mode == MUSE_NORM_INPUT_SCALED) {
+      g.ss_gain = gamma;
+      g.ss_gain_group_stride = c.gamma_shared ? 0 : L;
+    }
+    MUSE_CK((launch_gemm_bn<T, T, EPI_STORE_SS>(bn_g, md, md, mb, g, nsm, st)));
+  }
+  // (a8 + a9) per-expert RMSNorm and weighted combine
+  {
+    const int vec = 16 / static_cast<int>(sizeof(T));
+    const int threads = static_cast<int>(std::max<int64_t>(32, align_up(static_cast<size_t>(L / vec), 32)));
+    k_combine<T><<<static_cast<unsigned>(Tn), threads, 0, st>>>(
+        topk_idx, topk_w, inv, ss, static_cast<int>(L / 32), y, reinterpret_cast<const T*>(gamma),
+        c.gamma_shared ? 0 : L, static_cast<int>(L), static_cast<int>(k), c.eps, cbuf);
+    MUSE_CK(cudaGetLastError());
+  }
+  // (a10) unpooler
+  return dense_gemm<T, T>(W_unpool, D, cbuf, Tn, L, out, bn_d, status, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+void muse_moe_config_init(muse_moe_config* cfg) {
+  if (cfg == nullptr) return;
+  std::memset(cfg, 0, sizeof(*cfg));
+  cfg->top_k = 1;
+  cfg->dtype = MUSE_BF16;
+  cfg->eps = 1e-6f;
+  cfg->router_mode = MUSE_ROUTER_SOFTMAX;
+  cfg->router_logit_scale = 1.0f;
+  cfg->routed_scaling = 1.0f;
+  cfg->norm_mode = MUSE_NORM_CENTRED;
+  cfg->pre_norm_eps = 1e-5f;
+}
+
+muse_status muse_latent_moe_workspace_size(const muse_moe_config* cfg, size_t* bytes) {
+  if (bytes == nullptr) return MUSE_ERR_INVALID_ARG;
+  const muse_status s = validate_sizes(cfg);
+  if (s != MUSE_OK) return s;
+  *bytes = make_layout(*cfg).pub.total;
+  return MUSE_OK;
+}
+
+muse_status muse_latent_moe_workspace_layout(const muse_moe_config* cfg, muse_moe_workspace_layout* layout) {
+  if (layout == nullptr) return MUSE_ERR_INVALID_ARG;
+  const muse_status s = validate_sizes(cfg);
+  if (s != MUSE_OK) return s;
+  *layout = make_layout(*cfg).pub;
+  return MUSE_OK;
+}
+
+muse_status muse_latent_moe_forward(const muse_moe_config* cfg, const void* x, const void* W_router,
+                                    const void* W_pool, const void* W_gate, const void* W_up, const void* W_down,
+                                    const void* gamma, const void* W_unpool, void* out, void* stream) {
+  muse_status s = validate_sizes(cfg);
+  if (s != MUSE_OK) return s;
+  const void* ptrs[] = {x, W_router, W_pool, W_gate, W_up, W_down, gamma, W_unpool, out};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return MUSE_ERR_INVALID_ARG;
+  if (cfg->router_bias != nullptr && (reinterpret_cast<uintptr_t>(cfg->router_bias) & 3u)) return MUSE_ERR_INVALID_ARG;
+  const Layout lay = make_layout(*cfg);
+  if (cfg->workspace == nullptr || (reinterpret_cast<uintptr_t>(cfg->workspace) & (kAlign - 1)))
+    return MUSE_ERR_WORKSPACE;
+  if (cfg->workspace_bytes < lay.pub.total) return MUSE_ERR_WORKSPACE;
+  if (encode_fn() == nullptr) return MUSE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cfg->dtype == MUSE_BF16)
+    return forward_impl<__nv_bfloat16>(*cfg, lay, x, W_router, W_pool, W_gate, W_up, W_down, gamma, W_unpool, out, st);
+  return forward_impl<float>(*cfg, lay, x, W_router, W_pool, W_gate, W_up, W_down, gamma, W_unpool, out, st);
+}
+
+muse_status muse_latent_moe_forward_host_io(const muse_moe_config* cfg, const void* x_host, void* x_dev,
+                                            const void* W_router, const void* W_pool, const void* W_gate,
+                                            const void* W_up, const void* W_down, const void* gamma,
+                                            const void* W_unpool, void* out_dev, void* out_host, void* stream) {
+  muse_status s = validate_sizes(cfg);
+  if (s != MUSE_OK) return s;
+  if (x_host == nullptr || out_host == nullptr || x_dev == nullptr || out_dev == nullptr) return MUSE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t bytes = static_cast<size_t>(cfg->T) * cfg->D * act_size(*cfg);
+  if (cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return MUSE_ERR_CUDA;
+  s = muse_latent_moe_forward(cfg, x_dev, W_router, W_pool, W_gate, W_up, W_down, gamma, W_unpool, out_dev, stream);
+  if (s != MUSE_OK) return s;
+  if (cudaMemcpyAsync(out_host, out_dev, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) return MUSE_ERR_CUDA;
+  return MUSE_OK;
+}
+
+muse_status muse_latent_moe_last_device_status(const muse_moe_config* cfg, void* stream, uint32_t* detail) {
+  muse_status s = validate_sizes(cfg);
+  if (s != MUSE_OK) return s;
+  if (cfg->workspace == nullptr) return MUSE_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MUSE_ERR_CUDA;
+  uint32_t word[2] = {0, 0};
+  const Layout lay = make_layout(*cfg);
+  if (cudaMemcpy(word, static_cast<uint8_t*>(cfg->workspace) + lay.pub.status, sizeof(word),
+                 cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MUSE_ERR_CUDA;
+  if (detail != nullptr) *detail = word[1];
+  return static_cast<muse_status>(word[0]);
+}
+
+const char* muse_status_string(muse_status s) {
+  switch (s) {
+    case MUSE_OK: return "ok";
+    case MUSE_ERR_INVALID_ARG: return "invalid argument";
+    case MUSE_ERR_UNSUPPORTED: return "unsupported shape or mode";
+    case MUSE_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case MUSE_ERR_CUDA: return "CUDA call failed";
+    case MUSE_ERR_TIMEOUT: return "device-side wait timed out";
+    case MUSE_ERR_DEVICE: return "device-side check failed";
+  }
+  return "unknown status";
+}
+
+int32_t muse_latent_moe_launch_count(const muse_moe_config* cfg) {
+  if (validate_sizes(cfg) != MUSE_OK) return -1;
+  // router, top-k, hist, tiles, rows, pooler, gather, gate/up, down, combine, unpooler
+  return 11;
+}
+
+}  // extern "C"

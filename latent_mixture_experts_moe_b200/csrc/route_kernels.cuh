@@ -1,0 +1,310 @@
+// route_kernels.cuh -- the non-GEMM steps of the latent-MoE block:
+//   router logits in FP32 FMA (float32 workloads only), top-k selection and weights,
+//   token -> expert permutation (histogram, padded prefix sum, device tile lists,
+//   stable rank), gather into expert order, and the per-expert-RMSNorm weighted combine.
+// All of them are deterministic: integer atomics only for counts, fixed-order FP32 sums.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "gemm_umma.cuh"
+
+namespace muse {
+
+__device__ __forceinline__ float neg_inf() { return -__int_as_float(0x7f800000); }
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Exclusive prefix sum over the block (blockDim.x a multiple of 32, <= 1024); *total
+// receives the block sum. Every thread of the block must call it.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* total) {
+  __shared__ int warp_tot[32];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += u;
+  }
+  __syncthreads();
+  if (lane == 31) warp_tot[w] = inc;
+  __syncthreads();
+  if (w == 0) {
+    int x = lane < nw ? warp_tot[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += u;
+    }
+    warp_tot[lane] = x;  // inclusive over warps
+  }
+  __syncthreads();
+  const int before = (w == 0) ? 0 : warp_tot[w - 1];
+  *total = warp_tot[nw - 1];
+  return before + inc - v;
+}
+
+// --------------------------------------------------------------------------------------
+// (a1, float32 workloads) router logits l[t, e] = sum_d W_router[e, d] x[t, d] in FP32
+// FMA, so routing decisions of float32 inputs see FP32 and not TF32 products.
+// One block per token, a warp per expert, lanes stride over d, fixed-order reduction.
+// --------------------------------------------------------------------------------------
+__global__ void k_router_logits_f32(const float* __restrict__ x, const float* __restrict__ Wr,
+                                    int D, int E, float* __restrict__ logits) {
+  const int t = blockIdx.x;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const float* xr = x + static_cast<int64_t>(t) * D;
+  for (int e = w; e < E; e += nw) {
+    const float* wr = Wr + static_cast<int64_t>(e) * D;
+    float s = 0.0f;
+    for (int d = lane; d < D; d += 32) s = fmaf(wr[d], xr[d], s);
+    s = warp_sum(s);
+    if (lane == 0) logits[static_cast<int64_t>(t) * E + e] = s;
+  }
+}
+
+// --------------------------------------------------------------------------------------
+// (a2) top-k selection and routing weights, one warp per token.
+// key = l + b (softmax mode) or sigmoid(scale*l) + b (sigmoid mode); the k largest keys
+// are taken one at a time by a warp argmax with ties to the lower expert index, so
+// slot j holds the j-th largest key. Weights use the unbiased logits:
+//   softmax: g_j = exp(l_j - m) / sum_S exp(l - m)  (softmax over E renormalised on S)
+//   sigmoid: g_j = rsf * s_j / (sum_S s + 1e-15)
+// --------------------------------------------------------------------------------------
+__global__ void k_topk(const float* __restrict__ logits, int T, int E, int k,
+                       const float* __restrict__ bias, int mode, float scale, float rsf,
+                       int* __restrict__ idx_out, float* __restrict__ w_out,
+                       int* __restrict__ user_idx, float* __restrict__ user_w) {
+  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;  // warp-uniform
+  const float* l = logits + static_cast<int64_t>(t) * E;
+  const int npl = (E + 31) >> 5;
+  float key[32];
+  uint32_t taken = 0;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    key[i] = neg_inf();
+    if (i < npl) {
+      const int e = lane + 32 * i;
+      if (e < E) {
+        const float li = l[e];
+        float kv = (mode == 0) ? li : 1.0f / (1.0f + expf(-scale * li));
+        if (bias != nullptr) kv += bias[e];
+        key[i] = (kv == kv) ? kv : neg_inf();  // a NaN key never wins over a number
+      } else {
+        taken |= 1u << i;
+      }
+    } else {
+      taken |= 1u << i;
+    }
+  }
+  int my_sel = 0;
+  for (int j = 0; j < k; ++j) {
+    float bk = neg_inf();
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int e = lane + 32 * i;
+      if (!((taken >> i) & 1u) && (key[i] > bk || (key[i] == bk && e < bi))) {
+        bk = key[i];
+        bi = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ok > bk || (ok == bk && oi < bi)) {
+        bk = ok;
+        bi = oi;
+      }
+    }
+    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    if (lane == j) my_sel = bi;
+  }
+  const bool mine = lane < k;
+  const float lj = mine ? l[my_sel] : 0.0f;
+  float g;
+  if (mode == 0) {
+    const float m = warp_max(mine ? lj : neg_inf());
+    const float pj = mine ? expf(lj - m) : 0.0f;
+    g = pj / warp_sum(pj);
+  } else {
+    const float sj = mine ? 1.0f / (1.0f + expf(-scale * lj)) : 0.0f;
+    g = rsf * sj / (warp_sum(sj) + 1e-15f);
+  }
+  if (mine) {
+    const int64_t o = static_cast<int64_t>(t) * k + lane;
+    idx_out[o] = my_sel;
+    w_out[o] = g;
+    if (user_idx != nullptr) user_idx[o] = my_sel;
+    if (user_w != nullptr) user_w[o] = g;
+  }
+}
+
+// --------------------------------------------------------------------------------------
+// (a3) permutation, step 1: tokens per expert (integer atomics: exact, order-free).
+// --------------------------------------------------------------------------------------
+__global__ void k_expert_hist(const int* __restrict__ idx, int n, int E, int* __restrict__ counts,
+                              uint32_t* status) {
+  extern __shared__ int hist[];
+  for (int i = threadIdx.x; i < E; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  for (int a = blockIdx.x * blockDim.x + threadIdx.x; a < n; a += gridDim.x * blockDim.x) {
+    const int e = idx[a];
+    if (static_cast<unsigned>(e) < static_cast<unsigned>(E))
+      atomicAdd(&hist[e], 1);
+    else
+      record_status(status, kStatusDevice, 0x1000u);
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < E; i += blockDim.x)
+    if (hist[i]) atomicAdd(&counts[i], hist[i]);
+}
+
+// --------------------------------------------------------------------------------------
+// (a3) step 2 (one block, thread per expert): padded row offsets (each expert's rows
+// rounded up to a multiple of 16, the MMA's N granularity), the two grouped-GEMM tile
+// lists and the padding rows' token = -1. An expert's n rows split into
+// ceil(n / BN) near-equal chunks of a multiple of 16 rows; tiles are ordered expert,
+// feature tile, chunk, so the chunks sharing one weight tile run side by side.
+// --------------------------------------------------------------------------------------
+__global__ void k_build_tiles(const int* __restrict__ counts, int E, int BN, int mt_gu, int mt_dn,
+                              int* __restrict__ offsets, int4* __restrict__ tiles_gu,
+                              int* __restrict__ ntiles_gu, int4* __restrict__ tiles_dn,
+                              int* __restrict__ ntiles_dn, int* __restrict__ row_token) {
+  const int e = threadIdx.x;
+  const int n = (e < E) ? counts[e] : 0;
+  const int padded = (n + 15) & ~15;
+  int total_rows, total_gu, total_dn;
+  const int off = block_exclusive_scan(padded, &total_rows);
+  const int nch = (n + BN - 1) / BN;
+  const int chunk = nch ? ((((n + nch - 1) / nch) + 15) & ~15) : 0;
+  const int gu_off = block_exclusive_scan(nch * mt_gu, &total_gu);
+  const int dn_off = block_exclusive_scan(nch * mt_dn, &total_dn);
+  if (e < E) {
+    offsets[e] = off;
+    for (int ft = 0; ft < mt_gu; ++ft)
+      for (int ch = 0; ch < nch; ++ch)
+        tiles_gu[gu_off + ft * nch + ch] = make_int4(e, ft * 128, off + ch * chunk, min(chunk, n - ch * chunk));
+    for (int ft = 0; ft < mt_dn; ++ft)
+      for (int ch = 0; ch < nch; ++ch)
+        tiles_dn[dn_off + ft * nch + ch] = make_int4(e, ft * 128, off + ch * chunk, min(chunk, n - ch * chunk));
+    for (int r = off + n; r < off + padded; ++r) row_token[r] = -1;
+  }
+  if (threadIdx.x == 0) {
+    offsets[E] = total_rows;
+    *ntiles_gu = total_gu;
+    *ntiles_dn = total_dn;
+  }
+}
+
+// --------------------------------------------------------------------------------------
+// (a3) step 3 (block per expert): stable rank of each assignment a = t*k + j among the
+// assignments to the same expert, in increasing a (token ascending, slot ascending):
+// row = offsets[e] + rank; inv[a] = row, row_token[row] = t.
+// --------------------------------------------------------------------------------------
+__global__ void k_assign_rows(const int* __restrict__ idx, int n, int k, const int* __restrict__ counts,
+                              const int* __restrict__ offsets, int* __restrict__ inv,
+                              int* __restrict__ row_token) {
+  const int e = blockIdx.x;
+  const int cnt = counts[e];
+  if (cnt == 0) return;  // block-uniform
+  const int base_row = offsets[e];
+  int found = 0;
+  for (int a0 = 0; a0 < n && found < cnt; a0 += blockDim.x) {
+    const int a = a0 + threadIdx.x;
+    const int flag = (a < n && idx[a] == e) ? 1 : 0;
+    int tot;
+    const int rank = found + block_exclusive_scan(flag, &tot);
+    if (flag) {
+      const int row = base_row + rank;
+      inv[a] = row;
+      row_token[row] = a / k;
+    }
+    found += tot;
+  }
+}
+
+// --------------------------------------------------------------------------------------
+// (a3) gather: Zp[row] = z[row_token[row]] (zeros for padding rows), 16-byte vectors.
+// --------------------------------------------------------------------------------------
+__global__ void k_gather_rows(const int* __restrict__ row_token, const int* __restrict__ total_rows,
+                              const uint4* __restrict__ z, uint4* __restrict__ zp, int vec_per_row) {
+  const int64_t R = *total_rows;
+  const int64_t nvec = R * vec_per_row;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < nvec;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / vec_per_row;
+    const int c = static_cast<int>(i - r * vec_per_row);
+    const int tok = row_token[r];
+    zp[i] = (tok >= 0) ? z[static_cast<int64_t>(tok) * vec_per_row + c] : make_uint4(0, 0, 0, 0);
+  }
+}
+
+// --------------------------------------------------------------------------------------
+// (a8 + a9) per-expert RMSNorm applied inside the weighted combine, one block per token:
+//   c[t] = sum_j g_j * y_j / sqrt(ss_j / L + eps) * (1 + gamma[e_j])
+// j in routing order, FP32 accumulation, 16-byte loads. ss_j is the sum of the row's
+// L/32 partial sums of squares (fixed order) written by the down-projection epilogue;
+// in input-scaled mode those partials were taken of y * (1 + gamma) instead of y.
+// --------------------------------------------------------------------------------------
+template <typename T>
+__global__ void k_combine(const int* __restrict__ topk_idx, const float* __restrict__ topk_w,
+                          const int* __restrict__ inv, const float* __restrict__ ss, int ss_ld,
+                          const T* __restrict__ Y, const T* __restrict__ gamma, int64_t gamma_stride,
+                          int L, int k, float eps, T* __restrict__ c) {
+  constexpr int VEC = 16 / sizeof(T);
+  __shared__ float scale_s[32];
+  __shared__ int pos_s[32];
+  __shared__ int e_s[32];
+  const int t = blockIdx.x;
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    for (int j = 0; j < k; ++j) {
+      const int64_t a = static_cast<int64_t>(t) * k + j;
+      const int pos = inv[a];
+      float s = 0.0f;
+      for (int i = lane; i < ss_ld; i += 32) s += ss[static_cast<int64_t>(pos) * ss_ld + i];
+      s = warp_sum(s);
+      if (lane == 0) {
+        scale_s[j] = topk_w[a] * (1.0f / sqrtf(s / static_cast<float>(L) + eps));
+        pos_s[j] = pos;
+        e_s[j] = topk_idx[a];
+      }
+    }
+  }
+  __syncthreads();
+  const int f0 = threadIdx.x * VEC;
+  if (f0 >= L) return;
+  float acc[VEC];
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) acc[v] = 0.0f;
+  for (int j = 0; j < k; ++j) {
+    const uint4 yv = *reinterpret_cast<const uint4*>(Y + static_cast<int64_t>(pos_s[j]) * L + f0);
+    const uint4 gv = *reinterpret_cast<const uint4*>(gamma + e_s[j] * gamma_stride + f0);
+    const T* yy = reinterpret_cast<const T*>(&yv);
+    const T* gg = reinterpret_cast<const T*>(&gv);
+    const float sj = scale_s[j];
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) acc[v] = fmaf(sj * (1.0f + to_f32(gg[v])), to_f32(yy[v]), acc[v]);
+  }
+  uint4 ov;
+  T* oo = reinterpret_cast<T*>(&ov);
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) oo[v] = from_f32<T>(acc[v]);
+  *reinterpret_cast<uint4*>(c + static_cast<int64_t>(t) * L + f0) = ov;
+}
+
+}  // namespace muse

@@ -1,0 +1,140 @@
+"""Helpers of the GPU parity tests: run the CUDA path through the C ABI, run the FP64
+oracle on the same bytes, and compare with the tolerances the block is held to.
+
+Tolerances (for every workload):
+  * expert indices: the selected SET must equal the oracle's exactly, except for tokens
+    whose k-th and (k+1)-th oracle keys differ by less than TIE_TOL; for those the GPU
+    set must be one of the oracle's own valid alternatives, and the oracle output for
+    that alternative is the reference. The ORDER inside the set must be non-increasing
+    in the oracle's keys up to TIE_TOL (several orders are correct for near-equal keys);
+  * routing weights: |g_gpu - g_oracle| <= 2e-4 per selected expert;
+  * outputs: relative L2 error <= 1e-2 and max-abs error <= 5e-2 * rms(out).
+"""
+from __future__ import annotations
+
+import math
+from typing import Dict, Optional, Sequence
+
+import numpy as np
+import torch
+
+import latent_mixture_experts_moe_b200 as moe
+import oracle
+import workloads as W
+
+TIE_TOL = 1e-4
+G_TOL = 2e-4
+REL_L2 = 1e-2
+MAX_ABS_RMS = 5e-2
+
+
+def rel_l2(got: np.ndarray, ref: np.ndarray) -> float:
+    return float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300))
+
+
+def assert_close(got: np.ndarray, ref: np.ndarray, what: str, rel=REL_L2, max_abs_rms=MAX_ABS_RMS):
+    got = np.asarray(got, dtype=np.float64)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
+    r = rel_l2(got, ref)
+    rms = math.sqrt(float(np.mean(ref * ref)))
+    ma = float(np.abs(got - ref).max())
+    assert r <= rel, f"{what}: rel-L2 {r:.3e} > {rel}"
+    assert ma <= max_abs_rms * rms, f"{what}: max-abs {ma:.3e} > {max_abs_rms} * rms {rms:.3e}"
+    return r, ma / rms
+
+
+def ws_view(ws: torch.Tensor, off: int, dtype: torch.dtype, shape: Sequence[int]) -> torch.Tensor:
+    n = int(np.prod(shape)) * torch.tensor([], dtype=dtype).element_size()
+    return ws[off:off + n].view(dtype).view(*shape)
+
+
+class Run:
+    """One forward of the CUDA path with its routing outputs and workspace."""
+
+    def __init__(self, w: W.Workload, inp: Dict[str, torch.Tensor], T: Optional[int] = None, **modes):
+        T = T or w.T
+        self.w, self.T = w, T
+        weights = {k: v for k, v in inp.items() if k != "x"}
+        self.model = moe.LatentMoE(weights, T_max=T, k=w.k, eps=w.eps, **modes)
+        dev = inp["x"].device
+        self.idx = torch.full((T, w.k), -1, dtype=torch.int32, device=dev)
+        self.g = torch.zeros((T, w.k), dtype=torch.float32, device=dev)
+        self.out = self.model(inp["x"][:T], topk_idx=self.idx, topk_w=self.g)
+        torch.cuda.synchronize()
+        cfg = self.model.config(T, self.model.workspace)
+        code, detail = moe.last_device_status(cfg)
+        assert code == 0, f"device status {moe.STATUS.get(code)} detail {detail:#x}"
+        self.layout = moe.workspace_layout(cfg)
+
+    def inter(self, name: str, dtype, shape):
+        return ws_view(self.model.workspace, self.layout[name], dtype, shape)
+
+    def act(self):
+        return torch.float32 if self.w.dtype == "f32" else torch.bfloat16
+
+
+def host(t: torch.Tensor) -> np.ndarray:
+    return oracle.as_f64(t)
+
+
+def expert_source(inp: Dict[str, torch.Tensor]):
+    return lambda e: (inp["W_gate"][e], inp["W_up"][e], inp["W_down"][e])
+
+
+def oracle_block(w: W.Workload, inp: Dict[str, torch.Tensor], rows: np.ndarray, **kw) -> Dict[str, np.ndarray]:
+    """The oracle on token rows `rows` of x (tokens are independent)."""
+    x = host(inp["x"][torch.as_tensor(rows, device=inp["x"].device)])
+    bias = host(inp["router_bias"]) if "router_bias" in inp else None
+    return oracle.latent_moe_forward(x, host(inp["W_router"]), host(inp["W_pool"]), expert_source(inp),
+                                     host(inp["gamma"]), host(inp["W_unpool"]), w.k, w.eps, router_bias=bias,
+                                     **kw)
+
+
+def check_routing(ref: Dict[str, np.ndarray], gpu_idx: np.ndarray, gpu_g: np.ndarray, k: int):
+    """Returns the tokens whose GPU set is a valid alternative different from the oracle's
+    (near ties), after checking every token's set, order and weights."""
+    keys, ridx, rg = ref["keys"], ref["idx"], ref["g"]
+    alt_tokens = []
+    for t in range(gpu_idx.shape[0]):
+        gs, rs = set(gpu_idx[t].tolist()), set(ridx[t].tolist())
+        assert len(gs) == k, f"token {t}: repeated expert in {gpu_idx[t]}"
+        if gs != rs:
+            srt = np.sort(keys[t])[::-1]
+            gap = srt[k - 1] - srt[k] if k < keys.shape[1] else np.inf
+            assert gap < TIE_TOL, f"token {t}: GPU {sorted(gs)} vs oracle {sorted(rs)}, gap {gap:.2e}"
+            assert tuple(sorted(gs)) in oracle.topk_alternatives(keys[t], k, TIE_TOL), f"token {t}"
+            alt_tokens.append(t)
+        ko = keys[t][gpu_idx[t]]
+        assert np.all(np.diff(ko) <= TIE_TOL), f"token {t}: order {gpu_idx[t]} keys {ko}"
+        if gs == rs:
+            for j in range(k):
+                e = gpu_idx[t, j]
+                jr = int(np.nonzero(ridx[t] == e)[0][0])
+                assert abs(gpu_g[t, j] - rg[t, jr]) <= G_TOL, f"token {t} expert {e}: g {gpu_g[t, j]} vs {rg[t, jr]}"
+    return alt_tokens
+
+
+def oracle_on_gpu_alternatives(w, inp, rows, ref, gpu_idx, alt_tokens, **kw):
+    """For near-tie tokens, the oracle output under the oracle's alternative routing that
+    the GPU chose (found in oracle.topk_alternatives), with the oracle's own weights."""
+    out = ref["out"].copy()
+    for t in alt_tokens:
+        sel = np.array(sorted(gpu_idx[t].tolist(), key=lambda e: (-ref["keys"][t][e], e)))[None, :]
+        g = oracle.softmax_weights(ref["logits"][t:t + 1], sel)
+        r1 = oracle_block(w, inp, rows[t:t + 1], routing=(sel, g), **kw)
+        out[t] = r1["out"][0]
+    return out
+
+
+def expected_permutation(idx: np.ndarray, E: int):
+    """Integer definition of the expert-ordered rows: assignments a = t*k + j grouped by
+    expert, ascending a inside each expert, each expert's group padded to 16 rows."""
+    flat = idx.reshape(-1)
+    counts = np.bincount(flat, minlength=E)
+    padded = (counts + 15) // 16 * 16
+    offsets = np.concatenate([[0], np.cumsum(padded)])
+    inv = np.empty(flat.size, dtype=np.int64)
+    for e in range(E):
+        a = np.nonzero(flat == e)[0]
+        inv[a] = offsets[e] + np.arange(a.size)
+    return counts, offsets, inv

@@ -1,0 +1,178 @@
+"""GPU parity: the CUDA path (through the C ABI) against the FP64 oracle on the same
+seeded inputs. Small workloads are compared element by element, every intermediate too;
+full-size workloads on every routing decision and on sampled tokens' outputs.
+"""
+import numpy as np
+import pytest
+import torch
+
+import latent_mixture_experts_moe_b200 as moe
+import oracle
+import workloads as W
+from parity_util import (Run, assert_close, check_routing, expected_permutation, host, oracle_block,
+                         oracle_on_gpu_alternatives)
+
+pytestmark = pytest.mark.gpu
+
+
+def full_check(w, inp, run, rows=None, **modes):
+    """Routing, permutation, intermediates and output of `run` against the oracle."""
+    T = run.T
+    rows = np.arange(T) if rows is None else rows
+    ref = oracle_block(w, inp, rows)
+    gidx = run.idx.cpu().numpy()[rows]
+    gg = run.g.cpu().numpy()[rows]
+    alts = check_routing(ref, gidx, gg, w.k)
+    ref_out = oracle_on_gpu_alternatives(w, inp, rows, ref, gidx, alts)
+    out = host(run.out)[rows]
+    assert_close(out, ref_out, f"{w.name} out")
+    return ref, alts
+
+
+# ------------------------------------------------------------------------- small, exact
+@pytest.fixture(scope="module")
+def tiny():
+    w = W.WORKLOADS["tiny"]
+    return w, W.make_inputs(w, "cuda")
+
+
+@pytest.fixture(scope="module")
+def mid():
+    w = W.WORKLOADS["mid"]
+    return w, W.make_inputs(w, "cuda")
+
+
+@pytest.mark.parametrize("name", ["tiny", "mid"])
+def test_small_workload_every_intermediate(name, tiny, mid):
+    w, inp = {"tiny": tiny, "mid": mid}[name]
+    run = Run(w, inp)
+    ref, alts = full_check(w, inp, run)
+    act = run.act()
+    T, k, L, I, E = w.T, w.k, w.L, w.I, w.E
+    # router logits
+    logits = run.inter("logits", torch.float32, (T, E)).cpu().numpy()
+    assert_close(logits, ref["logits"], "logits", rel=1e-4, max_abs_rms=1e-3)
+    # pooler
+    assert_close(host(run.inter("z", act, (T, L))), ref["z"], "z")
+    if alts:
+        return
+    counts, offsets, inv = expected_permutation(ref["idx"], E)
+    R = run.layout["rows"]
+    assert np.array_equal(run.inter("expert_count", torch.int32, (E,)).cpu().numpy(), counts)
+    assert np.array_equal(run.inter("expert_offset", torch.int32, (E + 1,)).cpu().numpy(), offsets)
+    ginv = run.inter("inv", torch.int32, (T * k,)).cpu().numpy()
+    assert np.array_equal(ginv, inv)
+    rtok = run.inter("row_token", torch.int32, (R,)).cpu().numpy()
+    assert np.array_equal(rtok[inv], np.arange(T * k) // k)
+    # expert outputs before the norm, in expert order
+    y = host(run.inter("y", act, (R, L)))[ginv].reshape(T, k, L)
+    assert_close(y, ref["y"], "y")
+    ss = run.inter("ss", torch.float32, (R, L // 32)).cpu().numpy().astype(np.float64)[ginv].sum(1).reshape(T, k)
+    assert_close(ss, ref["ss"], "sum of squares", rel=2e-2)
+    assert_close(host(run.inter("c", act, (T, L))), ref["c"], "combined latent")
+
+
+def test_repeat_runs_are_bitwise_identical(mid):
+    w, inp = mid
+    a = Run(w, inp)
+    b = Run(w, inp)
+    assert torch.equal(a.out, b.out)
+    assert torch.equal(a.idx, b.idx) and torch.equal(a.g, b.g)
+
+
+def test_host_io_entry_point_matches_device_entry_point(mid):
+    w, inp = mid
+    run = Run(w, inp)
+    x_host = inp["x"].cpu().pin_memory()
+    out_host = torch.empty((w.T, w.D), dtype=inp["x"].dtype).pin_memory()
+    x_dev = torch.empty_like(inp["x"])
+    out_dev = torch.empty((w.T, w.D), dtype=inp["x"].dtype, device="cuda")
+    cfg = run.model.config(w.T, run.model.workspace)
+    moe.forward_host_io(cfg, x_host, x_dev, inp["W_router"], inp["W_pool"], inp["W_gate"], inp["W_up"],
+                        inp["W_down"], inp["gamma"], inp["W_unpool"], out_dev, out_host)
+    torch.cuda.synchronize()
+    assert torch.equal(out_host, run.out.cpu())
+
+
+# ------------------------------------------------------------------------- edge cases
+EDGE = [
+    # name, T, D, L, I, E, k, dtype, bias_kind
+    ("one_token", 1, 256, 128, 128, 8, 2, "bf16", None),
+    ("ragged_17", 17, 384, 256, 128, 16, 3, "bf16", None),
+    ("ragged_300_wide_I", 300, 256, 128, 384, 8, 2, "bf16", None),
+    ("empty_experts", 3, 256, 128, 128, 64, 2, "bf16", None),
+    ("expert_takes_all", 300, 256, 128, 128, 8, 2, "bf16", "all_to_0"),
+    ("k_equals_E", 40, 256, 128, 256, 4, 4, "bf16", None),
+    ("k_one", 33, 256, 256, 128, 16, 1, "bf16", None),
+    ("fp32_ragged", 37, 256, 256, 128, 8, 3, "f32", None),
+    ("many_tokens_per_expert", 1100, 256, 128, 128, 4, 2, "bf16", None),
+]
+
+
+@pytest.mark.parametrize("case", EDGE, ids=[c[0] for c in EDGE])
+def test_edge_cases(case):
+    name, T, D, L, I, E, k, dt, bias_kind = case
+    w = W.Workload(name, T=T, D=D, L=L, I=I, E=E, k=k, dtype=dt, seed=3)
+    inp = W.make_inputs(w, "cuda")
+    if bias_kind == "all_to_0":
+        b = torch.zeros(E, dtype=torch.float32)
+        b[0] = 100.0
+        inp["router_bias"] = b.cuda()
+    run = Run(w, inp)
+    ref, alts = full_check(w, inp, run)
+    if bias_kind == "all_to_0":
+        assert np.all(run.idx.cpu().numpy()[:, 0] == 0)
+    if not alts:
+        counts, offsets, inv = expected_permutation(ref["idx"], E)
+        assert np.array_equal(run.inter("inv", torch.int32, (T * k,)).cpu().numpy(), inv)
+
+
+# ------------------------------------------------------------------------- full size
+@pytest.fixture(scope="module")
+def full_weights():
+    w = W.WORKLOADS["prefill"]
+    inp = W.make_inputs(w, "cuda", names=["W_router", "W_pool", "W_gate", "W_up", "W_down", "gamma", "W_unpool"])
+    inp["x"] = W.make_tensor(w, "x", "cuda")
+    yield inp
+    del inp
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.slow
+def test_full_size_decode_all_tokens(full_weights):
+    w = W.WORKLOADS["decode"]
+    run = Run(w, full_weights, T=w.T)
+    full_check(w, full_weights, run)
+    # about 222 distinct experts are touched by 64 tokens x top-8 of 256
+    assert 180 <= len(np.unique(run.idx.cpu().numpy())) <= 256
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["prefill", "prefill_zipf"])
+def test_full_size_prefill_routing_and_sampled_tokens(name, full_weights):
+    w = W.WORKLOADS[name]
+    inp = dict(full_weights)
+    if w.routing == "zipf":
+        inp["router_bias"] = W.zipf_router_bias(w).cuda()
+    run = Run(w, inp)
+    # every routing decision against the oracle (router only: exact definition, all tokens)
+    x = host(inp["x"])
+    logits = oracle.router_logits(x, host(inp["W_router"]))
+    del x
+    bias = host(inp["router_bias"]) if "router_bias" in inp else None
+    idx, g, keys = oracle.route(logits, w.k, bias)
+    alts = check_routing({"keys": keys, "idx": idx, "g": g}, run.idx.cpu().numpy(), run.g.cpu().numpy(), w.k)
+    assert len(alts) <= 4
+    if not alts:
+        counts, offsets, inv = expected_permutation(idx, w.E)
+        assert np.array_equal(run.inter("expert_count", torch.int32, (w.E,)).cpu().numpy(), counts)
+        assert np.array_equal(run.inter("inv", torch.int32, (w.T * w.k,)).cpu().numpy(), inv)
+    if w.routing == "zipf":
+        loads = np.sort(np.bincount(run.idx.cpu().numpy().ravel(), minlength=w.E))[::-1]
+        target = W.zipf_target_loads(w.T, w.E, w.k).numpy()
+        assert loads[0] == w.T and loads[1] == w.T
+        assert np.abs(loads - target).sum() / (w.T * w.k) < 0.02
+    # sampled tokens through the whole block
+    rows = np.random.default_rng(7).choice(w.T, size=12, replace=False)
+    rows.sort()
+    full_check(w, inp, run, rows=rows)
