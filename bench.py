@@ -1,0 +1,441 @@
+#!/usr/bin/env python
+"""Latent-MoE block forward (Muse Spark Open shapes) on B200: tokens/s and roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload prefill|decode|prefill_zipf|mid|tiny] [--no-side]
+
+One step = one forward pass of the whole block (router, top-k, permutation, pooler,
+gather, gate/up + SwiGLU, down + sum of squares, per-expert norm + combine, unpooler)
+over one batch of synthetic tokens already resident in HBM, through the C ABI.
+Default workload: the full-width prefill layer (T=8192, D=8192, L=4096, I=4096,
+E=256, top-8, bf16); the decode layer (T=64) and the Zipf-skewed prefill are timed
+beside it and reported as sub-objects. Multi-GPU: one process per GPU, every rank a
+replica with its own tokens (weak scaling, no data-path collective), time = max over
+ranks of the CUDA-event time.
+
+Timing: W untimed warm-up steps, then K steps between CUDA events on the launching
+stream, with a barrier and a device synchronisation on both sides. Every step streams
+the expert weights (25.8 GB >> 126 MB L2), so inputs are larger than L2 and no flush is
+needed. Per-kernel durations come from events the library records between its launches.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {k: float(d[k]) for k in PEAKS_FALLBACK}, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+# ------------------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+    Q = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = f"GPU-{torch.cuda.get_device_properties(device_index).uuid}"
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-lms", "100", "-i", self.dev], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self, t0: float, t1: float):
+        rows = []
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(f[1]), float(f[2]), f[5:9]))
+            except ValueError:
+                continue
+        inside = [r for r in rows if t0 - 0.05 <= r[0] <= t1 + 0.05] or rows
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in inside for n, v in zip(names, r[3]) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": max(r[2] for r in inside),
+                "reasons": reasons, "samples": len(inside)}
+
+
+# ------------------------------------------------------------------------------ accounting
+def stage_work(w: W.Workload, n_touched: int):
+    """Algorithmic FLOPs and bytes of each launch (only the k selected experts, only the
+    distinct experts the routing touched; intermediates counted where a kernel's job is
+    to move them)."""
+    T, D, L, I, E, k = w.T, w.D, w.L, w.I, w.E, w.k
+    a = 2 if w.dtype == "bf16" else 4
+    A = T * k
+    return {
+        "router": (2 * T * E * D, T * D * a + E * D * a + T * E * 4),
+        "topk": (0, T * E * 4 + A * 8),
+        "expert_hist": (0, A * 4),
+        "tiles": (0, E * 8),
+        "assign_rows": (0, A * 8),
+        "pooler": (2 * T * L * D, T * D * a + L * D * a + T * L * a),
+        "gather": (0, T * L * a + A * L * a),
+        "gate_up_swiglu": (2 * A * L * 2 * I, n_touched * 2 * I * L * a + A * L * a + A * I * a),
+        "down_sumsq": (2 * A * I * L, n_touched * L * I * a + A * I * a + A * L * a + A * (L // 32) * 4),
+        "norm_combine": (0, A * L * a + A * (L // 32) * 4 + T * L * a + n_touched * L * a),
+        "unpooler": (2 * T * D * L, T * L * a + D * L * a + T * D * a),
+    }
+
+
+def step_work(w: W.Workload, n_touched: int):
+    T, D, L, I, E, k = w.T, w.D, w.L, w.I, w.E, w.k
+    a = 2 if w.dtype == "bf16" else 4
+    flops = 2 * T * (E * D + L * D + k * 3 * L * I + D * L)
+    byts = 2 * T * D * a + (E * D + 2 * L * D) * a + n_touched * (3 * L * I + L) * a
+    return flops, byts
+
+
+# ------------------------------------------------------------------------------ our arm
+def make_rank_inputs(w: W.Workload, rank: int, dev):
+    inp = W.make_inputs(w, dev, names=["W_router", "W_pool", "W_gate", "W_up", "W_down", "gamma", "W_unpool"])
+    x = torch.empty((w.T, w.D), dtype=W.TORCH_DTYPE[w.dtype], device=dev)
+    W.fill(x, w.seed, W.TID["x"], 1.0, start=rank * w.T * w.D)   # rank r: tokens [rT, (r+1)T)
+    inp["x"] = x
+    return inp
+
+
+def run_ours(w: W.Workload, inp, steps: int, warmup: int, rank: int, world: int, peaks, peak_kind,
+             sample_clocks: bool, e2e_steps: int):
+    import latent_mixture_experts_moe_b200 as moe
+    dev = inp["x"].device
+    weights = {k: v for k, v in inp.items() if k != "x"}
+    model = moe.LatentMoE(weights, T_max=w.T, k=w.k, eps=w.eps)
+    out = torch.empty((w.T, w.D), dtype=inp["x"].dtype, device=dev)
+    idx = torch.empty((w.T, w.k), dtype=torch.int32, device=dev)
+    nst = len(moe.STAGES)
+    stream = torch.cuda.current_stream()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)] for _ in range(steps)]
+    for row in ev:
+        for e in row:
+            e.record(stream)
+    handles = [moe.event_handles(row) for row in ev]
+    for _ in range(warmup):
+        model(inp["x"], out=out, topk_idx=idx)
+    torch.cuda.synchronize()
+    code, detail = moe.last_device_status(model.config(w.T, model.workspace))
+    if code != 0:
+        raise RuntimeError(f"device status {code} detail {detail:#x}")
+    clocks = ClockSampler(dev.index) if sample_clocks else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    wall0 = time.time()
+    t_start.record(stream)
+    for s in range(steps):
+        model(inp["x"], out=out, topk_idx=idx, stage_events=handles[s])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    wall1 = time.time()
+    barrier(world)
+    if clocks:
+        time.sleep(0.2)
+        clocks.stop()
+    ms = t_start.elapsed_time(t_end)
+    ms_max = all_max(ms, world, dev)
+    code, detail = moe.last_device_status(model.config(w.T, model.workspace))
+    if code != 0:
+        raise RuntimeError(f"device status {code} detail {detail:#x}")
+    stage_ms = [sum(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(steps)) / steps for i in range(nst)]
+    n_touched = int(torch.unique(idx).numel())
+    work = stage_work(w, n_touched)
+    dom = max(range(nst), key=lambda i: stage_ms[i])
+    dname = moe.STAGES[dom]
+    fl, by = work[dname]
+    t_dom = stage_ms[dom] * 1e-3
+    t_tensor = fl / (peaks["bf16_tflops_sustained"] * 1e12)
+    t_hbm = by / (peaks["hbm_gbs"] * 1e9)
+    if t_tensor >= t_hbm:
+        roof = {"bound": "tensor", "achieved": fl / t_dom / 1e12, "peak": peaks["bf16_tflops_sustained"],
+                "unit": "TFLOP/s"}
+        roof["frac_of_burst_peak"] = fl / t_dom / 1e12 / peaks["bf16_tflops"]
+    else:
+        roof = {"bound": "hbm", "achieved": by / t_dom / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["kernel"] = dname
+    roof["peak_source"] = f"{peak_kind} ({'sustained' if roof['bound'] == 'tensor' else 'copy'})"
+    roof["algorithmic_flops"] = fl
+    roof["algorithmic_bytes"] = by
+    roof["traffic"] = measured_traffic(dname, w)
+    sf, sb = step_work(w, n_touched)
+    t_step = ms_max / steps * 1e-3
+    step_roof = max(sf / (peaks["bf16_tflops_sustained"] * 1e12), sb / (peaks["hbm_gbs"] * 1e9))
+    res = {
+        "value": world * w.T * steps / (ms_max * 1e-3),
+        "ms_per_step": ms_max / steps,
+        "stage_ms": {moe.STAGES[i]: round(stage_ms[i], 4) for i in range(nst)},
+        "roofline": roof,
+        "step": {"tflops": sf / t_step / 1e12, "gbs": sb / t_step / 1e9, "roofline_ms": step_roof * 1e3,
+                 "frac_of_step_roofline": step_roof / t_step, "distinct_experts": n_touched},
+        "wall_s": wall1 - wall0,
+        "gpu_launches": steps * moe.launch_count(model.config(w.T)),
+    }
+    if clocks:
+        res["clocks"] = clocks.summary(wall0, wall1)
+    if e2e_steps > 0:
+        res["e2e"] = run_e2e(w, model, inp, e2e_steps, world, dev)
+    return res
+
+
+def run_e2e(w, model, inp, steps, world, dev):
+    """Same metric through the host-buffer entry point: per step, H2D of x from pinned
+    memory, the forward, and D2H of out, all inside the timed region."""
+    import latent_mixture_experts_moe_b200 as moe
+    x_host = inp["x"].cpu().pin_memory()
+    out_host = torch.empty((w.T, w.D), dtype=inp["x"].dtype).pin_memory()
+    x_dev = torch.empty_like(inp["x"])
+    out_dev = torch.empty((w.T, w.D), dtype=inp["x"].dtype, device=dev)
+    cfg = model.config(w.T, model.workspace)
+    wt = model.w
+    args = (wt["W_router"], wt["W_pool"], wt["W_gate"], wt["W_up"], wt["W_down"], wt["gamma"], wt["W_unpool"])
+    for _ in range(2):
+        moe.forward_host_io(cfg, x_host, x_dev, *args, out_dev, out_host)
+    barrier(world)
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        moe.forward_host_io(cfg, x_host, x_dev, *args, out_dev, out_host)
+    e.record()
+    torch.cuda.synchronize()
+    ms = all_max(s.elapsed_time(e), world, dev)
+    nbytes = w.T * w.D * (2 if w.dtype == "bf16" else 4)
+    return {"value": world * w.T * steps / (ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": nbytes,
+            "d2h_bytes_per_step": nbytes, "ms_per_step": ms / steps}
+
+
+def measured_traffic(kernel: str, w: W.Workload):
+    """DRAM bytes per launch from the committed ncu summary, if it matches this kernel
+    source and workload; else None."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+        ent = d.get(f"{w.name}:{kernel}")
+        if ent is None or ent.get("src_sha") != kernel_source_sha():
+            return None
+        return ent["bytes_per_launch"]
+    except (ValueError, KeyError):
+        return None
+
+
+def kernel_source_sha():
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("gemm_umma.cuh", "ptx.cuh", "route_kernels.cuh", "muse_moe.cu"):
+        h.update(open(os.path.join(ROOT, "latent_mixture_experts_moe_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+# ------------------------------------------------------------------------------ oracle arm
+def oracle_sample(w: W.Workload, n_tokens: int, dev, widen: bool):
+    """Host copies of what the oracle needs for tokens [0, n) of the workload: those x
+    rows, the shared weights and the experts their routing touches (generated on `dev`
+    with the shared seeded generator). widen=True converts them to float64 up front."""
+    import oracle
+    xr = torch.empty((n_tokens, w.D), dtype=W.TORCH_DTYPE[w.dtype], device=dev)
+    W.fill(xr, w.seed, W.TID["x"], 1.0)
+    shared = {n: W.make_tensor(w, n, dev).cpu() for n in ("W_router", "W_pool", "gamma", "W_unpool")}
+    x = xr.cpu()
+    bias = W.zipf_router_bias(w) if w.routing == "zipf" else None
+    logits = oracle.router_logits(oracle.as_f64(x), oracle.as_f64(shared["W_router"]))
+    idx, _, _ = oracle.route(logits, w.k, None if bias is None else oracle.as_f64(bias))
+    experts = {}
+    for e in np.unique(idx):
+        experts[int(e)] = tuple(W.expert_slab(w, n, int(e), dev).cpu() for n in ("W_gate", "W_up", "W_down"))
+    if widen:
+        x = oracle.as_f64(x)
+        shared = {n: oracle.as_f64(v) for n, v in shared.items()}
+        experts = {e: tuple(oracle.as_f64(m) for m in v) for e, v in experts.items()}
+        bias = None if bias is None else oracle.as_f64(bias)
+    return x, shared, bias, experts
+
+
+def time_oracle(w, x, shared, bias, experts):
+    """Wall time of one oracle forward (as_f64 is a no-op on pre-widened arrays)."""
+    import oracle
+    f = oracle.as_f64
+    t0 = time.perf_counter()
+    oracle.latent_moe_forward(f(x), f(shared["W_router"]), f(shared["W_pool"]), lambda e: experts[e],
+                              f(shared["gamma"]), f(shared["W_unpool"]), w.k, w.eps,
+                              router_bias=None if bias is None else f(bias))
+    return time.perf_counter() - t0
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def cpu_baseline(w: W.Workload, dev, n_tokens: int):
+    x, shared, bias, experts = oracle_sample(w, n_tokens, dev, widen=False)
+    dt = time_oracle(w, x, shared, bias, experts)
+    return {"value": n_tokens / dt, "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
+            "sample": f"first {n_tokens} tokens of the {w.name} workload (T={w.T}) through the FP64 numpy "
+                      f"oracle, widening bf16 weights to f64 included; {len(experts)} distinct experts; {dt:.1f} s"}
+
+
+def run_reference(w: W.Workload, args, dev):
+    """The FP64 oracle as the reference arm: every step runs the workload's first token
+    through the whole block, on weights widened to float64 before timing."""
+    x, shared, bias, experts = oracle_sample(w, 1, dev, widen=True)
+    times = [time_oracle(w, x, shared, bias, experts) for _ in range(args.warmup + args.steps)][args.warmup:]
+    total = sum(times)
+    value = args.steps / total
+    return {
+        "metric": metric_name(), "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(w), "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
+                         "sample": f"token 0 of the {w.name} workload per step, FP64 numpy oracle, "
+                                   f"weights pre-widened to f64"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ------------------------------------------------------------------------------ plumbing
+def metric_name():
+    return "latent-MoE layer tokens/s on 1 B200 (T=8192 prefill, T=64 decode); % roofline"
+
+
+def config_dict(w: W.Workload):
+    return {"workload": f"{w.name}: latent-MoE layer T={w.T} D={w.D} L={w.L} I={w.I} E={w.E} top-{w.k} "
+                        f"{w.dtype} {w.routing} routing",
+            "T": w.T, "D": w.D, "L": w.L, "I": w.I, "E": w.E, "top_k": w.k, "routing": w.routing,
+            "l2": "inputs larger than L2: each step streams the touched experts' weights (up to 25.8 GB)"}
+
+
+_DIST = {"on": False}
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def all_max(v: float, world: int, dev) -> float:
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="prefill", choices=list(W.WORKLOADS))
+    ap.add_argument("--no-side", action="store_true", help="skip the decode / skewed side workloads")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle cpu_baseline")
+    ap.add_argument("--cpu-tokens", type=int, default=4)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=dev)
+    w = W.WORKLOADS[args.workload]
+    try:
+        if args.impl == "reference":
+            if rank == 0:
+                print(json.dumps(run_reference(w, args, dev)), flush=True)
+            return
+        peaks, peak_kind = load_peaks()
+        inp = make_rank_inputs(w, rank, dev)
+        main_res = run_ours(w, inp, args.steps, args.warmup, rank, world, peaks, peak_kind, True,
+                            e2e_steps=min(args.steps, 20))
+        side = {}
+        if not args.no_side and w.name == "prefill":
+            wd = W.WORKLOADS["decode"]
+            xd = torch.empty((wd.T, wd.D), dtype=inp["x"].dtype, device=dev)
+            W.fill(xd, wd.seed, W.TID["x"], 1.0, start=rank * wd.T * wd.D)
+            inp_d = dict(inp, x=xd)
+            side["decode"] = run_ours(wd, inp_d, max(args.steps, 50), args.warmup, rank, world, peaks, peak_kind,
+                                      False, e2e_steps=0)
+            wz = W.WORKLOADS["prefill_zipf"]
+            inp_z = dict(inp, router_bias=W.zipf_router_bias(wz).to(dev))
+            side["prefill_zipf"] = run_ours(wz, inp_z, args.steps, args.warmup, rank, world, peaks, peak_kind,
+                                            False, e2e_steps=0)
+        if rank == 0:
+            line = {
+                "metric": metric_name(), "value": main_res["value"], "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": main_res["ms_per_step"],
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+                "data": "synthetic (seeded counter-based N(0,1) inputs, N(0,1/fan_in) weights)",
+                "config": dict(config_dict(w), parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
+                "roofline": main_res["roofline"], "step_roofline": main_res["step"],
+                "stage_ms": main_res["stage_ms"], "gpu_launches": main_res["gpu_launches"],
+                "clocks": main_res.get("clocks"), "e2e": main_res.get("e2e"),
+            }
+            for name, r in side.items():
+                line[name] = {"value": r["value"], "unit": "tokens/s", "ms_per_step": r["ms_per_step"],
+                              "roofline": r["roofline"], "step_roofline": r["step"], "stage_ms": r["stage_ms"]}
+            if world == 1 and not args.no_cpu:
+                line["cpu_baseline"] = cpu_baseline(w, dev, args.cpu_tokens)
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -94,6 +94,9 @@ typedef struct muse_moe_config {
   size_t workspace_bytes;
   int32_t* topk_idx_out;      /* optional device [T, k] int32: selected experts       */
   float* topk_w_out;          /* optional device [T, k] float32: their weights        */
+  void* const* stage_events;  /* optional: launch_count + 1 cudaEvent_t handles; event i
+                                 is recorded on the stream before launch i and the last
+                                 after the final launch (per-kernel device timing)     */
 } muse_moe_config;
 
 /* Byte offsets of the intermediates inside the workspace after a forward call, for

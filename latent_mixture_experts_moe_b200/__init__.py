@@ -41,7 +41,8 @@ class Config(ctypes.Structure):
                 ("norm_mode", ctypes.c_int32), ("gamma_shared", ctypes.c_int32),
                 ("pre_norm_gain", ctypes.c_void_p), ("pre_norm_eps", ctypes.c_float),
                 ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
-                ("topk_idx_out", ctypes.c_void_p), ("topk_w_out", ctypes.c_void_p)]
+                ("topk_idx_out", ctypes.c_void_p), ("topk_w_out", ctypes.c_void_p),
+                ("stage_events", ctypes.c_void_p)]
 
 
 class WorkspaceLayout(ctypes.Structure):
@@ -151,6 +152,19 @@ def forward_host_io(cfg: Config, x_host, x_dev, W_router, W_pool, W_gate, W_up, 
     _check(code, "muse_latent_moe_forward_host_io")
 
 
+STAGES = ("router", "topk", "expert_hist", "tiles", "assign_rows", "pooler", "gather", "gate_up_swiglu",
+          "down_sumsq", "norm_combine", "unpooler")
+
+
+def event_handles(events) -> "ctypes.Array":
+    """ctypes array of the raw cudaEvent_t handles of torch.cuda.Event objects (each
+    recorded once beforehand so that it exists)."""
+    arr = (ctypes.c_void_p * len(events))()
+    for i, ev in enumerate(events):
+        arr[i] = int(ev.cuda_event)
+    return arr
+
+
 def last_device_status(cfg: Config, stream=None):
     detail = ctypes.c_uint32(0)
     code = lib().muse_latent_moe_last_device_status(ctypes.byref(cfg), _stream_handle(stream), ctypes.byref(detail))
@@ -186,13 +200,16 @@ class LatentMoE:
             c.workspace_bytes = workspace.numel()
         return c
 
-    def __call__(self, x, out=None, stream=None, topk_idx=None, topk_w=None):
+    def __call__(self, x, out=None, stream=None, topk_idx=None, topk_w=None, stage_events=None):
+        """stage_events: optional ctypes array of launch_count + 1 cudaEvent_t handles."""
         import torch
         T = x.shape[0]
         if T > self.T_max:
             raise ValueError(f"T={T} exceeds T_max={self.T_max}")
         cfg = self.config(T, self.workspace)
         cfg.topk_idx_out, cfg.topk_w_out = _ptr(topk_idx), _ptr(topk_w)
+        if stage_events is not None:
+            cfg.stage_events = ctypes.cast(stage_events, ctypes.c_void_p)
         if out is None:
             out = torch.empty((T, self.dims["D"]), dtype=x.dtype, device=x.device)
         w = self.w

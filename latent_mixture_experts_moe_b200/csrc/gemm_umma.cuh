@@ -11,8 +11,8 @@
 //
 // Roles (192 threads, one CTA per SM):
 //   warp 0      TMA producer: A tile 128 x 128 B (+ a second A tile for gate/up) and the
-//               token tile as N/16 boxes of 16 rows, 128-byte swizzle, into a STAGES-deep
-//               ring guarded by full/empty mbarriers;
+//               token tile in at most 5 boxes of 16..256 rows (one box for a full tile),
+//               128-byte swizzle, into a STAGES-deep ring guarded by full/empty mbarriers;
 //   warp 1      TMEM allocator and UMMA issuer (one thread): 4 x K=16 (bf16) or K=8 (tf32)
 //               MMAs per stage, tcgen05.commit frees the stage; a commit per tile hands
 //               the accumulator to the epilogue;
@@ -22,8 +22,9 @@
 //               EPI_STORE_SS  y -> Y plus per-token partial sums of y^2 over the warp's
 //                             32 features (for the per-expert RMSNorm), from the FP32
 //                             accumulator before rounding.
-// Single-accumulator modes double-buffer the TMEM accumulator so the epilogue of tile i
-// overlaps the MMAs of tile i+1.
+// With MT = 2 two 128-row weight tiles share each token tile (256 features per CTA tile,
+// or gate + up of 128 features); with MT = 1 the TMEM accumulator is double-buffered so
+// the epilogue of tile i overlaps the MMAs of tile i+1.
 //
 // Work list: either a device-built list of int4 {group, m0, row0, n} (grouped expert
 // GEMMs; built by the routing kernels, never read by the host) or implicit dense
@@ -48,6 +49,7 @@ struct GemmArgs {
   const int* num_tiles_dev;  // grouped: device tile count
   int num_tiles;             // dense: m_tiles * ceil(T / BN)
   int m_tiles;               // dense: tiles along M
+  int m_step;                // dense: features per tile (128 * MT)
   int rows_per_group;        // rows of A per group (expert); A row = group * this + m0
   int m_valid;               // valid output features per group (stores masked beyond)
   int T;                     // dense: token rows of B
@@ -83,9 +85,14 @@ __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) { retu
 template <>
 __device__ __forceinline__ float from_f32<float>(float v) { return v; }
 
-template <int BN, int EPI>
+// MT = 128-row weight tiles per CTA: 2 puts two accumulators behind one token tile
+// (gate and up for EPI_SWIGLU; two adjacent 128-feature blocks otherwise), which halves
+// the operand bytes the CTA loads per MMA cycle compared with MT = 1.
+template <int BN, int EPI, int MT>
 struct GemmShape {
-  static constexpr bool kDual = (EPI == EPI_SWIGLU);
+  static constexpr bool kDual = (MT == 2);
+  static_assert(MT == 1 || MT == 2, "MT is 1 or 2");
+  static_assert(EPI != EPI_SWIGLU || MT == 2, "SwiGLU needs the gate and up accumulators");
   static constexpr uint32_t kABytes = 128u * 128u;              // 128 rows x 128 B
   static constexpr uint32_t kBBytes = static_cast<uint32_t>(BN) * 128u;
   static constexpr uint32_t kStageBytes = kABytes * (kDual ? 2u : 1u) + kBBytes;
@@ -115,7 +122,7 @@ __device__ __forceinline__ void gemm_tile(const GemmArgs& p, int t, int BN, int&
     const int mt = t % p.m_tiles;
     const int ch = t / p.m_tiles;
     g = 0;
-    m0 = mt * 128;
+    m0 = mt * p.m_step;
     row0 = ch * BN;
     n = min(BN, p.T - row0);
   }
@@ -137,11 +144,18 @@ __device__ __forceinline__ float transpose_reduce32(float (&v)[32], int lane) {
   return v[0];
 }
 
-template <typename TIn, typename TOut, int BN, int EPI>
-__global__ void __launch_bounds__(192, 1)
-    k_umma_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
-                const __grid_constant__ CUtensorMap tmB, const GemmArgs p) {
-  using S = GemmShape<BN, EPI>;
+// Tensor maps of one launch: the weight operand (a second one for the up projection)
+// and the token operand with boxes of 16 << i rows, i = 0..4, so that a tile of n rows
+// loads in popcount(ceil(n / 16)) copies (one copy for a full 256-row tile).
+struct TmaMaps {
+  CUtensorMap a;
+  CUtensorMap a2;
+  CUtensorMap b[5];
+};
+
+template <typename TIn, typename TOut, int BN, int EPI, int MT>
+__global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ TmaMaps maps, const GemmArgs p) {
+  using S = GemmShape<BN, EPI, MT>;
   constexpr bool kDual = S::kDual;
   constexpr int kStages = S::kStages;
   constexpr bool kTF32 = ElemTraits<TIn>::kTF32;
@@ -172,9 +186,9 @@ __global__ void __launch_bounds__(192, 1)
     }
     *abort_flag = 0;
     fence_mbar_init();
-    prefetch_tmap(&tmA);
-    if (kDual) prefetch_tmap(&tmA2);
-    prefetch_tmap(&tmB);
+    prefetch_tmap(&maps.a);
+    if (kDual) prefetch_tmap(&maps.a2);
+    for (int i = 0; i < 5 && (16 << i) <= BN; ++i) prefetch_tmap(&maps.b[i]);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_holder), S::kTmemCols);
@@ -207,10 +221,19 @@ __global__ void __launch_bounds__(192, 1)
           mbar_arrive_expect_tx(full_bar(stage), bytes);
           const uint32_t sA = smem_u32(smem + stage * S::kStageBytes);
           const int kc = kb * static_cast<int>(128 / sizeof(TIn));
-          tma_load_2d(sA, &tmA, full_bar(stage), kc, a_row);
-          if (kDual) tma_load_2d(sA + S::kABytes, &tmA2, full_bar(stage), kc, a_row);
+          tma_load_2d(sA, &maps.a, full_bar(stage), kc, a_row);
+          // second weight tile: the up projection at the same rows, or the next 128 rows
+          if (kDual) tma_load_2d(sA + S::kABytes, &maps.a2, full_bar(stage), kc, EPI == EPI_SWIGLU ? a_row : a_row + 128);
           const uint32_t sB = sA + S::kABytes * (kDual ? 2u : 1u);
-          for (int j = 0; j < nb16; ++j) tma_load_2d(sB + 2048u * j, &tmB, full_bar(stage), kc, row0 + 16 * j);
+          // largest boxes first: 16-row block offset j16 advances by each box's height
+          int j16 = 0;
+#pragma unroll
+          for (int i = 4; i >= 0; --i) {
+            if ((16 << i) <= BN && (nb16 >> i) & 1) {
+              tma_load_2d(sB + 2048u * j16, &maps.b[i], full_bar(stage), kc, row0 + 16 * j16);
+              j16 += 1 << i;
+            }
+          }
           issued_mask |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
           if (++stage == kStages) {
@@ -296,20 +319,16 @@ __global__ void __launch_bounds__(192, 1)
       const bool ready = mbar_wait(accf_bar(acc), acc_phase, abort_flag, p.status, 0x400u + acc);
       if (!__all_sync(0xffffffffu, ready)) break;
       tc_fence_after();
-      const int f = m0 + q * 32 + lane;  // output feature of this thread (within group)
-      const bool f_ok = f < p.m_valid;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc) * S::kAccCols;
       TOut* out = reinterpret_cast<TOut*>(p.out);
-      float gain1 = 1.0f;
-      if (EPI == EPI_STORE_SS && p.ss_gain != nullptr && f_ok)
-        gain1 = 1.0f + to_f32(reinterpret_cast<const TIn*>(p.ss_gain)[g * p.ss_gain_group_stride + f]);
       const int nchunks = (n + 31) >> 5;
-      for (int c = 0; c < nchunks; ++c) {
-        uint32_t v[32];
-        tmem_ld32(taddr + 32u * c, v);
-        if constexpr (kDual) {
-          uint32_t u[32];
+      if constexpr (EPI == EPI_SWIGLU) {
+        const int f = m0 + q * 32 + lane;  // output feature of this thread (within group)
+        const bool f_ok = f < p.m_valid;
+        for (int c = 0; c < nchunks; ++c) {
+          uint32_t v[32], u[32];
+          tmem_ld32(taddr + 32u * c, v);
           tmem_ld32(taddr + BN + 32u * c, u);
           tmem_ld_wait();
 #pragma unroll
@@ -319,24 +338,36 @@ __global__ void __launch_bounds__(192, 1)
             const float h = a / (1.0f + __expf(-a)) * __uint_as_float(u[i]);
             if (tok < n && f_ok) out[(static_cast<int64_t>(row0) + tok) * p.ld_out + f] = from_f32<TOut>(h);
           }
-        } else {
-          tmem_ld_wait();
+        }
+      } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int tok = c * 32 + i;
-            if (tok < n && f_ok)
-              out[(static_cast<int64_t>(row0) + tok) * p.ld_out + f] = from_f32<TOut>(__uint_as_float(v[i]));
-          }
-          if constexpr (EPI == EPI_STORE_SS) {
-            float sq[32];
+        for (int half = 0; half < MT; ++half) {
+          const int f = m0 + half * 128 + q * 32 + lane;
+          const bool f_ok = f < p.m_valid;
+          float gain1 = 1.0f;
+          if (EPI == EPI_STORE_SS && p.ss_gain != nullptr && f_ok)
+            gain1 = 1.0f + to_f32(reinterpret_cast<const TIn*>(p.ss_gain)[g * p.ss_gain_group_stride + f]);
+          for (int c = 0; c < nchunks; ++c) {
+            uint32_t v[32];
+            tmem_ld32(taddr + static_cast<uint32_t>(half * BN) + 32u * c, v);
+            tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-              const float y = __uint_as_float(v[i]) * gain1;
-              sq[i] = f_ok ? y * y : 0.0f;
+              const int tok = c * 32 + i;
+              if (tok < n && f_ok)
+                out[(static_cast<int64_t>(row0) + tok) * p.ld_out + f] = from_f32<TOut>(__uint_as_float(v[i]));
             }
-            const float tot = transpose_reduce32(sq, lane);
-            const int tok = c * 32 + lane;
-            if (tok < n) p.ss[(static_cast<int64_t>(row0) + tok) * p.ss_ld + (m0 >> 5) + q] = tot;
+            if constexpr (EPI == EPI_STORE_SS) {
+              float sq[32];
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const float y = __uint_as_float(v[i]) * gain1;
+                sq[i] = f_ok ? y * y : 0.0f;
+              }
+              const float tot = transpose_reduce32(sq, lane);
+              const int tok = c * 32 + lane;
+              if (tok < n) p.ss[(static_cast<int64_t>(row0) + tok) * p.ss_ld + ((m0 + half * 128) >> 5) + q] = tot;
+            }
           }
         }
       }

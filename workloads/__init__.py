@@ -57,6 +57,9 @@ WORKLOADS: Dict[str, Workload] = {
     "prefill": Workload("prefill", T=8192, D=8192, L=4096, I=4096, E=256, k=8, dtype="bf16"),
     "prefill_zipf": Workload("prefill_zipf", T=8192, D=8192, L=4096, I=4096, E=256, k=8,
                              dtype="bf16", routing="zipf"),
+    # full-width layer with 16 experts and 256 tokens per expert: the prefill tile
+    # shapes on ~2 GB of device memory (profiling captures)
+    "prefill_e16": Workload("prefill_e16", T=2048, D=8192, L=4096, I=4096, E=16, k=2, dtype="bf16"),
 }
 
 # tensor ids of the generator (fixed, part of the workload definition)
