@@ -157,6 +157,32 @@ MUSE_API muse_status muse_latent_moe_forward_host_io(const muse_moe_config* cfg,
 MUSE_API muse_status muse_latent_moe_last_device_status(const muse_moe_config* cfg, void* stream,
                                                uint32_t* detail);
 
+/* Forward pass for callers that cannot allocate device memory at all: a plug-in whose
+ * host application owns every allocation, code that runs where cudaMalloc is not
+ * permitted or would stall the device, or a service with a fixed memory budget. It is
+ * muse_latent_moe_forward with the workspace taken from a scratch array compiled into
+ * this library (a file-scope __device__ array of MUSE_STATIC_SCRATCH_BYTES, held by
+ * every GPU that loads the library until the process exits) instead of from
+ * cfg->workspace, which is ignored. The pages describe nothing like it: it exists
+ * for callers of this library only.
+ *   - Sizes whose workspace (muse_latent_moe_workspace_size) exceeds
+ *     MUSE_STATIC_SCRATCH_BYTES are rejected with MUSE_ERR_WORKSPACE before any launch.
+ *   - It allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ *   - The first call on each device looks up the array's device address with that
+ *     device current; make that first call before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents (each call
+ *     clears what must start at zero). Calls whose work overlaps on the GPU -- on two
+ *     streams, or on one device from two threads without ordering -- race on it: order
+ *     them on one stream or serialise them.
+ *   - The device-side status word lives in that shared array and is not readable
+ *     through muse_latent_moe_last_device_status. */
+#define MUSE_STATIC_SCRATCH_BYTES (16u << 20)
+MUSE_API muse_status muse_latent_moe_forward_static_scratch(const muse_moe_config* cfg, const void* x,
+                                                            const void* W_router, const void* W_pool,
+                                                            const void* W_gate, const void* W_up,
+                                                            const void* W_down, const void* gamma,
+                                                            const void* W_unpool, void* out, void* stream);
+
 /* Static string for a status code. */
 MUSE_API const char* muse_status_string(muse_status s);
 

@@ -24,7 +24,10 @@ STATUS = {0: "MUSE_OK", 1: "MUSE_ERR_INVALID_ARG", 2: "MUSE_ERR_UNSUPPORTED", 3:
 # every extern "C" entry point of include/muse_moe.h
 EXPORTS = ("muse_moe_config_init", "muse_latent_moe_workspace_size", "muse_latent_moe_workspace_layout",
            "muse_latent_moe_forward", "muse_latent_moe_forward_host_io", "muse_latent_moe_last_device_status",
-           "muse_status_string", "muse_latent_moe_launch_count")
+           "muse_status_string", "muse_latent_moe_launch_count", "muse_latent_moe_forward_static_scratch")
+
+# size of the library's built-in scratch array (MUSE_STATIC_SCRATCH_BYTES)
+STATIC_SCRATCH_BYTES = 16 << 20
 
 
 class MuseError(RuntimeError):
@@ -76,6 +79,8 @@ def lib() -> ctypes.CDLL:
         L.muse_latent_moe_last_device_status.restype = ctypes.c_int
         L.muse_status_string.argtypes = [ctypes.c_int]
         L.muse_status_string.restype = ctypes.c_char_p
+        L.muse_latent_moe_forward_static_scratch.argtypes = [cp] + [vp] * 10
+        L.muse_latent_moe_forward_static_scratch.restype = ctypes.c_int
         L.muse_latent_moe_launch_count.argtypes = [cp]
         L.muse_latent_moe_launch_count.restype = ctypes.c_int32
         _lib = L
@@ -141,6 +146,16 @@ def forward(cfg: Config, x, W_router, W_pool, W_gate, W_up, W_down, gamma, W_unp
                                          _ptr(W_up), _ptr(W_down), _ptr(gamma), _ptr(W_unpool), _ptr(out),
                                          _stream_handle(stream))
     _check(code, "muse_latent_moe_forward")
+
+
+def forward_static_scratch(cfg: Config, x, W_router, W_pool, W_gate, W_up, W_down, gamma, W_unpool, out,
+                           stream=None) -> None:
+    """Forward through the allocation-free entry point (workspace = the library's built-in
+    scratch array; cfg.workspace is ignored). For callers that cannot allocate device memory."""
+    code = lib().muse_latent_moe_forward_static_scratch(ctypes.byref(cfg), _ptr(x), _ptr(W_router), _ptr(W_pool),
+                                                        _ptr(W_gate), _ptr(W_up), _ptr(W_down), _ptr(gamma),
+                                                        _ptr(W_unpool), _ptr(out), _stream_handle(stream))
+    _check(code, "muse_latent_moe_forward_static_scratch")
 
 
 def forward_host_io(cfg: Config, x_host, x_dev, W_router, W_pool, W_gate, W_up, W_down, gamma, W_unpool,

@@ -356,6 +356,29 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
   return MUSE_OK;
 }
 
+// Scratch for muse_latent_moe_forward_static_scratch: a fixed array in device global
+// memory, so that entry point never allocates. In host code this name stands for the
+// symbol, not a device address; the address comes from cudaGetSymbolAddress.
+__device__ __align__(256) uint8_t g_static_scratch[MUSE_STATIC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_scratch_mu;
+void* g_static_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_static_scratch on the current device, looked up once per device.
+muse_status static_scratch_address(void** ptr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MUSE_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+  if (g_static_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return MUSE_ERR_CUDA;
+    g_static_scratch_ptr[dev] = p;
+  }
+  *ptr = g_static_scratch_ptr[dev];
+  return MUSE_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -423,6 +446,22 @@ muse_status muse_latent_moe_forward_host_io(const muse_moe_config* cfg, const vo
   if (s != MUSE_OK) return s;
   if (cudaMemcpyAsync(out_host, out_dev, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) return MUSE_ERR_CUDA;
   return MUSE_OK;
+}
+
+muse_status muse_latent_moe_forward_static_scratch(const muse_moe_config* cfg, const void* x, const void* W_router,
+                                                  const void* W_pool, const void* W_gate, const void* W_up,
+                                                  const void* W_down, const void* gamma, const void* W_unpool,
+                                                  void* out, void* stream) {
+  const muse_status s = validate_sizes(cfg);
+  if (s != MUSE_OK) return s;
+  if (make_layout(*cfg).pub.total > MUSE_STATIC_SCRATCH_BYTES) return MUSE_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  const muse_status a = static_scratch_address(&scratch);
+  if (a != MUSE_OK) return a;
+  muse_moe_config c = *cfg;
+  c.workspace = scratch;
+  c.workspace_bytes = MUSE_STATIC_SCRATCH_BYTES;
+  return muse_latent_moe_forward(&c, x, W_router, W_pool, W_gate, W_up, W_down, gamma, W_unpool, out, stream);
 }
 
 muse_status muse_latent_moe_last_device_status(const muse_moe_config* cfg, void* stream, uint32_t* detail) {
