@@ -186,7 +186,8 @@ MUSE_API muse_status muse_latent_moe_forward_static_scratch(const muse_moe_confi
 /* Static string for a status code. */
 MUSE_API const char* muse_status_string(muse_status s);
 
-/* Number of kernel launches one forward call makes for cfg's sizes (for accounting). */
+/* Number of kernel launches one forward call makes for cfg (11; 12 with a pre-expert
+ * norm). stage_events must hold this many + 1 events. */
 MUSE_API int32_t muse_latent_moe_launch_count(const muse_moe_config* cfg);
 
 #ifdef __cplusplus

@@ -98,7 +98,7 @@ def _check(code: int, where: str) -> None:
 
 def make_config(T: int, D: int, L: int, I: int, E: int, k: int, dtype: str = "bf16", eps: float = 1e-6,
                 router_mode: int = ROUTER_SOFTMAX, router_logit_scale: float = 1.0, routed_scaling: float = 1.0,
-                norm_mode: int = NORM_CENTRED, gamma_shared: bool = False) -> Config:
+                norm_mode: int = NORM_CENTRED, gamma_shared: bool = False, pre_norm_eps: float = 1e-5) -> Config:
     c = Config()
     lib().muse_moe_config_init(ctypes.byref(c))
     c.T, c.D, c.L, c.I, c.E, c.top_k = T, D, L, I, E, k
@@ -106,6 +106,7 @@ def make_config(T: int, D: int, L: int, I: int, E: int, k: int, dtype: str = "bf
     c.eps = eps
     c.router_mode, c.router_logit_scale, c.routed_scaling = router_mode, router_logit_scale, routed_scaling
     c.norm_mode, c.gamma_shared = norm_mode, int(gamma_shared)
+    c.pre_norm_eps = pre_norm_eps
     return c
 
 
@@ -190,7 +191,8 @@ class LatentMoE:
     """Holds the block's device weights and a workspace; calling it runs the forward.
 
     weights: dict with W_router, W_pool, W_gate, W_up, W_down, gamma, W_unpool (torch
-    CUDA tensors in the layouts of include/muse_moe.h); router_bias optional.
+    CUDA tensors in the layouts of include/muse_moe.h); router_bias and pre_norm_gain
+    optional. modes: make_config keywords (router_mode, norm_mode, gamma_shared, ...).
     """
 
     def __init__(self, weights: Dict, T_max: int, k: int, eps: float = 1e-6, **modes):
@@ -210,6 +212,8 @@ class LatentMoE:
         c = make_config(T, d["D"], d["L"], d["I"], d["E"], d["k"], self.dtype, d["eps"], **self.modes)
         if self.w.get("router_bias") is not None:
             c.router_bias = _ptr(self.w["router_bias"])
+        if self.w.get("pre_norm_gain") is not None:
+            c.pre_norm_gain = _ptr(self.w["pre_norm_gain"])
         if workspace is not None:
             c.workspace = _ptr(workspace)
             c.workspace_bytes = workspace.numel()

@@ -292,6 +292,15 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
     if (s != MUSE_OK) return s;
     MUSE_CK(mark());
   }
+  // pages' pre_expert_norm on z (optional)
+  if (c.pre_norm_gain != nullptr) {
+    const int vec = 16 / static_cast<int>(sizeof(T));
+    const int threads = static_cast<int>(std::max<int64_t>(32, align_up(static_cast<size_t>(L / vec), 32)));
+    k_prenorm_rows<T><<<static_cast<unsigned>(Tn), threads, 0, st>>>(z, reinterpret_cast<const T*>(c.pre_norm_gain),
+                                                                    static_cast<int>(L), c.pre_norm_eps);
+    MUSE_CK(cudaGetLastError());
+    MUSE_CK(mark());
+  }
   // (a5) gather into expert order
   {
     const int vpr = static_cast<int>(L * sizeof(T) / 16);
@@ -421,6 +430,8 @@ muse_status muse_latent_moe_forward(const muse_moe_config* cfg, const void* x, c
   for (const void* p : ptrs)
     if (p == nullptr || !aligned16(p)) return MUSE_ERR_INVALID_ARG;
   if (cfg->router_bias != nullptr && (reinterpret_cast<uintptr_t>(cfg->router_bias) & 3u)) return MUSE_ERR_INVALID_ARG;
+  if (cfg->pre_norm_gain != nullptr && !aligned16(cfg->pre_norm_gain)) return MUSE_ERR_INVALID_ARG;
+  if (cfg->pre_norm_gain != nullptr && !(cfg->pre_norm_eps >= 0.0f)) return MUSE_ERR_INVALID_ARG;
   const Layout lay = make_layout(*cfg);
   if (cfg->workspace == nullptr || (reinterpret_cast<uintptr_t>(cfg->workspace) & (kAlign - 1)))
     return MUSE_ERR_WORKSPACE;
@@ -495,7 +506,8 @@ const char* muse_status_string(muse_status s) {
 int32_t muse_latent_moe_launch_count(const muse_moe_config* cfg) {
   if (validate_sizes(cfg) != MUSE_OK) return -1;
   // router, top-k, hist, tiles, rows, pooler, gather, gate/up, down, combine, unpooler
-  return 11;
+  // (+ the optional pre-expert norm, which is launched between pooler and gather)
+  return cfg->pre_norm_gain != nullptr ? 12 : 11;
 }
 
 }  // extern "C"

@@ -239,6 +239,46 @@ __global__ void k_assign_rows(const int* __restrict__ idx, int n, int k, const i
 }
 
 // --------------------------------------------------------------------------------------
+// pages' pre_expert_norm (optional): centred RMSNorm of each pooled row in place,
+// z <- z / sqrt(mean(z^2) + eps) * (1 + w), FP32 statistics, one block per token.
+// --------------------------------------------------------------------------------------
+template <typename T>
+__global__ void k_prenorm_rows(T* __restrict__ z, const T* __restrict__ w, int L, float eps) {
+  constexpr int VEC = 16 / sizeof(T);
+  __shared__ float part[32];
+  __shared__ float scale_s;
+  T* row = z + static_cast<int64_t>(blockIdx.x) * L;
+  const int f0 = threadIdx.x * VEC;
+  uint4 v = make_uint4(0, 0, 0, 0);
+  float ss = 0.0f;
+  if (f0 < L) {
+    v = *reinterpret_cast<const uint4*>(row + f0);
+    const T* vv = reinterpret_cast<const T*>(&v);
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) ss = fmaf(to_f32(vv[i]), to_f32(vv[i]), ss);
+  }
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float t = threadIdx.x < (blockDim.x >> 5) ? part[threadIdx.x] : 0.0f;
+    t = warp_sum(t);
+    if (threadIdx.x == 0) scale_s = 1.0f / sqrtf(t / static_cast<float>(L) + eps);
+  }
+  __syncthreads();
+  if (f0 < L) {
+    const uint4 gv = *reinterpret_cast<const uint4*>(w + f0);
+    const T* vv = reinterpret_cast<const T*>(&v);
+    const T* gg = reinterpret_cast<const T*>(&gv);
+    uint4 ov;
+    T* oo = reinterpret_cast<T*>(&ov);
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) oo[i] = from_f32<T>(to_f32(vv[i]) * scale_s * (1.0f + to_f32(gg[i])));
+    *reinterpret_cast<uint4*>(row + f0) = ov;
+  }
+}
+
+// --------------------------------------------------------------------------------------
 // (a3) gather: Zp[row] = z[row_token[row]] (zeros for padding rows), 16-byte vectors.
 // --------------------------------------------------------------------------------------
 __global__ void k_gather_rows(const int* __restrict__ row_token, const int* __restrict__ total_rows,

@@ -49,7 +49,8 @@ def ws_view(ws: torch.Tensor, off: int, dtype: torch.dtype, shape: Sequence[int]
 
 
 class Run:
-    """One forward of the CUDA path with its routing outputs and workspace."""
+    """One forward of the CUDA path with its routing outputs and workspace (modes: the
+    keyword arguments of latent_mixture_experts_moe_b200.make_config)."""
 
     def __init__(self, w: W.Workload, inp: Dict[str, torch.Tensor], T: Optional[int] = None, **modes):
         T = T or w.T
@@ -85,6 +86,8 @@ def oracle_block(w: W.Workload, inp: Dict[str, torch.Tensor], rows: np.ndarray, 
     """The oracle on token rows `rows` of x (tokens are independent)."""
     x = host(inp["x"][torch.as_tensor(rows, device=inp["x"].device)])
     bias = host(inp["router_bias"]) if "router_bias" in inp else None
+    if "pre_norm_gain" in inp:
+        kw = dict(kw, pre_norm_gain=host(inp["pre_norm_gain"]))
     return oracle.latent_moe_forward(x, host(inp["W_router"]), host(inp["W_pool"]), expert_source(inp),
                                      host(inp["gamma"]), host(inp["W_unpool"]), w.k, w.eps, router_bias=bias,
                                      **kw)
@@ -120,7 +123,11 @@ def oracle_on_gpu_alternatives(w, inp, rows, ref, gpu_idx, alt_tokens, **kw):
     out = ref["out"].copy()
     for t in alt_tokens:
         sel = np.array(sorted(gpu_idx[t].tolist(), key=lambda e: (-ref["keys"][t][e], e)))[None, :]
-        g = oracle.softmax_weights(ref["logits"][t:t + 1], sel)
+        if kw.get("router_mode", "softmax") == "sigmoid":
+            g = oracle.sigmoid_weights(ref["logits"][t:t + 1], sel, kw.get("logit_scale", 1.0),
+                                       kw.get("routed_scaling", 1.0))
+        else:
+            g = oracle.softmax_weights(ref["logits"][t:t + 1], sel)
         r1 = oracle_block(w, inp, rows[t:t + 1], routing=(sel, g), **kw)
         out[t] = r1["out"][0]
     return out

@@ -15,15 +15,15 @@ from parity_util import (Run, assert_close, check_routing, expected_permutation,
 pytestmark = pytest.mark.gpu
 
 
-def full_check(w, inp, run, rows=None, **modes):
+def full_check(w, inp, run, rows=None, **oracle_modes):
     """Routing, permutation, intermediates and output of `run` against the oracle."""
     T = run.T
     rows = np.arange(T) if rows is None else rows
-    ref = oracle_block(w, inp, rows)
+    ref = oracle_block(w, inp, rows, **oracle_modes)
     gidx = run.idx.cpu().numpy()[rows]
     gg = run.g.cpu().numpy()[rows]
     alts = check_routing(ref, gidx, gg, w.k)
-    ref_out = oracle_on_gpu_alternatives(w, inp, rows, ref, gidx, alts)
+    ref_out = oracle_on_gpu_alternatives(w, inp, rows, ref, gidx, alts, **oracle_modes)
     out = host(run.out)[rows]
     assert_close(out, ref_out, f"{w.name} out")
     return ref, alts
@@ -127,6 +127,37 @@ def test_edge_cases(case):
     if not alts:
         counts, offsets, inv = expected_permutation(ref["idx"], E)
         assert np.array_equal(run.inter("inv", torch.int32, (T * k,)).cpu().numpy(), inv)
+
+
+# ------------------------------------------------------------------------- released mode
+PAGES = [
+    # name, T, D, L, I, E, k
+    ("pages_mid", 256, 2048, 1024, 1024, 64, 4),
+    ("pages_ragged", 37, 512, 256, 384, 16, 8),
+]
+
+
+@pytest.mark.parametrize("case", PAGES, ids=[c[0] for c in PAGES])
+def test_pages_released_mode(case):
+    """The block as the pages describe the released model (deep dive §4.2-4.4, Norm
+    gates page): sigmoid router on the logits times 1/sqrt(D/256) with a selection-only
+    bias and s/(sum s + 1e-15) weights; centred pre-expert norm (eps 1e-5) on z; ONE
+    input-scaled post-expert norm gain shared by every expert (eps 1e-8)."""
+    name, T, D, L, I, E, k = case
+    w = W.Workload(name, T=T, D=D, L=L, I=I, E=E, k=k, dtype="bf16", eps=1e-8, seed=5)
+    inp = W.make_inputs(w, "cuda")
+    inp["gamma"] = inp["gamma"][0].contiguous()                      # one shared [L] gain
+    pre = torch.empty(L, dtype=torch.bfloat16, device="cuda")
+    inp["pre_norm_gain"] = W.fill(pre, w.seed, 11, 0.3)
+    inp["router_bias"] = (W.normal_f64(w.seed, 12, 0, E) * 0.05).to(torch.float32).cuda()
+    scale = 1.0 / np.sqrt(D / 256)
+    run = Run(w, inp, router_mode=moe.ROUTER_SIGMOID, router_logit_scale=scale, routed_scaling=1.0,
+              norm_mode=moe.NORM_INPUT_SCALED, gamma_shared=True, pre_norm_eps=1e-5)
+    ref, alts = full_check(w, inp, run, router_mode="sigmoid", logit_scale=scale, routed_scaling=1.0,
+                           norm_mode="input_scaled", pre_norm_eps=1e-5)
+    assert_close(host(run.inter("z", run.act(), (T, L))), ref["z"], "normalised latent z")
+    g = run.g.cpu().numpy()
+    assert np.allclose(g.sum(1), 1.0, atol=1e-5)                     # convex combination
 
 
 # ------------------------------------------------------------------------- full size
