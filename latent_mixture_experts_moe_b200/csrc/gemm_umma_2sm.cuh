@@ -1,0 +1,295 @@
+// gemm_umma_2sm.cuh -- the same contraction as gemm_umma.cuh on a CTA pair (a cluster of
+// two CTAs on one TPC) with cta_group::2 UMMAs, for tiles of up to 256 tokens (prefill):
+//
+//   the pair tile is 256 (or 512) output features x N <= 256 tokens; each CTA stages
+//   128 weight rows per weight tile and HALF of the token tile (N/2 rows) in its own
+//   shared memory; the leader CTA (cluster rank 0) issues M = 256 MMAs that read both
+//   CTAs' tiles, and each CTA's TMEM receives its own 128 feature rows x N columns.
+//
+// Per SM and MMA cycle this moves 48 bytes of operands (gate/up; 512-feature down tiles)
+// or 64 (256-feature tiles) instead of 64 / 96 for one CTA, and the ring holds more
+// stages. Synchronisation:
+//   * both CTAs' TMA copies complete on the LEADER's full barrier (cta_group::2 form of the
+//     copy, no multicast); only the leader posts the expected bytes of both halves;
+//   * the leader's tcgen05.commit multicasts "stage free" to both CTAs' empty barriers and
+//     "accumulator ready" to both CTAs' accumulator barriers;
+//   * both CTAs' epilogue warps release the accumulator on the leader's barrier (8 arrivals,
+//     remote ones through the cluster window);
+//   * a cluster barrier after initialisation and before TMEM is freed keeps each CTA alive
+//     while its partner may still touch its barriers, shared memory or TMEM.
+// Every wait is bounded as in gemm_umma.cuh.
+#pragma once
+
+#include "gemm_umma.cuh"
+
+namespace muse {
+
+template <int EPI, int MT>
+struct Gemm2Shape {
+  static constexpr bool kDual = (MT == 2);
+  static_assert(MT == 1 || MT == 2, "MT is 1 or 2");
+  static_assert(EPI != EPI_SWIGLU || MT == 2, "SwiGLU needs the gate and up accumulators");
+  static constexpr int kBN = 256;                               // tokens per pair tile
+  static constexpr uint32_t kABytes = 128u * 128u;              // 128 weight rows x 128 B
+  static constexpr uint32_t kBBytes = 128u * 128u;              // 128 token rows x 128 B
+  static constexpr uint32_t kStageBytes = kABytes * MT + kBBytes;
+  static constexpr int kSmemBudget = 227 * 1024 - 1024 - 256;
+  static constexpr int kStagesFit = kSmemBudget / static_cast<int>(kStageBytes);
+  static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
+  static constexpr int kAccStages = kDual ? 1 : 2;
+  static constexpr uint32_t kAccCols = 256u * MT;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes + 256;
+  // output features covered by one pair tile
+  static constexpr int kFeatStep = (EPI == EPI_SWIGLU) ? 256 : 256 * MT;
+  static_assert(kAccCols * kAccStages <= kTmemCols, "accumulators exceed TMEM");
+};
+
+template <typename TOut, int EPI, int MT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+    k_umma_gemm_2sm(const __grid_constant__ TmaMaps maps, const GemmArgs p) {
+  using S = Gemm2Shape<EPI, MT>;
+  using TIn = __nv_bfloat16;
+  constexpr bool kDual = S::kDual;
+  constexpr int kStages = S::kStages;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * S::kStageBytes);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = (rank == 0);
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+  const uint32_t bar0 = smem_u32(bars);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
+  auto accf_bar = [&](int a) { return bar0 + 8u * (2 * kStages + a); };
+  auto acce_bar = [&](int a) { return bar0 + 8u * (2 * kStages + 2 + a); };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(accf_bar(a), 1);
+      mbar_init(acce_bar(a), 8);  // 4 epilogue warps in each CTA of the pair
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&maps.a);
+    if (kDual) prefetch_tmap(&maps.a2);
+    for (int i = 0; i < 4; ++i) prefetch_tmap(&maps.b[i]);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_holder), S::kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // partner barriers are initialised before anyone signals them
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const int num_tiles = (p.tiles != nullptr) ? *p.num_tiles_dev : p.num_tiles;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_phase = 0;
+      bool ok = true;
+      for (int t = pair; ok && t < num_tiles; t += npairs) {
+        int g, m0, row0, n;
+        gemm_tile(p, t, S::kBN, g, m0, row0, n);
+        const int N = (n + 31) & ~31;
+        const int half = N >> 1;             // token rows staged by each CTA
+        const int nb16 = half >> 4;          // 1..8 blocks of 16 rows
+        const uint32_t bytes_pair = 2u * (S::kABytes * MT + static_cast<uint32_t>(half) * 128u);
+        const int a_row = g * p.rows_per_group + m0 + static_cast<int>(rank) * 128;
+        const int a2_row = (EPI == EPI_SWIGLU) ? a_row : a_row + 256;
+        const int b_row = row0 + static_cast<int>(rank) * half;
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait<true>(empty_bar(stage), phase ^ 1u, abort_flag, p.status, 0x500u + stage)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = mapa_shared(full_bar(stage), 0);
+          if (leader) mbar_arrive_expect_tx(full_bar(stage), bytes_pair);
+          const uint32_t sA = smem_u32(smem + stage * S::kStageBytes);
+          const int kc = kb * 64;
+          tma_load_2d_pair(sA, &maps.a, fb, kc, a_row);
+          if (kDual) tma_load_2d_pair(sA + S::kABytes, &maps.a2, fb, kc, a2_row);
+          const uint32_t sB = sA + S::kABytes * MT;
+          int j16 = 0;
+#pragma unroll
+          for (int i = 3; i >= 0; --i) {
+            if ((nb16 >> i) & 1) {
+              tma_load_2d_pair(sB + 2048u * j16, &maps.b[i], fb, kc, b_row + 16 * j16);
+              j16 += 1 << i;
+            }
+          }
+          issued_mask |= 1u << stage;
+          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok && leader) {
+        // the leader's full barriers count both CTAs' copies: let them land
+        for (int s = 0; s < kStages; ++s)
+          if (issued_mask & (1u << s)) mbar_wait_drain(full_bar(s), (issued_phase >> s) & 1u);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- UMMA issuer (leader)
+    if (lane == 0 && leader) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      bool issued_any = false;
+      for (int t = pair; ok && t < num_tiles; t += npairs) {
+        int g, m0, row0, n;
+        gemm_tile(p, t, S::kBN, g, m0, row0, n);
+        const uint32_t N = static_cast<uint32_t>((n + 31) & ~31);
+        const uint32_t idesc = idesc_f32acc(1u, 256u, N);
+        if (!mbar_wait<true>(acce_bar(acc), acc_phase ^ 1u, abort_flag, p.status, 0x600u + acc)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_base + static_cast<uint32_t>(acc) * S::kAccCols;
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait<true>(full_bar(stage), phase, abort_flag, p.status, 0x700u + stage)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sA = smem_u32(smem + stage * S::kStageBytes);
+          const uint32_t sB = sA + S::kABytes * MT;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
+            const uint64_t db = sdesc_k_sw128(sB + 32u * kk);
+            umma_pair_bf16(d, sdesc_k_sw128(sA + 32u * kk), db, idesc, accum);
+            if (kDual) umma_pair_bf16(d + 256u, sdesc_k_sw128(sA + S::kABytes + 32u * kk), db, idesc, accum);
+          }
+          issued_any = true;
+          tc_commit_pair(empty_bar(stage), 0x3);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit_pair(accf_bar(acc), 0x3);
+        if (S::kAccStages == 2) {
+          acc ^= 1;
+          if (acc == 0) acc_phase ^= 1u;
+        } else {
+          acc_phase ^= 1u;
+        }
+      }
+      if (!ok && issued_any) {
+        tc_commit_pair(accf_bar(acc), 0x3);
+        mbar_wait_drain(accf_bar(acc), acc_phase);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- epilogue (both CTAs)
+    const int q = warp & 3;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = pair; t < num_tiles; t += npairs) {
+      int g, m0, row0, n;
+      gemm_tile(p, t, S::kBN, g, m0, row0, n);
+      const bool ready = mbar_wait<true>(accf_bar(acc), acc_phase, abort_flag, p.status, 0x800u + acc);
+      if (!__all_sync(0xffffffffu, ready)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                             static_cast<uint32_t>(acc) * S::kAccCols;
+      TOut* out = reinterpret_cast<TOut*>(p.out);
+      const int nchunks = (n + 31) >> 5;
+      const int fbase = m0 + static_cast<int>(rank) * 128 + q * 32 + lane;
+      if constexpr (EPI == EPI_SWIGLU) {
+        const int f = fbase;
+        const bool f_ok = f < p.m_valid;
+        for (int c = 0; c < nchunks; ++c) {
+          uint32_t v[32], u[32];
+          tmem_ld32(taddr + 32u * c, v);
+          tmem_ld32(taddr + 256u + 32u * c, u);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int tok = c * 32 + i;
+            const float a = __uint_as_float(v[i]);
+            const float h = a / (1.0f + __expf(-a)) * __uint_as_float(u[i]);
+            if (tok < n && f_ok) out[(static_cast<int64_t>(row0) + tok) * p.ld_out + f] = from_f32<TOut>(h);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int h = 0; h < MT; ++h) {
+          const int f = fbase + h * 256;
+          const bool f_ok = f < p.m_valid;
+          float gain1 = 1.0f;
+          if (EPI == EPI_STORE_SS && p.ss_gain != nullptr && f_ok)
+            gain1 = 1.0f + to_f32(reinterpret_cast<const TIn*>(p.ss_gain)[g * p.ss_gain_group_stride + f]);
+          for (int c = 0; c < nchunks; ++c) {
+            uint32_t v[32];
+            tmem_ld32(taddr + static_cast<uint32_t>(h * 256) + 32u * c, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int tok = c * 32 + i;
+              if (tok < n && f_ok)
+                out[(static_cast<int64_t>(row0) + tok) * p.ld_out + f] = from_f32<TOut>(__uint_as_float(v[i]));
+            }
+            if constexpr (EPI == EPI_STORE_SS) {
+              float sq[32];
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const float y = __uint_as_float(v[i]) * gain1;
+                sq[i] = f_ok ? y * y : 0.0f;
+              }
+              const float tot = transpose_reduce32(sq, lane);
+              const int tok = c * 32 + lane;
+              const int col = (m0 + h * 256 + static_cast<int>(rank) * 128) >> 5;
+              if (tok < n) p.ss[(static_cast<int64_t>(row0) + tok) * p.ss_ld + col + q] = tot;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(acce_bar(acc), 0));
+      if (S::kAccStages == 2) {
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      } else {
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // neither CTA leaves while its partner may still signal or read it
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, S::kTmemCols);
+  }
+}
+
+}  // namespace muse

@@ -18,6 +18,7 @@
 
 #include "../../include/muse_moe.h"
 #include "gemm_umma.cuh"
+#include "gemm_umma_2sm.cuh"
 #include "route_kernels.cuh"
 
 using namespace muse;
@@ -165,6 +166,24 @@ cudaError_t launch_gemm_bn(int bn, int mt, const TmaMaps& maps, const GemmArgs& 
   }
 }
 
+template <typename TOut, int EPI, int MT>
+cudaError_t launch_gemm_2sm(const TmaMaps& maps, const GemmArgs& args, int pairs, cudaStream_t st) {
+  auto kern = k_umma_gemm_2sm<TOut, EPI, MT>;
+  const size_t smem = Gemm2Shape<EPI, MT>::kSmemBytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  kern<<<2 * pairs, 192, smem, st>>>(maps, args);
+  return cudaGetLastError();
+}
+
+// How a GEMM is tiled: on one SM (mt weight tiles of 128 rows per CTA) or on a CTA pair
+// (cta_group::2; 256 * mt features per pair tile, tiles of up to 256 tokens).
+struct GemmPlan {
+  bool pair;
+  int mt;
+  int step;  // output features per tile
+};
+
 // weight operand map(s) with 128-row boxes and the token operand with 16..256-row boxes
 bool make_maps(TmaMaps* m, const void* a, const void* a2, int64_t a_rows, const void* b, int64_t b_rows, int64_t K,
                bool bf16) {
@@ -190,20 +209,42 @@ muse_status dense_gemm(const void* W, int64_t M, const void* X, int64_t T, int64
   const bool bf = sizeof(TIn) == 2;
   if (!make_maps(&maps, W, nullptr, M, X, T, K, bf)) return MUSE_ERR_CUDA;
   GemmArgs g = base_args(status);
-  // two 128-row weight tiles per CTA when that still leaves at least a full wave of tiles
   const int nsm = sm_count();
-  const int mt = (cdiv(M, 256) * cdiv(T, bn) >= nsm) ? 2 : 1;
-  g.m_step = 128 * mt;
-  g.m_tiles = static_cast<int>(cdiv(M, g.m_step));
-  g.num_tiles = static_cast<int>(g.m_tiles * cdiv(T, bn));
   g.rows_per_group = 0;
   g.m_valid = static_cast<int>(M);
   g.T = static_cast<int>(T);
   g.k_blocks = static_cast<int>(cdiv(K * sizeof(TIn), 128));
   g.out = out;
   g.ld_out = M;
+  // a CTA pair per 256 features x 256 tokens when that fills at least one wave of pairs
+  if (bf && bn == 256 && cdiv(M, 256) * cdiv(T, 256) >= nsm / 2) {
+    g.m_step = 256;
+    g.m_tiles = static_cast<int>(cdiv(M, 256));
+    g.num_tiles = static_cast<int>(g.m_tiles * cdiv(T, 256));
+    const int pairs = std::min(g.num_tiles, nsm / 2);
+    return launch_gemm_2sm<TOut, EPI_STORE, 1>(maps, g, pairs, st) == cudaSuccess ? MUSE_OK : MUSE_ERR_CUDA;
+  }
+  // two 128-row weight tiles per CTA when that still leaves at least a full wave of tiles
+  const int mt = (cdiv(M, 256) * cdiv(T, bn) >= nsm) ? 2 : 1;
+  g.m_step = 128 * mt;
+  g.m_tiles = static_cast<int>(cdiv(M, g.m_step));
+  g.num_tiles = static_cast<int>(g.m_tiles * cdiv(T, bn));
   const int grid = std::min(g.num_tiles, nsm);
   return launch_gemm_bn<TIn, TOut, EPI_STORE>(bn, mt, maps, g, grid, st) == cudaSuccess ? MUSE_OK : MUSE_ERR_CUDA;
+}
+
+// Grouped-GEMM plans. gate/up: a CTA pair per 256 features when tiles hold up to 256
+// tokens (bf16), else one CTA per 128 features (gate and up accumulators). down: a pair
+// per 512 features (two accumulators) or 256, else one CTA per 256 or 128 features.
+GemmPlan plan_gate_up(const muse_moe_config& c, int bn_g) {
+  if (c.dtype == MUSE_BF16 && bn_g == 256 && c.I % 256 == 0) return {true, 2, 256};
+  return {false, 2, 128};
+}
+GemmPlan plan_down(const muse_moe_config& c, int bn_g) {
+  if (c.dtype == MUSE_BF16 && bn_g == 256 && c.L % 512 == 0) return {true, 2, 512};
+  if (c.dtype == MUSE_BF16 && bn_g == 256 && c.L % 256 == 0) return {true, 1, 256};
+  if (bn_g == 256 && c.L % 256 == 0) return {false, 2, 256};
+  return {false, 1, 128};
 }
 
 #define MUSE_CK(x)                                 \
@@ -239,8 +280,7 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
   const int64_t assign = Tn * k;
   const int nsm = sm_count();
   const int bn_d = dense_bn(c), bn_g = grouped_bn(c);
-  // the down projection takes 256 features per tile when tiles hold up to 256 tokens
-  const int mt_dn = (bn_g == 256 && L % 256 == 0) ? 2 : 1;
+  const GemmPlan pgu = plan_gate_up(c, bn_g), pdn = plan_down(c, bn_g);
 
   MUSE_CK(cudaMemsetAsync(status, 0, 16, st));
   MUSE_CK(cudaMemsetAsync(counts, 0, sizeof(int) * E, st));
@@ -276,9 +316,9 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
     MUSE_CK(cudaGetLastError());
     MUSE_CK(mark());
     const int threads = static_cast<int>(align_up(static_cast<size_t>(E), 32));
-    k_build_tiles<<<1, threads, 0, st>>>(counts, static_cast<int>(E), bn_g, static_cast<int>(I / 128),
-                                         static_cast<int>(L / (128 * mt_dn)), 128 * mt_dn, offsets, tiles_gu,
-                                         ntiles, tiles_dn, ntiles + 1, row_token);
+    k_build_tiles<<<1, threads, 0, st>>>(counts, static_cast<int>(E), bn_g, static_cast<int>(I / pgu.step), pgu.step,
+                                         static_cast<int>(L / pdn.step), pdn.step, offsets, tiles_gu, ntiles,
+                                         tiles_dn, ntiles + 1, row_token);
     MUSE_CK(cudaGetLastError());
     MUSE_CK(mark());
     k_assign_rows<<<static_cast<unsigned>(E), 1024, 0, st>>>(topk_idx, static_cast<int>(assign), static_cast<int>(k),
@@ -322,7 +362,11 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
     g.k_blocks = static_cast<int>(L * sizeof(T) / 128);
     g.out = h;
     g.ld_out = I;
-    MUSE_CK((launch_gemm_bn<T, T, EPI_SWIGLU>(bn_g, 2, maps, g, nsm, st)));
+    if (pgu.pair) {
+      MUSE_CK((launch_gemm_2sm<T, EPI_SWIGLU, 2>(maps, g, nsm / 2, st)));
+    } else {
+      MUSE_CK((launch_gemm_bn<T, T, EPI_SWIGLU>(bn_g, 2, maps, g, nsm, st)));
+    }
     MUSE_CK(mark());
   }
   // (a7) down projection + sum-of-squares partials
@@ -343,7 +387,13 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
       g.ss_gain = gamma;
       g.ss_gain_group_stride = c.gamma_shared ? 0 : L;
     }
-    MUSE_CK((launch_gemm_bn<T, T, EPI_STORE_SS>(bn_g, mt_dn, maps, g, nsm, st)));
+    if (pdn.pair && pdn.mt == 2) {
+      MUSE_CK((launch_gemm_2sm<T, EPI_STORE_SS, 2>(maps, g, nsm / 2, st)));
+    } else if (pdn.pair) {
+      MUSE_CK((launch_gemm_2sm<T, EPI_STORE_SS, 1>(maps, g, nsm / 2, st)));
+    } else {
+      MUSE_CK((launch_gemm_bn<T, T, EPI_STORE_SS>(bn_g, pdn.mt, maps, g, nsm, st)));
+    }
     MUSE_CK(mark());
   }
   // (a8 + a9) per-expert RMSNorm and weighted combine

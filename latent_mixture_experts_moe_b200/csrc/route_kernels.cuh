@@ -176,13 +176,13 @@ __global__ void k_expert_hist(const int* __restrict__ idx, int n, int E, int* __
 // --------------------------------------------------------------------------------------
 // (a3) step 2 (one block, thread per expert): padded row offsets (each expert's rows
 // rounded up to a multiple of 16, the MMA's N granularity), the two grouped-GEMM tile
-// lists (gate/up tiles 128 features apart, down tiles step_dn apart) and the padding
+// lists (gate/up tiles step_gu features apart, down tiles step_dn apart) and the padding
 // rows' token = -1. An expert's n rows split into
 // ceil(n / BN) near-equal chunks of a multiple of 16 rows; tiles are ordered expert,
 // feature tile, chunk, so the chunks sharing one weight tile run side by side.
 // --------------------------------------------------------------------------------------
-__global__ void k_build_tiles(const int* __restrict__ counts, int E, int BN, int mt_gu, int mt_dn, int step_dn,
-                              int* __restrict__ offsets, int4* __restrict__ tiles_gu,
+__global__ void k_build_tiles(const int* __restrict__ counts, int E, int BN, int mt_gu, int step_gu, int mt_dn,
+                              int step_dn, int* __restrict__ offsets, int4* __restrict__ tiles_gu,
                               int* __restrict__ ntiles_gu, int4* __restrict__ tiles_dn,
                               int* __restrict__ ntiles_dn, int* __restrict__ row_token) {
   const int e = threadIdx.x;
@@ -198,7 +198,7 @@ __global__ void k_build_tiles(const int* __restrict__ counts, int E, int BN, int
     offsets[e] = off;
     for (int ft = 0; ft < mt_gu; ++ft)
       for (int ch = 0; ch < nch; ++ch)
-        tiles_gu[gu_off + ft * nch + ch] = make_int4(e, ft * 128, off + ch * chunk, min(chunk, n - ch * chunk));
+        tiles_gu[gu_off + ft * nch + ch] = make_int4(e, ft * step_gu, off + ch * chunk, min(chunk, n - ch * chunk));
     for (int ft = 0; ft < mt_dn; ++ft)
       for (int ch = 0; ch < nch; ++ch)
         tiles_dn[dn_off + ft * nch + ch] = make_int4(e, ft * step_dn, off + ch * chunk, min(chunk, n - ch * chunk));

@@ -106,8 +106,12 @@ EDGE = [
     ("k_one", 33, 256, 256, 128, 16, 1, "bf16", None),
     ("fp32_ragged", 37, 256, 256, 128, 8, 3, "f32", None),
     ("many_tokens_per_expert", 1100, 256, 128, 128, 4, 2, "bf16", None),
-    # 256-feature tiles: the unpooler has >= one wave of 256-wide tiles, down has L % 256 == 0
+    # 256-feature tiles: the unpooler has >= one wave of 256-wide tiles, down has L % 256 == 0;
+    # with I % 256 == 0 and L % 512 == 0 gate/up and down run on CTA pairs (cta_group::2)
     ("wide_tiles", 4864, 2048, 512, 256, 8, 2, "bf16", None),
+    # CTA pairs with ragged token chunks (about 388 rows per expert in two chunks), down
+    # on 256-feature pair tiles (L % 512 != 0)
+    ("pair_ragged", 777, 512, 256, 512, 4, 2, "bf16", None),
 ]
 
 
