@@ -151,6 +151,7 @@ struct TmaMaps {
   CUtensorMap a;
   CUtensorMap a2;
   CUtensorMap b[5];
+  CUtensorMap out;  // output [rows, features], 16-row x 128-feature boxes (CTA-pair bf16 stores)
 };
 
 template <typename TIn, typename TOut, int BN, int EPI, int MT>

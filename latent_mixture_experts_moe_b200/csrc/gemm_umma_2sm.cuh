@@ -20,6 +20,8 @@
 // Every wait is bounded as in gemm_umma.cuh.
 #pragma once
 
+#include <type_traits>
+
 #include "gemm_umma.cuh"
 
 namespace muse {
@@ -33,20 +35,28 @@ struct Gemm2Shape {
   static constexpr uint32_t kABytes = 128u * 128u;              // 128 weight rows x 128 B
   static constexpr uint32_t kBBytes = 128u * 128u;              // 128 token rows x 128 B
   static constexpr uint32_t kStageBytes = kABytes * MT + kBBytes;
-  static constexpr int kSmemBudget = 227 * 1024 - 1024 - 256;
+  // output staging for TMA stores: per epilogue group 2 buffers x 32 token rows x 128
+  // features of bf16
+  static constexpr uint32_t kOutBufBytes = 32u * 128u * 2u;
+  static constexpr uint32_t kOutBytes = 2u * 2u * kOutBufBytes;
+  static constexpr int kSmemBudget = 227 * 1024 - 1024 - 256 - static_cast<int>(kOutBytes);
   static constexpr int kStagesFit = kSmemBudget / static_cast<int>(kStageBytes);
   static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
   static constexpr int kAccStages = kDual ? 1 : 2;
   static constexpr uint32_t kAccCols = 256u * MT;
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes + 256;
+  static constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes + kOutBytes + 256;
   // output features covered by one pair tile
   static constexpr int kFeatStep = (EPI == EPI_SWIGLU) ? 256 : 256 * MT;
   static_assert(kAccCols * kAccStages <= kTmemCols, "accumulators exceed TMEM");
 };
 
+// 10 warps: 0 TMA producer, 1 TMEM owner + UMMA issuer (leader), 2..9 epilogue in two
+// groups of four (one warp per TMEM lane quadrant each) taking alternate token chunks
+constexpr int kPairThreads = 320;
+
 template <typename TOut, int EPI, int MT>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     k_umma_gemm_2sm(const __grid_constant__ TmaMaps maps, const GemmArgs p) {
   using S = Gemm2Shape<EPI, MT>;
   using TIn = __nv_bfloat16;
@@ -55,7 +65,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * S::kStageBytes);
+  uint8_t* out_stage = smem + kStages * S::kStageBytes;  // 1024-aligned
+  uint64_t* bars = reinterpret_cast<uint64_t*>(out_stage + S::kOutBytes);
+  constexpr bool kTmaStore = std::is_same<TOut, __nv_bfloat16>::value;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -78,13 +90,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(accf_bar(a), 1);
-      mbar_init(acce_bar(a), 8);  // 4 epilogue warps in each CTA of the pair
+      mbar_init(acce_bar(a), 16);  // 8 epilogue warps in each CTA of the pair
     }
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&maps.a);
     if (kDual) prefetch_tmap(&maps.a2);
     for (int i = 0; i < 4; ++i) prefetch_tmap(&maps.b[i]);
+    if (kTmaStore) prefetch_tmap(&maps.out);
   }
   if (warp == 1) {
     tmem_alloc_pair(smem_u32(tmem_holder), S::kTmemCols);
@@ -208,7 +221,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- epilogue (both CTAs)
+    // bf16 outputs go through a double-buffered shared tile [32 tokens][128 features] and
+    // leave as TMA stores of 16-row boxes (one thread issues them); a 16-row box never
+    // reaches past an expert's 16-padded rows, and TMA clips at the tensor's edge.
     const int q = warp & 3;
+    const int fl = q * 32 + lane;  // feature of this thread within the CTA's 128
+    const int grp = (warp - 2) >> 2;  // epilogue group: chunks c with c % 2 == grp
+    const bool elected = ((warp & ~4) == 2 && lane == 0);  // warp 2 or 6
+    uint8_t* grp_stage = out_stage + grp * 2 * S::kOutBufBytes;
+    int sbuf = 0;
+    auto emit = [&](const float (&val)[32], int c, int col0, int row0, int n, bool f_ok, int f) {
+      TOut* out = reinterpret_cast<TOut*>(p.out);
+      if constexpr (kTmaStore) {
+        if (elected) bulk_wait_group_read<1>();  // the buffer's previous store has read it
+        epilogue_group_bar_sync(grp);
+        __nv_bfloat16* buf = reinterpret_cast<__nv_bfloat16*>(grp_stage + sbuf * S::kOutBufBytes);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) buf[i * 128 + fl] = __float2bfloat16_rn(val[i]);
+        fence_proxy_async_smem();
+        epilogue_group_bar_sync(grp);
+        if (elected) {
+          const uint32_t src = smem_u32(buf);
+          if (c * 32 < n) tma_store_2d(&maps.out, src, col0, row0 + c * 32);
+          if (c * 32 + 16 < n) tma_store_2d(&maps.out, src + S::kOutBufBytes / 2, col0, row0 + c * 32 + 16);
+          bulk_commit_group();
+        }
+        sbuf ^= 1;
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int tok = c * 32 + i;
+          if (tok < n && f_ok) out[(static_cast<int64_t>(row0) + tok) * p.ld_out + f] = from_f32<TOut>(val[i]);
+        }
+      }
+    };
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = pair; t < num_tiles; t += npairs) {
@@ -219,55 +265,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc) * S::kAccCols;
-      TOut* out = reinterpret_cast<TOut*>(p.out);
       const int nchunks = (n + 31) >> 5;
-      const int fbase = m0 + static_cast<int>(rank) * 128 + q * 32 + lane;
+      const int col_cta = m0 + static_cast<int>(rank) * 128;  // first feature of this CTA
       if constexpr (EPI == EPI_SWIGLU) {
-        const int f = fbase;
+        const int f = col_cta + fl;
         const bool f_ok = f < p.m_valid;
-        for (int c = 0; c < nchunks; ++c) {
+        for (int c = grp; c < nchunks; c += 2) {
           uint32_t v[32], u[32];
           tmem_ld32(taddr + 32u * c, v);
           tmem_ld32(taddr + 256u + 32u * c, u);
           tmem_ld_wait();
+          float hv[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const int tok = c * 32 + i;
             const float a = __uint_as_float(v[i]);
-            const float h = a / (1.0f + __expf(-a)) * __uint_as_float(u[i]);
-            if (tok < n && f_ok) out[(static_cast<int64_t>(row0) + tok) * p.ld_out + f] = from_f32<TOut>(h);
+            hv[i] = __fdividef(a, 1.0f + __expf(-a)) * __uint_as_float(u[i]);  // SiLU(gate) * up
           }
+          emit(hv, c, col_cta, row0, n, f_ok, f);
         }
       } else {
 #pragma unroll
         for (int h = 0; h < MT; ++h) {
-          const int f = fbase + h * 256;
+          const int f = col_cta + h * 256 + fl;
           const bool f_ok = f < p.m_valid;
           float gain1 = 1.0f;
           if (EPI == EPI_STORE_SS && p.ss_gain != nullptr && f_ok)
             gain1 = 1.0f + to_f32(reinterpret_cast<const TIn*>(p.ss_gain)[g * p.ss_gain_group_stride + f]);
-          for (int c = 0; c < nchunks; ++c) {
+          for (int c = grp; c < nchunks; c += 2) {
             uint32_t v[32];
             tmem_ld32(taddr + static_cast<uint32_t>(h * 256) + 32u * c, v);
             tmem_ld_wait();
+            float yv[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int tok = c * 32 + i;
-              if (tok < n && f_ok)
-                out[(static_cast<int64_t>(row0) + tok) * p.ld_out + f] = from_f32<TOut>(__uint_as_float(v[i]));
-            }
+            for (int i = 0; i < 32; ++i) yv[i] = __uint_as_float(v[i]);
             if constexpr (EPI == EPI_STORE_SS) {
               float sq[32];
 #pragma unroll
               for (int i = 0; i < 32; ++i) {
-                const float y = __uint_as_float(v[i]) * gain1;
+                const float y = yv[i] * gain1;
                 sq[i] = f_ok ? y * y : 0.0f;
               }
               const float tot = transpose_reduce32(sq, lane);
               const int tok = c * 32 + lane;
-              const int col = (m0 + h * 256 + static_cast<int>(rank) * 128) >> 5;
-              if (tok < n) p.ss[(static_cast<int64_t>(row0) + tok) * p.ss_ld + col + q] = tot;
+              if (tok < n) p.ss[(static_cast<int64_t>(row0) + tok) * p.ss_ld + ((col_cta + h * 256) >> 5) + q] = tot;
             }
+            emit(yv, c, col_cta + h * 256, row0, n, f_ok, f);
           }
         }
       }
@@ -281,6 +323,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         acc_phase ^= 1u;
       }
     }
+    if (kTmaStore && elected) bulk_wait_group_all();  // stores done before the CTA leaves
   }
 
   tc_fence_before();

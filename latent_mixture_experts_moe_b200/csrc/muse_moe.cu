@@ -16,7 +16,7 @@
 #include <cstring>
 #include <mutex>
 
-#include "../../include/muse_moe.h"
+#include "muse_moe.h"
 #include "gemm_umma.cuh"
 #include "gemm_umma_2sm.cuh"
 #include "route_kernels.cuh"
@@ -135,6 +135,20 @@ bool make_map(CUtensorMap* m, const void* base, bool bf16, int64_t K, int64_t ro
   return r == CUDA_SUCCESS;
 }
 
+// Output map for TMA stores: rows x cols bf16 row-major, boxes of 16 rows x 128 columns,
+// no swizzle (the epilogue stages tiles row-major in shared memory).
+bool make_out_map(CUtensorMap* m, void* base, int64_t rows, int64_t cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  cuuint32_t box[2] = {128u, 16u};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 int sm_count() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
@@ -172,7 +186,7 @@ cudaError_t launch_gemm_2sm(const TmaMaps& maps, const GemmArgs& args, int pairs
   const size_t smem = Gemm2Shape<EPI, MT>::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  kern<<<2 * pairs, 192, smem, st>>>(maps, args);
+  kern<<<2 * pairs, kPairThreads, smem, st>>>(maps, args);
   return cudaGetLastError();
 }
 
@@ -218,6 +232,7 @@ muse_status dense_gemm(const void* W, int64_t M, const void* X, int64_t T, int64
   g.ld_out = M;
   // a CTA pair per 256 features x 256 tokens when that fills at least one wave of pairs
   if (bf && bn == 256 && cdiv(M, 256) * cdiv(T, 256) >= nsm / 2) {
+    if (sizeof(TOut) == 2 && !make_out_map(&maps.out, out, T, M)) return MUSE_ERR_CUDA;
     g.m_step = 256;
     g.m_tiles = static_cast<int>(cdiv(M, 256));
     g.num_tiles = static_cast<int>(g.m_tiles * cdiv(T, 256));
@@ -363,6 +378,7 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
     g.out = h;
     g.ld_out = I;
     if (pgu.pair) {
+      if (!make_out_map(&maps.out, h, R, I)) return MUSE_ERR_CUDA;
       MUSE_CK((launch_gemm_2sm<T, EPI_SWIGLU, 2>(maps, g, nsm / 2, st)));
     } else {
       MUSE_CK((launch_gemm_bn<T, T, EPI_SWIGLU>(bn_g, 2, maps, g, nsm, st)));
@@ -387,6 +403,7 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
       g.ss_gain = gamma;
       g.ss_gain_group_stride = c.gamma_shared ? 0 : L;
     }
+    if (pdn.pair && !make_out_map(&maps.out, y, R, L)) return MUSE_ERR_CUDA;
     if (pdn.pair && pdn.mt == 2) {
       MUSE_CK((launch_gemm_2sm<T, EPI_STORE_SS, 2>(maps, g, nsm / 2, st)));
     } else if (pdn.pair) {

@@ -222,6 +222,33 @@ __host__ __device__ constexpr uint32_t idesc_f32acc(uint32_t ab, uint32_t M, uin
   return (1u << 4) | (ab << 7) | (ab << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
+// ------------------------------------------------------------------------ TMA stores
+// 2-D tile store shared (this CTA) -> global, tracked by the issuing thread's bulk groups.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, uint32_t src, int32_t c0, int32_t c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(src), "r"(c0), "r"(c1)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// waits until at most N of this thread's bulk groups still read their shared source
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// waits until all of this thread's bulk groups have completed
+__device__ __forceinline__ void bulk_wait_group_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// orders this thread's generic-proxy shared-memory writes before later async-proxy reads
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// named barrier 1 over the 128 epilogue threads
+__device__ __forceinline__ void epilogue_bar_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// named barrier 1 + grp over one group of 4 epilogue warps (128 threads)
+__device__ __forceinline__ void epilogue_group_bar_sync(int grp) {
+  asm volatile("bar.sync %0, 128;" ::"r"(1 + grp) : "memory");
+}
+
 // ------------------------------------------------------------------------ CTA pairs
 // (cluster of 2 CTAs on one TPC driving cta_group::2 MMAs; still no multicast loads)
 __device__ __forceinline__ uint32_t cluster_ctarank() {
