@@ -359,8 +359,9 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
   // (a5) gather into expert order
   {
     const int vpr = static_cast<int>(L * sizeof(T) / 16);
-    k_gather_rows<<<4 * nsm, 256, 0, st>>>(row_token, offsets + E, reinterpret_cast<const uint4*>(z),
-                                           reinterpret_cast<uint4*>(zp), vpr);
+    const int rows_grid = static_cast<int>(std::min<int64_t>(lay.pub.rows, 16 * nsm));
+    k_gather_rows<<<rows_grid, 128, 0, st>>>(row_token, offsets + E, reinterpret_cast<const uint4*>(z),
+                                            reinterpret_cast<uint4*>(zp), vpr);
     MUSE_CK(cudaGetLastError());
     MUSE_CK(mark());
   }
@@ -416,7 +417,9 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
   // (a8 + a9) per-expert RMSNorm and weighted combine
   {
     const int vec = 16 / static_cast<int>(sizeof(T));
-    const int threads = static_cast<int>(std::max<int64_t>(32, align_up(static_cast<size_t>(L / vec), 32)));
+    // a vector per thread up to 256 threads; one warp per selected row for the scales
+    const int threads = static_cast<int>(
+        std::max<int64_t>(32 * std::min<int64_t>(k, 8), std::min<int64_t>(256, align_up(static_cast<size_t>(L / vec), 32))));
     k_combine<T><<<static_cast<unsigned>(Tn), threads, 0, st>>>(
         topk_idx, topk_w, inv, ss, static_cast<int>(L / 32), y, reinterpret_cast<const T*>(gamma),
         c.gamma_shared ? 0 : L, static_cast<int>(L), static_cast<int>(k), c.eps, cbuf);

@@ -279,18 +279,21 @@ __global__ void k_prenorm_rows(T* __restrict__ z, const T* __restrict__ w, int L
 }
 
 // --------------------------------------------------------------------------------------
-// (a3) gather: Zp[row] = z[row_token[row]] (zeros for padding rows), 16-byte vectors.
+// (a3) gather: Zp[row] = z[row_token[row]] (zeros for padding rows), 16-byte vectors;
+// one block per row (grid-strided), every thread moving several independent vectors.
 // --------------------------------------------------------------------------------------
 __global__ void k_gather_rows(const int* __restrict__ row_token, const int* __restrict__ total_rows,
                               const uint4* __restrict__ z, uint4* __restrict__ zp, int vec_per_row) {
-  const int64_t R = *total_rows;
-  const int64_t nvec = R * vec_per_row;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < nvec;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = i / vec_per_row;
-    const int c = static_cast<int>(i - r * vec_per_row);
+  const int R = *total_rows;
+  for (int r = blockIdx.x; r < R; r += gridDim.x) {
     const int tok = row_token[r];
-    zp[i] = (tok >= 0) ? z[static_cast<int64_t>(tok) * vec_per_row + c] : make_uint4(0, 0, 0, 0);
+    uint4* dst = zp + static_cast<int64_t>(r) * vec_per_row;
+    if (tok >= 0) {
+      const uint4* src = z + static_cast<int64_t>(tok) * vec_per_row;
+      for (int c = threadIdx.x; c < vec_per_row; c += blockDim.x) dst[c] = src[c];
+    } else {
+      for (int c = threadIdx.x; c < vec_per_row; c += blockDim.x) dst[c] = make_uint4(0, 0, 0, 0);
+    }
   }
 }
 
@@ -311,41 +314,41 @@ __global__ void k_combine(const int* __restrict__ topk_idx, const float* __restr
   __shared__ int pos_s[32];
   __shared__ int e_s[32];
   const int t = blockIdx.x;
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
-    for (int j = 0; j < k; ++j) {
-      const int64_t a = static_cast<int64_t>(t) * k + j;
-      const int pos = inv[a];
-      float s = 0.0f;
-      for (int i = lane; i < ss_ld; i += 32) s += ss[static_cast<int64_t>(pos) * ss_ld + i];
-      s = warp_sum(s);
-      if (lane == 0) {
-        scale_s[j] = topk_w[a] * (1.0f / sqrtf(s / static_cast<float>(L) + eps));
-        pos_s[j] = pos;
-        e_s[j] = topk_idx[a];
-      }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  // the k row scales in parallel, one warp per selected row
+  for (int j = warp; j < k; j += nw) {
+    const int64_t a = static_cast<int64_t>(t) * k + j;
+    const int pos = inv[a];
+    float s = 0.0f;
+    for (int i = lane; i < ss_ld; i += 32) s += ss[static_cast<int64_t>(pos) * ss_ld + i];
+    s = warp_sum(s);
+    if (lane == 0) {
+      scale_s[j] = topk_w[a] * (1.0f / sqrtf(s / static_cast<float>(L) + eps));
+      pos_s[j] = pos;
+      e_s[j] = topk_idx[a];
     }
   }
   __syncthreads();
-  const int f0 = threadIdx.x * VEC;
-  if (f0 >= L) return;
-  float acc[VEC];
+  for (int f0 = threadIdx.x * VEC; f0 < L; f0 += blockDim.x * VEC) {
+    float acc[VEC];
 #pragma unroll
-  for (int v = 0; v < VEC; ++v) acc[v] = 0.0f;
-  for (int j = 0; j < k; ++j) {
-    const uint4 yv = *reinterpret_cast<const uint4*>(Y + static_cast<int64_t>(pos_s[j]) * L + f0);
-    const uint4 gv = *reinterpret_cast<const uint4*>(gamma + e_s[j] * gamma_stride + f0);
-    const T* yy = reinterpret_cast<const T*>(&yv);
-    const T* gg = reinterpret_cast<const T*>(&gv);
-    const float sj = scale_s[j];
+    for (int v = 0; v < VEC; ++v) acc[v] = 0.0f;
+#pragma unroll 8
+    for (int j = 0; j < k; ++j) {
+      const uint4 yv = *reinterpret_cast<const uint4*>(Y + static_cast<int64_t>(pos_s[j]) * L + f0);
+      const uint4 gv = *reinterpret_cast<const uint4*>(gamma + e_s[j] * gamma_stride + f0);
+      const T* yy = reinterpret_cast<const T*>(&yv);
+      const T* gg = reinterpret_cast<const T*>(&gv);
+      const float sj = scale_s[j];
 #pragma unroll
-    for (int v = 0; v < VEC; ++v) acc[v] = fmaf(sj * (1.0f + to_f32(gg[v])), to_f32(yy[v]), acc[v]);
+      for (int v = 0; v < VEC; ++v) acc[v] = fmaf(sj * (1.0f + to_f32(gg[v])), to_f32(yy[v]), acc[v]);
+    }
+    uint4 ov;
+    T* oo = reinterpret_cast<T*>(&ov);
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) oo[v] = from_f32<T>(acc[v]);
+    *reinterpret_cast<uint4*>(c + static_cast<int64_t>(t) * L + f0) = ov;
   }
-  uint4 ov;
-  T* oo = reinterpret_cast<T*>(&ov);
-#pragma unroll
-  for (int v = 0; v < VEC; ++v) oo[v] = from_f32<T>(acc[v]);
-  *reinterpret_cast<uint4*>(c + static_cast<int64_t>(t) * L + f0) = ov;
 }
 
 }  // namespace muse
