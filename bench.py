@@ -132,11 +132,21 @@ def step_work(w: W.Workload, n_touched: int):
 
 
 # ------------------------------------------------------------------------------ our arm
+def rank_tokens(w: W.Workload, rank: int, dev) -> torch.Tensor:
+    """Rank r's batch: tokens [rT, (r+1)T) of the workload's one seeded token stream, so N
+    replicas together process N*T distinct tokens (weak scaling, no data-path exchange)."""
+    x = torch.empty((w.T, w.D), dtype=W.TORCH_DTYPE[w.dtype], device=dev)
+    return W.fill(x, w.seed, W.TID["x"], 1.0, start=rank * w.T * w.D)
+
+
+def job_tokens_per_s(world: int, T: int, steps: int, ms_max: float) -> float:
+    """Whole-job throughput: tokens of all ranks over the slowest rank's time."""
+    return world * T * steps / (ms_max * 1e-3)
+
+
 def make_rank_inputs(w: W.Workload, rank: int, dev):
     inp = W.make_inputs(w, dev, names=["W_router", "W_pool", "W_gate", "W_up", "W_down", "gamma", "W_unpool"])
-    x = torch.empty((w.T, w.D), dtype=W.TORCH_DTYPE[w.dtype], device=dev)
-    W.fill(x, w.seed, W.TID["x"], 1.0, start=rank * w.T * w.D)   # rank r: tokens [rT, (r+1)T)
-    inp["x"] = x
+    inp["x"] = rank_tokens(w, rank, dev)
     return inp
 
 
@@ -209,7 +219,7 @@ def run_ours(w: W.Workload, inp, steps: int, warmup: int, rank: int, world: int,
     t_step = ms_max / steps * 1e-3
     step_roof = max(sf / (peaks["bf16_tflops_sustained"] * 1e12), sb / (peaks["hbm_gbs"] * 1e9))
     res = {
-        "value": world * w.T * steps / (ms_max * 1e-3),
+        "value": job_tokens_per_s(world, w.T, steps, ms_max),
         "ms_per_step": ms_max / steps,
         "stage_ms": {moe.STAGES[i]: round(stage_ms[i], 4) for i in range(nst)},
         "roofline": roof,
@@ -248,7 +258,7 @@ def run_e2e(w, model, inp, steps, world, dev):
     torch.cuda.synchronize()
     ms = all_max(s.elapsed_time(e), world, dev)
     nbytes = w.T * w.D * (2 if w.dtype == "bf16" else 4)
-    return {"value": world * w.T * steps / (ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": nbytes,
+    return {"value": job_tokens_per_s(world, w.T, steps, ms), "unit": "tokens/s", "h2d_bytes_per_step": nbytes,
             "d2h_bytes_per_step": nbytes, "ms_per_step": ms / steps}
 
 
@@ -406,9 +416,7 @@ def main():
         side = {}
         if not args.no_side and w.name == "prefill":
             wd = W.WORKLOADS["decode"]
-            xd = torch.empty((wd.T, wd.D), dtype=inp["x"].dtype, device=dev)
-            W.fill(xd, wd.seed, W.TID["x"], 1.0, start=rank * wd.T * wd.D)
-            inp_d = dict(inp, x=xd)
+            inp_d = dict(inp, x=rank_tokens(wd, rank, dev))
             side["decode"] = run_ours(wd, inp_d, max(args.steps, 50), args.warmup, rank, world, peaks, peak_kind,
                                       False, e2e_steps=0)
             wz = W.WORKLOADS["prefill_zipf"]

@@ -183,6 +183,14 @@ MUSE_API muse_status muse_latent_moe_forward_static_scratch(const muse_moe_confi
                                                             const void* W_down, const void* gamma,
                                                             const void* W_unpool, void* out, void* stream);
 
+/* Self-test of the device-side bounded waits every kernel of this library uses: launches
+ * one small kernel whose single waiting thread waits on an mbarrier that nothing ever
+ * completes, with a limit of limit_ns nanoseconds (1 .. 10^10), on `stream`. The wait
+ * gives up, the kernel ends normally and status_dev (caller-owned device uint32[2],
+ * zero it first) receives {MUSE_ERR_TIMEOUT, detail}; the context stays usable. Returns
+ * MUSE_OK once launched, MUSE_ERR_INVALID_ARG for a null pointer or a limit out of range. */
+MUSE_API muse_status muse_selftest_bounded_wait(uint64_t limit_ns, uint32_t* status_dev, void* stream);
+
 /* Static string for a status code. */
 MUSE_API const char* muse_status_string(muse_status s);
 

@@ -24,7 +24,8 @@ STATUS = {0: "MUSE_OK", 1: "MUSE_ERR_INVALID_ARG", 2: "MUSE_ERR_UNSUPPORTED", 3:
 # every extern "C" entry point of include/muse_moe.h
 EXPORTS = ("muse_moe_config_init", "muse_latent_moe_workspace_size", "muse_latent_moe_workspace_layout",
            "muse_latent_moe_forward", "muse_latent_moe_forward_host_io", "muse_latent_moe_last_device_status",
-           "muse_status_string", "muse_latent_moe_launch_count", "muse_latent_moe_forward_static_scratch")
+           "muse_status_string", "muse_latent_moe_launch_count", "muse_latent_moe_forward_static_scratch",
+           "muse_selftest_bounded_wait")
 
 # size of the library's built-in scratch array (MUSE_STATIC_SCRATCH_BYTES)
 STATIC_SCRATCH_BYTES = 16 << 20
@@ -81,6 +82,8 @@ def lib() -> ctypes.CDLL:
         L.muse_status_string.restype = ctypes.c_char_p
         L.muse_latent_moe_forward_static_scratch.argtypes = [cp] + [vp] * 10
         L.muse_latent_moe_forward_static_scratch.restype = ctypes.c_int
+        L.muse_selftest_bounded_wait.argtypes = [ctypes.c_uint64, vp, vp]
+        L.muse_selftest_bounded_wait.restype = ctypes.c_int
         L.muse_latent_moe_launch_count.argtypes = [cp]
         L.muse_latent_moe_launch_count.restype = ctypes.c_int32
         _lib = L
@@ -179,6 +182,12 @@ def event_handles(events) -> "ctypes.Array":
     for i, ev in enumerate(events):
         arr[i] = int(ev.cuda_event)
     return arr
+
+
+def selftest_bounded_wait(limit_ns: int, status_dev, stream=None) -> None:
+    """Run the device-side bounded-wait self-test (status_dev: zeroed CUDA int32[2])."""
+    _check(lib().muse_selftest_bounded_wait(int(limit_ns), _ptr(status_dev), _stream_handle(stream)),
+           "muse_selftest_bounded_wait")
 
 
 def last_device_status(cfg: Config, stream=None):

@@ -560,6 +560,12 @@ muse_status muse_latent_moe_last_device_status(const muse_moe_config* cfg, void*
   return static_cast<muse_status>(word[0]);
 }
 
+muse_status muse_selftest_bounded_wait(uint64_t limit_ns, uint32_t* status_dev, void* stream) {
+  if (status_dev == nullptr || limit_ns < 1 || limit_ns > 10000000000ull) return MUSE_ERR_INVALID_ARG;
+  k_selftest_wait<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns, status_dev);
+  return cudaGetLastError() == cudaSuccess ? MUSE_OK : MUSE_ERR_CUDA;
+}
+
 const char* muse_status_string(muse_status s) {
   switch (s) {
     case MUSE_OK: return "ok";

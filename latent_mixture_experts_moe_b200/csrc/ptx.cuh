@@ -77,14 +77,14 @@ __device__ __forceinline__ void record_status(uint32_t* status, uint32_t code, u
 // sets *abort and records MUSE_ERR_TIMEOUT with `detail` -- so no wait can hang the GPU.
 template <bool kClusterScope = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
-                                          uint32_t* status, uint32_t detail) {
+                                          uint32_t* status, uint32_t detail, uint64_t limit_ns = kWaitLimitNs) {
   auto test = [&]() { return kClusterScope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
   if (test()) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (test()) return true;
     if (*abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       *abort = 1;
       record_status(status, kStatusTimeout, detail);
       return false;

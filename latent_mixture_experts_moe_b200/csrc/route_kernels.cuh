@@ -351,4 +351,24 @@ __global__ void k_combine(const int* __restrict__ topk_idx, const float* __restr
   }
 }
 
+// --------------------------------------------------------------------------------------
+// Self-test of the bounded waits: one thread waits on an mbarrier that nothing will ever
+// complete, through the same mbar_wait the GEMMs use, with a short limit; the timeout is
+// recorded in status (a completed wait would be recorded as a device error).
+// --------------------------------------------------------------------------------------
+__global__ void k_selftest_wait(uint64_t limit_ns, uint32_t* status) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (mbar_wait(smem_u32(&bar), 0u, &abort_flag, status, 0x5E1Fu, limit_ns))
+      record_status(status, kStatusDevice, 0x5E1Fu);
+  }
+}
+
 }  // namespace muse

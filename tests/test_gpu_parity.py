@@ -133,6 +133,31 @@ def test_edge_cases(case):
         assert np.array_equal(run.inter("inv", torch.int32, (T * k,)).cpu().numpy(), inv)
 
 
+# ------------------------------------------------------------------------- failure detection
+def test_bounded_wait_times_out_and_the_context_stays_usable(tiny):
+    """A wait that nothing completes gives up after its limit and reports
+    MUSE_ERR_TIMEOUT through the status word; no trap, no hang, and the next forward runs."""
+    status = torch.zeros(2, dtype=torch.int32, device="cuda")
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    moe.selftest_bounded_wait(2_000_000, status)          # 2 ms limit
+    end.record()
+    torch.cuda.synchronize()
+    assert status.tolist() == [5, 0x5E1F]                  # MUSE_ERR_TIMEOUT, the wait's id
+    assert start.elapsed_time(end) >= 2.0
+    w, inp = tiny
+    run = Run(w, inp)                                      # the context is still usable
+    full_check(w, inp, run)
+
+
+def test_selftest_rejects_bad_arguments():
+    lib = moe.lib()
+    assert lib.muse_selftest_bounded_wait(1000, None, None) == 1
+    status = torch.zeros(2, dtype=torch.int32, device="cuda")
+    assert lib.muse_selftest_bounded_wait(0, status.data_ptr(), None) == 1
+    assert lib.muse_selftest_bounded_wait(10**11, status.data_ptr(), None) == 1
+
+
 # ------------------------------------------------------------------------- released mode
 PAGES = [
     # name, T, D, L, I, E, k
