@@ -21,6 +21,7 @@ needed. Per-kernel durations come from events the library records between its la
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import json
 import math
@@ -107,6 +108,7 @@ def stage_work(w: W.Workload, n_touched: int):
     to move them)."""
     T, D, L, I, E, k = w.T, w.D, w.L, w.I, w.E, w.k
     a = 2 if w.dtype == "bf16" else 4
+    ab = 0.5625 if w.experts == "nvfp4" else a      # bytes per expert weight
     A = T * k
     return {
         "router": (2 * T * E * D, T * D * a + E * D * a + T * E * 4),
@@ -116,8 +118,8 @@ def stage_work(w: W.Workload, n_touched: int):
         "assign_rows": (0, A * 8),
         "pooler": (2 * T * L * D, T * D * a + L * D * a + T * L * a),
         "gather": (0, T * L * a + A * L * a),
-        "gate_up_swiglu": (2 * A * L * 2 * I, n_touched * 2 * I * L * a + A * L * a + A * I * a),
-        "down_sumsq": (2 * A * I * L, n_touched * L * I * a + A * I * a + A * L * a + A * (L // 32) * 4),
+        "gate_up_swiglu": (2 * A * L * 2 * I, n_touched * 2 * I * L * ab + A * L * a + A * I * a),
+        "down_sumsq": (2 * A * I * L, n_touched * L * I * ab + A * I * a + A * L * a + A * (L // 32) * 4),
         "norm_combine": (0, A * L * a + A * (L // 32) * 4 + T * L * a + n_touched * L * a),
         "unpooler": (2 * T * D * L, T * L * a + D * L * a + T * D * a),
     }
@@ -126,8 +128,9 @@ def stage_work(w: W.Workload, n_touched: int):
 def step_work(w: W.Workload, n_touched: int):
     T, D, L, I, E, k = w.T, w.D, w.L, w.I, w.E, w.k
     a = 2 if w.dtype == "bf16" else 4
+    ab = 0.5625 if w.experts == "nvfp4" else a
     flops = 2 * T * (E * D + L * D + k * 3 * L * I + D * L)
-    byts = 2 * T * D * a + (E * D + 2 * L * D) * a + n_touched * (3 * L * I + L) * a
+    byts = 2 * T * D * a + (E * D + 2 * L * D) * a + n_touched * (3 * L * I * ab + L * a)
     return flops, byts
 
 
@@ -392,6 +395,7 @@ def main():
     ap.add_argument("--workload", default="prefill", choices=list(W.WORKLOADS))
     ap.add_argument("--no-side", action="store_true", help="skip the decode / skewed side workloads")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle cpu_baseline")
+    ap.add_argument("--no-nvfp4", action="store_true", help="skip the NVFP4-expert side workloads")
     ap.add_argument("--cpu-tokens", type=int, default=4)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -423,6 +427,18 @@ def main():
             inp_z = dict(inp, router_bias=W.zipf_router_bias(wz).to(dev))
             side["prefill_zipf"] = run_ours(wz, inp_z, args.steps, args.warmup, rank, world, peaks, peak_kind,
                                             False, e2e_steps=0)
+            if not args.no_nvfp4:
+                # NVFP4 experts (quantised from the same bf16 weights): T=4096 and a T=64 decode
+                wq = W.WORKLOADS["nvfp4"]
+                q = W.make_inputs(wq, dev, names=["W_gate", "W_up", "W_down"])
+                inp_q = dict({k: v for k, v in inp.items() if k not in ("W_gate", "W_up", "W_down")}, **q)
+                inp_q["x"] = rank_tokens(wq, rank, dev)
+                side["nvfp4"] = run_ours(wq, inp_q, args.steps, args.warmup, rank, world, peaks, peak_kind,
+                                         False, e2e_steps=0)
+                wqd = dataclasses.replace(wq, name="nvfp4_decode", T=64)
+                inp_qd = dict(inp_q, x=rank_tokens(wqd, rank, dev))
+                side["nvfp4_decode"] = run_ours(wqd, inp_qd, max(args.steps, 50), args.warmup, rank, world, peaks,
+                                                peak_kind, False, e2e_steps=0)
         if rank == 0:
             line = {
                 "metric": metric_name(), "value": main_res["value"], "unit": "tokens/s", "n_gpus": world,

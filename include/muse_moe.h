@@ -65,6 +65,23 @@ typedef enum muse_router_mode {
                                  key = s + b, g = rsf * s / (sum_S s + 1e-15)          */
 } muse_router_mode;
 
+typedef enum muse_expert_weights {
+  MUSE_EXPERTS_DENSE = 0,     /* W_gate / W_up / W_down are dense tensors of cfg->dtype   */
+  MUSE_EXPERTS_NVFP4 = 1      /* each points to a muse_nvfp4_weight (below); bf16 only    */
+} muse_expert_weights;
+
+/* One NVFP4 expert weight tensor [E, out, in] (deep dive §7.3-7.4: 4-bit values, one FP8
+ * E4M3 scale per 16 weights; 0.5625 bytes per weight): element (e, o, i) is
+ *   e2m1(nibble) * e4m3(block_scales[e, o, i / 16]) * matrix_scale[e],
+ * the nibble being the low half of codes[e, o, i / 2] for even i, the high half for odd i.
+ * E2M1 and E4M3 are the OCP MX v1.0 FP4 and FP8 formats. The struct lives in host memory;
+ * its pointers are device memory, 16-byte aligned. */
+typedef struct muse_nvfp4_weight {
+  const void* codes;          /* uint8 [E, out, in/2]                                 */
+  const void* block_scales;   /* uint8 (E4M3) [E, out, in/16]                          */
+  const float* matrix_scale;  /* float [E]                                            */
+} muse_nvfp4_weight;
+
 typedef enum muse_norm_mode {
   MUSE_NORM_CENTRED = 0,      /* y / sqrt(mean(y^2)+eps) * (1+gamma)                   */
   MUSE_NORM_INPUT_SCALED = 1  /* u / sqrt(mean(u^2)+eps), u = y * (1+gamma)           */
@@ -97,6 +114,7 @@ typedef struct muse_moe_config {
   void* const* stage_events;  /* optional: launch_count + 1 cudaEvent_t handles; event i
                                  is recorded on the stream before launch i and the last
                                  after the final launch (per-kernel device timing)     */
+  int32_t expert_weights;     /* muse_expert_weights                                  */
 } muse_moe_config;
 
 /* Byte offsets of the intermediates inside the workspace after a forward call, for
@@ -132,6 +150,8 @@ MUSE_API muse_status muse_latent_moe_workspace_layout(const muse_moe_config* cfg
                                              muse_moe_workspace_layout* layout);
 
 /* Forward pass of the block on device buffers (layouts above); enqueued on `stream`
+ * (with cfg->expert_weights == MUSE_EXPERTS_NVFP4, W_gate / W_up / W_down are host
+ * pointers to muse_nvfp4_weight descriptions of device tensors)
  * (a cudaStream_t, NULL = legacy default stream). Pointers must be device memory,
  * 16-byte aligned; `out` must not alias an input. Returns without synchronising. */
 MUSE_API muse_status muse_latent_moe_forward(const muse_moe_config* cfg, const void* x,

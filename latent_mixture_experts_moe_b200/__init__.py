@@ -16,6 +16,7 @@ LIB_PATH = os.path.join(PKG, "libmuse_moe.so")
 
 MUSE_F32, MUSE_BF16 = 0, 1
 ROUTER_SOFTMAX, ROUTER_SIGMOID = 0, 1
+EXPERTS_DENSE, EXPERTS_NVFP4 = 0, 1
 NORM_CENTRED, NORM_INPUT_SCALED = 0, 1
 
 STATUS = {0: "MUSE_OK", 1: "MUSE_ERR_INVALID_ARG", 2: "MUSE_ERR_UNSUPPORTED", 3: "MUSE_ERR_WORKSPACE",
@@ -46,7 +47,11 @@ class Config(ctypes.Structure):
                 ("pre_norm_gain", ctypes.c_void_p), ("pre_norm_eps", ctypes.c_float),
                 ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
                 ("topk_idx_out", ctypes.c_void_p), ("topk_w_out", ctypes.c_void_p),
-                ("stage_events", ctypes.c_void_p)]
+                ("stage_events", ctypes.c_void_p), ("expert_weights", ctypes.c_int32)]
+
+
+class Nvfp4Weight(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("block_scales", ctypes.c_void_p), ("matrix_scale", ctypes.c_void_p)]
 
 
 class WorkspaceLayout(ctypes.Structure):
@@ -132,6 +137,8 @@ def launch_count(cfg: Config) -> int:
 def _ptr(t) -> int:
     if t is None:
         return 0
+    if isinstance(t, ctypes.Structure):
+        return ctypes.addressof(t)
     if not t.is_contiguous():
         raise ValueError("tensors must be contiguous")
     return int(t.data_ptr())
@@ -206,9 +213,18 @@ class LatentMoE:
 
     def __init__(self, weights: Dict, T_max: int, k: int, eps: float = 1e-6, **modes):
         import torch
-        self.w = weights
+        self.w = dict(weights)
         E, D = weights["W_router"].shape
-        _, I, L = weights["W_gate"].shape
+        self.nvfp4 = "W_gate_codes" in weights
+        if self.nvfp4:
+            # NVFP4 experts: <name>_codes [E, out, in/2], <name>_scales [E, out, in/16], <name>_mscale [E]
+            _, I, L2 = weights["W_gate_codes"].shape
+            L = 2 * L2
+            for n in ("W_gate", "W_up", "W_down"):
+                self.w[n] = Nvfp4Weight(_ptr(weights[n + "_codes"]), _ptr(weights[n + "_scales"]),
+                                        _ptr(weights[n + "_mscale"]))
+        else:
+            _, I, L = weights["W_gate"].shape
         self.dtype = {torch.float32: "f32", torch.bfloat16: "bf16"}[weights["W_router"].dtype]
         self.dims = dict(D=int(D), L=int(L), I=int(I), E=int(E), k=k, eps=eps)
         self.modes = modes
@@ -219,6 +235,8 @@ class LatentMoE:
     def config(self, T: int, workspace=None) -> Config:
         d = self.dims
         c = make_config(T, d["D"], d["L"], d["I"], d["E"], d["k"], self.dtype, d["eps"], **self.modes)
+        if self.nvfp4:
+            c.expert_weights = EXPERTS_NVFP4
         if self.w.get("router_bias") is not None:
             c.router_bias = _ptr(self.w["router_bias"])
         if self.w.get("pre_norm_gain") is not None:

@@ -1,0 +1,395 @@
+// gemm_umma_fp4.cuh -- the grouped expert GEMMs with NVFP4 expert weights (W4A16):
+//
+//   C[token, f] = mscale[e] * sum_k (e2m1(code[f, k]) * e4m3(scale[f, k / 16])) * X[token, k]
+//
+// Weights stay 4-bit in HBM (0.5 B per weight + one E4M3 byte per 16): TMA brings the packed
+// codes of a 128-row x 64-K tile (4 KB) into shared memory, four converter warps expand it
+// into the bf16 128-byte-swizzled tile the UMMA reads (code x block scale is exact in bf16:
+// at most 2 + 4 significant bits), and the per-matrix FP32 scale multiplies the FP32
+// accumulator in the epilogue. Tokens (bf16) are the B operand as in gemm_umma.cuh.
+//
+// Roles (320 threads, one CTA per SM): warp 0 TMA producer (codes + token tile), warp 1 TMEM
+// owner + UMMA issuer, warps 2..5 epilogue, warps 6..9 converters (thread i of them expands
+// weight row i of each 128-row tile, its block scales read from global memory one k-block
+// ahead). Barriers per stage: full (TMA bytes), conv (4 converter warps), empty (UMMA commit).
+// Every wait is bounded (ptx.cuh).
+#pragma once
+
+#include "gemm_umma.cuh"
+
+namespace muse {
+
+struct Fp4Args {
+  const uint8_t* scales_a;   // E4M3 block scales of the matrix behind maps.a  [rows, scale_ld]
+  const uint8_t* scales_a2;  // ... behind maps.a2 (gate/up: the up matrix; else = scales_a)
+  const float* mscale_a;     // per-group (expert) matrix scales of maps.a
+  const float* mscale_a2;
+  int scale_ld;              // bytes per weight row of block scales (K / 16)
+};
+
+template <int BN, int EPI, int MT>
+struct Fp4Shape {
+  static constexpr uint32_t kABytes = 128u * 128u;   // bf16 tile written by the converters
+  static constexpr uint32_t kCodeBytes = 128u * 32u; // packed codes of 128 rows x 64 K
+  static constexpr uint32_t kBBytes = static_cast<uint32_t>(BN) * 128u;
+  static constexpr uint32_t kStageBytes = kABytes * MT + kBBytes + kCodeBytes * MT;
+  static constexpr int kSmemBudget = 227 * 1024 - 1024 - 1024;   // alignment, LUT + barriers
+  static constexpr int kStagesFit = kSmemBudget / static_cast<int>(kStageBytes);
+  static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
+  static constexpr int kAccStages = MT == 2 ? 1 : 2;
+  static constexpr uint32_t kAccCols = static_cast<uint32_t>(BN) * MT;
+  static constexpr uint32_t kColsNeeded = kAccCols * kAccStages;
+  static constexpr uint32_t kTmemCols = kColsNeeded <= 32 ? 32 : kColsNeeded <= 64 ? 64
+                                        : kColsNeeded <= 128 ? 128 : kColsNeeded <= 256 ? 256 : 512;
+  static constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes + 1024;
+  static_assert(kStages >= 2, "tile too large for the shared-memory ring");
+  static_assert(EPI != EPI_SWIGLU || MT == 2, "SwiGLU needs the gate and up accumulators");
+};
+
+constexpr int kFp4Threads = 320;
+
+// 4 codes (the low 16 bits of w: nibbles k0..k3) -> 4 bf16 in two words, low element
+// first. Magnitude bytes come from two 8-entry byte tables (byte-permute lookups), the
+// sign goes to bit 15 of each half.
+__device__ __forceinline__ void e2m1x4_to_bf16(uint32_t w, uint32_t& o0, uint32_t& o1) {
+  const uint32_t sel = w & 0x7777u;
+  // |value| as bf16: high bytes {00,3F,3F,3F,40,40,40,40}, low {00,00,80,C0,00,40,80,C0}
+  const uint32_t hi = __byte_perm(0x3F3F3F00u, 0x40404040u, sel);
+  const uint32_t lo = __byte_perm(0xC0800000u, 0xC0804000u, sel);
+  o0 = __byte_perm(lo, hi, 0x5140u) | ((w << 12) & 0x8000u) | ((w << 24) & 0x80000000u);
+  o1 = __byte_perm(lo, hi, 0x7362u) | ((w << 4) & 0x8000u) | ((w << 16) & 0x80000000u);
+}
+
+__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
+  __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162*>(&a);
+  __nv_bfloat162 y = *reinterpret_cast<__nv_bfloat162*>(&b);
+  __nv_bfloat162 r = __hmul2(x, y);
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
+// Expands one 64-weight row segment (32 code bytes at `codes`, 4 E4M3 scales in `s4`) into
+// the 128-byte row `r` of a 128-byte-swizzled bf16 tile at `tile` (16-byte chunk c of row r
+// sits at chunk position c ^ (r & 7)).
+__device__ __forceinline__ void expand_row(const uint8_t* codes, uint32_t s4, const uint16_t* lut, uint8_t* tile,
+                                           int r) {
+  const uint4 c0 = *reinterpret_cast<const uint4*>(codes);
+  const uint4 c1 = *reinterpret_cast<const uint4*>(codes + 16);
+  const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+  uint8_t* row = tile + r * 128;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t sb = lut[(s4 >> (8 * (i >> 1))) & 0xFFu];   // one scale per 16 weights
+    const uint32_t s2 = sb | (sb << 16);
+    uint32_t a0, a1, b0, b1;
+    e2m1x4_to_bf16(words[i], a0, a1);
+    e2m1x4_to_bf16(words[i] >> 16, b0, b1);
+    uint4 v;
+    v.x = bf16x2_mul(a0, s2);
+    v.y = bf16x2_mul(a1, s2);
+    v.z = bf16x2_mul(b0, s2);
+    v.w = bf16x2_mul(b1, s2);
+    *reinterpret_cast<uint4*>(row + ((i ^ (r & 7)) << 4)) = v;
+  }
+}
+
+template <int BN, int EPI, int MT>
+__global__ void __launch_bounds__(kFp4Threads, 1)
+    k_umma_gemm_fp4(const __grid_constant__ TmaMaps maps, const GemmArgs p, const Fp4Args q4) {
+  using S = Fp4Shape<BN, EPI, MT>;
+  using TOut = __nv_bfloat16;
+  constexpr int kStages = S::kStages;
+  constexpr bool kDual = (MT == 2);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint16_t* lut = reinterpret_cast<uint16_t*>(smem + kStages * S::kStageBytes);       // 256 x bf16
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * S::kStageBytes + 512);
+  // bars: full[kStages], conv[kStages], empty[kStages], acc_full[2], acc_empty[2]
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 3 * kStages + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t bar0 = smem_u32(bars);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto conv_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (2 * kStages + s); };
+  auto accf_bar = [&](int a) { return bar0 + 8u * (3 * kStages + a); };
+  auto acce_bar = [&](int a) { return bar0 + 8u * (3 * kStages + 2 + a); };
+  auto a_tile = [&](int s, int m) { return smem + s * S::kStageBytes + m * S::kABytes; };
+  auto b_tile = [&](int s) { return smem + s * S::kStageBytes + MT * S::kABytes; };
+  auto code_tile = [&](int s, int m) { return smem + s * S::kStageBytes + MT * S::kABytes + S::kBBytes + m * S::kCodeBytes; };
+
+  // E4M3 -> bf16 (exact: at most 4 significant bits, 2^-9 .. 448); S.1111.111 -> NaN
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) {
+    const uint32_t s = (i >> 7) & 1, e = (i >> 3) & 15, m = i & 7;
+    float v;
+    if (e == 15 && m == 7) {
+      v = __int_as_float(0x7FC00000);
+    } else if (e == 0) {
+      v = static_cast<float>(m) * 0.001953125f;  // m * 2^-9
+    } else {
+      v = __int_as_float(static_cast<int>(((e + 120u) << 23) | (m << 20)));
+    }
+    if (s) v = -v;
+    lut[i] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(conv_bar(s), 4);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(accf_bar(a), 1);
+      mbar_init(acce_bar(a), 4);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&maps.a);
+    if (kDual) prefetch_tmap(&maps.a2);
+    for (int i = 0; i < 5 && (16 << i) <= BN; ++i) prefetch_tmap(&maps.b[i]);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), S::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const int num_tiles = *p.num_tiles_dev;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+        int g, m0, row0, n;
+        gemm_tile(p, t, BN, g, m0, row0, n);
+        const int nb16 = (n + 15) >> 4;
+        const uint32_t bytes = S::kCodeBytes * MT + static_cast<uint32_t>(nb16) * 2048u;
+        const int a_row = g * p.rows_per_group + m0;
+        const int a2_row = EPI == EPI_SWIGLU ? a_row : a_row + 128;
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.status, 0x900u + stage)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(full_bar(stage), bytes);
+          tma_load_2d(smem_u32(code_tile(stage, 0)), &maps.a, full_bar(stage), kb * 32, a_row);
+          if (kDual) tma_load_2d(smem_u32(code_tile(stage, 1)), &maps.a2, full_bar(stage), kb * 32, a2_row);
+          const uint32_t sB = smem_u32(b_tile(stage));
+          const int kc = kb * 64;
+          int j16 = 0;
+#pragma unroll
+          for (int i = 4; i >= 0; --i) {
+            if ((16 << i) <= BN && (nb16 >> i) & 1) {
+              tma_load_2d(sB + 2048u * j16, &maps.b[i], full_bar(stage), kc, row0 + 16 * j16);
+              j16 += 1 << i;
+            }
+          }
+          issued_mask |= 1u << stage;
+          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        for (int s = 0; s < kStages; ++s)
+          if (issued_mask & (1u << s)) mbar_wait_drain(full_bar(s), (issued_phase >> s) & 1u);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- UMMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      bool issued_any = false;
+      for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+        int g, m0, row0, n;
+        gemm_tile(p, t, BN, g, m0, row0, n);
+        const uint32_t N = static_cast<uint32_t>((n + 15) & ~15);
+        const uint32_t idesc = idesc_f32acc(1u, 128u, N);
+        if (!mbar_wait(acce_bar(acc), acc_phase ^ 1u, abort_flag, p.status, 0xA00u + acc)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_base + static_cast<uint32_t>(acc) * S::kAccCols;
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, p.status, 0xB00u + stage) ||
+              !mbar_wait(conv_bar(stage), phase, abort_flag, p.status, 0xC00u + stage)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sA = smem_u32(a_tile(stage, 0));
+          const uint32_t sB = smem_u32(b_tile(stage));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
+            const uint64_t db = sdesc_k_sw128(sB + 32u * kk);
+            umma<false>(d, sdesc_k_sw128(sA + 32u * kk), db, idesc, accum);
+            if (kDual) umma<false>(d + BN, sdesc_k_sw128(sA + S::kABytes + 32u * kk), db, idesc, accum);
+          }
+          issued_any = true;
+          tc_commit(empty_bar(stage));
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(accf_bar(acc));
+        if (S::kAccStages == 2) {
+          acc ^= 1;
+          if (acc == 0) acc_phase ^= 1u;
+        } else {
+          acc_phase ^= 1u;
+        }
+      }
+      if (!ok && issued_any) {
+        tc_commit(accf_bar(acc));
+        mbar_wait_drain(accf_bar(acc), acc_phase);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 6) {
+    // ---------------------------------------------------------------- converters
+    const int r = threadIdx.x - 192;  // weight row of the tile this thread expands
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+      int g, m0, row0, n;
+      gemm_tile(p, t, BN, g, m0, row0, n);
+      const int a_row = g * p.rows_per_group + m0;
+      const int a2_row = EPI == EPI_SWIGLU ? a_row : a_row + 128;
+      const uint8_t* sc_a = q4.scales_a + static_cast<int64_t>(a_row + r) * q4.scale_ld;
+      const uint8_t* sc_a2 = q4.scales_a2 + static_cast<int64_t>(a2_row + r) * q4.scale_ld;
+      uint32_t s_a = *reinterpret_cast<const uint32_t*>(sc_a);
+      uint32_t s_a2 = kDual ? *reinterpret_cast<const uint32_t*>(sc_a2) : 0u;
+      bool ok = true;
+      for (int kb = 0; kb < p.k_blocks; ++kb) {
+        // next k-block's 4 scales per row, loaded while this one converts
+        uint32_t n_a = 0, n_a2 = 0;
+        if (kb + 1 < p.k_blocks) {
+          n_a = *reinterpret_cast<const uint32_t*>(sc_a + 4 * (kb + 1));
+          if (kDual) n_a2 = *reinterpret_cast<const uint32_t*>(sc_a2 + 4 * (kb + 1));
+        }
+        const bool ready = mbar_wait(full_bar(stage), phase, abort_flag, p.status, 0xD00u + stage);
+        if (!__all_sync(0xffffffffu, ready)) {
+          ok = false;
+          break;
+        }
+        expand_row(code_tile(stage, 0) + r * 32, s_a, lut, a_tile(stage, 0), r);
+        if (kDual) expand_row(code_tile(stage, 1) + r * 32, s_a2, lut, a_tile(stage, 1), r);
+        fence_proxy_async_smem();  // generic-proxy writes -> the tensor core's reads
+        __syncwarp();
+        if (lane == 0) mbar_arrive(conv_bar(stage));
+        s_a = n_a;
+        s_a2 = n_a2;
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int q = warp & 3;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+      int g, m0, row0, n;
+      gemm_tile(p, t, BN, g, m0, row0, n);
+      const bool ready = mbar_wait(accf_bar(acc), acc_phase, abort_flag, p.status, 0xE00u + acc);
+      if (!__all_sync(0xffffffffu, ready)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                             static_cast<uint32_t>(acc) * S::kAccCols;
+      TOut* out = reinterpret_cast<TOut*>(p.out);
+      const int nchunks = (n + 31) >> 5;
+      const float ms_a = q4.mscale_a[g];
+      if constexpr (EPI == EPI_SWIGLU) {
+        const float ms_u = q4.mscale_a2[g];
+        const int f = m0 + q * 32 + lane;
+        const bool f_ok = f < p.m_valid;
+        for (int c = 0; c < nchunks; ++c) {
+          uint32_t v[32], u[32];
+          tmem_ld32(taddr + 32u * c, v);
+          tmem_ld32(taddr + BN + 32u * c, u);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int tok = c * 32 + i;
+            const float a = __uint_as_float(v[i]) * ms_a;
+            const float h = __fdividef(a, 1.0f + __expf(-a)) * (__uint_as_float(u[i]) * ms_u);
+            if (tok < n && f_ok) out[(static_cast<int64_t>(row0) + tok) * p.ld_out + f] = from_f32<TOut>(h);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int half = 0; half < MT; ++half) {
+          const int f = m0 + half * 128 + q * 32 + lane;
+          const bool f_ok = f < p.m_valid;
+          float gain1 = 1.0f;
+          if (EPI == EPI_STORE_SS && p.ss_gain != nullptr && f_ok)
+            gain1 = 1.0f + to_f32(reinterpret_cast<const __nv_bfloat16*>(p.ss_gain)[g * p.ss_gain_group_stride + f]);
+          for (int c = 0; c < nchunks; ++c) {
+            uint32_t v[32];
+            tmem_ld32(taddr + static_cast<uint32_t>(half * BN) + 32u * c, v);
+            tmem_ld_wait();
+            float yv[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) yv[i] = __uint_as_float(v[i]) * ms_a;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int tok = c * 32 + i;
+              if (tok < n && f_ok) out[(static_cast<int64_t>(row0) + tok) * p.ld_out + f] = from_f32<TOut>(yv[i]);
+            }
+            if constexpr (EPI == EPI_STORE_SS) {
+              float sq[32];
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const float y = yv[i] * gain1;
+                sq[i] = f_ok ? y * y : 0.0f;
+              }
+              const float tot = transpose_reduce32(sq, lane);
+              const int tok = c * 32 + lane;
+              if (tok < n) p.ss[(static_cast<int64_t>(row0) + tok) * p.ss_ld + ((m0 + half * 128) >> 5) + q] = tot;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acce_bar(acc));
+      if (S::kAccStages == 2) {
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      } else {
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, S::kTmemCols);
+  }
+}
+
+}  // namespace muse

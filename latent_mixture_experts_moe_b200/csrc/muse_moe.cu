@@ -19,6 +19,7 @@
 #include "muse_moe.h"
 #include "gemm_umma.cuh"
 #include "gemm_umma_2sm.cuh"
+#include "gemm_umma_fp4.cuh"
 #include "route_kernels.cuh"
 
 using namespace muse;
@@ -80,6 +81,8 @@ Layout make_layout(const muse_moe_config& c) {
   return l;
 }
 
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
 muse_status validate_sizes(const muse_moe_config* c) {
   if (c == nullptr) return MUSE_ERR_INVALID_ARG;
   if (c->T < 1 || c->D < 1 || c->L < 1 || c->I < 1 || c->E < 1) return MUSE_ERR_INVALID_ARG;
@@ -95,10 +98,16 @@ muse_status validate_sizes(const muse_moe_config* c) {
   if (c->T * c->top_k + 16 * c->E > (int64_t(1) << 30) || c->E * std::max(c->I, c->L) > (int64_t(1) << 31) - 1)
     return MUSE_ERR_UNSUPPORTED;
   if (c->T > (int64_t(1) << 24)) return MUSE_ERR_UNSUPPORTED;
+  if (c->expert_weights != MUSE_EXPERTS_DENSE && c->expert_weights != MUSE_EXPERTS_NVFP4) return MUSE_ERR_INVALID_ARG;
+  if (c->expert_weights == MUSE_EXPERTS_NVFP4 && c->dtype != MUSE_BF16) return MUSE_ERR_UNSUPPORTED;
   return MUSE_OK;
 }
 
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool valid_nvfp4(const void* w) {
+  const muse_nvfp4_weight* q = static_cast<const muse_nvfp4_weight*>(w);
+  return q != nullptr && q->codes != nullptr && q->block_scales != nullptr && q->matrix_scale != nullptr &&
+         aligned16(q->codes) && aligned16(q->block_scales) && (reinterpret_cast<uintptr_t>(q->matrix_scale) & 3u) == 0;
+}
 
 // ---------------------------------------------------------------------- tensor maps
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -133,6 +142,20 @@ bool make_map(CUtensorMap* m, const void* base, bool bf16, int64_t K, int64_t ro
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// Packed 4-bit codes: rows x (K/2) bytes, boxes of 128 rows x 32 bytes (64 weights),
+// no swizzle (the converter warps read them).
+bool make_code_map(CUtensorMap* m, const void* base, int64_t rows, int64_t K) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
+  cuuint32_t box[2] = {32u, 128u};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Output map for TMA stores: rows x cols bf16 row-major, boxes of 16 rows x 128 columns,
@@ -177,6 +200,30 @@ cudaError_t launch_gemm_bn(int bn, int mt, const TmaMaps& maps, const GemmArgs& 
                                  : launch_gemm<TIn, TOut, 32, EPI, 1>(maps, args, grid, st);
     return mt == 2 ? launch_gemm<TIn, TOut, 256, EPI, 2>(maps, args, grid, st)
                    : launch_gemm<TIn, TOut, 256, EPI, 1>(maps, args, grid, st);
+  }
+}
+
+template <int BN, int EPI, int MT>
+cudaError_t launch_gemm_fp4_t(const TmaMaps& maps, const GemmArgs& args, const Fp4Args& q4, int grid, cudaStream_t st) {
+  auto kern = k_umma_gemm_fp4<BN, EPI, MT>;
+  const size_t smem = Fp4Shape<BN, EPI, MT>::kSmemBytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kFp4Threads, smem, st>>>(maps, args, q4);
+  return cudaGetLastError();
+}
+
+template <int EPI>
+cudaError_t launch_gemm_fp4(int bn, int mt, const TmaMaps& maps, const GemmArgs& args, const Fp4Args& q4, int grid,
+                            cudaStream_t st) {
+  if constexpr (EPI == EPI_SWIGLU) {
+    return bn == 32 ? launch_gemm_fp4_t<32, EPI, 2>(maps, args, q4, grid, st)
+                    : launch_gemm_fp4_t<256, EPI, 2>(maps, args, q4, grid, st);
+  } else {
+    if (bn == 32) return mt == 2 ? launch_gemm_fp4_t<32, EPI, 2>(maps, args, q4, grid, st)
+                                 : launch_gemm_fp4_t<32, EPI, 1>(maps, args, q4, grid, st);
+    return mt == 2 ? launch_gemm_fp4_t<256, EPI, 2>(maps, args, q4, grid, st)
+                   : launch_gemm_fp4_t<256, EPI, 1>(maps, args, q4, grid, st);
   }
 }
 
@@ -252,10 +299,13 @@ muse_status dense_gemm(const void* W, int64_t M, const void* X, int64_t T, int64
 // tokens (bf16), else one CTA per 128 features (gate and up accumulators). down: a pair
 // per 512 features (two accumulators) or 256, else one CTA per 256 or 128 features.
 GemmPlan plan_gate_up(const muse_moe_config& c, int bn_g) {
+  if (c.expert_weights == MUSE_EXPERTS_NVFP4) return {false, 2, 128};
   if (c.dtype == MUSE_BF16 && bn_g == 256 && c.I % 256 == 0) return {true, 2, 256};
   return {false, 2, 128};
 }
 GemmPlan plan_down(const muse_moe_config& c, int bn_g) {
+  if (c.expert_weights == MUSE_EXPERTS_NVFP4) return (bn_g == 256 && c.L % 256 == 0) ? GemmPlan{false, 2, 256}
+                                                                                      : GemmPlan{false, 1, 128};
   if (c.dtype == MUSE_BF16 && bn_g == 256 && c.L % 512 == 0) return {true, 2, 512};
   if (c.dtype == MUSE_BF16 && bn_g == 256 && c.L % 256 == 0) return {true, 1, 256};
   if (bn_g == 256 && c.L % 256 == 0) return {false, 2, 256};
@@ -368,8 +418,21 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
   const int64_t R = lay.pub.rows;
   // (a6) gate/up + SwiGLU
   {
+    const bool fp4 = c.expert_weights == MUSE_EXPERTS_NVFP4;
     TmaMaps maps;
-    if (!make_maps(&maps, W_gate, W_up, E * I, zp, R, L, bf)) return MUSE_ERR_CUDA;
+    Fp4Args q4{};
+    if (fp4) {
+      const muse_nvfp4_weight* wg = static_cast<const muse_nvfp4_weight*>(W_gate);
+      const muse_nvfp4_weight* wu = static_cast<const muse_nvfp4_weight*>(W_up);
+      std::memset(&maps, 0, sizeof(maps));
+      if (!make_code_map(&maps.a, wg->codes, E * I, L) || !make_code_map(&maps.a2, wu->codes, E * I, L)) return MUSE_ERR_CUDA;
+      for (int i = 0; i < 5; ++i)
+        if (!make_map(&maps.b[i], zp, bf, L, R, 16 << i)) return MUSE_ERR_CUDA;
+      q4 = Fp4Args{static_cast<const uint8_t*>(wg->block_scales), static_cast<const uint8_t*>(wu->block_scales),
+                   wg->matrix_scale, wu->matrix_scale, static_cast<int>(L / 16)};
+    } else if (!make_maps(&maps, W_gate, W_up, E * I, zp, R, L, bf)) {
+      return MUSE_ERR_CUDA;
+    }
     GemmArgs g = base_args(status);
     g.tiles = tiles_gu;
     g.num_tiles_dev = ntiles;
@@ -378,7 +441,9 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
     g.k_blocks = static_cast<int>(L * sizeof(T) / 128);
     g.out = h;
     g.ld_out = I;
-    if (pgu.pair) {
+    if (fp4) {
+      MUSE_CK(launch_gemm_fp4<EPI_SWIGLU>(bn_g, 2, maps, g, q4, nsm, st));
+    } else if (pgu.pair) {
       if (!make_out_map(&maps.out, h, R, I)) return MUSE_ERR_CUDA;
       MUSE_CK((launch_gemm_2sm<T, EPI_SWIGLU, 2>(maps, g, nsm / 2, st)));
     } else {
@@ -388,8 +453,20 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
   }
   // (a7) down projection + sum-of-squares partials
   {
+    const bool fp4 = c.expert_weights == MUSE_EXPERTS_NVFP4;
     TmaMaps maps;
-    if (!make_maps(&maps, W_down, nullptr, E * L, h, R, I, bf)) return MUSE_ERR_CUDA;
+    Fp4Args q4{};
+    if (fp4) {
+      const muse_nvfp4_weight* wd = static_cast<const muse_nvfp4_weight*>(W_down);
+      std::memset(&maps, 0, sizeof(maps));
+      if (!make_code_map(&maps.a, wd->codes, E * L, I) || !make_code_map(&maps.a2, wd->codes, E * L, I)) return MUSE_ERR_CUDA;
+      for (int i = 0; i < 5; ++i)
+        if (!make_map(&maps.b[i], h, bf, I, R, 16 << i)) return MUSE_ERR_CUDA;
+      q4 = Fp4Args{static_cast<const uint8_t*>(wd->block_scales), static_cast<const uint8_t*>(wd->block_scales),
+                   wd->matrix_scale, wd->matrix_scale, static_cast<int>(I / 16)};
+    } else if (!make_maps(&maps, W_down, nullptr, E * L, h, R, I, bf)) {
+      return MUSE_ERR_CUDA;
+    }
     GemmArgs g = base_args(status);
     g.tiles = tiles_dn;
     g.num_tiles_dev = ntiles + 1;
@@ -405,7 +482,9 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
       g.ss_gain_group_stride = c.gamma_shared ? 0 : L;
     }
     if (pdn.pair && !make_out_map(&maps.out, y, R, L)) return MUSE_ERR_CUDA;
-    if (pdn.pair && pdn.mt == 2) {
+    if (fp4) {
+      MUSE_CK(launch_gemm_fp4<EPI_STORE_SS>(bn_g, pdn.mt, maps, g, q4, nsm, st));
+    } else if (pdn.pair && pdn.mt == 2) {
       MUSE_CK((launch_gemm_2sm<T, EPI_STORE_SS, 2>(maps, g, nsm / 2, st)));
     } else if (pdn.pair) {
       MUSE_CK((launch_gemm_2sm<T, EPI_STORE_SS, 1>(maps, g, nsm / 2, st)));
@@ -496,9 +575,17 @@ muse_status muse_latent_moe_forward(const muse_moe_config* cfg, const void* x, c
                                     const void* gamma, const void* W_unpool, void* out, void* stream) {
   muse_status s = validate_sizes(cfg);
   if (s != MUSE_OK) return s;
-  const void* ptrs[] = {x, W_router, W_pool, W_gate, W_up, W_down, gamma, W_unpool, out};
+  const void* ptrs[] = {x, W_router, W_pool, gamma, W_unpool, out};
   for (const void* p : ptrs)
     if (p == nullptr || !aligned16(p)) return MUSE_ERR_INVALID_ARG;
+  const void* experts[] = {W_gate, W_up, W_down};
+  for (const void* p : experts) {
+    if (cfg->expert_weights == MUSE_EXPERTS_NVFP4) {
+      if (!valid_nvfp4(p)) return MUSE_ERR_INVALID_ARG;
+    } else if (p == nullptr || !aligned16(p)) {
+      return MUSE_ERR_INVALID_ARG;
+    }
+  }
   if (cfg->router_bias != nullptr && (reinterpret_cast<uintptr_t>(cfg->router_bias) & 3u)) return MUSE_ERR_INVALID_ARG;
   if (cfg->pre_norm_gain != nullptr && !aligned16(cfg->pre_norm_gain)) return MUSE_ERR_INVALID_ARG;
   if (cfg->pre_norm_gain != nullptr && !(cfg->pre_norm_eps >= 0.0f)) return MUSE_ERR_INVALID_ARG;

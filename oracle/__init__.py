@@ -5,3 +5,4 @@ against. Only tests/, __graft_entry__.smoke() and bench.py's cpu_baseline / refe
 leg may import it. It shares no code with the CUDA library and never imports it.
 """
 from .latent_moe import *  # noqa: F401,F403
+from .nvfp4 import *  # noqa: F401,F403

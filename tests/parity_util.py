@@ -79,6 +79,12 @@ def host(t: torch.Tensor) -> np.ndarray:
 
 
 def expert_source(inp: Dict[str, torch.Tensor]):
+    if "W_gate_codes" in inp:
+        # NVFP4 experts: the oracle runs on exactly the dequantised codes
+        def deq(name, e):
+            return oracle.dequantize_nvfp4(inp[name + "_codes"][e].cpu().numpy(), inp[name + "_scales"][e].cpu().numpy(),
+                                           float(inp[name + "_mscale"][e]))
+        return lambda e: (deq("W_gate", e), deq("W_up", e), deq("W_down", e))
     return lambda e: (inp["W_gate"][e], inp["W_up"][e], inp["W_down"][e])
 
 

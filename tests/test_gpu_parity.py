@@ -189,6 +189,50 @@ def test_pages_released_mode(case):
     assert np.allclose(g.sum(1), 1.0, atol=1e-5)                     # convex combination
 
 
+# ------------------------------------------------------------------------- NVFP4 experts
+NVFP4 = [
+    # name, T, D, L, I, E, k  (bn 32 tiles; bn 256 tiles with 256-feature down tiles; ragged)
+    ("nvfp4_mid", 256, 2048, 1024, 1024, 64, 4),
+    ("nvfp4_wide", 1100, 512, 512, 512, 4, 2),
+    ("nvfp4_ragged", 37, 256, 256, 384, 8, 3),
+]
+NVFP4_REL_L2 = 2e-2   # the block's NVFP4 tolerance against the oracle on the same codes
+
+
+@pytest.mark.parametrize("case", NVFP4, ids=[c[0] for c in NVFP4])
+def test_nvfp4_experts(case):
+    name, T, D, L, I, E, k = case
+    w = W.Workload(name, T=T, D=D, L=L, I=I, E=E, k=k, dtype="bf16", seed=9, experts="nvfp4")
+    inp = W.make_inputs(w, "cuda")
+    run = Run(w, inp)
+    rows = np.arange(T)
+    ref = oracle_block(w, inp, rows)
+    gidx = run.idx.cpu().numpy()
+    alts = check_routing(ref, gidx, run.g.cpu().numpy(), w.k)
+    ref_out = oracle_on_gpu_alternatives(w, inp, rows, ref, gidx, alts)
+    r, _ = assert_close(host(run.out), ref_out, f"{name} out", rel=NVFP4_REL_L2)
+    print(f"{name}: rel-L2 {r:.2e}")
+    if not alts:
+        R = run.layout["rows"]
+        ginv = run.inter("inv", torch.int32, (T * k,)).cpu().numpy()
+        y = host(run.inter("y", torch.bfloat16, (R, L)))[ginv].reshape(T, k, L)
+        assert_close(y, ref["y"], f"{name} expert outputs", rel=NVFP4_REL_L2)
+
+
+@pytest.mark.slow
+def test_full_size_nvfp4_layer_sampled_tokens():
+    w = W.WORKLOADS["nvfp4"]
+    inp = W.make_inputs(w, "cuda")
+    run = Run(w, inp)
+    rows = np.sort(np.random.default_rng(3).choice(w.T, size=10, replace=False))
+    ref = oracle_block(w, inp, rows)
+    gidx = run.idx.cpu().numpy()[rows]
+    alts = check_routing(ref, gidx, run.g.cpu().numpy()[rows], w.k)
+    ref_out = oracle_on_gpu_alternatives(w, inp, rows, ref, gidx, alts)
+    r, _ = assert_close(host(run.out)[rows], ref_out, "nvfp4 layer out", rel=NVFP4_REL_L2)
+    print(f"nvfp4 full layer: rel-L2 {r:.2e}")
+
+
 # ------------------------------------------------------------------------- full size
 @pytest.fixture(scope="module")
 def full_weights():

@@ -336,3 +336,41 @@ def test_parameter_and_flop_accounting():
     # 2 x active parameters, less the two 4096-entry norm gains the FLOP count leaves out
     assert flops == 2 * (a["params_active_per_token"] - 2 * L)
     assert round(flops / 1e6, 1) == a["moe_mflops_per_token_printed"]
+
+
+# ------------------------------------------------------------------ NVFP4 decoding
+def test_e2m1_table():
+    for s in lines("fp4_e2m1.txt"):
+        code, val = s.split()
+        got = oracle.decode_e2m1(int(code))
+        assert got == float(val) and np.signbit(got) == val.startswith("-")
+
+
+def test_e4m3_values_and_every_byte_against_torch():
+    for s in lines("fp8_e4m3.txt"):
+        b, val = s.split()
+        got = float(oracle.decode_e4m3(int(b, 16)))
+        assert (np.isnan(got) and val == "nan") or got == float(val)
+    import torch
+    allb = torch.arange(256, dtype=torch.uint8)
+    ref = allb.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = oracle.decode_e4m3(np.arange(256))
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    assert np.array_equal(got[~np.isnan(got)], ref[~np.isnan(ref)])
+
+
+def test_nibble_order_and_dequantisation():
+    codes = np.array([[0x21, 0xF7]], dtype=np.uint8)          # values 1,2 | 7,15
+    assert oracle.unpack_nibbles(codes).tolist() == [[1, 2, 7, 15]]
+    # one row of 16 weights: codes 0..15, block scale 2.0 (0x40), matrix scale 0.25
+    packed = np.array([[lo | (hi << 4) for lo, hi in zip(range(0, 16, 2), range(1, 16, 2))]], dtype=np.uint8)
+    w = oracle.dequantize_nvfp4(packed, np.array([[0x40]], dtype=np.uint8), 0.25)
+    table = np.array([float(s.split()[1]) for s in lines("fp4_e2m1.txt")])
+    np.testing.assert_array_equal(w[0], table * 2.0 * 0.25)
+
+
+def test_nvfp4_bytes_per_weight():
+    # deep dive §7.3: 0.5625 bytes per weight (4 bits + one FP8 scale per 16 weights)
+    assert oracle.NVFP4_BYTES_PER_WEIGHT == 0.5625
+    out, k = 64, 256
+    assert (out * k // 2 + out * k // 16) / (out * k) == 0.5625

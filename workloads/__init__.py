@@ -45,6 +45,7 @@ class Workload:
     eps: float = 1e-6
     routing: str = "uniform"   # "uniform" (no bias) or "zipf" (selection bias, s=1.2)
     seed: int = 0
+    experts: str = "bf16"      # expert weight storage: "bf16" (the dtype) or "nvfp4"
 
     def with_tokens(self, T: int) -> "Workload":
         return dataclasses.replace(self, T=T)
@@ -60,6 +61,8 @@ WORKLOADS: Dict[str, Workload] = {
     # full-width layer with 16 experts and 256 tokens per expert: the prefill tile
     # shapes on ~2 GB of device memory (profiling captures)
     "prefill_e16": Workload("prefill_e16", T=2048, D=8192, L=4096, I=4096, E=16, k=2, dtype="bf16"),
+    # full layer with NVFP4 expert weights (router, pooler, unpooler and activations bf16)
+    "nvfp4": Workload("nvfp4", T=4096, D=8192, L=4096, I=4096, E=256, k=8, dtype="bf16", experts="nvfp4"),
 }
 
 # tensor ids of the generator (fixed, part of the workload definition)
@@ -176,11 +179,70 @@ def expert_slab(w: Workload, name: str, e: int, device="cpu",
 
 
 def make_inputs(w: Workload, device="cpu", names=None) -> Dict[str, torch.Tensor]:
+    """The workload's tensors. For NVFP4 experts, W_gate / W_up / W_down are replaced by
+    <name>_codes, <name>_scales and <name>_mscale (see quantize_nvfp4), each expert
+    quantised from the same bf16 weights a bf16 workload would use."""
     names = names or list(shapes(w).keys())
-    out = {n: make_tensor(w, n, device) for n in names}
+    out = {}
+    for n in names:
+        if w.experts == "nvfp4" and n in ("W_gate", "W_up", "W_down"):
+            out.update(make_nvfp4_experts(w, n, device))
+        else:
+            out[n] = make_tensor(w, n, device)
     if w.routing == "zipf":
         out["router_bias"] = zipf_router_bias(w).to(device)
     return out
+
+
+# ----------------------------------------------------------------------------------------
+# NVFP4 expert weights: 4-bit E2M1 values, one E4M3 scale per 16 weights of a row, one
+# float32 scale per expert matrix (the format the deep dive's §7.4 describes). The
+# quantiser is part of input generation; any quantiser would do for parity, since both
+# sides read the same codes.
+# ----------------------------------------------------------------------------------------
+_E2M1_MIDPOINTS = (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0)
+_E2M1_TIES_UP = (0.75, 1.75, 3.5)   # midpoints whose upper neighbour has the even mantissa
+
+
+def _e2m1_codes(q: torch.Tensor) -> torch.Tensor:
+    """Round to nearest E2M1 value (ties to even), saturating at +-6; returns codes 0..15."""
+    a = q.abs().clamp(max=6.0)
+    mag = torch.zeros_like(a, dtype=torch.uint8)
+    for mid in _E2M1_MIDPOINTS:
+        mag += (a > mid).to(torch.uint8)
+    for mid in _E2M1_TIES_UP:
+        mag += (a == mid).to(torch.uint8)
+    return mag | (torch.signbit(q).to(torch.uint8) << 3)
+
+
+def quantize_nvfp4(wt: torch.Tensor):
+    """[out, in] weights -> (codes uint8 [out, in/2] low nibble first, block scales uint8
+    E4M3 [out, in/16], matrix scale float). Matrix scale amax/(6*448); block scale
+    E4M3(amax_block / (6 * matrix scale)); code E2M1(w / (block * matrix scale))."""
+    x = wt.to(torch.float32)
+    out_dim, in_dim = x.shape
+    amax = float(x.abs().max())
+    ms = amax / (6.0 * 448.0) if amax > 0 else 1.0
+    blocks = x.view(out_dim, in_dim // 16, 16)
+    bscale = (blocks.abs().amax(-1) / (6.0 * ms)).clamp(max=448.0).to(torch.float8_e4m3fn)
+    denom = bscale.to(torch.float32) * ms
+    q = torch.where(denom[..., None] > 0, blocks / denom[..., None].clamp(min=1e-30), torch.zeros_like(blocks))
+    codes = _e2m1_codes(q).view(out_dim, in_dim // 2, 2)
+    packed = codes[..., 0] | (codes[..., 1] << 4)
+    return packed.contiguous(), bscale.view(torch.uint8).contiguous(), ms
+
+
+def make_nvfp4_experts(w: Workload, name: str, device="cpu") -> Dict[str, torch.Tensor]:
+    shp = shapes(w)[name]
+    E, rows, cols = shp
+    codes = torch.empty((E, rows, cols // 2), dtype=torch.uint8, device=device)
+    scales = torch.empty((E, rows, cols // 16), dtype=torch.uint8, device=device)
+    mscale = torch.empty(E, dtype=torch.float32, device=device)
+    for e in range(E):
+        c, s, m = quantize_nvfp4(expert_slab(w, name, e, device))
+        codes[e], scales[e], mscale[e] = c, s, m
+    return {f"{name}_codes": codes, f"{name}_scales": scales, f"{name}_mscale": mscale}
+
 
 
 # ----------------------------------------------------------------------------------------
