@@ -435,7 +435,7 @@ def main():
                 inp_q["x"] = rank_tokens(wq, rank, dev)
                 side["nvfp4"] = run_ours(wq, inp_q, args.steps, args.warmup, rank, world, peaks, peak_kind,
                                          False, e2e_steps=0)
-                wqd = dataclasses.replace(wq, name="nvfp4_decode", T=64)
+                wqd = W.WORKLOADS["nvfp4_decode"]
                 inp_qd = dict(inp_q, x=rank_tokens(wqd, rank, dev))
                 side["nvfp4_decode"] = run_ours(wqd, inp_qd, max(args.steps, 50), args.warmup, rank, world, peaks,
                                                 peak_kind, False, e2e_steps=0)

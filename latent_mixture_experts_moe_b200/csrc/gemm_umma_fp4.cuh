@@ -2,17 +2,22 @@
 //
 //   C[token, f] = mscale[e] * sum_k (e2m1(code[f, k]) * e4m3(scale[f, k / 16])) * X[token, k]
 //
-// Weights stay 4-bit in HBM (0.5 B per weight + one E4M3 byte per 16): TMA brings the packed
-// codes of a 128-row x 64-K tile (4 KB) into shared memory, four converter warps expand it
-// into the bf16 128-byte-swizzled tile the UMMA reads (code x block scale is exact in bf16:
-// at most 2 + 4 significant bits), and the per-matrix FP32 scale multiplies the FP32
-// accumulator in the epilogue. Tokens (bf16) are the B operand as in gemm_umma.cuh.
+// Weights stay 4-bit in HBM (0.5 B per weight + one E4M3 byte per 16 weights). TMA brings the
+// packed codes of a 128-row x 64-K tile (4 KB) and the token tile into shared memory; eight
+// converter warps expand each code row into 64 bf16 values (code x block scale is exact in
+// bf16: at most 2 + 4 significant bits) and write them straight into TENSOR MEMORY, where the
+// UMMA takes its A operand (kind::f16 with A in TMEM: 128 lanes x 32 columns per 64-K tile,
+// two K elements per column). The dequantised weights never touch shared memory, which
+// leaves its bandwidth to the TMA copies and the token operand. The per-matrix FP32 scale
+// multiplies the FP32 accumulator in the epilogue.
 //
-// Roles (320 threads, one CTA per SM): warp 0 TMA producer (codes + token tile), warp 1 TMEM
-// owner + UMMA issuer, warps 2..5 epilogue, warps 6..9 converters (thread i of them expands
-// weight row i of each 128-row tile, its block scales read from global memory one k-block
-// ahead). Barriers per stage: full (TMA bytes), conv (4 converter warps), empty (UMMA commit).
-// Every wait is bounded (ptx.cuh).
+// Roles (448 threads, one CTA per SM): warp 0 TMA producer (codes + token tile, a deep ring:
+// 4-bit stages are small), warp 1 TMEM owner + UMMA issuer, warps 2..5 epilogue, warps 6..13
+// converters (warp w expands weight rows 32*(w%4) .. +31 -- the TMEM lanes it may write -- of
+// tile (w-6)/4; block scales read from global memory 8 k-blocks at a time). TMEM columns:
+// accumulators from 0, converted weight slots (2 or 3 of 32 * MT columns) after them.
+// Barriers: per TMA stage full (bytes) / empty (UMMA commit); per converted slot conv
+// (converter warps) / cfree (UMMA commit). Every wait is bounded (ptx.cuh).
 #pragma once
 
 #include "gemm_umma.cuh"
@@ -29,35 +34,44 @@ struct Fp4Args {
 
 template <int BN, int EPI, int MT>
 struct Fp4Shape {
-  static constexpr uint32_t kABytes = 128u * 128u;   // bf16 tile written by the converters
-  static constexpr uint32_t kCodeBytes = 128u * 32u; // packed codes of 128 rows x 64 K
+  static_assert(BN == 32 || BN == 128 || BN == 192, "token tiles of 32, 128 or 192 rows");
+  static constexpr uint32_t kCodeBytes = 128u * 32u;  // packed codes of 128 rows x 64 K
   static constexpr uint32_t kBBytes = static_cast<uint32_t>(BN) * 128u;
-  static constexpr uint32_t kStageBytes = kABytes * MT + kBBytes + kCodeBytes * MT;
-  static constexpr int kSmemBudget = 227 * 1024 - 1024 - 1024;   // alignment, LUT + barriers
+  static constexpr uint32_t kStageBytes = kBBytes + kCodeBytes * MT;   // TMA ring stage
+  static constexpr int kSmemBudget = 227 * 1024 - 1024 - 1024;         // alignment, LUT + barriers
   static constexpr int kStagesFit = kSmemBudget / static_cast<int>(kStageBytes);
-  static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
+  static constexpr int kStages = kStagesFit > 16 ? 16 : kStagesFit;
   static constexpr int kAccStages = MT == 2 ? 1 : 2;
   static constexpr uint32_t kAccCols = static_cast<uint32_t>(BN) * MT;
-  static constexpr uint32_t kColsNeeded = kAccCols * kAccStages;
-  static constexpr uint32_t kTmemCols = kColsNeeded <= 32 ? 32 : kColsNeeded <= 64 ? 64
-                                        : kColsNeeded <= 128 ? 128 : kColsNeeded <= 256 ? 256 : 512;
+  static constexpr uint32_t kTmemCols = 512;
+  // converted weight tiles in the TMEM columns the accumulators leave: 3 slots (measured
+  // best for decode-sized tiles; deeper did worse), or as many as fit
+  static constexpr uint32_t kConvCols = 32u * MT;         // TMEM columns per slot
+  static constexpr uint32_t kConvCol0 = kAccCols * kAccStages;
+  static constexpr int kConvFit = static_cast<int>((kTmemCols - kConvCol0) / kConvCols);
+  static constexpr int kConvSlots = kConvFit > 3 ? 3 : kConvFit;
   static constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes + 1024;
+  static_assert(kConvSlots >= 2, "no TMEM room for converted weight tiles");
   static_assert(kStages >= 2, "tile too large for the shared-memory ring");
+  static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte alignment of swizzled tiles");
   static_assert(EPI != EPI_SWIGLU || MT == 2, "SwiGLU needs the gate and up accumulators");
 };
 
-constexpr int kFp4Threads = 320;
+// warps 0 producer, 1 UMMA issuer, 2..5 epilogue, 6..13 converters (with MT = 1, 10..13 idle)
+constexpr int kFp4Threads = 448;
 
 // 4 codes (the low 16 bits of w: nibbles k0..k3) -> 4 bf16 in two words, low element
-// first. Magnitude bytes come from two 8-entry byte tables (byte-permute lookups), the
-// sign goes to bit 15 of each half.
+// first, with byte-permute lookups: the magnitude (nibble bits 0-2) selects the high and low
+// byte of |value| from two 8-entry tables, the sign (nibble bit 3) selects 0x00 or 0x80 to
+// OR into the high byte.
 __device__ __forceinline__ void e2m1x4_to_bf16(uint32_t w, uint32_t& o0, uint32_t& o1) {
   const uint32_t sel = w & 0x7777u;
   // |value| as bf16: high bytes {00,3F,3F,3F,40,40,40,40}, low {00,00,80,C0,00,40,80,C0}
-  const uint32_t hi = __byte_perm(0x3F3F3F00u, 0x40404040u, sel);
+  const uint32_t sgn = __byte_perm(0u, 0x80808080u, (w >> 1) & 0x4444u);
+  const uint32_t hi = __byte_perm(0x3F3F3F00u, 0x40404040u, sel) | sgn;
   const uint32_t lo = __byte_perm(0xC0800000u, 0xC0804000u, sel);
-  o0 = __byte_perm(lo, hi, 0x5140u) | ((w << 12) & 0x8000u) | ((w << 24) & 0x80000000u);
-  o1 = __byte_perm(lo, hi, 0x7362u) | ((w << 4) & 0x8000u) | ((w << 16) & 0x80000000u);
+  o0 = __byte_perm(lo, hi, 0x5140u);
+  o1 = __byte_perm(lo, hi, 0x7362u);
 }
 
 __device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
@@ -67,15 +81,27 @@ __device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
   return *reinterpret_cast<uint32_t*>(&r);
 }
 
-// Expands one 64-weight row segment (32 code bytes at `codes`, 4 E4M3 scales in `s4`) into
-// the 128-byte row `r` of a 128-byte-swizzled bf16 tile at `tile` (16-byte chunk c of row r
-// sits at chunk position c ^ (r & 7)).
-__device__ __forceinline__ void expand_row(const uint8_t* codes, uint32_t s4, const uint16_t* lut, uint8_t* tile,
-                                           int r) {
+// E4M3 byte -> bf16 bits (exact: at most 4 significant bits, 2^-9 .. 448), S.1111.111 -> NaN
+__device__ __forceinline__ uint32_t e4m3_to_bf16_bits(uint32_t b) {
+  const uint32_t s = (b >> 7) & 1u, e = (b >> 3) & 15u, m = b & 7u;
+  float v;
+  if (e == 15u && m == 7u) {
+    v = __int_as_float(0x7FC00000);
+  } else if (e == 0u) {
+    v = static_cast<float>(m) * 0.001953125f;  // m * 2^-9
+  } else {
+    v = __int_as_float(static_cast<int>(((e + 120u) << 23) | (m << 20)));
+  }
+  return __bfloat16_as_ushort(__float2bfloat16_rn(s ? -v : v));
+}
+
+// One 64-weight row segment (32 code bytes at `codes`, 4 E4M3 scales in `s4`) -> 32 words of
+// bf16 pairs (K elements 2j, 2j+1 in word j), the TMEM column order of the A operand.
+__device__ __forceinline__ void expand_row(const uint8_t* codes, uint32_t s4, const uint16_t* lut,
+                                           uint32_t (&out)[32]) {
   const uint4 c0 = *reinterpret_cast<const uint4*>(codes);
   const uint4 c1 = *reinterpret_cast<const uint4*>(codes + 16);
   const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-  uint8_t* row = tile + r * 128;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const uint32_t sb = lut[(s4 >> (8 * (i >> 1))) & 0xFFu];   // one scale per 16 weights
@@ -83,12 +109,10 @@ __device__ __forceinline__ void expand_row(const uint8_t* codes, uint32_t s4, co
     uint32_t a0, a1, b0, b1;
     e2m1x4_to_bf16(words[i], a0, a1);
     e2m1x4_to_bf16(words[i] >> 16, b0, b1);
-    uint4 v;
-    v.x = bf16x2_mul(a0, s2);
-    v.y = bf16x2_mul(a1, s2);
-    v.z = bf16x2_mul(b0, s2);
-    v.w = bf16x2_mul(b1, s2);
-    *reinterpret_cast<uint4*>(row + ((i ^ (r & 7)) << 4)) = v;
+    out[4 * i + 0] = bf16x2_mul(a0, s2);
+    out[4 * i + 1] = bf16x2_mul(a1, s2);
+    out[4 * i + 2] = bf16x2_mul(b0, s2);
+    out[4 * i + 3] = bf16x2_mul(b1, s2);
   }
 }
 
@@ -102,43 +126,36 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint16_t* lut = reinterpret_cast<uint16_t*>(smem + kStages * S::kStageBytes);       // 256 x bf16
+  constexpr int kConv = S::kConvSlots;
+  uint16_t* lut = reinterpret_cast<uint16_t*>(smem + kStages * S::kStageBytes);  // 256 x bf16
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * S::kStageBytes + 512);
-  // bars: full[kStages], conv[kStages], empty[kStages], acc_full[2], acc_empty[2]
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 3 * kStages + 4);
+  // bars: full[kStages], empty[kStages], conv[kConv], cfree[kConv], acc_full[2], acc_empty[2]
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 2 * kConv + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t bar0 = smem_u32(bars);
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
-  auto conv_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
-  auto empty_bar = [&](int s) { return bar0 + 8u * (2 * kStages + s); };
-  auto accf_bar = [&](int a) { return bar0 + 8u * (3 * kStages + a); };
-  auto acce_bar = [&](int a) { return bar0 + 8u * (3 * kStages + 2 + a); };
-  auto a_tile = [&](int s, int m) { return smem + s * S::kStageBytes + m * S::kABytes; };
-  auto b_tile = [&](int s) { return smem + s * S::kStageBytes + MT * S::kABytes; };
-  auto code_tile = [&](int s, int m) { return smem + s * S::kStageBytes + MT * S::kABytes + S::kBBytes + m * S::kCodeBytes; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
+  auto conv_bar = [&](int c) { return bar0 + 8u * (2 * kStages + c); };
+  auto cfree_bar = [&](int c) { return bar0 + 8u * (2 * kStages + kConv + c); };
+  auto accf_bar = [&](int a) { return bar0 + 8u * (2 * kStages + 2 * kConv + a); };
+  auto acce_bar = [&](int a) { return bar0 + 8u * (2 * kStages + 2 * kConv + 2 + a); };
+  auto b_tile = [&](int s) { return smem + s * S::kStageBytes; };
+  auto code_tile = [&](int s, int m) { return smem + s * S::kStageBytes + S::kBBytes + m * S::kCodeBytes; };
+  // TMEM column of converted weight tile m of slot c
+  auto conv_col = [&](int c, int m) { return S::kConvCol0 + static_cast<uint32_t>(c) * S::kConvCols + 32u * m; };
 
-  // E4M3 -> bf16 (exact: at most 4 significant bits, 2^-9 .. 448); S.1111.111 -> NaN
-  for (int i = threadIdx.x; i < 256; i += blockDim.x) {
-    const uint32_t s = (i >> 7) & 1, e = (i >> 3) & 15, m = i & 7;
-    float v;
-    if (e == 15 && m == 7) {
-      v = __int_as_float(0x7FC00000);
-    } else if (e == 0) {
-      v = static_cast<float>(m) * 0.001953125f;  // m * 2^-9
-    } else {
-      v = __int_as_float(static_cast<int>(((e + 120u) << 23) | (m << 20)));
-    }
-    if (s) v = -v;
-    lut[i] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
-  }
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) lut[i] = static_cast<uint16_t>(e4m3_to_bf16_bits(i));
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(full_bar(s), 1);
-      mbar_init(conv_bar(s), 4);
       mbar_init(empty_bar(s), 1);
+    }
+    for (int c = 0; c < kConv; ++c) {
+      mbar_init(conv_bar(c), 4 * MT);
+      mbar_init(cfree_bar(c), 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(accf_bar(a), 1);
@@ -186,7 +203,7 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
           const int kc = kb * 64;
           int j16 = 0;
 #pragma unroll
-          for (int i = 4; i >= 0; --i) {
+          for (int i = 3; i >= 0; --i) {
             if ((16 << i) <= BN && (nb16 >> i) & 1) {
               tma_load_2d(sB + 2048u * j16, &maps.b[i], full_bar(stage), kc, row0 + 16 * j16);
               j16 += 1 << i;
@@ -209,8 +226,8 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------------- UMMA issuer
     if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
+      int stage = 0, cs = 0;
+      uint32_t phase = 0, cphase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
@@ -228,25 +245,29 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
         const uint32_t d = tmem_base + static_cast<uint32_t>(acc) * S::kAccCols;
         for (int kb = 0; kb < p.k_blocks; ++kb) {
           if (!mbar_wait(full_bar(stage), phase, abort_flag, p.status, 0xB00u + stage) ||
-              !mbar_wait(conv_bar(stage), phase, abort_flag, p.status, 0xC00u + stage)) {
+              !mbar_wait(conv_bar(cs), cphase, abort_flag, p.status, 0xC00u + cs)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sA = smem_u32(a_tile(stage, 0));
           const uint32_t sB = smem_u32(b_tile(stage));
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
             const uint64_t db = sdesc_k_sw128(sB + 32u * kk);
-            umma<false>(d, sdesc_k_sw128(sA + 32u * kk), db, idesc, accum);
-            if (kDual) umma<false>(d + BN, sdesc_k_sw128(sA + S::kABytes + 32u * kk), db, idesc, accum);
+            umma_ts_bf16(d, tmem_base + conv_col(cs, 0) + 8u * kk, db, idesc, accum);
+            if (kDual) umma_ts_bf16(d + BN, tmem_base + conv_col(cs, 1) + 8u * kk, db, idesc, accum);
           }
           issued_any = true;
           tc_commit(empty_bar(stage));
+          tc_commit(cfree_bar(cs));
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1u;
+          }
+          if (++cs == kConv) {
+            cs = 0;
+            cphase ^= 1u;
           }
         }
         if (!ok) break;
@@ -266,44 +287,71 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
     __syncwarp();
   } else if (warp >= 6) {
     // ---------------------------------------------------------------- converters
-    const int r = threadIdx.x - 192;  // weight row of the tile this thread expands
-    int stage = 0;
-    uint32_t phase = 0;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
-      int g, m0, row0, n;
-      gemm_tile(p, t, BN, g, m0, row0, n);
-      const int a_row = g * p.rows_per_group + m0;
-      const int a2_row = EPI == EPI_SWIGLU ? a_row : a_row + 128;
-      const uint8_t* sc_a = q4.scales_a + static_cast<int64_t>(a_row + r) * q4.scale_ld;
-      const uint8_t* sc_a2 = q4.scales_a2 + static_cast<int64_t>(a2_row + r) * q4.scale_ld;
-      uint32_t s_a = *reinterpret_cast<const uint32_t*>(sc_a);
-      uint32_t s_a2 = kDual ? *reinterpret_cast<const uint32_t*>(sc_a2) : 0u;
+    const int mat = (warp - 6) >> 2;  // which 128-row weight tile: 0 = maps.a, 1 = maps.a2
+    const int quad = warp & 3;        // TMEM lane quadrant this warp may write
+    const int r = quad * 32 + lane;   // weight row (= TMEM lane) this thread expands
+    if (mat < MT) {
+      int stage = 0, cs = 0;
+      uint32_t phase = 0, cphase = 0;
       bool ok = true;
-      for (int kb = 0; kb < p.k_blocks; ++kb) {
-        // next k-block's 4 scales per row, loaded while this one converts
-        uint32_t n_a = 0, n_a2 = 0;
-        if (kb + 1 < p.k_blocks) {
-          n_a = *reinterpret_cast<const uint32_t*>(sc_a + 4 * (kb + 1));
-          if (kDual) n_a2 = *reinterpret_cast<const uint32_t*>(sc_a2 + 4 * (kb + 1));
-        }
-        const bool ready = mbar_wait(full_bar(stage), phase, abort_flag, p.status, 0xD00u + stage);
-        if (!__all_sync(0xffffffffu, ready)) {
-          ok = false;
-          break;
-        }
-        expand_row(code_tile(stage, 0) + r * 32, s_a, lut, a_tile(stage, 0), r);
-        if (kDual) expand_row(code_tile(stage, 1) + r * 32, s_a2, lut, a_tile(stage, 1), r);
-        fence_proxy_async_smem();  // generic-proxy writes -> the tensor core's reads
-        __syncwarp();
-        if (lane == 0) mbar_arrive(conv_bar(stage));
-        s_a = n_a;
-        s_a2 = n_a2;
-        if (++stage == kStages) {
-          stage = 0;
-          phase ^= 1u;
+      const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+      for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+        int g, m0, row0, n;
+        gemm_tile(p, t, BN, g, m0, row0, n);
+        const int a_row = g * p.rows_per_group + m0;
+        const int row = (mat == 0 ? a_row : (EPI == EPI_SWIGLU ? a_row : a_row + 128)) + r;
+        const uint8_t* sc = (mat == 0 ? q4.scales_a : q4.scales_a2) + static_cast<int64_t>(row) * q4.scale_ld;
+        // the row's block scales for 8 k-blocks are one 32-byte sector: two 16-byte loads
+        // (when rows are 16-byte aligned), the next sector loaded while this one is used
+        auto load8 = [&](int kb0, uint32_t (&dst)[8]) {
+          if (kb0 + 8 <= p.k_blocks && (q4.scale_ld & 15) == 0) {  // 16-byte aligned rows
+            const uint4 u0 = *reinterpret_cast<const uint4*>(sc + 4 * kb0);
+            const uint4 u1 = *reinterpret_cast<const uint4*>(sc + 4 * kb0 + 16);
+            dst[0] = u0.x; dst[1] = u0.y; dst[2] = u0.z; dst[3] = u0.w;
+            dst[4] = u1.x; dst[5] = u1.y; dst[6] = u1.z; dst[7] = u1.w;
+          } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              dst[j] = kb0 + j < p.k_blocks ? *reinterpret_cast<const uint32_t*>(sc + 4 * (kb0 + j)) : 0u;
+          }
+        };
+        uint32_t cur[8], nxt[8];
+        load8(0, cur);
+        for (int kb0 = 0; ok && kb0 < p.k_blocks; kb0 += 8) {
+          if (kb0 + 8 < p.k_blocks) load8(kb0 + 8, nxt);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int kb = kb0 + j;
+            if (kb < p.k_blocks) {
+              const bool ready = mbar_wait(full_bar(stage), phase, abort_flag, p.status, 0xD00u + stage) &&
+                                 mbar_wait(cfree_bar(cs), cphase ^ 1u, abort_flag, p.status, 0xF00u + cs);
+              if (!__all_sync(0xffffffffu, ready)) {
+                ok = false;
+              } else {
+                tc_fence_after();
+                uint32_t v[32];
+                expand_row(code_tile(stage, mat) + r * 32, cur[j], lut, v);
+                tmem_st32(lane_base + conv_col(cs, mat), v);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(conv_bar(cs));
+                if (++stage == kStages) {
+                  stage = 0;
+                  phase ^= 1u;
+                }
+                if (++cs == kConv) {
+                  cs = 0;
+                  cphase ^= 1u;
+                }
+              }
+            }
+            if (!ok) break;
+          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j) cur[j] = nxt[j];
         }
       }
-      if (!ok) break;
     }
   } else {
     // ---------------------------------------------------------------- epilogue

@@ -32,7 +32,10 @@ int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // ---------------------------------------------------------------------- tile sizing
 // tokens per grouped-GEMM tile: small tiles when experts see few tokens (decode)
-int grouped_bn(const muse_moe_config& c) { return (c.T * c.top_k) <= 32 * c.E ? 32 : 256; }
+int grouped_bn(const muse_moe_config& c) {
+  if ((c.T * c.top_k) <= 32 * c.E) return 32;
+  return c.expert_weights == MUSE_EXPERTS_NVFP4 ? 192 : 256;  // NVFP4: accumulators leave TMEM room for weights
+}
 int dense_bn(const muse_moe_config& c) { return c.T <= 32 ? 32 : 256; }
 
 struct Layout {
@@ -218,12 +221,12 @@ cudaError_t launch_gemm_fp4(int bn, int mt, const TmaMaps& maps, const GemmArgs&
                             cudaStream_t st) {
   if constexpr (EPI == EPI_SWIGLU) {
     return bn == 32 ? launch_gemm_fp4_t<32, EPI, 2>(maps, args, q4, grid, st)
-                    : launch_gemm_fp4_t<256, EPI, 2>(maps, args, q4, grid, st);
+                    : launch_gemm_fp4_t<192, EPI, 2>(maps, args, q4, grid, st);
   } else {
     if (bn == 32) return mt == 2 ? launch_gemm_fp4_t<32, EPI, 2>(maps, args, q4, grid, st)
                                  : launch_gemm_fp4_t<32, EPI, 1>(maps, args, q4, grid, st);
-    return mt == 2 ? launch_gemm_fp4_t<256, EPI, 2>(maps, args, q4, grid, st)
-                   : launch_gemm_fp4_t<256, EPI, 1>(maps, args, q4, grid, st);
+    return mt == 2 ? launch_gemm_fp4_t<192, EPI, 2>(maps, args, q4, grid, st)
+                   : launch_gemm_fp4_t<192, EPI, 1>(maps, args, q4, grid, st);
   }
 }
 
@@ -304,8 +307,7 @@ GemmPlan plan_gate_up(const muse_moe_config& c, int bn_g) {
   return {false, 2, 128};
 }
 GemmPlan plan_down(const muse_moe_config& c, int bn_g) {
-  if (c.expert_weights == MUSE_EXPERTS_NVFP4) return (bn_g == 256 && c.L % 256 == 0) ? GemmPlan{false, 2, 256}
-                                                                                      : GemmPlan{false, 1, 128};
+  if (c.expert_weights == MUSE_EXPERTS_NVFP4) return c.L % 256 == 0 ? GemmPlan{false, 2, 256} : GemmPlan{false, 1, 128};
   if (c.dtype == MUSE_BF16 && bn_g == 256 && c.L % 512 == 0) return {true, 2, 512};
   if (c.dtype == MUSE_BF16 && bn_g == 256 && c.L % 256 == 0) return {true, 1, 256};
   if (bn_g == 256 && c.L % 256 == 0) return {false, 2, 256};

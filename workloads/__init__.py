@@ -63,6 +63,11 @@ WORKLOADS: Dict[str, Workload] = {
     "prefill_e16": Workload("prefill_e16", T=2048, D=8192, L=4096, I=4096, E=16, k=2, dtype="bf16"),
     # full layer with NVFP4 expert weights (router, pooler, unpooler and activations bf16)
     "nvfp4": Workload("nvfp4", T=4096, D=8192, L=4096, I=4096, E=256, k=8, dtype="bf16", experts="nvfp4"),
+    "nvfp4_decode": Workload("nvfp4_decode", T=64, D=8192, L=4096, I=4096, E=256, k=8, dtype="bf16",
+                             experts="nvfp4"),
+    # decode-like NVFP4 case on ~1 GB of weights (2-3 tokens per expert; profiling captures)
+    "nvfp4_decode_e32": Workload("nvfp4_decode_e32", T=32, D=8192, L=4096, I=4096, E=32, k=2, dtype="bf16",
+                                 experts="nvfp4"),
 }
 
 # tensor ids of the generator (fixed, part of the workload definition)
