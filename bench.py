@@ -284,7 +284,8 @@ def measured_traffic(kernel: str, w: W.Workload):
 def kernel_source_sha():
     import hashlib
     h = hashlib.sha256()
-    for f in ("gemm_umma.cuh", "ptx.cuh", "route_kernels.cuh", "muse_moe.cu"):
+    from latent_mixture_experts_moe_b200.build import KERNEL_SOURCES
+    for f in KERNEL_SOURCES:
         h.update(open(os.path.join(ROOT, "latent_mixture_experts_moe_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 

@@ -61,6 +61,8 @@ struct GemmArgs {
   const void* ss_gain;       // EPI_STORE_SS: optional gain offsets; squares y*(1+gain)
   int64_t ss_gain_group_stride;  // elements between groups' gains (0 = shared)
   uint32_t* status;          // workspace status word
+  int* tile_counter;         // CTA-pair kernel: tiles are claimed from this counter (zero
+                             // before the launch); nullptr: static round robin over pairs
 };
 
 template <typename TIn>

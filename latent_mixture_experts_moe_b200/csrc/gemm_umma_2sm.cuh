@@ -17,6 +17,14 @@
 //     remote ones through the cluster window);
 //   * a cluster barrier after initialisation and before TMEM is freed keeps each CTA alive
 //     while its partner may still touch its barriers, shared memory or TMEM.
+// Tile scheduling: with a tile counter the leader's producer claims the pair's next tile
+// from it (atomicAdd) when it is about to load it, and hands the index to every role of
+// both CTAs through a 4-deep ring in shared memory (the partner's copy is written through
+// the cluster window; full / empty mbarriers per slot). Pairs that become free one after
+// the other take consecutive tiles, and the tile list orders the token chunks of one
+// expert's feature tile side by side, so the pairs that share a weight tile stream it at
+// the same time and DRAM delivers it once (a static round robin lets them drift apart by
+// more than L2 can bridge). Without a counter the pairs take tiles round robin.
 // Every wait is bounded as in gemm_umma.cuh.
 #pragma once
 
@@ -39,13 +47,18 @@ struct Gemm2Shape {
   // features of bf16
   static constexpr uint32_t kOutBufBytes = 32u * 128u * 2u;
   static constexpr uint32_t kOutBytes = 2u * 2u * kOutBufBytes;
-  static constexpr int kSmemBudget = 227 * 1024 - 1024 - 256 - static_cast<int>(kOutBytes);
+  static constexpr int kSmemBudget = 227 * 1024 - 1024 - 512 - static_cast<int>(kOutBytes);
   static constexpr int kStagesFit = kSmemBudget / static_cast<int>(kStageBytes);
   static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
   static constexpr int kAccStages = kDual ? 1 : 2;
   static constexpr uint32_t kAccCols = 256u * MT;
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes + kOutBytes + 256;
+  static constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes + kOutBytes + 512;
+  // tile-index ring (dynamic scheduling): slots, and the readers of each slot -- the
+  // leader's UMMA thread and 8 epilogue warps, the partner's producer and 8 epilogue warps
+  static constexpr int kSched = 4;
+  static constexpr int kSchedReaders = 1 + 8 + 1 + 8;
+  static_assert(8 * (2 * kStages + 4 + 2 * kSched) + 8 + 4 * kSched <= 512, "barrier area");
   // output features covered by one pair tile
   static constexpr int kFeatStep = (EPI == EPI_SWIGLU) ? 256 : 256 * MT;
   static_assert(kAccCols * kAccStages <= kTmemCols, "accumulators exceed TMEM");
@@ -68,8 +81,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   uint8_t* out_stage = smem + kStages * S::kStageBytes;  // 1024-aligned
   uint64_t* bars = reinterpret_cast<uint64_t*>(out_stage + S::kOutBytes);
   constexpr bool kTmaStore = std::is_same<TOut, __nv_bfloat16>::value;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 4);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 4 + 2 * S::kSched);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  volatile int* sched_ring = reinterpret_cast<volatile int*>(tmem_holder + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -82,6 +96,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
   auto accf_bar = [&](int a) { return bar0 + 8u * (2 * kStages + a); };
   auto acce_bar = [&](int a) { return bar0 + 8u * (2 * kStages + 2 + a); };
+  auto sfull_bar = [&](int s) { return bar0 + 8u * (2 * kStages + 4 + s); };
+  auto sempty_bar = [&](int s) { return bar0 + 8u * (2 * kStages + 4 + S::kSched + s); };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -91,6 +107,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     for (int a = 0; a < 2; ++a) {
       mbar_init(accf_bar(a), 1);
       mbar_init(acce_bar(a), 16);  // 8 epilogue warps in each CTA of the pair
+    }
+    for (int s = 0; s < S::kSched; ++s) {
+      mbar_init(sfull_bar(s), 1);
+      mbar_init(sempty_bar(s), S::kSchedReaders);  // used on the leader
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -109,6 +129,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const int num_tiles = (p.tiles != nullptr) ? *p.num_tiles_dev : p.num_tiles;
+  const bool dyn = (p.tile_counter != nullptr);
+
+  // The pair's i-th tile: -1 past the end, -2 when a wait gave up. The leader's producer
+  // claims and publishes it; every other role receives it and then frees the slot.
+  auto claim_tile = [&](int i) -> int {
+    const int t = dyn ? atomicAdd(p.tile_counter, 1) : pair + i * npairs;
+    return t < num_tiles ? t : -1;
+  };
+  auto publish_tile = [&](int i, int t) -> bool {
+    if (!dyn) return true;
+    const int s = i % S::kSched;
+    const uint32_t ph = static_cast<uint32_t>(i / S::kSched) & 1u;
+    if (!mbar_wait<true>(sempty_bar(s), ph ^ 1u, abort_flag, p.status, 0x900u + s)) return false;
+    sched_ring[s] = t;
+    st_shared_cluster_u32(mapa_shared(smem_u32(const_cast<int*>(sched_ring + s)), 1), static_cast<uint32_t>(t));
+    mbar_arrive(sfull_bar(s));
+    mbar_arrive_cluster(mapa_shared(sfull_bar(s), 1));  // release: orders the store above
+    return true;
+  };
+  auto receive_tile = [&](int i, uint32_t code) -> int {
+    if (!dyn) {
+      const int t = pair + i * npairs;
+      return t < num_tiles ? t : -1;
+    }
+    const int s = i % S::kSched;
+    const uint32_t ph = static_cast<uint32_t>(i / S::kSched) & 1u;
+    if (!mbar_wait<true>(sfull_bar(s), ph, abort_flag, p.status, code + s)) return -2;
+    return sched_ring[s];
+  };
+  auto release_tile = [&](int i) {
+    if (!dyn) return;
+    const uint32_t b = sempty_bar(i % S::kSched);
+    if (leader) {
+      mbar_arrive(b);
+    } else {
+      mbar_arrive_cluster(mapa_shared(b, 0));
+    }
+  };
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer (both CTAs)
@@ -117,7 +175,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_phase = 0;
       bool ok = true;
-      for (int t = pair; ok && t < num_tiles; t += npairs) {
+      for (int i = 0; ok; ++i) {
+        int t;
+        if (leader) {
+          t = claim_tile(i);
+          if (!publish_tile(i, t)) {
+            ok = false;
+            break;
+          }
+        } else {
+          t = receive_tile(i, 0x940u);
+          if (t == -2) {
+            ok = false;
+            break;
+          }
+          release_tile(i);
+        }
+        if (t < 0) break;
         int g, m0, row0, n;
         gemm_tile(p, t, S::kBN, g, m0, row0, n);
         const int N = (n + 31) & ~31;
@@ -171,7 +245,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       bool issued_any = false;
-      for (int t = pair; ok && t < num_tiles; t += npairs) {
+      for (int i = 0; ok; ++i) {
+        const int t = receive_tile(i, 0x980u);
+        if (t == -2) {
+          ok = false;
+          break;
+        }
+        release_tile(i);
+        if (t < 0) break;
         int g, m0, row0, n;
         gemm_tile(p, t, S::kBN, g, m0, row0, n);
         const uint32_t N = static_cast<uint32_t>((n + 31) & ~31);
@@ -257,7 +338,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     };
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = pair; t < num_tiles; t += npairs) {
+    for (int i = 0;; ++i) {
+      int t = receive_tile(i, 0x9C0u);
+      if (!__all_sync(0xffffffffu, t != -2)) break;
+      t = __shfl_sync(0xffffffffu, t, 0);
+      __syncwarp();
+      if (lane == 0) release_tile(i);
+      if (t < 0) break;
       int g, m0, row0, n;
       gemm_tile(p, t, S::kBN, g, m0, row0, n);
       const bool ready = mbar_wait<true>(accf_bar(acc), acc_phase, abort_flag, p.status, 0x800u + acc);

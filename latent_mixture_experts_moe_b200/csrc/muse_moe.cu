@@ -40,7 +40,7 @@ int dense_bn(const muse_moe_config& c) { return c.T <= 32 ? 32 : 256; }
 
 struct Layout {
   muse_moe_workspace_layout pub;
-  size_t tiles_gu, tiles_dn, ntiles;  // int4 lists and two int counters
+  size_t tiles_gu, tiles_dn, ntiles;  // int4 lists; int[8]: tile counts [0..1], tile counters [4..7]
   int64_t max_tiles_gu, max_tiles_dn;
 };
 
@@ -65,7 +65,7 @@ Layout make_layout(const muse_moe_config& c) {
   l.pub.status = take(16);
   l.pub.expert_count = take(sizeof(int32_t) * E);
   l.pub.expert_offset = take(sizeof(int32_t) * (E + 1));
-  l.ntiles = take(sizeof(int32_t) * 2);
+  l.ntiles = take(sizeof(int32_t) * 8);
   l.pub.logits = take(sizeof(float) * T * E);
   l.pub.topk_idx = take(sizeof(int32_t) * assign);
   l.pub.topk_w = take(sizeof(float) * assign);
@@ -268,7 +268,7 @@ GemmArgs base_args(uint32_t* status) {
 // dense C[T, M] = X[T, K] W[M, K]^T
 template <typename TIn, typename TOut>
 muse_status dense_gemm(const void* W, int64_t M, const void* X, int64_t T, int64_t K, void* out, int bn,
-                       uint32_t* status, cudaStream_t st) {
+                       uint32_t* status, int* tile_counter, cudaStream_t st) {
   TmaMaps maps;
   const bool bf = sizeof(TIn) == 2;
   if (!make_maps(&maps, W, nullptr, M, X, T, K, bf)) return MUSE_ERR_CUDA;
@@ -286,6 +286,7 @@ muse_status dense_gemm(const void* W, int64_t M, const void* X, int64_t T, int64
     g.m_step = 256;
     g.m_tiles = static_cast<int>(cdiv(M, 256));
     g.num_tiles = static_cast<int>(g.m_tiles * cdiv(T, 256));
+    g.tile_counter = tile_counter;
     const int pairs = std::min(g.num_tiles, nsm / 2);
     return launch_gemm_2sm<TOut, EPI_STORE, 1>(maps, g, pairs, st) == cudaSuccess ? MUSE_OK : MUSE_ERR_CUDA;
   }
@@ -360,7 +361,7 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
 
   // (a1) router logits
   if (bf) {
-    muse_status s = dense_gemm<T, float>(W_router, E, x, Tn, D, logits, bn_d, status, st);
+    muse_status s = dense_gemm<T, float>(W_router, E, x, Tn, D, logits, bn_d, status, nullptr, st);
     if (s != MUSE_OK) return s;
   } else {
     k_router_logits_f32<<<static_cast<unsigned>(Tn), 256, 0, st>>>(reinterpret_cast<const float*>(x),
@@ -385,7 +386,7 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
     const int threads = static_cast<int>(align_up(static_cast<size_t>(E), 32));
     k_build_tiles<<<1, threads, 0, st>>>(counts, static_cast<int>(E), bn_g, static_cast<int>(I / pgu.step), pgu.step,
                                          static_cast<int>(L / pdn.step), pdn.step, offsets, tiles_gu, ntiles,
-                                         tiles_dn, ntiles + 1, row_token);
+                                         tiles_dn, ntiles + 1, ntiles + 4, row_token);
     MUSE_CK(cudaGetLastError());
     MUSE_CK(mark());
     k_assign_rows<<<static_cast<unsigned>(E), 1024, 0, st>>>(topk_idx, static_cast<int>(assign), static_cast<int>(k),
@@ -395,7 +396,7 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
   }
   // (a4) pooler
   {
-    muse_status s = dense_gemm<T, T>(W_pool, L, x, Tn, D, z, bn_d, status, st);
+    muse_status s = dense_gemm<T, T>(W_pool, L, x, Tn, D, z, bn_d, status, ntiles + 6, st);
     if (s != MUSE_OK) return s;
     MUSE_CK(mark());
   }
@@ -438,6 +439,7 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
     GemmArgs g = base_args(status);
     g.tiles = tiles_gu;
     g.num_tiles_dev = ntiles;
+    g.tile_counter = ntiles + 4;
     g.rows_per_group = static_cast<int>(I);
     g.m_valid = static_cast<int>(I);
     g.k_blocks = static_cast<int>(L * sizeof(T) / 128);
@@ -472,6 +474,7 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
     GemmArgs g = base_args(status);
     g.tiles = tiles_dn;
     g.num_tiles_dev = ntiles + 1;
+    g.tile_counter = ntiles + 5;
     g.rows_per_group = static_cast<int>(L);
     g.m_valid = static_cast<int>(L);
     g.k_blocks = static_cast<int>(I * sizeof(T) / 128);
@@ -509,7 +512,7 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
   }
   // (a10) unpooler
   {
-    muse_status s = dense_gemm<T, T>(W_unpool, D, cbuf, Tn, L, out, bn_d, status, st);
+    muse_status s = dense_gemm<T, T>(W_unpool, D, cbuf, Tn, L, out, bn_d, status, ntiles + 7, st);
     if (s != MUSE_OK) return s;
   }
   MUSE_CK(mark());

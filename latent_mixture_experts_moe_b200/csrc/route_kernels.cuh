@@ -179,12 +179,14 @@ __global__ void k_expert_hist(const int* __restrict__ idx, int n, int E, int* __
 // lists (gate/up tiles step_gu features apart, down tiles step_dn apart) and the padding
 // rows' token = -1. An expert's n rows split into
 // ceil(n / BN) near-equal chunks of a multiple of 16 rows; tiles are ordered expert,
-// feature tile, chunk, so the chunks sharing one weight tile run side by side.
+// feature tile, chunk, so the chunks sharing one weight tile run side by side. Also
+// zeroes the tile counters the CTA-pair GEMMs of the forward claim tiles from.
 // --------------------------------------------------------------------------------------
 __global__ void k_build_tiles(const int* __restrict__ counts, int E, int BN, int mt_gu, int step_gu, int mt_dn,
                               int step_dn, int* __restrict__ offsets, int4* __restrict__ tiles_gu,
                               int* __restrict__ ntiles_gu, int4* __restrict__ tiles_dn,
-                              int* __restrict__ ntiles_dn, int* __restrict__ row_token) {
+                              int* __restrict__ ntiles_dn, int* __restrict__ tile_counters,
+                              int* __restrict__ row_token) {
   const int e = threadIdx.x;
   const int n = (e < E) ? counts[e] : 0;
   const int padded = (n + 15) & ~15;
@@ -208,6 +210,7 @@ __global__ void k_build_tiles(const int* __restrict__ counts, int E, int BN, int
     offsets[E] = total_rows;
     *ntiles_gu = total_gu;
     *ntiles_dn = total_dn;
+    for (int i = 0; i < 4; ++i) tile_counters[i] = 0;  // the CTA-pair GEMMs of this forward
   }
 }
 
