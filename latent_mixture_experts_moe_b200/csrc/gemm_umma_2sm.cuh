@@ -354,50 +354,89 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                              static_cast<uint32_t>(acc) * S::kAccCols;
       const int nchunks = (n + 31) >> 5;
       const int col_cta = m0 + static_cast<int>(rank) * 128;  // first feature of this CTA
+      // This group's chunks are c = grp, grp + 2, ... < nchunks (m of them). TMEM loads are
+      // issued one step ahead of the arithmetic that uses them, into two register buffers,
+      // with the loops unrolled so that no buffer is carried around a loop. (10 warps per
+      // CTA leave 168 registers a thread: three warps share one quarter of the register
+      // file on two of the four schedulers.)
+      const int m = nchunks > grp ? (nchunks - grp + 1) >> 1 : 0;
       if constexpr (EPI == EPI_SWIGLU) {
+        // per chunk two steps of 16 tokens; buffers hold gate and up of one step
         const int f = col_cta + fl;
         const bool f_ok = f < p.m_valid;
-        for (int c = grp; c < nchunks; c += 2) {
-          uint32_t v[32], u[32];
-          tmem_ld32(taddr + 32u * c, v);
-          tmem_ld32(taddr + 256u + 32u * c, u);
-          tmem_ld_wait();
-          float hv[32];
+        constexpr int kMaxM = S::kBN / 64;
+        auto load = [&](int c, int half, uint32_t (&gu)[32]) {
+          const uint32_t a = taddr + static_cast<uint32_t>(32 * c + 16 * half);
+          tmem_ld16(a, *reinterpret_cast<uint32_t(*)[16]>(&gu[0]));
+          tmem_ld16(a + 256u, *reinterpret_cast<uint32_t(*)[16]>(&gu[16]));
+        };
+        auto swiglu16 = [&](const uint32_t (&gu)[32], float* hv) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float a = __uint_as_float(v[i]);
-            hv[i] = __fdividef(a, 1.0f + __expf(-a)) * __uint_as_float(u[i]);  // SiLU(gate) * up
-          }
+          for (int i = 0; i < 16; ++i) hv[i] = silu_tanh(__uint_as_float(gu[i])) * __uint_as_float(gu[16 + i]);
+        };
+        uint32_t ba[32], bb[32];
+        if (m > 0) load(grp, 0, ba);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < kMaxM; ++j) {
+          if (j >= m) break;
+          const int c = grp + 2 * j;
+          float hv[32];
+          load(c, 1, bb);
+          swiglu16(ba, hv);
+          tmem_ld_wait();
+          if (j + 1 < m) load(c + 2, 0, ba);
+          swiglu16(bb, hv + 16);
           emit(hv, c, col_cta, row0, n, f_ok, f);
+          tmem_ld_wait();
         }
       } else {
+        float gain1[MT];
+        bool fok[MT];
 #pragma unroll
         for (int h = 0; h < MT; ++h) {
           const int f = col_cta + h * 256 + fl;
-          const bool f_ok = f < p.m_valid;
-          float gain1 = 1.0f;
-          if (EPI == EPI_STORE_SS && p.ss_gain != nullptr && f_ok)
-            gain1 = 1.0f + to_f32(reinterpret_cast<const TIn*>(p.ss_gain)[g * p.ss_gain_group_stride + f]);
-          for (int c = grp; c < nchunks; c += 2) {
-            uint32_t v[32];
-            tmem_ld32(taddr + static_cast<uint32_t>(h * 256) + 32u * c, v);
-            tmem_ld_wait();
-            float yv[32];
+          fok[h] = f < p.m_valid;
+          gain1[h] = 1.0f;
+          if (EPI == EPI_STORE_SS && p.ss_gain != nullptr && fok[h])
+            gain1[h] = 1.0f + to_f32(reinterpret_cast<const TIn*>(p.ss_gain)[g * p.ss_gain_group_stride + f]);
+        }
+        constexpr int kItems = MT * (S::kBN / 64);
+        const int valid = MT * m;  // item j: chunk grp + 2 * (j / MT), accumulator half j % MT
+        auto addr = [&](int j) {
+          return taddr + static_cast<uint32_t>((j % MT) * 256 + 32 * (grp + 2 * (j / MT)));
+        };
+        auto process = [&](const uint32_t (&v)[32], int j) {
+          const int h = j % MT;
+          const int c = grp + 2 * (j / MT);
+          float yv[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) yv[i] = __uint_as_float(v[i]);
-            if constexpr (EPI == EPI_STORE_SS) {
-              float sq[32];
+          for (int i = 0; i < 32; ++i) yv[i] = __uint_as_float(v[i]);
+          emit(yv, c, col_cta + h * 256, row0, n, fok[h], col_cta + h * 256 + fl);
+          if constexpr (EPI == EPI_STORE_SS) {
 #pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const float y = yv[i] * gain1;
-                sq[i] = f_ok ? y * y : 0.0f;
-              }
-              const float tot = transpose_reduce32(sq, lane);
-              const int tok = c * 32 + lane;
-              if (tok < n) p.ss[(static_cast<int64_t>(row0) + tok) * p.ss_ld + ((col_cta + h * 256) >> 5) + q] = tot;
+            for (int i = 0; i < 32; ++i) {
+              const float y = yv[i] * gain1[h];
+              yv[i] = fok[h] ? y * y : 0.0f;
             }
-            emit(yv, c, col_cta + h * 256, row0, n, f_ok, f);
+            const float tot = transpose_reduce32(yv, lane);
+            const int tok = c * 32 + lane;
+            if (tok < n) p.ss[(static_cast<int64_t>(row0) + tok) * p.ss_ld + ((col_cta + h * 256) >> 5) + q] = tot;
           }
+        };
+        uint32_t va[32], vb[32];
+        if (valid > 0) tmem_ld32(addr(0), va);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < kItems; j += 2) {
+          if (j >= valid) break;
+          if (j + 1 < valid) tmem_ld32(addr(j + 1), vb);
+          process(va, j);
+          tmem_ld_wait();
+          if (j + 1 >= valid) break;
+          if (j + 2 < valid) tmem_ld32(addr(j + 2), va);
+          process(vb, j + 1);
+          tmem_ld_wait();
         }
       }
       tc_fence_before();
