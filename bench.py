@@ -17,6 +17,8 @@ Timing: W untimed warm-up steps, then K steps between CUDA events on the launchi
 stream, with a barrier and a device synchronisation on both sides. Every step streams
 the expert weights (25.8 GB >> 126 MB L2), so inputs are larger than L2 and no flush is
 needed. Per-kernel durations come from events the library records between its launches.
+Decode workloads are also timed as replays of one CUDA graph of the forward
+("graph_replay"), which takes the host's per-launch work out of the step.
 """
 from __future__ import annotations
 
@@ -153,8 +155,42 @@ def make_rank_inputs(w: W.Workload, rank: int, dev):
     return inp
 
 
+def time_graph(w: W.Workload, model, inp, out, idx, steps: int, warmup: int, world: int, dev):
+    """The same forward captured once in a CUDA graph and replayed: CUDA-event time of
+    `steps` replays (max over ranks), no host work between launches."""
+    import latent_mixture_experts_moe_b200 as moe
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        model(inp["x"], out=out, topk_idx=idx)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        model(inp["x"], out=out, topk_idx=idx)
+    for _ in range(warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    stream = torch.cuda.current_stream()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        graph.replay()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = all_max(t0.elapsed_time(t1), world, dev)
+    code, detail = moe.last_device_status(model.config(w.T, model.workspace))
+    del graph
+    if code != 0:
+        raise RuntimeError(f"device status {code} detail {detail:#x} under graph replay")
+    return {"value": job_tokens_per_s(world, w.T, steps, ms), "unit": "tokens/s", "ms_per_step": ms / steps,
+            "steps": steps}
+
+
 def run_ours(w: W.Workload, inp, steps: int, warmup: int, rank: int, world: int, peaks, peak_kind,
-             sample_clocks: bool, e2e_steps: int):
+             sample_clocks: bool, e2e_steps: int, graph_steps: int = 0):
     import latent_mixture_experts_moe_b200 as moe
     dev = inp["x"].device
     weights = {k: v for k, v in inp.items() if k != "x"}
@@ -235,6 +271,8 @@ def run_ours(w: W.Workload, inp, steps: int, warmup: int, rank: int, world: int,
         res["clocks"] = clocks.summary(wall0, wall1)
     if e2e_steps > 0:
         res["e2e"] = run_e2e(w, model, inp, e2e_steps, world, dev)
+    if graph_steps > 0:
+        res["graph"] = time_graph(w, model, inp, out, idx, graph_steps, warmup, world, dev)
     return res
 
 
@@ -417,13 +455,14 @@ def main():
         peaks, peak_kind = load_peaks()
         inp = make_rank_inputs(w, rank, dev)
         main_res = run_ours(w, inp, args.steps, args.warmup, rank, world, peaks, peak_kind, True,
-                            e2e_steps=min(args.steps, 20))
+                            e2e_steps=min(args.steps, 20),
+                            graph_steps=args.steps if w.name.endswith("decode") else 0)
         side = {}
         if not args.no_side and w.name == "prefill":
             wd = W.WORKLOADS["decode"]
             inp_d = dict(inp, x=rank_tokens(wd, rank, dev))
             side["decode"] = run_ours(wd, inp_d, max(args.steps, 50), args.warmup, rank, world, peaks, peak_kind,
-                                      False, e2e_steps=0)
+                                      False, e2e_steps=0, graph_steps=max(args.steps, 50))
             wz = W.WORKLOADS["prefill_zipf"]
             inp_z = dict(inp, router_bias=W.zipf_router_bias(wz).to(dev))
             side["prefill_zipf"] = run_ours(wz, inp_z, args.steps, args.warmup, rank, world, peaks, peak_kind,
@@ -451,9 +490,13 @@ def main():
                 "stage_ms": main_res["stage_ms"], "gpu_launches": main_res["gpu_launches"],
                 "clocks": main_res.get("clocks"), "e2e": main_res.get("e2e"),
             }
+            if "graph" in main_res:
+                line["graph_replay"] = main_res["graph"]
             for name, r in side.items():
                 line[name] = {"value": r["value"], "unit": "tokens/s", "ms_per_step": r["ms_per_step"],
                               "roofline": r["roofline"], "step_roofline": r["step"], "stage_ms": r["stage_ms"]}
+                if "graph" in r:
+                    line[name]["graph_replay"] = r["graph"]
             if world == 1 and not args.no_cpu:
                 line["cpu_baseline"] = cpu_baseline(w, dev, args.cpu_tokens)
             print(json.dumps(line), flush=True)

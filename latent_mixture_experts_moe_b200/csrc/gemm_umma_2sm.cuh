@@ -194,10 +194,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         if (t < 0) break;
         int g, m0, row0, n;
         gemm_tile(p, t, S::kBN, g, m0, row0, n);
-        const int N = (n + 31) & ~31;
-        const int half = N >> 1;             // token rows staged by each CTA
-        const int nb16 = half >> 4;          // 1..8 blocks of 16 rows
-        const uint32_t bytes_pair = 2u * (S::kABytes * MT + static_cast<uint32_t>(half) * 128u);
+        // N = n rounded up to 16 (the M = 256 MMA's N granularity); each CTA stages N / 2
+        // token rows, a multiple of 8, loaded as 16-row boxes: the last box may carry 8 rows
+        // past the half (the partner's first rows, or zero fill past the tensor), which
+        // still lie inside the stage's 128-row B area and count in the expected bytes
+        const int N = (n + 15) & ~15;
+        const int half = N >> 1;             // token rows the MMA reads from this CTA
+        const int nb16 = (half + 15) >> 4;   // 1..8 boxes of 16 rows
+        const uint32_t bytes_pair = 2u * (S::kABytes * MT + static_cast<uint32_t>(nb16) * 2048u);
         const int a_row = g * p.rows_per_group + m0 + static_cast<int>(rank) * 128;
         const int a2_row = (EPI == EPI_SWIGLU) ? a_row : a_row + 256;
         const int b_row = row0 + static_cast<int>(rank) * half;
@@ -255,7 +259,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         if (t < 0) break;
         int g, m0, row0, n;
         gemm_tile(p, t, S::kBN, g, m0, row0, n);
-        const uint32_t N = static_cast<uint32_t>((n + 31) & ~31);
+        const uint32_t N = static_cast<uint32_t>((n + 15) & ~15);
         const uint32_t idesc = idesc_f32acc(1u, 256u, N);
         if (!mbar_wait<true>(acce_bar(acc), acc_phase ^ 1u, abort_flag, p.status, 0x600u + acc)) {
           ok = false;

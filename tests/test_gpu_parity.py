@@ -94,6 +94,48 @@ def test_host_io_entry_point_matches_device_entry_point(mid):
     assert torch.equal(out_host, run.out.cpu())
 
 
+# ------------------------------------------------------------------------- CUDA graphs
+GRAPH = [
+    # name, T, D, L, I, E, k: decode-sized tiles (one-CTA kernels), and CTA-pair tiles whose
+    # tile counters must be re-zeroed inside every replay
+    ("graph_small_tiles", 96, 1024, 512, 512, 32, 4),
+    ("graph_pair_tiles", 1024, 1024, 512, 512, 4, 2),
+]
+
+
+@pytest.mark.parametrize("case", GRAPH, ids=[c[0] for c in GRAPH])
+def test_cuda_graph_replay_matches_eager(case):
+    """The forward captured once in a CUDA graph and replayed gives the eager result bit for
+    bit, also after new tokens are written into the captured input buffer."""
+    import dataclasses
+    name, T, D, L, I, E, k = case
+    w = W.Workload(name, T=T, D=D, L=L, I=I, E=E, k=k, dtype="bf16", seed=11)
+    inp = W.make_inputs(w, "cuda")
+    model = moe.LatentMoE({n: v for n, v in inp.items() if n != "x"}, T_max=T, k=k, eps=w.eps)
+    x = inp["x"].clone()
+    out_g = torch.empty((T, D), dtype=torch.bfloat16, device="cuda")
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        model(x, out=out_g)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        model(x, out=out_g)
+    x2 = W.make_inputs(dataclasses.replace(w, seed=12), "cuda", names=["x"])["x"]
+    for xs in (inp["x"], x2, inp["x"]):
+        x.copy_(xs)
+        graph.replay()
+        torch.cuda.synchronize()
+        eager = model(xs.clone())
+        torch.cuda.synchronize()
+        assert torch.equal(out_g, eager)
+    code, detail = moe.last_device_status(model.config(T, model.workspace))
+    assert code == 0, f"status {code} detail {detail:#x}"
+    del graph
+
+
 # ------------------------------------------------------------------------- edge cases
 EDGE = [
     # name, T, D, L, I, E, k, dtype, bias_kind
