@@ -115,6 +115,25 @@ typedef struct muse_moe_config {
                                  is recorded on the stream before launch i and the last
                                  after the final launch (per-kernel device timing)     */
   int32_t expert_weights;     /* muse_expert_weights                                  */
+  /* The feed-forward sublayer around the block (deep dive §2.1 steps 6-7, §5.2 residual
+   * gate, §5.3 norm table); each step is off when its pointer is NULL. With all three,
+   * x is the decoder layer's residual stream and out its next value:
+   *   xn  = x / sqrt(mean(x^2) + ffn_pre_eps) * (1 + ffn_pre_gain)   (centred RMSNorm;
+   *         the router and the pooler read xn instead of x)
+   *   f   = the block applied to xn
+   *   v   = f * (1 + ffn_post_gain);  fn = v / sqrt(mean(v^2) + ffn_post_eps)
+   *   out = alpha * x + beta * fn, beta = sigmoid(g / T),
+   *         alpha = sqrt(max(sigmoid(-g / T) * (1 + beta), residual_gate_eps)),
+   *   with g = residual_gate, T = residual_gate_temperature; statistics and gate
+   *   coefficients in FP32, out rounded once to cfg->dtype. Without the gate
+   *   out = fn (or f); without the post norm the gate mixes x and f. */
+  const void* ffn_pre_gain;   /* device [D] gain offsets in cfg->dtype, or NULL       */
+  float ffn_pre_eps;          /* pages: 1e-5                                          */
+  const void* ffn_post_gain;  /* device [D] gain offsets in cfg->dtype, or NULL       */
+  float ffn_post_eps;         /* pages: 1e-8                                          */
+  const float* residual_gate; /* device [D] float32 gate parameters g, or NULL        */
+  float residual_gate_temperature; /* pages: 0.3                                      */
+  float residual_gate_eps;    /* floor of alpha^2; pages: 1e-3                         */
 } muse_moe_config;
 
 /* Byte offsets of the intermediates inside the workspace after a forward call, for
@@ -135,11 +154,16 @@ typedef struct muse_moe_workspace_layout {
   size_t y;             /* act   [R, L]  expert outputs before the norm               */
   size_t ss;            /* float [R, L/32] partial sums of y^2 per 32 columns         */
   size_t c;             /* act   [T, L]  combined latent                              */
+  size_t xn;            /* act   [T, D]  normalised input (with ffn_pre_gain; else 0)  */
+  size_t ss_out;        /* float [T, D/32] partial sums of v^2 per 32 columns (with
+                           ffn_post_gain; else 0)                                     */
   size_t total;         /* bytes required                                             */
   int64_t rows;         /* R: upper bound of padded rows                              */
 } muse_moe_workspace_layout;
 
-/* Fills defaults: router softmax, scale 1, rsf 1, norm centred per expert, eps 1e-6. */
+/* Fills defaults: router softmax, scale 1, rsf 1, norm centred per expert, eps 1e-6;
+ * sublayer steps off, with the pages' epsilons (1e-5, 1e-8), temperature 0.3 and
+ * alpha^2 floor 1e-3 ready for when their pointers are set. */
 MUSE_API void muse_moe_config_init(muse_moe_config* cfg);
 
 /* Workspace bytes for cfg's sizes (cfg->workspace is not read). */
@@ -214,8 +238,11 @@ MUSE_API muse_status muse_selftest_bounded_wait(uint64_t limit_ns, uint32_t* sta
 /* Static string for a status code. */
 MUSE_API const char* muse_status_string(muse_status s);
 
-/* Number of kernel launches one forward call makes for cfg (11; 12 with a pre-expert
- * norm). stage_events must hold this many + 1 events. */
+/* Number of kernel launches one forward call makes for cfg: 11, plus one each for the
+ * pre-expert norm, the pre-FFN norm, and the post-FFN norm / residual gate (one kernel
+ * finishes both). In launch order: [ffn pre norm], router, top-k, histogram, tiles,
+ * assign rows, pooler, [pre-expert norm], gather, gate/up, down, norm + combine,
+ * unpooler, [post norm / gate]. stage_events must hold this many + 1 events. */
 MUSE_API int32_t muse_latent_moe_launch_count(const muse_moe_config* cfg);
 
 #ifdef __cplusplus

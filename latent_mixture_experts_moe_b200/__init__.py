@@ -47,7 +47,11 @@ class Config(ctypes.Structure):
                 ("pre_norm_gain", ctypes.c_void_p), ("pre_norm_eps", ctypes.c_float),
                 ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
                 ("topk_idx_out", ctypes.c_void_p), ("topk_w_out", ctypes.c_void_p),
-                ("stage_events", ctypes.c_void_p), ("expert_weights", ctypes.c_int32)]
+                ("stage_events", ctypes.c_void_p), ("expert_weights", ctypes.c_int32),
+                ("ffn_pre_gain", ctypes.c_void_p), ("ffn_pre_eps", ctypes.c_float),
+                ("ffn_post_gain", ctypes.c_void_p), ("ffn_post_eps", ctypes.c_float),
+                ("residual_gate", ctypes.c_void_p), ("residual_gate_temperature", ctypes.c_float),
+                ("residual_gate_eps", ctypes.c_float)]
 
 
 class Nvfp4Weight(ctypes.Structure):
@@ -57,7 +61,7 @@ class Nvfp4Weight(ctypes.Structure):
 class WorkspaceLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in ("status", "expert_count", "expert_offset", "logits", "topk_idx",
                                               "topk_w", "inv", "row_token", "z", "zp", "h", "y", "ss", "c",
-                                              "total")] + [("rows", ctypes.c_int64)]
+                                              "xn", "ss_out", "total")] + [("rows", ctypes.c_int64)]
 
 
 _lib: Optional[ctypes.CDLL] = None
@@ -106,7 +110,9 @@ def _check(code: int, where: str) -> None:
 
 def make_config(T: int, D: int, L: int, I: int, E: int, k: int, dtype: str = "bf16", eps: float = 1e-6,
                 router_mode: int = ROUTER_SOFTMAX, router_logit_scale: float = 1.0, routed_scaling: float = 1.0,
-                norm_mode: int = NORM_CENTRED, gamma_shared: bool = False, pre_norm_eps: float = 1e-5) -> Config:
+                norm_mode: int = NORM_CENTRED, gamma_shared: bool = False, pre_norm_eps: float = 1e-5,
+                ffn_pre_eps: float = 1e-5, ffn_post_eps: float = 1e-8, residual_gate_temperature: float = 0.3,
+                residual_gate_eps: float = 1e-3) -> Config:
     c = Config()
     lib().muse_moe_config_init(ctypes.byref(c))
     c.T, c.D, c.L, c.I, c.E, c.top_k = T, D, L, I, E, k
@@ -115,6 +121,8 @@ def make_config(T: int, D: int, L: int, I: int, E: int, k: int, dtype: str = "bf
     c.router_mode, c.router_logit_scale, c.routed_scaling = router_mode, router_logit_scale, routed_scaling
     c.norm_mode, c.gamma_shared = norm_mode, int(gamma_shared)
     c.pre_norm_eps = pre_norm_eps
+    c.ffn_pre_eps, c.ffn_post_eps = ffn_pre_eps, ffn_post_eps
+    c.residual_gate_temperature, c.residual_gate_eps = residual_gate_temperature, residual_gate_eps
     return c
 
 
@@ -182,6 +190,19 @@ STAGES = ("router", "topk", "expert_hist", "tiles", "assign_rows", "pooler", "ga
           "down_sumsq", "norm_combine", "unpooler")
 
 
+def stages(cfg: Config):
+    """Names of the kernels one forward launches for cfg, in launch order (STAGES plus the
+    optional sublayer pre-norm, pre-expert norm and sublayer post-norm / residual gate)."""
+    names = list(STAGES)
+    if cfg.pre_norm_gain:
+        names.insert(names.index("gather"), "pre_expert_norm")
+    if cfg.ffn_pre_gain:
+        names.insert(0, "ffn_pre_norm")
+    if cfg.ffn_post_gain or cfg.residual_gate:
+        names.append("ffn_post_norm_gate")
+    return tuple(names)
+
+
 def event_handles(events) -> "ctypes.Array":
     """ctypes array of the raw cudaEvent_t handles of torch.cuda.Event objects (each
     recorded once beforehand so that it exists)."""
@@ -207,7 +228,8 @@ class LatentMoE:
     """Holds the block's device weights and a workspace; calling it runs the forward.
 
     weights: dict with W_router, W_pool, W_gate, W_up, W_down, gamma, W_unpool (torch
-    CUDA tensors in the layouts of include/muse_moe.h); router_bias and pre_norm_gain
+    CUDA tensors in the layouts of include/muse_moe.h); router_bias, pre_norm_gain and the
+    feed-forward sublayer's ffn_pre_gain, ffn_post_gain and residual_gate (float32) are
     optional. modes: make_config keywords (router_mode, norm_mode, gamma_shared, ...).
     """
 
@@ -239,8 +261,9 @@ class LatentMoE:
             c.expert_weights = EXPERTS_NVFP4
         if self.w.get("router_bias") is not None:
             c.router_bias = _ptr(self.w["router_bias"])
-        if self.w.get("pre_norm_gain") is not None:
-            c.pre_norm_gain = _ptr(self.w["pre_norm_gain"])
+        for name in ("pre_norm_gain", "ffn_pre_gain", "ffn_post_gain", "residual_gate"):
+            if self.w.get(name) is not None:
+                setattr(c, name, _ptr(self.w[name]))
         if workspace is not None:
             c.workspace = _ptr(workspace)
             c.workspace_bytes = workspace.numel()

@@ -79,6 +79,8 @@ Layout make_layout(const muse_moe_config& c) {
   l.pub.y = take(as * rows * c.L);
   l.pub.ss = take(sizeof(float) * rows * (c.L / 32));
   l.pub.c = take(as * T * c.L);
+  l.pub.xn = c.ffn_pre_gain != nullptr ? take(as * T * c.D) : 0;
+  l.pub.ss_out = c.ffn_post_gain != nullptr ? take(sizeof(float) * T * (c.D / 32)) : 0;
   l.pub.total = o;
   l.pub.rows = rows;
   return l;
@@ -265,10 +267,18 @@ GemmArgs base_args(uint32_t* status) {
   return g;
 }
 
+// Sum-of-squares partials of a dense GEMM's output (EPI_STORE_SS): ss[t, f / 32] over
+// 32-column groups of (acc * (1 + gain[f])).
+struct DenseSS {
+  float* ss = nullptr;
+  int ld = 0;
+  const void* gain = nullptr;
+};
+
 // dense C[T, M] = X[T, K] W[M, K]^T
-template <typename TIn, typename TOut>
+template <typename TIn, typename TOut, int EPI = EPI_STORE>
 muse_status dense_gemm(const void* W, int64_t M, const void* X, int64_t T, int64_t K, void* out, int bn,
-                       uint32_t* status, int* tile_counter, cudaStream_t st) {
+                       uint32_t* status, int* tile_counter, cudaStream_t st, DenseSS sq = DenseSS{}) {
   TmaMaps maps;
   const bool bf = sizeof(TIn) == 2;
   if (!make_maps(&maps, W, nullptr, M, X, T, K, bf)) return MUSE_ERR_CUDA;
@@ -280,6 +290,10 @@ muse_status dense_gemm(const void* W, int64_t M, const void* X, int64_t T, int64
   g.k_blocks = static_cast<int>(cdiv(K * sizeof(TIn), 128));
   g.out = out;
   g.ld_out = M;
+  g.ss = sq.ss;
+  g.ss_ld = sq.ld;
+  g.ss_gain = sq.gain;
+  g.ss_gain_group_stride = 0;
   // a CTA pair per 256 features x 256 tokens when that fills at least one wave of pairs
   if (bf && bn == 256 && cdiv(M, 256) * cdiv(T, 256) >= nsm / 2) {
     if (sizeof(TOut) == 2 && !make_out_map(&maps.out, out, T, M)) return MUSE_ERR_CUDA;
@@ -288,7 +302,7 @@ muse_status dense_gemm(const void* W, int64_t M, const void* X, int64_t T, int64
     g.num_tiles = static_cast<int>(g.m_tiles * cdiv(T, 256));
     g.tile_counter = tile_counter;
     const int pairs = std::min(g.num_tiles, nsm / 2);
-    return launch_gemm_2sm<TOut, EPI_STORE, 1>(maps, g, pairs, st) == cudaSuccess ? MUSE_OK : MUSE_ERR_CUDA;
+    return launch_gemm_2sm<TOut, EPI, 1>(maps, g, pairs, st) == cudaSuccess ? MUSE_OK : MUSE_ERR_CUDA;
   }
   // two 128-row weight tiles per CTA when that still leaves at least a full wave of tiles
   const int mt = (cdiv(M, 256) * cdiv(T, bn) >= nsm) ? 2 : 1;
@@ -296,7 +310,7 @@ muse_status dense_gemm(const void* W, int64_t M, const void* X, int64_t T, int64
   g.m_tiles = static_cast<int>(cdiv(M, g.m_step));
   g.num_tiles = static_cast<int>(g.m_tiles * cdiv(T, bn));
   const int grid = std::min(g.num_tiles, nsm);
-  return launch_gemm_bn<TIn, TOut, EPI_STORE>(bn, mt, maps, g, grid, st) == cudaSuccess ? MUSE_OK : MUSE_ERR_CUDA;
+  return launch_gemm_bn<TIn, TOut, EPI>(bn, mt, maps, g, grid, st) == cudaSuccess ? MUSE_OK : MUSE_ERR_CUDA;
 }
 
 // Grouped-GEMM plans. gate/up: a CTA pair per 256 features when tiles hold up to 256
@@ -359,12 +373,23 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
   };
   MUSE_CK(mark());
 
+  // feed-forward sublayer pre-norm (optional): the router and the pooler read xn
+  const void* xin = x;
+  if (c.ffn_pre_gain != nullptr) {
+    T* xn = reinterpret_cast<T*>(at(lay.pub.xn));
+    k_rmsnorm_rows<T><<<static_cast<unsigned>(Tn), 256, 0, st>>>(reinterpret_cast<const T*>(x), xn,
+                                                                 reinterpret_cast<const T*>(c.ffn_pre_gain),
+                                                                 static_cast<int>(D), c.ffn_pre_eps);
+    MUSE_CK(cudaGetLastError());
+    MUSE_CK(mark());
+    xin = xn;
+  }
   // (a1) router logits
   if (bf) {
-    muse_status s = dense_gemm<T, float>(W_router, E, x, Tn, D, logits, bn_d, status, nullptr, st);
+    muse_status s = dense_gemm<T, float>(W_router, E, xin, Tn, D, logits, bn_d, status, nullptr, st);
     if (s != MUSE_OK) return s;
   } else {
-    k_router_logits_f32<<<static_cast<unsigned>(Tn), 256, 0, st>>>(reinterpret_cast<const float*>(x),
+    k_router_logits_f32<<<static_cast<unsigned>(Tn), 256, 0, st>>>(reinterpret_cast<const float*>(xin),
                                                                   reinterpret_cast<const float*>(W_router),
                                                                   static_cast<int>(D), static_cast<int>(E), logits);
     MUSE_CK(cudaGetLastError());
@@ -396,16 +421,14 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
   }
   // (a4) pooler
   {
-    muse_status s = dense_gemm<T, T>(W_pool, L, x, Tn, D, z, bn_d, status, ntiles + 6, st);
+    muse_status s = dense_gemm<T, T>(W_pool, L, xin, Tn, D, z, bn_d, status, ntiles + 6, st);
     if (s != MUSE_OK) return s;
     MUSE_CK(mark());
   }
   // pages' pre_expert_norm on z (optional)
   if (c.pre_norm_gain != nullptr) {
-    const int vec = 16 / static_cast<int>(sizeof(T));
-    const int threads = static_cast<int>(std::max<int64_t>(32, align_up(static_cast<size_t>(L / vec), 32)));
-    k_prenorm_rows<T><<<static_cast<unsigned>(Tn), threads, 0, st>>>(z, reinterpret_cast<const T*>(c.pre_norm_gain),
-                                                                    static_cast<int>(L), c.pre_norm_eps);
+    k_rmsnorm_rows<T><<<static_cast<unsigned>(Tn), 256, 0, st>>>(z, z, reinterpret_cast<const T*>(c.pre_norm_gain),
+                                                                 static_cast<int>(L), c.pre_norm_eps);
     MUSE_CK(cudaGetLastError());
     MUSE_CK(mark());
   }
@@ -510,12 +533,32 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
     MUSE_CK(cudaGetLastError());
     MUSE_CK(mark());
   }
-  // (a10) unpooler
+  // (a10) unpooler; with the sublayer post-norm its epilogue also writes the partial sums
+  // of (f * (1 + w))^2
+  const bool post = c.ffn_post_gain != nullptr;
   {
-    muse_status s = dense_gemm<T, T>(W_unpool, D, cbuf, Tn, L, out, bn_d, status, ntiles + 7, st);
+    muse_status s;
+    if (post) {
+      DenseSS sq;
+      sq.ss = reinterpret_cast<float*>(at(lay.pub.ss_out));
+      sq.ld = static_cast<int>(D / 32);
+      sq.gain = c.ffn_post_gain;
+      s = dense_gemm<T, T, EPI_STORE_SS>(W_unpool, D, cbuf, Tn, L, out, bn_d, status, ntiles + 7, st, sq);
+    } else {
+      s = dense_gemm<T, T>(W_unpool, D, cbuf, Tn, L, out, bn_d, status, ntiles + 7, st);
+    }
     if (s != MUSE_OK) return s;
   }
   MUSE_CK(mark());
+  // feed-forward sublayer post-norm and residual gate (optional), in place on out
+  if (post || c.residual_gate != nullptr) {
+    k_ffn_finish<T><<<static_cast<unsigned>(Tn), 256, 0, st>>>(
+        reinterpret_cast<T*>(out), reinterpret_cast<const T*>(x), reinterpret_cast<const float*>(at(lay.pub.ss_out)),
+        static_cast<int>(D / 32), reinterpret_cast<const T*>(c.ffn_post_gain), c.ffn_post_eps, c.residual_gate,
+        1.0f / c.residual_gate_temperature, c.residual_gate_eps, static_cast<int>(D));
+    MUSE_CK(cudaGetLastError());
+    MUSE_CK(mark());
+  }
   return MUSE_OK;
 }
 
@@ -557,6 +600,10 @@ void muse_moe_config_init(muse_moe_config* cfg) {
   cfg->routed_scaling = 1.0f;
   cfg->norm_mode = MUSE_NORM_CENTRED;
   cfg->pre_norm_eps = 1e-5f;
+  cfg->ffn_pre_eps = 1e-5f;
+  cfg->ffn_post_eps = 1e-8f;
+  cfg->residual_gate_temperature = 0.3f;
+  cfg->residual_gate_eps = 1e-3f;
 }
 
 muse_status muse_latent_moe_workspace_size(const muse_moe_config* cfg, size_t* bytes) {
@@ -594,6 +641,13 @@ muse_status muse_latent_moe_forward(const muse_moe_config* cfg, const void* x, c
   if (cfg->router_bias != nullptr && (reinterpret_cast<uintptr_t>(cfg->router_bias) & 3u)) return MUSE_ERR_INVALID_ARG;
   if (cfg->pre_norm_gain != nullptr && !aligned16(cfg->pre_norm_gain)) return MUSE_ERR_INVALID_ARG;
   if (cfg->pre_norm_gain != nullptr && !(cfg->pre_norm_eps >= 0.0f)) return MUSE_ERR_INVALID_ARG;
+  if (cfg->ffn_pre_gain != nullptr && (!aligned16(cfg->ffn_pre_gain) || !(cfg->ffn_pre_eps >= 0.0f)))
+    return MUSE_ERR_INVALID_ARG;
+  if (cfg->ffn_post_gain != nullptr && (!aligned16(cfg->ffn_post_gain) || !(cfg->ffn_post_eps >= 0.0f)))
+    return MUSE_ERR_INVALID_ARG;
+  if (cfg->residual_gate != nullptr &&
+      (!aligned16(cfg->residual_gate) || !(cfg->residual_gate_temperature > 0.0f) || !(cfg->residual_gate_eps >= 0.0f)))
+    return MUSE_ERR_INVALID_ARG;
   const Layout lay = make_layout(*cfg);
   if (cfg->workspace == nullptr || (reinterpret_cast<uintptr_t>(cfg->workspace) & (kAlign - 1)))
     return MUSE_ERR_WORKSPACE;
@@ -673,9 +727,11 @@ const char* muse_status_string(muse_status s) {
 
 int32_t muse_latent_moe_launch_count(const muse_moe_config* cfg) {
   if (validate_sizes(cfg) != MUSE_OK) return -1;
-  // router, top-k, hist, tiles, rows, pooler, gather, gate/up, down, combine, unpooler
-  // (+ the optional pre-expert norm, which is launched between pooler and gather)
-  return cfg->pre_norm_gain != nullptr ? 12 : 11;
+  // router, top-k, hist, tiles, rows, pooler, gather, gate/up, down, combine, unpooler,
+  // and the optional sublayer pre-norm (first), pre-expert norm (between pooler and
+  // gather) and sublayer post-norm / residual gate (last)
+  return 11 + (cfg->pre_norm_gain != nullptr) + (cfg->ffn_pre_gain != nullptr) +
+         (cfg->ffn_post_gain != nullptr || cfg->residual_gate != nullptr);
 }
 
 }  // extern "C"

@@ -241,43 +241,105 @@ __global__ void k_assign_rows(const int* __restrict__ idx, int n, int k, const i
   }
 }
 
+// Sum over the block in a fixed order (a butterfly inside each warp, then every warp
+// sums the warp totals the same way), so equal inputs give equal bits on every run and
+// every thread receives the total. part: 32 floats of shared memory.
+__device__ __forceinline__ float block_sum(float v, float* part) {
+  v = warp_sum(v);
+  __syncthreads();  // part may still be read by a previous call
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = v;
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  float t = lane < static_cast<int>(blockDim.x >> 5) ? part[lane] : 0.0f;
+  return warp_sum(t);
+}
+
 // --------------------------------------------------------------------------------------
-// pages' pre_expert_norm (optional): centred RMSNorm of each pooled row in place,
-// z <- z / sqrt(mean(z^2) + eps) * (1 + w), FP32 statistics, one block per token.
+// Centred RMSNorm of rows of n elements (one block per row, FP32 statistics):
+//   out = in / sqrt(mean(in^2) + eps) * (1 + w)
+// Used for the pages' pre_expert_norm on z (in place, in == out) and for the feed-
+// forward sublayer's pre-norm on x (deep dive §2.1 step 6, §5.3 table). Two passes over
+// the row: the second re-reads it from cache.
 // --------------------------------------------------------------------------------------
 template <typename T>
-__global__ void k_prenorm_rows(T* __restrict__ z, const T* __restrict__ w, int L, float eps) {
+__global__ void k_rmsnorm_rows(const T* in, T* out, const T* __restrict__ w, int n, float eps) {
   constexpr int VEC = 16 / sizeof(T);
   __shared__ float part[32];
-  __shared__ float scale_s;
-  T* row = z + static_cast<int64_t>(blockIdx.x) * L;
-  const int f0 = threadIdx.x * VEC;
-  uint4 v = make_uint4(0, 0, 0, 0);
+  const T* irow = in + static_cast<int64_t>(blockIdx.x) * n;
+  T* orow = out + static_cast<int64_t>(blockIdx.x) * n;
   float ss = 0.0f;
-  if (f0 < L) {
-    v = *reinterpret_cast<const uint4*>(row + f0);
+  for (int c = threadIdx.x * VEC; c < n; c += blockDim.x * VEC) {
+    const uint4 v = *reinterpret_cast<const uint4*>(irow + c);
     const T* vv = reinterpret_cast<const T*>(&v);
 #pragma unroll
     for (int i = 0; i < VEC; ++i) ss = fmaf(to_f32(vv[i]), to_f32(vv[i]), ss);
   }
-  ss = warp_sum(ss);
-  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = ss;
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    float t = threadIdx.x < (blockDim.x >> 5) ? part[threadIdx.x] : 0.0f;
-    t = warp_sum(t);
-    if (threadIdx.x == 0) scale_s = 1.0f / sqrtf(t / static_cast<float>(L) + eps);
-  }
-  __syncthreads();
-  if (f0 < L) {
-    const uint4 gv = *reinterpret_cast<const uint4*>(w + f0);
+  const float scale = 1.0f / sqrtf(block_sum(ss, part) / static_cast<float>(n) + eps);
+  for (int c = threadIdx.x * VEC; c < n; c += blockDim.x * VEC) {
+    const uint4 v = *reinterpret_cast<const uint4*>(irow + c);
+    const uint4 gv = *reinterpret_cast<const uint4*>(w + c);
     const T* vv = reinterpret_cast<const T*>(&v);
     const T* gg = reinterpret_cast<const T*>(&gv);
     uint4 ov;
     T* oo = reinterpret_cast<T*>(&ov);
 #pragma unroll
-    for (int i = 0; i < VEC; ++i) oo[i] = from_f32<T>(to_f32(vv[i]) * scale_s * (1.0f + to_f32(gg[i])));
-    *reinterpret_cast<uint4*>(row + f0) = ov;
+    for (int i = 0; i < VEC; ++i) oo[i] = from_f32<T>(to_f32(vv[i]) * scale * (1.0f + to_f32(gg[i])));
+    *reinterpret_cast<uint4*>(orow + c) = ov;
+  }
+}
+
+// --------------------------------------------------------------------------------------
+// Feed-forward sublayer, after the unpooler (deep dive §2.1 step 7, §5.2, §5.3), in place
+// on out = f, one block per token:
+//   post norm (post_gain != NULL): v = f * (1 + w), fn = v / sqrt(mean(v^2) + post_eps),
+//     mean(v^2) from the unpooler epilogue's partial sums ss[t, 0 .. D/32) of squares of
+//     the FP32 accumulator times (1 + w), the scale applied to the stored f;
+//   residual gate (gate != NULL): out = alpha * x + beta * fn, beta = sigmoid(g / T),
+//     alpha = sqrt(max(sigmoid(-g / T) * (1 + beta), gate_eps)), coefficients in FP32.
+// --------------------------------------------------------------------------------------
+template <typename T>
+__global__ void k_ffn_finish(T* __restrict__ out, const T* __restrict__ x, const float* __restrict__ ss, int ss_ld,
+                             const T* __restrict__ post_gain, float post_eps, const float* __restrict__ gate,
+                             float inv_temp, float gate_eps, int D) {
+  constexpr int VEC = 16 / sizeof(T);
+  __shared__ float part[32];
+  const int64_t t = blockIdx.x;
+  float scale = 1.0f;
+  if (post_gain != nullptr) {  // uniform over the grid
+    float s = 0.0f;
+    for (int i = threadIdx.x; i < ss_ld; i += blockDim.x) s += ss[t * ss_ld + i];
+    scale = 1.0f / sqrtf(block_sum(s, part) / static_cast<float>(D) + post_eps);
+  }
+  T* orow = out + t * D;
+  const T* xrow = x + t * D;
+  for (int c = threadIdx.x * VEC; c < D; c += blockDim.x * VEC) {
+    const uint4 fv4 = *reinterpret_cast<const uint4*>(orow + c);
+    const T* fv = reinterpret_cast<const T*>(&fv4);
+    float f[VEC];
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) f[i] = to_f32(fv[i]);
+    if (post_gain != nullptr) {
+      const uint4 gv4 = *reinterpret_cast<const uint4*>(post_gain + c);
+      const T* gv = reinterpret_cast<const T*>(&gv4);
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) f[i] = f[i] * (1.0f + to_f32(gv[i])) * scale;
+    }
+    if (gate != nullptr) {
+      const uint4 xv4 = *reinterpret_cast<const uint4*>(xrow + c);
+      const T* xv = reinterpret_cast<const T*>(&xv4);
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) {
+        const float wg = gate[c + i] * inv_temp;
+        const float beta = 1.0f / (1.0f + expf(-wg));
+        const float alpha = sqrtf(fmaxf((1.0f / (1.0f + expf(wg))) * (1.0f + beta), gate_eps));
+        f[i] = alpha * to_f32(xv[i]) + beta * f[i];
+      }
+    }
+    uint4 ov;
+    T* oo = reinterpret_cast<T*>(&ov);
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) oo[i] = from_f32<T>(f[i]);
+    *reinterpret_cast<uint4*>(orow + c) = ov;
   }
 }
 

@@ -29,7 +29,10 @@ Readings where the pages are open or disagree (each is listed in the design doc):
     the "routing order" the combine sums in;
   * per-expert output norm: centred form with a per-expert gain (default); the pages'
     shared input-scaled form is `norm_mode="input_scaled"`;
-  * no pre-expert norm unless `pre_norm_gain` is given (pages: centred, eps 1e-5).
+  * no pre-expert norm unless `pre_norm_gain` is given (pages: centred, eps 1e-5);
+  * the feed-forward sublayer around the block (pre-norm, post-norm, residual gate;
+    deep dive §2.1 steps 6-7, §5.2, §5.3) only when its parameters are given; gains are
+    used as 1 + w exactly (the pages' ports round 1 + w to bfloat16 first).
 
 Parity pins (tests/test_oracle_pins.py): every function here is pinned by a worked
 example printed on the pages, a closed form, a brute-force enumeration or an
@@ -46,7 +49,8 @@ __all__ = [
     "router_logits", "select_topk", "softmax_weights", "sigmoid_weights", "route",
     "topk_alternatives", "pooler", "silu", "expert_ffn", "centred_rmsnorm",
     "input_scaled_rmsnorm", "combine", "unpooler", "latent_moe_forward", "as_f64",
-    "moe_flops_per_token", "expert_param_count",
+    "moe_flops_per_token", "expert_param_count", "residual_gate_coefficients", "residual_gate",
+    "round_bf16",
 ]
 
 Array = np.ndarray
@@ -200,6 +204,35 @@ def combine(n: Array, g: Array) -> Array:
 
 
 # ---------------------------------------------------------------------------------------
+# the feed-forward sublayer around the block -- deep dive §2.1 steps 6-7 and §5.3 norm
+# table (pre_feedforward_layernorm: centred, eps 1e-5; post_feedforward_layernorm:
+# scale first, then normalise, eps 1e-8), §5.2 norm-preserving residual gate
+# ---------------------------------------------------------------------------------------
+def round_bf16(a: Array) -> Array:
+    """Round float64 values to the nearest bfloat16 (8 significant bits, ties to even),
+    returned as float64. Used where the pages' implementation stores an activation in
+    bfloat16 before a decision is taken on it."""
+    m, e = np.frexp(np.asarray(a, dtype=np.float64))
+    return np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)
+
+
+def residual_gate_coefficients(gate: Array, temperature: float = 0.3, floor: float = 1e-3):
+    """Per-channel (alpha, beta) of the residual gate with parameters g:
+    beta = sigmoid(g / T) weights the branch, alpha = sqrt(max(sigmoid(-g / T) * (1 + beta),
+    floor)) the residual stream; where the floor is inactive alpha^2 = 1 - beta^2."""
+    w = gate / temperature
+    beta = _sigmoid(w)
+    alpha = np.sqrt(np.maximum(_sigmoid(-w) * (1.0 + beta), floor))
+    return alpha, beta
+
+
+def residual_gate(x: Array, f: Array, gate: Array, temperature: float = 0.3, floor: float = 1e-3) -> Array:
+    """alpha * x + beta * f per channel: x the residual stream, f the normalised branch."""
+    alpha, beta = residual_gate_coefficients(gate, temperature, floor)
+    return alpha * x + beta * f
+
+
+# ---------------------------------------------------------------------------------------
 # the whole block
 # ---------------------------------------------------------------------------------------
 def latent_moe_forward(x: Array, W_router: Array, W_pool: Array, experts: ExpertSource,
@@ -208,17 +241,33 @@ def latent_moe_forward(x: Array, W_router: Array, W_pool: Array, experts: Expert
                        logit_scale: float = 1.0, routed_scaling: float = 1.0,
                        norm_mode: str = "centred", pre_norm_gain: Optional[Array] = None,
                        pre_norm_eps: float = 1e-5, routing: Optional[Tuple[Array, Array]] = None,
-                       ) -> Dict[str, Array]:
+                       ffn_pre_gain: Optional[Array] = None, ffn_pre_eps: float = 1e-5,
+                       ffn_post_gain: Optional[Array] = None, ffn_post_eps: float = 1e-8,
+                       gate: Optional[Array] = None, gate_temperature: float = 0.3, gate_floor: float = 1e-3,
+                       xn_round: Optional[str] = None) -> Dict[str, Array]:
     """Forward pass of the latent-MoE block for every row of x, in float64.
 
     experts: (W_gate [E,I,L], W_up [E,I,L], W_down [E,L,I]) or a callable e -> the three
     [out, in] matrices of expert e (so full-size weights need not sit in host memory).
     gamma: [E, L] per-expert gain offsets, or [L] for one shared gain.
     routing: optional (idx, g) from one of this oracle's own alternative routings.
+    ffn_pre_gain / ffn_post_gain / gate: the feed-forward sublayer's pre-norm, post-norm
+    and residual gate around the block; x is then the residual stream and out its next
+    value: xn = centred(x), f = block(xn), fn = input-scaled(f), out = alpha x + beta fn.
+    xn_round="bf16" rounds xn to bfloat16 before the router and the pooler read it, as the
+    pages' implementation stores it (the routing decision is then taken on the same values
+    the bfloat16 kernels see).
 
-    Returns every intermediate: logits, keys, idx, g, z, y [T,k,L], ss [T,k], n, c, out.
+    Returns every intermediate: xn, logits, keys, idx, g, z, y [T,k,L], ss [T,k], n, c,
+    f (the block's output), out.
     """
     T = x.shape[0]
+    x_res = x
+    if ffn_pre_gain is not None:
+        x = centred_rmsnorm(x, ffn_pre_gain, ffn_pre_eps)
+        if xn_round == "bf16":
+            x = round_bf16(x)
+    xn = x
     logits = router_logits(x, W_router)                                  # (a1)
     idx, g, keys = route(logits, k, router_bias, router_mode, logit_scale, routed_scaling)
     if routing is not None:
@@ -241,10 +290,13 @@ def latent_moe_forward(x: Array, W_router: Array, W_pool: Array, experts: Expert
     else:
         raise ValueError(norm_mode)
     c = combine(n, g)                                                    # (a9)
-    out = unpooler(c, W_unpool)                                          # (a10)
+    f = unpooler(c, W_unpool)                                            # (a10)
     ss = np.sum(y * y, axis=-1)
-    return {"logits": logits, "keys": keys, "idx": idx, "g": g, "z": z, "y": y, "ss": ss,
-            "n": n, "c": c, "out": out}
+    out = f if ffn_post_gain is None else input_scaled_rmsnorm(f, ffn_post_gain, ffn_post_eps)
+    if gate is not None:
+        out = residual_gate(x_res, out, gate, gate_temperature, gate_floor)
+    return {"xn": xn, "logits": logits, "keys": keys, "idx": idx, "g": g, "z": z, "y": y, "ss": ss,
+            "n": n, "c": c, "f": f, "out": out}
 
 
 # ---------------------------------------------------------------------------------------

@@ -94,6 +94,11 @@ def oracle_block(w: W.Workload, inp: Dict[str, torch.Tensor], rows: np.ndarray, 
     bias = host(inp["router_bias"]) if "router_bias" in inp else None
     if "pre_norm_gain" in inp:
         kw = dict(kw, pre_norm_gain=host(inp["pre_norm_gain"]))
+    for name, key in (("ffn_pre_gain", "ffn_pre_gain"), ("ffn_post_gain", "ffn_post_gain"), ("residual_gate", "gate")):
+        if name in inp:
+            kw = dict(kw, **{key: host(inp[name])})
+    if "ffn_pre_gain" in inp and w.dtype == "bf16":
+        kw = dict(kw, xn_round="bf16")
     return oracle.latent_moe_forward(x, host(inp["W_router"]), host(inp["W_pool"]), expert_source(inp),
                                      host(inp["gamma"]), host(inp["W_unpool"]), w.k, w.eps, router_bias=bias,
                                      **kw)

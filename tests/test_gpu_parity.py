@@ -136,6 +136,49 @@ def test_cuda_graph_replay_matches_eager(case):
     del graph
 
 
+# ------------------------------------------------- feed-forward sublayer around the block
+SUBLAYER = [
+    # name, T, D, L, I, E, k, dtype, steps (pre-norm, post-norm, residual gate)
+    ("sublayer_all_mid", 256, 2048, 1024, 1024, 64, 4, "bf16", ("pre", "post", "gate")),
+    ("sublayer_pre_only", 64, 1024, 512, 512, 16, 2, "bf16", ("pre",)),
+    ("sublayer_post_gate", 64, 1024, 512, 512, 16, 2, "bf16", ("post", "gate")),
+    ("sublayer_gate_only", 48, 1024, 512, 512, 16, 2, "bf16", ("gate",)),
+    ("sublayer_all_f32", 37, 256, 256, 128, 8, 3, "f32", ("pre", "post", "gate")),
+    # the unpooler on CTA pairs (>= one wave of 256 x 256 tiles) with the squares epilogue
+    ("sublayer_all_pair_unpooler", 1280, 4096, 512, 512, 8, 2, "bf16", ("pre", "post", "gate")),
+]
+SUBLAYER_KEYS = {"pre": "ffn_pre_gain", "post": "ffn_post_gain", "gate": "residual_gate"}
+
+
+@pytest.mark.parametrize("case", SUBLAYER, ids=[c[0] for c in SUBLAYER])
+def test_feedforward_sublayer(case):
+    name, T, D, L, I, E, k, dt, steps = case
+    w = W.Workload(name, T=T, D=D, L=L, I=I, E=E, k=k, dtype=dt, seed=5)
+    inp = W.make_inputs(w, "cuda")
+    sub = W.sublayer_inputs(w, "cuda")
+    for st in steps:
+        inp[SUBLAYER_KEYS[st]] = sub[SUBLAYER_KEYS[st]]
+    run = Run(w, inp)
+    ref, alts = full_check(w, inp, run)
+    cfg = run.model.config(T, run.model.workspace)
+    n_launch = moe.launch_count(cfg)
+    assert n_launch == 11 + ("pre" in steps) + ("post" in steps or "gate" in steps)
+    names = moe.stages(cfg)
+    assert len(names) == n_launch
+    if "pre" in steps:
+        assert names[0] == "ffn_pre_norm"
+        xn = host(run.inter("xn", run.act(), (T, D)))
+        assert_close(xn, ref["xn"], "xn", rel=5e-3, max_abs_rms=2e-2)
+    # every stage event is recorded once per launch, in order
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(n_launch + 1)]
+    for e in ev:
+        e.record()
+    out2 = run.model(inp["x"], stage_events=moe.event_handles(ev))
+    torch.cuda.synchronize()
+    assert torch.equal(out2, run.out)
+    assert all(ev[i].elapsed_time(ev[i + 1]) >= 0.0 for i in range(n_launch))
+
+
 # ------------------------------------------------------------------------- edge cases
 EDGE = [
     # name, T, D, L, I, E, k, dtype, bias_kind

@@ -374,3 +374,108 @@ def test_nvfp4_bytes_per_weight():
     assert oracle.NVFP4_BYTES_PER_WEIGHT == 0.5625
     out, k = 64, 256
     assert (out * k // 2 + out * k // 16) / (out * k) == 0.5625
+
+
+# ----------------------------------------------- feed-forward sublayer around the block
+def _decimals(s):
+    return len(s.split(".")[1]) if "." in s else 0
+
+
+def test_residual_gate_table():
+    """Every row of the gate table (deep dive §5.2): beta, alpha, alpha^2 + beta^2 and the
+    rotation angle, each to one unit in its last printed digit."""
+    rows = list(lines("residual_gate.txt"))
+    assert len(rows) == 5
+    for s in rows:
+        f = s.split()
+        g = float(f[0])
+        alpha, beta = oracle.residual_gate_coefficients(np.array([g]))
+        got = [beta[0], alpha[0], alpha[0] ** 2 + beta[0] ** 2, math.degrees(math.atan2(beta[0], alpha[0]))]
+        for printed, v in zip(f[1:], got):
+            assert abs(v - float(printed)) <= 10.0 ** -_decimals(printed), (g, printed, v)
+
+
+def test_residual_gate_four_channel_example():
+    x = np.array([1.0, -1.0, 1.0, -1.0])
+    f = np.array([1.0, 1.0, -1.0, -1.0])
+    for s in lines("residual_gate_example.txt"):
+        v = floats(s)
+        out = oracle.residual_gate(x, f, np.full(4, v[0]))
+        np.testing.assert_allclose(out, v[1:5], atol=1e-3)
+        assert abs(math.sqrt(np.mean(out * out)) - v[5]) <= 1e-3
+    # plain addition leaves the unit circle (RMS 1.414 on the page)
+    assert abs(math.sqrt(np.mean((x + f) ** 2)) - 1.414) <= 1e-3
+
+
+def test_residual_gate_floor_and_norm_preservation():
+    """alpha^2 + beta^2 = 1 exactly while the floor is inactive, which the page places at
+    beta > 0.9995, i.e. g > 2.28; above it alpha stays sqrt(1e-3) and the sum tends to
+    1.001. A gate of unit-RMS orthogonal inputs keeps RMS 1 (deep dive §5.2)."""
+    g = np.linspace(-6.0, 2.27, 2001)
+    a, b = oracle.residual_gate_coefficients(g)
+    np.testing.assert_allclose(a * a + b * b, 1.0, rtol=0, atol=1e-13)
+    a, b = oracle.residual_gate_coefficients(np.array([2.29, 5.0, 40.0]))
+    np.testing.assert_allclose(a, math.sqrt(1e-3), rtol=1e-13)
+    assert np.all(a * a + b * b > 1.0) and abs(a[-1] ** 2 + b[-1] ** 2 - 1.001) < 1e-12
+    # threshold where sigmoid(-w)(1 + sigmoid(w)) = 1e-3, to the page's two decimals
+    thr = 0.3 * math.log(math.sqrt(0.999) / (1.0 - math.sqrt(0.999)))
+    assert round(thr, 2) == 2.28
+    # a beta of 0.5 sits at g = 0, and beta -> 0 passes the residual stream unchanged
+    assert oracle.residual_gate_coefficients(np.array([0.0]))[1][0] == 0.5
+    x = RNG.normal(size=64)
+    np.testing.assert_allclose(oracle.residual_gate(x, RNG.normal(size=64), np.full(64, -30.0)), x, atol=1e-12)
+    # rotation: orthogonal unit-RMS x and f (Hadamard rows) keep RMS 1 for any gate value
+    # shared by the channels (the page's example); the cross terms cancel over channels
+    h = np.array([[1, 1, 1, 1], [1, -1, 1, -1], [1, 1, -1, -1], [1, -1, -1, 1]], dtype=float)
+    for gv in RNG.uniform(-2.0, 2.2, size=20):
+        for i, j in ((1, 2), (0, 3), (2, 3)):
+            out = oracle.residual_gate(h[i], h[j], np.full(4, gv))
+            assert abs(np.mean(out * out) - 1.0) < 1e-13
+
+
+def test_sublayer_pre_norm_makes_the_block_scale_invariant():
+    """With the centred pre-norm (gain 0, eps 0) the block sees x / rms(x), so scaling the
+    residual stream leaves the branch output unchanged; without it the output is not."""
+    b = _random_block(T=9)
+    kw = dict(ffn_pre_gain=np.zeros(b["x"].shape[1]), ffn_pre_eps=0.0)
+    ref = _fwd(b, k=2, **kw)
+    got = _fwd(dict(b, x=3.7 * b["x"]), k=2, **kw)
+    np.testing.assert_allclose(got["f"], ref["f"], rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(np.sqrt(np.mean(ref["xn"] ** 2, axis=1)), 1.0, atol=1e-12)
+    assert not np.allclose(_fwd(dict(b, x=3.7 * b["x"]), k=2)["out"], _fwd(b, k=2)["out"])
+
+
+def test_sublayer_post_norm_and_gate():
+    """The post-norm branch has RMS sqrt(ms / (ms + eps)) whatever the block computed (the
+    page's unit-RMS write, §5.3), its direction is f * (1 + w); a gate of beta -> 0 returns
+    the residual stream and of beta -> 1 (floor off) the normalised branch."""
+    b = _random_block(T=7)
+    D = b["x"].shape[1]
+    w = RNG.normal(size=D) * 0.3
+    r = _fwd(b, k=2, ffn_post_gain=w, ffn_post_eps=1e-8)
+    v = r["f"] * (1 + w)
+    ms = np.mean(v * v, axis=1)
+    np.testing.assert_allclose(np.sqrt(np.mean(r["out"] ** 2, axis=1)), np.sqrt(ms / (ms + 1e-8)), rtol=1e-12)
+    cos = np.sum(r["out"] * v, axis=1) / np.linalg.norm(r["out"], axis=1) / np.linalg.norm(v, axis=1)
+    np.testing.assert_allclose(cos, 1.0, atol=1e-12)
+    low = _fwd(b, k=2, ffn_post_gain=w, gate=np.full(D, -40.0))
+    np.testing.assert_allclose(low["out"], b["x"], atol=1e-12)
+    # g = 12: beta = 1 - 4e-18, alpha = 2.9e-9 once the floor is switched off
+    high = _fwd(b, k=2, ffn_post_gain=w, gate=np.full(D, 12.0), gate_floor=0.0)
+    np.testing.assert_allclose(high["out"], r["out"], atol=1e-7)
+
+
+def test_round_bf16_against_torch_and_ties():
+    """Nearest bfloat16, ties to even: equal to torch's float32 -> bfloat16 conversion on
+    float32 inputs, and the hand cases of the 8-bit significand."""
+    import torch
+    v = RNG.normal(size=20000) * np.exp(RNG.uniform(-20, 20, size=20000))
+    v32 = v.astype(np.float32).astype(np.float64)
+    ref = torch.from_numpy(v32).to(torch.float32).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(oracle.round_bf16(v32), ref)
+    # 1 + 2^-8 is halfway between 1 and 1 + 2^-7: ties to the even significand (1)
+    assert oracle.round_bf16(1.0 + 2.0 ** -8) == 1.0
+    # 1 + 3 * 2^-8 is halfway between 1 + 2^-7 and 1 + 2^-6: ties to 1 + 2^-6
+    assert oracle.round_bf16(1.0 + 3 * 2.0 ** -8) == 1.0 + 2.0 ** -6
+    assert oracle.round_bf16(1.0 + 2.0 ** -8 + 2.0 ** -30) == 1.0 + 2.0 ** -7
+    assert oracle.round_bf16(-3.0) == -3.0 and oracle.round_bf16(0.0) == 0.0

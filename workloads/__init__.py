@@ -183,6 +183,24 @@ def expert_slab(w: Workload, name: str, e: int, device="cpu",
     return fill(t, w.seed, TID[name], stddev(w, name), start=e * per)
 
 
+SUBLAYER_TID = {"ffn_pre_gain": 12, "ffn_post_gain": 13, "residual_gate": 14}
+
+
+def sublayer_inputs(w: Workload, device="cpu") -> Dict[str, torch.Tensor]:
+    """Parameters of the feed-forward sublayer around the block: the pre- and post-norm
+    gain offsets [D] ~ N(0, 0.1) (variance, like gamma) in the workload dtype, and the
+    residual gate's parameters g [D] ~ N(0, 1) in float32 -- wider than the N(0, 0.02^2)
+    initialisation the pages quote, so that beta spans (0, 1) and some channels reach
+    the alpha^2 floor (g > 2.28)."""
+    out = {}
+    for n in ("ffn_pre_gain", "ffn_post_gain"):
+        t = torch.empty((w.D,), dtype=TORCH_DTYPE[w.dtype], device=device)
+        out[n] = fill(t, w.seed, SUBLAYER_TID[n], math.sqrt(0.1))
+    g = torch.empty((w.D,), dtype=torch.float32, device=device)
+    out["residual_gate"] = fill(g, w.seed, SUBLAYER_TID["residual_gate"], 1.0)
+    return out
+
+
 def make_inputs(w: Workload, device="cpu", names=None) -> Dict[str, torch.Tensor]:
     """The workload's tensors. For NVFP4 experts, W_gate / W_up / W_down are replaced by
     <name>_codes, <name>_scales and <name>_mscale (see quantize_nvfp4), each expert
