@@ -17,7 +17,9 @@ Timing: W untimed warm-up steps, then K steps between CUDA events on the launchi
 stream, with a barrier and a device synchronisation on both sides. Every step streams
 the expert weights (25.8 GB >> 126 MB L2), so inputs are larger than L2 and no flush is
 needed. Per-kernel durations come from events the library records between its launches.
-Decode workloads are also timed as replays of one CUDA graph of the forward
+The side line "prefill_sublayer" runs the same layer inside its feed-forward sublayer
+(pre-norm, block, post-norm, residual gate). Decode workloads are also timed as replays
+of one CUDA graph of the forward
 ("graph_replay"), which takes the host's per-launch work out of the step.
 """
 from __future__ import annotations
@@ -124,6 +126,11 @@ def stage_work(w: W.Workload, n_touched: int):
         "down_sumsq": (2 * A * I * L, n_touched * L * I * ab + A * I * a + A * L * a + A * (L // 32) * 4),
         "norm_combine": (0, A * L * a + A * (L // 32) * 4 + T * L * a + n_touched * L * a),
         "unpooler": (2 * T * D * L, T * L * a + D * L * a + T * D * a),
+        # optional steps: pre-expert norm on z; the feed-forward sublayer's pre-norm on x
+        # and post-norm + residual gate (out, x, partial sums, gains, gate parameters)
+        "pre_expert_norm": (0, 2 * T * L * a + L * a),
+        "ffn_pre_norm": (0, 2 * T * D * a + D * a),
+        "ffn_post_norm_gate": (0, 3 * T * D * a + T * (D // 32) * 4 + D * (a + 4)),
     }
 
 
@@ -197,7 +204,8 @@ def run_ours(w: W.Workload, inp, steps: int, warmup: int, rank: int, world: int,
     model = moe.LatentMoE(weights, T_max=w.T, k=w.k, eps=w.eps)
     out = torch.empty((w.T, w.D), dtype=inp["x"].dtype, device=dev)
     idx = torch.empty((w.T, w.k), dtype=torch.int32, device=dev)
-    nst = len(moe.STAGES)
+    stage_names = moe.stages(model.config(w.T))
+    nst = len(stage_names)
     stream = torch.cuda.current_stream()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)] for _ in range(steps)]
     for row in ev:
@@ -237,7 +245,7 @@ def run_ours(w: W.Workload, inp, steps: int, warmup: int, rank: int, world: int,
     n_touched = int(torch.unique(idx).numel())
     work = stage_work(w, n_touched)
     dom = max(range(nst), key=lambda i: stage_ms[i])
-    dname = moe.STAGES[dom]
+    dname = stage_names[dom]
     fl, by = work[dname]
     t_dom = stage_ms[dom] * 1e-3
     t_tensor = fl / (peaks["bf16_tflops_sustained"] * 1e12)
@@ -260,7 +268,7 @@ def run_ours(w: W.Workload, inp, steps: int, warmup: int, rank: int, world: int,
     res = {
         "value": job_tokens_per_s(world, w.T, steps, ms_max),
         "ms_per_step": ms_max / steps,
-        "stage_ms": {moe.STAGES[i]: round(stage_ms[i], 4) for i in range(nst)},
+        "stage_ms": {stage_names[i]: round(stage_ms[i], 4) for i in range(nst)},
         "roofline": roof,
         "step": {"tflops": sf / t_step / 1e12, "gbs": sb / t_step / 1e9, "roofline_ms": step_roof * 1e3,
                  "frac_of_step_roofline": step_roof / t_step, "distinct_experts": n_touched},
@@ -467,6 +475,10 @@ def main():
             inp_z = dict(inp, router_bias=W.zipf_router_bias(wz).to(dev))
             side["prefill_zipf"] = run_ours(wz, inp_z, args.steps, args.warmup, rank, world, peaks, peak_kind,
                                             False, e2e_steps=0)
+            # the whole feed-forward sublayer: pre-norm, the block, post-norm, residual gate
+            inp_s = dict(inp, **W.sublayer_inputs(w, dev))
+            side["prefill_sublayer"] = run_ours(w, inp_s, args.steps, args.warmup, rank, world, peaks, peak_kind,
+                                                False, e2e_steps=0)
             if not args.no_nvfp4:
                 # NVFP4 experts (quantised from the same bf16 weights): T=4096 and a T=64 decode
                 wq = W.WORKLOADS["nvfp4"]

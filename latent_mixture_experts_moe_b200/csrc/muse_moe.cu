@@ -552,10 +552,13 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
   MUSE_CK(mark());
   // feed-forward sublayer post-norm and residual gate (optional), in place on out
   if (post || c.residual_gate != nullptr) {
-    k_ffn_finish<T><<<static_cast<unsigned>(Tn), 256, 0, st>>>(
+    const int vec = 16 / static_cast<int>(sizeof(T));
+    const dim3 grid(static_cast<unsigned>(cdiv(Tn, kFinishRows)),
+                    static_cast<unsigned>(cdiv(D, static_cast<int64_t>(kFinishThreads) * vec)));
+    k_ffn_finish<T><<<grid, kFinishThreads, 0, st>>>(
         reinterpret_cast<T*>(out), reinterpret_cast<const T*>(x), reinterpret_cast<const float*>(at(lay.pub.ss_out)),
         static_cast<int>(D / 32), reinterpret_cast<const T*>(c.ffn_post_gain), c.ffn_post_eps, c.residual_gate,
-        1.0f / c.residual_gate_temperature, c.residual_gate_eps, static_cast<int>(D));
+        1.0f / c.residual_gate_temperature, c.residual_gate_eps, static_cast<int>(D), static_cast<int>(Tn));
     MUSE_CK(cudaGetLastError());
     MUSE_CK(mark());
   }

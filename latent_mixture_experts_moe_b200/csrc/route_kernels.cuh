@@ -290,56 +290,94 @@ __global__ void k_rmsnorm_rows(const T* in, T* out, const T* __restrict__ w, int
 
 // --------------------------------------------------------------------------------------
 // Feed-forward sublayer, after the unpooler (deep dive §2.1 step 7, §5.2, §5.3), in place
-// on out = f, one block per token:
+// on out = f; a block covers kFinishRows tokens x kFinishThreads vectors of channels, so
+// each thread computes its channels' gate coefficients once for many tokens:
 //   post norm (post_gain != NULL): v = f * (1 + w), fn = v / sqrt(mean(v^2) + post_eps),
 //     mean(v^2) from the unpooler epilogue's partial sums ss[t, 0 .. D/32) of squares of
 //     the FP32 accumulator times (1 + w), the scale applied to the stored f;
 //   residual gate (gate != NULL): out = alpha * x + beta * fn, beta = sigmoid(g / T),
 //     alpha = sqrt(max(sigmoid(-g / T) * (1 + beta), gate_eps)), coefficients in FP32.
 // --------------------------------------------------------------------------------------
+constexpr int kFinishRows = 32;     // tokens per block
+constexpr int kFinishThreads = 256;  // one 16-byte vector of channels per thread
+
 template <typename T>
-__global__ void k_ffn_finish(T* __restrict__ out, const T* __restrict__ x, const float* __restrict__ ss, int ss_ld,
-                             const T* __restrict__ post_gain, float post_eps, const float* __restrict__ gate,
-                             float inv_temp, float gate_eps, int D) {
+__global__ void __launch_bounds__(kFinishThreads) k_ffn_finish(
+    T* __restrict__ out, const T* __restrict__ x, const float* __restrict__ ss, int ss_ld,
+    const T* __restrict__ post_gain, float post_eps, const float* __restrict__ gate, float inv_temp,
+    float gate_eps, int D, int T_rows) {
   constexpr int VEC = 16 / sizeof(T);
-  __shared__ float part[32];
-  const int64_t t = blockIdx.x;
-  float scale = 1.0f;
-  if (post_gain != nullptr) {  // uniform over the grid
-    float s = 0.0f;
-    for (int i = threadIdx.x; i < ss_ld; i += blockDim.x) s += ss[t * ss_ld + i];
-    scale = 1.0f / sqrtf(block_sum(s, part) / static_cast<float>(D) + post_eps);
-  }
-  T* orow = out + t * D;
-  const T* xrow = x + t * D;
-  for (int c = threadIdx.x * VEC; c < D; c += blockDim.x * VEC) {
-    const uint4 fv4 = *reinterpret_cast<const uint4*>(orow + c);
-    const T* fv = reinterpret_cast<const T*>(&fv4);
-    float f[VEC];
-#pragma unroll
-    for (int i = 0; i < VEC; ++i) f[i] = to_f32(fv[i]);
+  __shared__ float scale_s[kFinishRows];
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kFinishRows;  // x: token blocks (up to 2^31 - 1)
+  const int rows = min(kFinishRows, T_rows - static_cast<int>(t0));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // post-norm scale of each of the block's tokens: one warp per token, fixed order
+  for (int r = warp; r < rows; r += kFinishThreads / 32) {
+    float sc = 1.0f;
     if (post_gain != nullptr) {
-      const uint4 gv4 = *reinterpret_cast<const uint4*>(post_gain + c);
-      const T* gv = reinterpret_cast<const T*>(&gv4);
-#pragma unroll
-      for (int i = 0; i < VEC; ++i) f[i] = f[i] * (1.0f + to_f32(gv[i])) * scale;
+      float s = 0.0f;
+      for (int i = lane; i < ss_ld; i += 32) s += ss[(t0 + r) * ss_ld + i];
+      sc = 1.0f / sqrtf(warp_sum(s) / static_cast<float>(D) + post_eps);
     }
-    if (gate != nullptr) {
-      const uint4 xv4 = *reinterpret_cast<const uint4*>(xrow + c);
-      const T* xv = reinterpret_cast<const T*>(&xv4);
+    if (lane == 0) scale_s[r] = sc;
+  }
+  __syncthreads();
+  const int c = (blockIdx.y * kFinishThreads + threadIdx.x) * VEC;  // y: channel slices
+  if (c >= D) return;
+  // this thread's channels: gain and gate coefficients, once for all rows
+  float gain[VEC], alpha[VEC], beta[VEC];
 #pragma unroll
-      for (int i = 0; i < VEC; ++i) {
-        const float wg = gate[c + i] * inv_temp;
-        const float beta = 1.0f / (1.0f + expf(-wg));
-        const float alpha = sqrtf(fmaxf((1.0f / (1.0f + expf(wg))) * (1.0f + beta), gate_eps));
-        f[i] = alpha * to_f32(xv[i]) + beta * f[i];
+  for (int i = 0; i < VEC; ++i) {
+    gain[i] = 1.0f;
+    alpha[i] = 0.0f;
+    beta[i] = 1.0f;
+  }
+  if (post_gain != nullptr) {
+    const uint4 gv4 = *reinterpret_cast<const uint4*>(post_gain + c);
+    const T* gv = reinterpret_cast<const T*>(&gv4);
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) gain[i] = 1.0f + to_f32(gv[i]);
+  }
+  if (gate != nullptr) {
+#pragma unroll
+    for (int i = 0; i < VEC; i += 4) {
+      const float4 g4 = *reinterpret_cast<const float4*>(gate + c + i);
+      const float gg[4] = {g4.x, g4.y, g4.z, g4.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float wg = gg[j] * inv_temp;
+        beta[i + j] = 1.0f / (1.0f + expf(-wg));
+        alpha[i + j] = sqrtf(fmaxf((1.0f / (1.0f + expf(wg))) * (1.0f + beta[i + j]), gate_eps));
       }
     }
-    uint4 ov;
-    T* oo = reinterpret_cast<T*>(&ov);
+  }
+  // rows four at a time: loads first, then arithmetic and stores
+  for (int r0 = 0; r0 < rows; r0 += 4) {
+    uint4 fv4[4], xv4[4];
 #pragma unroll
-    for (int i = 0; i < VEC; ++i) oo[i] = from_f32<T>(f[i]);
-    *reinterpret_cast<uint4*>(orow + c) = ov;
+    for (int j = 0; j < 4; ++j) {
+      fv4[j] = make_uint4(0, 0, 0, 0);
+      xv4[j] = make_uint4(0, 0, 0, 0);
+      if (r0 + j < rows) {
+        fv4[j] = *reinterpret_cast<const uint4*>(out + (t0 + r0 + j) * D + c);
+        if (gate != nullptr) xv4[j] = *reinterpret_cast<const uint4*>(x + (t0 + r0 + j) * D + c);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (r0 + j >= rows) break;
+      const T* fv = reinterpret_cast<const T*>(&fv4[j]);
+      const T* xv = reinterpret_cast<const T*>(&xv4[j]);
+      const float sc = scale_s[r0 + j];
+      uint4 ov;
+      T* oo = reinterpret_cast<T*>(&ov);
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) {
+        const float f = to_f32(fv[i]) * gain[i] * sc;
+        oo[i] = from_f32<T>(gate != nullptr ? alpha[i] * to_f32(xv[i]) + beta[i] * f : f);
+      }
+      *reinterpret_cast<uint4*>(out + (t0 + r0 + j) * D + c) = ov;
+    }
   }
 }
 
