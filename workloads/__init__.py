@@ -183,7 +183,7 @@ def expert_slab(w: Workload, name: str, e: int, device="cpu",
     return fill(t, w.seed, TID[name], stddev(w, name), start=e * per)
 
 
-SUBLAYER_TID = {"ffn_pre_gain": 12, "ffn_post_gain": 13, "residual_gate": 14}
+SUBLAYER_TID = {"ffn_pre_gain": 13, "ffn_post_gain": 14, "residual_gate": 15}
 
 
 def sublayer_inputs(w: Workload, device="cpu") -> Dict[str, torch.Tensor]:
