@@ -50,7 +50,7 @@ __all__ = [
     "topk_alternatives", "pooler", "silu", "expert_ffn", "centred_rmsnorm",
     "input_scaled_rmsnorm", "combine", "unpooler", "latent_moe_forward", "as_f64",
     "moe_flops_per_token", "expert_param_count", "residual_gate_coefficients", "residual_gate",
-    "round_bf16",
+    "round_bf16", "nvfp4_activation",
 ]
 
 Array = np.ndarray
@@ -168,12 +168,27 @@ def silu(a: Array) -> Array:
     return a * _sigmoid(a)
 
 
-def expert_ffn(z: Array, W_gate: Array, W_up: Array, W_down: Array) -> Array:
-    """Rows of z [n, L] through one expert; W_gate/W_up [I, L], W_down [L, I]."""
+def expert_ffn(z: Array, W_gate: Array, W_up: Array, W_down: Array,
+               act: Optional[Callable[[Array], Array]] = None) -> Array:
+    """Rows of z [n, L] through one expert; W_gate/W_up [I, L], W_down [L, I]. act, when
+    given, maps each GEMM's activation operand (z, then the SwiGLU output h) to the values
+    the GEMM multiplies (the W4A4 mode's quantise-dequantise)."""
+    if act is not None:
+        z = act(z)
     a = z @ W_gate.T
     u = z @ W_up.T
     h = silu(a) * u
+    if act is not None:
+        h = act(h)
     return h @ W_down.T
+
+
+def nvfp4_activation(v: Array) -> Array:
+    """W4A4 operand of an expert GEMM: the activation as the kernels store it (bfloat16),
+    quantised per 16 to E2M1 codes with E4M3 scales, and dequantised (oracle.nvfp4)."""
+    from .nvfp4 import dequantize_activations_nvfp4, quantize_activations_nvfp4
+    codes, scales = quantize_activations_nvfp4(round_bf16(v))
+    return dequantize_activations_nvfp4(codes, scales)
 
 
 # ---------------------------------------------------------------------------------------
@@ -244,7 +259,7 @@ def latent_moe_forward(x: Array, W_router: Array, W_pool: Array, experts: Expert
                        ffn_pre_gain: Optional[Array] = None, ffn_pre_eps: float = 1e-5,
                        ffn_post_gain: Optional[Array] = None, ffn_post_eps: float = 1e-8,
                        gate: Optional[Array] = None, gate_temperature: float = 0.3, gate_floor: float = 1e-3,
-                       xn_round: Optional[str] = None) -> Dict[str, Array]:
+                       xn_round: Optional[str] = None, act_format: str = "bf16") -> Dict[str, Array]:
     """Forward pass of the latent-MoE block for every row of x, in float64.
 
     experts: (W_gate [E,I,L], W_up [E,I,L], W_down [E,L,I]) or a callable e -> the three
@@ -256,7 +271,8 @@ def latent_moe_forward(x: Array, W_router: Array, W_pool: Array, experts: Expert
     value: xn = centred(x), f = block(xn), fn = input-scaled(f), out = alpha x + beta fn.
     xn_round="bf16" rounds xn to bfloat16 before the router and the pooler read it, as the
     pages' implementation stores it (the routing decision is then taken on the same values
-    the bfloat16 kernels see).
+    the bfloat16 kernels see). act_format="nvfp4" runs the expert GEMMs W4A4: their
+    activation operands (z rows, SwiGLU outputs) go through nvfp4_activation.
 
     Returns every intermediate: xn, logits, keys, idx, g, z, y [T,k,L], ss [T,k], n, c,
     f (the block's output), out.
@@ -281,7 +297,8 @@ def latent_moe_forward(x: Array, W_router: Array, W_pool: Array, experts: Expert
     for e in np.unique(idx):                                             # (a3) dispatch
         tok, slot = np.nonzero(idx == e)
         Wg, Wu, Wd = get(int(e))
-        y[tok, slot, :] = expert_ffn(z[tok], as_f64(Wg), as_f64(Wu), as_f64(Wd))  # (a6, a7)
+        act = nvfp4_activation if act_format == "nvfp4" else None
+        y[tok, slot, :] = expert_ffn(z[tok], as_f64(Wg), as_f64(Wu), as_f64(Wd), act)  # (a6, a7)
     gam = gamma[idx] if gamma.ndim == 2 else np.broadcast_to(gamma, (T, k, L))
     if norm_mode == "centred":                                           # (a8)
         n = centred_rmsnorm(y, gam, eps)

@@ -1,4 +1,5 @@
-"""FP64 decoding of NVFP4 expert weights (test infrastructure, part of the oracle).
+"""FP64 decoding of NVFP4 expert weights and the NVFP4 activation quantiser (test
+infrastructure, part of the oracle).
 
 Storage, per expert matrix W[e] of shape [out, in] (Muse Spark Open deep dive, §7.3 bytes
 bullet and §7.4 NVFP4 paragraph: 4-bit values, one FP8 E4M3 scale per 16 weights,
@@ -14,12 +15,21 @@ The 4-bit value is FP4 E2M1 of the OCP Microscaling (MX) formats specification v
 or NaN. E4M3 (deep dive §7.4: 4 exponent bits, 3 mantissa bits) is the OCP 8-bit float of
 the same specification: bias 7, subnormal when the exponent is 0, S.1111.111 is NaN, no
 infinities, largest value 448.
+
+Activations of the W4A4 mode (deep dive §7.4: the released checkpoint quantises both
+operands of the expert GEMMs) use the same element and block formats without a tensor
+scale: per block of 16 consecutive values of a row, scale = E4M3(amax / 6) and code =
+E2M1(value / scale), both rounded to nearest with ties to even, E2M1 saturating at 6. The
+arithmetic is single precision, as the kernels do it (the rounding decisions are then taken
+in the same precision on both sides): amax and value / scale are float32 operations on the
+float32 value of the stored bfloat16 activation.
 """
 from __future__ import annotations
 
 import numpy as np
 
-__all__ = ["decode_e2m1", "decode_e4m3", "unpack_nibbles", "dequantize_nvfp4", "NVFP4_BYTES_PER_WEIGHT"]
+__all__ = ["decode_e2m1", "decode_e4m3", "unpack_nibbles", "dequantize_nvfp4", "NVFP4_BYTES_PER_WEIGHT",
+           "round_e4m3", "round_e2m1", "quantize_activations_nvfp4", "dequantize_activations_nvfp4"]
 
 # 4 bits per value plus one byte per 16 values
 NVFP4_BYTES_PER_WEIGHT = 0.5 + 1.0 / 16.0
@@ -60,3 +70,55 @@ def dequantize_nvfp4(codes, scales, matrix_scale) -> np.ndarray:
     vals = decode_e2m1(unpack_nibbles(codes))
     blk = np.repeat(decode_e4m3(scales), 16, axis=-1)
     return vals * blk * float(matrix_scale)
+
+
+# the 127 finite non-negative E4M3 values in byte order (bytes 0x00 .. 0x7E), increasing
+_E4M3_POS = decode_e4m3(np.arange(127))
+# the 8 E2M1 magnitudes in code order (codes 0 .. 7), increasing
+_E2M1_POS = decode_e2m1(np.arange(8))
+
+
+def _nearest_even(table: np.ndarray, v: np.ndarray) -> np.ndarray:
+    """Index of the entry of the increasing table nearest to each v >= 0 (ties to the
+    even index, values past the end to the last entry)."""
+    v = np.asarray(v, dtype=np.float64)
+    hi = np.clip(np.searchsorted(table, v, side="left"), 1, len(table) - 1)
+    lo = hi - 1
+    dl, dh = v - table[lo], table[hi] - v
+    pick = np.where(dl < dh, lo, np.where(dh < dl, hi, np.where(lo % 2 == 0, lo, hi)))
+    return np.where(v >= table[-1], len(table) - 1, pick)
+
+
+def round_e4m3(v) -> np.ndarray:
+    """E4M3 byte nearest to each non-negative value (ties to even, saturating at 448)."""
+    return _nearest_even(_E4M3_POS, v).astype(np.uint8)
+
+
+def round_e2m1(q) -> np.ndarray:
+    """4-bit E2M1 code nearest to each value (ties to even, saturating at +-6); the sign
+    bit is set only for a negative value whose magnitude code is not 0."""
+    q = np.asarray(q, dtype=np.float64)
+    mag = _nearest_even(_E2M1_POS, np.abs(q)).astype(np.uint8)
+    return np.where((q < 0) & (mag > 0), mag | 8, mag).astype(np.uint8)
+
+
+def quantize_activations_nvfp4(x):
+    """Rows [..., n] (n a multiple of 16; values exactly representable in float32) ->
+    (codes uint8 [..., n/2] low nibble first, scales uint8 E4M3 [..., n/16])."""
+    x32 = np.asarray(x, dtype=np.float32)
+    blocks = x32.reshape(x32.shape[:-1] + (x32.shape[-1] // 16, 16))
+    amax = np.max(np.abs(blocks), axis=-1)                          # exact
+    s = (amax / np.float32(6.0)).astype(np.float32)                  # one float32 division
+    sbyte = round_e4m3(s.astype(np.float64))
+    sdec = decode_e4m3(sbyte).astype(np.float32)                     # exact in float32
+    with np.errstate(divide="ignore", invalid="ignore"):
+        q = np.where(sdec[..., None] > 0, blocks / sdec[..., None], np.float32(0.0)).astype(np.float32)
+    codes = round_e2m1(q.astype(np.float64)).reshape(x32.shape)
+    packed = (codes[..., 0::2] | (codes[..., 1::2] << 4)).astype(np.uint8)
+    return packed, sbyte
+
+
+def dequantize_activations_nvfp4(codes, scales) -> np.ndarray:
+    """FP64 values [..., n] of quantised activations."""
+    vals = decode_e2m1(unpack_nibbles(codes))
+    return vals * np.repeat(decode_e4m3(scales), 16, axis=-1)

@@ -479,3 +479,78 @@ def test_round_bf16_against_torch_and_ties():
     assert oracle.round_bf16(1.0 + 3 * 2.0 ** -8) == 1.0 + 2.0 ** -6
     assert oracle.round_bf16(1.0 + 2.0 ** -8 + 2.0 ** -30) == 1.0 + 2.0 ** -7
     assert oracle.round_bf16(-3.0) == -3.0 and oracle.round_bf16(0.0) == 0.0
+
+
+# ------------------------------------------------------------- NVFP4 activations (W4A4)
+def test_e2m1_rounding_table():
+    for s in lines("e2m1_rounding.txt"):
+        v, code = s.split()
+        assert int(oracle.round_e2m1(np.float32(float(v)).astype(np.float64))) == int(code), s
+
+
+def test_e2m1_rounding_is_nearest_with_ties_to_even():
+    """Brute force over random values: the code's value is the nearest E2M1 value, and at
+    an exact tie the code with mantissa bit 0 wins."""
+    ties = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    q = np.concatenate([RNG.uniform(-8, 8, 5000), ties, -ties])
+    codes = oracle.round_e2m1(q)
+    got = oracle.decode_e2m1(codes)
+    allv = oracle.decode_e2m1(np.arange(16))
+    for v, c, g in zip(q, codes, got):
+        d = np.abs(np.clip(v, -6, 6) - allv)
+        assert abs(np.clip(v, -6, 6) - g) <= d.min() + 1e-12
+        ties = np.nonzero(np.abs(d - d.min()) < 1e-12)[0]
+        if len(set(allv[ties])) > 1:
+            assert c & 1 == 0
+
+
+def test_round_e4m3_against_torch():
+    """Nearest E4M3 with ties to even equals torch's float32 -> float8_e4m3fn conversion for
+    every value in range, including all exact midpoints between neighbours."""
+    import torch
+    tab = oracle.decode_e4m3(np.arange(127))
+    mids = (tab[:-1] + tab[1:]) / 2
+    v = np.concatenate([RNG.uniform(0, 448, 20000), np.exp(RNG.uniform(-12, 6, 20000)), mids, tab]).astype(np.float32)
+    v = v[v <= 448]
+    ref = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(oracle.round_e4m3(v.astype(np.float64)), ref)
+    assert int(oracle.round_e4m3(np.array([1000.0]))[0]) == 0x7E          # saturates at 448
+
+
+def test_activation_quantiser_properties():
+    """Per block of 16: the scale is E4M3(amax / 6); the block's largest magnitude maps to
+    code 6 or 7 (4 or 6 times the scale); values already on the grid of a block come back
+    exactly; a zero block gives zero codes and scale; low nibble = even element."""
+    x = RNG.normal(size=(5, 64)).astype(np.float32)
+    codes, sc = oracle.quantize_activations_nvfp4(x)
+    assert codes.shape == (5, 32) and sc.shape == (5, 4)
+    amax = np.abs(x.reshape(5, 4, 16)).max(-1)
+    np.testing.assert_array_equal(sc, oracle.round_e4m3((amax / np.float32(6)).astype(np.float32).astype(np.float64)))
+    deq = oracle.dequantize_activations_nvfp4(codes, sc).reshape(5, 4, 16)
+    top = np.argmax(np.abs(x.reshape(5, 4, 16)), -1)
+    ratio = np.abs(np.take_along_axis(deq, top[..., None], -1)[..., 0]) / oracle.decode_e4m3(sc)
+    assert np.all((ratio == 4.0) | (ratio == 6.0))
+    # a block whose values are E2M1 values times an E4M3 scale of amax/6 round-trips exactly
+    grid = np.array([0, .5, 1, 1.5, 2, 3, 4, 6, -.5, -1, -1.5, -2, -3, -4, -6, 6], dtype=np.float32) * np.float32(0.375)
+    c2, s2 = oracle.quantize_activations_nvfp4(grid[None, :])
+    np.testing.assert_array_equal(oracle.dequantize_activations_nvfp4(c2, s2)[0], grid)
+    c3, s3 = oracle.quantize_activations_nvfp4(np.zeros((1, 16), np.float32))
+    assert not c3.any() and not s3.any()
+    c4, _ = oracle.quantize_activations_nvfp4(np.array([[6, -6] + [0] * 14], np.float32))
+    assert c4[0, 0] == 0x7 | (0xF << 4)
+
+
+def test_w4a4_expert_matches_dequantised_operands():
+    """The W4A4 expert equals the plain expert run on quantise-dequantised operands, and
+    its error against the unquantised expert is of the size 4-bit activations give."""
+    b = _random_block(T=6, D=32, L=32, I=48, E=3)
+    ref = _fwd(b, k=2)
+    got = _fwd(b, k=2, act_format="nvfp4")
+    rel = np.linalg.norm(got["y"] - ref["y"]) / np.linalg.norm(ref["y"])
+    assert 0.01 < rel < 0.3
+    z = b["x"] @ b["W_pool"].T
+    e = int(got["idx"][0, 0])
+    zq = oracle.nvfp4_activation(z[:1])
+    a = zq @ b["W_gate"][e].T
+    h = oracle.nvfp4_activation(a / (1 + np.exp(-a)) * (zq @ b["W_up"][e].T))
+    np.testing.assert_allclose(got["y"][0, 0], (h @ b["W_down"][e].T)[0], rtol=1e-12, atol=1e-12)
