@@ -131,16 +131,21 @@ def stage_work(w: W.Workload, n_touched: int):
         "pre_expert_norm": (0, 2 * T * L * a + L * a),
         "ffn_pre_norm": (0, 2 * T * D * a + D * a),
         "ffn_post_norm_gate": (0, 3 * T * D * a + T * (D // 32) * 4 + D * (a + 4)),
+        # W4A4: latent rows gathered and quantised (0.5625 B per value out), h quantised
+        "gather_quant": (0, T * L * a + A * L * 0.5625),
+        "quant_h": (0, A * I * a + A * I * 0.5625),
     }
 
 
 def step_work(w: W.Workload, n_touched: int):
+    """(FLOPs, bytes, the FLOPs that run on the FP4 tensor path) of one step."""
     T, D, L, I, E, k = w.T, w.D, w.L, w.I, w.E, w.k
     a = 2 if w.dtype == "bf16" else 4
     ab = 0.5625 if w.experts == "nvfp4" else a
     flops = 2 * T * (E * D + L * D + k * 3 * L * I + D * L)
     byts = 2 * T * D * a + (E * D + 2 * L * D) * a + n_touched * (3 * L * I * ab + L * a)
-    return flops, byts
+    fp4_flops = 2 * T * k * 3 * L * I if w.act == "nvfp4" else 0
+    return flops, byts, fp4_flops
 
 
 # ------------------------------------------------------------------------------ our arm
@@ -201,7 +206,8 @@ def run_ours(w: W.Workload, inp, steps: int, warmup: int, rank: int, world: int,
     import latent_mixture_experts_moe_b200 as moe
     dev = inp["x"].device
     weights = {k: v for k, v in inp.items() if k != "x"}
-    model = moe.LatentMoE(weights, T_max=w.T, k=w.k, eps=w.eps)
+    modes = {"act_format": moe.ACT_NVFP4} if w.act == "nvfp4" else {}
+    model = moe.LatentMoE(weights, T_max=w.T, k=w.k, eps=w.eps, **modes)
     out = torch.empty((w.T, w.D), dtype=inp["x"].dtype, device=dev)
     idx = torch.empty((w.T, w.k), dtype=torch.int32, device=dev)
     stage_names = moe.stages(model.config(w.T))
@@ -248,23 +254,29 @@ def run_ours(w: W.Workload, inp, steps: int, warmup: int, rank: int, world: int,
     dname = stage_names[dom]
     fl, by = work[dname]
     t_dom = stage_ms[dom] * 1e-3
-    t_tensor = fl / (peaks["bf16_tflops_sustained"] * 1e12)
+    # W4A4 expert GEMMs run on the FP4 tensor path: its peak is the measured bf16 peak times
+    # the nominal dense FP4 / BF16 ratio (9 / 2.25 PFLOP/s)
+    fp4_gemm = w.act == "nvfp4" and dname in ("gate_up_swiglu", "down_sumsq")
+    ratio = 4.0 if fp4_gemm else 1.0
+    t_tensor = fl / (ratio * peaks["bf16_tflops_sustained"] * 1e12)
     t_hbm = by / (peaks["hbm_gbs"] * 1e9)
     if t_tensor >= t_hbm:
-        roof = {"bound": "tensor", "achieved": fl / t_dom / 1e12, "peak": peaks["bf16_tflops_sustained"],
+        roof = {"bound": "tensor", "achieved": fl / t_dom / 1e12, "peak": ratio * peaks["bf16_tflops_sustained"],
                 "unit": "TFLOP/s"}
-        roof["frac_of_burst_peak"] = fl / t_dom / 1e12 / peaks["bf16_tflops"]
+        roof["frac_of_burst_peak"] = fl / t_dom / 1e12 / (ratio * peaks["bf16_tflops"])
     else:
         roof = {"bound": "hbm", "achieved": by / t_dom / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["kernel"] = dname
-    roof["peak_source"] = f"{peak_kind} ({'sustained' if roof['bound'] == 'tensor' else 'copy'})"
+    roof["peak_source"] = f"{peak_kind} ({'sustained' if roof['bound'] == 'tensor' else 'copy'})" + \
+        (" x 4 (nominal FP4 / BF16 dense ratio)" if fp4_gemm and roof["bound"] == "tensor" else "")
     roof["algorithmic_flops"] = fl
     roof["algorithmic_bytes"] = by
     roof["traffic"] = measured_traffic(dname, w)
-    sf, sb = step_work(w, n_touched)
+    sf, sb, sf4 = step_work(w, n_touched)
     t_step = ms_max / steps * 1e-3
-    step_roof = max(sf / (peaks["bf16_tflops_sustained"] * 1e12), sb / (peaks["hbm_gbs"] * 1e9))
+    bf16_peak = peaks["bf16_tflops_sustained"] * 1e12
+    step_roof = max((sf - sf4) / bf16_peak + sf4 / (4.0 * bf16_peak), sb / (peaks["hbm_gbs"] * 1e9))
     res = {
         "value": job_tokens_per_s(world, w.T, steps, ms_max),
         "ms_per_step": ms_max / steps,
@@ -491,6 +503,12 @@ def main():
                 inp_qd = dict(inp_q, x=rank_tokens(wqd, rank, dev))
                 side["nvfp4_decode"] = run_ours(wqd, inp_qd, max(args.steps, 50), args.warmup, rank, world, peaks,
                                                 peak_kind, False, e2e_steps=0)
+                # the same weights with NVFP4 activations (W4A4, tcgen05 kind::mxf4nvf4)
+                side["nvfp4_w4a4"] = run_ours(W.WORKLOADS["nvfp4_w4a4"], inp_q, args.steps, args.warmup, rank, world,
+                                              peaks, peak_kind, False, e2e_steps=0)
+                side["nvfp4_w4a4_decode"] = run_ours(W.WORKLOADS["nvfp4_w4a4_decode"], inp_qd, max(args.steps, 50),
+                                                     args.warmup, rank, world, peaks, peak_kind, False, e2e_steps=0,
+                                                     graph_steps=max(args.steps, 50))
         if rank == 0:
             line = {
                 "metric": metric_name(), "value": main_res["value"], "unit": "tokens/s", "n_gpus": world,

@@ -82,6 +82,17 @@ typedef struct muse_nvfp4_weight {
   const float* matrix_scale;  /* float [E]                                            */
 } muse_nvfp4_weight;
 
+/* Format of the expert GEMMs' activation operands (with NVFP4 expert weights). */
+typedef enum muse_act_format {
+  MUSE_ACT_BF16 = 0,          /* W4A16: activations stay bf16                           */
+  MUSE_ACT_NVFP4 = 1          /* W4A4 (deep dive §7.4): the latent rows and the SwiGLU
+                                 output are quantised per 16 values to E2M1 codes with an
+                                 E4M3 scale E4M3(amax / 6) (nearest, ties to even, float32
+                                 arithmetic, no tensor scale) and the tensor core reads
+                                 both operands as 4-bit codes; requires NVFP4 experts and
+                                 L, I multiples of 256                                   */
+} muse_act_format;
+
 typedef enum muse_norm_mode {
   MUSE_NORM_CENTRED = 0,      /* y / sqrt(mean(y^2)+eps) * (1+gamma)                   */
   MUSE_NORM_INPUT_SCALED = 1  /* u / sqrt(mean(u^2)+eps), u = y * (1+gamma)           */
@@ -134,6 +145,7 @@ typedef struct muse_moe_config {
   const float* residual_gate; /* device [D] float32 gate parameters g, or NULL        */
   float residual_gate_temperature; /* pages: 0.3                                      */
   float residual_gate_eps;    /* floor of alpha^2; pages: 1e-3                         */
+  int32_t act_format;         /* muse_act_format of the expert GEMMs' activations      */
 } muse_moe_config;
 
 /* Byte offsets of the intermediates inside the workspace after a forward call, for
@@ -157,6 +169,10 @@ typedef struct muse_moe_workspace_layout {
   size_t xn;            /* act   [T, D]  normalised input (with ffn_pre_gain; else 0)  */
   size_t ss_out;        /* float [T, D/32] partial sums of v^2 per 32 columns (with
                            ffn_post_gain; else 0)                                     */
+  size_t zq_codes;      /* uint8 [R, L/2]  W4A4: quantised expert-ordered latent rows   */
+  size_t zq_scales;     /* uint8 [R, L/16] their E4M3 block scales                     */
+  size_t hq_codes;      /* uint8 [R, I/2]  W4A4: quantised SwiGLU output (else 0)      */
+  size_t hq_scales;     /* uint8 [R, I/16]                                             */
   size_t total;         /* bytes required                                             */
   int64_t rows;         /* R: upper bound of padded rows                              */
 } muse_moe_workspace_layout;
@@ -235,14 +251,24 @@ MUSE_API muse_status muse_latent_moe_forward_static_scratch(const muse_moe_confi
  * MUSE_OK once launched, MUSE_ERR_INVALID_ARG for a null pointer or a limit out of range. */
 MUSE_API muse_status muse_selftest_bounded_wait(uint64_t limit_ns, uint32_t* status_dev, void* stream);
 
+/* The W4A4 activation quantiser on its own (the step the forward applies to the latent rows
+ * and to h, muse_act_format): rows x K bf16 values (device, row-major, 16-byte aligned, K a
+ * multiple of 16) -> codes uint8 [rows, K/2] (two E2M1 codes per byte, low nibble = even
+ * element; 16-byte aligned) and scales uint8 [rows, K/16] (E4M3), per block of 16 values
+ * scale = E4M3(amax / 6), code = E2M1(value / scale), nearest with ties to even, float32
+ * arithmetic. Enqueued on `stream`; INVALID_ARG for null / misaligned pointers or sizes. */
+MUSE_API muse_status muse_quantize_nvfp4_rows(const void* src, int64_t rows, int64_t K, void* codes,
+                                              void* scales, void* stream);
+
 /* Static string for a status code. */
 MUSE_API const char* muse_status_string(muse_status s);
 
 /* Number of kernel launches one forward call makes for cfg: 11, plus one each for the
- * pre-expert norm, the pre-FFN norm, and the post-FFN norm / residual gate (one kernel
- * finishes both). In launch order: [ffn pre norm], router, top-k, histogram, tiles,
- * assign rows, pooler, [pre-expert norm], gather, gate/up, down, norm + combine,
- * unpooler, [post norm / gate]. stage_events must hold this many + 1 events. */
+ * pre-expert norm, the pre-FFN norm, the post-FFN norm / residual gate (one kernel
+ * finishes both) and the W4A4 quantisation of h. In launch order: [ffn pre norm], router,
+ * top-k, histogram, tiles, assign rows, pooler, [pre-expert norm], gather (W4A4: gather and
+ * quantise), gate/up, [quantise h], down, norm + combine, unpooler, [post norm / gate].
+ * stage_events must hold this many + 1 events. */
 MUSE_API int32_t muse_latent_moe_launch_count(const muse_moe_config* cfg);
 
 #ifdef __cplusplus

@@ -17,6 +17,7 @@ LIB_PATH = os.path.join(PKG, "libmuse_moe.so")
 MUSE_F32, MUSE_BF16 = 0, 1
 ROUTER_SOFTMAX, ROUTER_SIGMOID = 0, 1
 EXPERTS_DENSE, EXPERTS_NVFP4 = 0, 1
+ACT_BF16, ACT_NVFP4 = 0, 1
 NORM_CENTRED, NORM_INPUT_SCALED = 0, 1
 
 STATUS = {0: "MUSE_OK", 1: "MUSE_ERR_INVALID_ARG", 2: "MUSE_ERR_UNSUPPORTED", 3: "MUSE_ERR_WORKSPACE",
@@ -26,7 +27,7 @@ STATUS = {0: "MUSE_OK", 1: "MUSE_ERR_INVALID_ARG", 2: "MUSE_ERR_UNSUPPORTED", 3:
 EXPORTS = ("muse_moe_config_init", "muse_latent_moe_workspace_size", "muse_latent_moe_workspace_layout",
            "muse_latent_moe_forward", "muse_latent_moe_forward_host_io", "muse_latent_moe_last_device_status",
            "muse_status_string", "muse_latent_moe_launch_count", "muse_latent_moe_forward_static_scratch",
-           "muse_selftest_bounded_wait")
+           "muse_selftest_bounded_wait", "muse_quantize_nvfp4_rows")
 
 # size of the library's built-in scratch array (MUSE_STATIC_SCRATCH_BYTES)
 STATIC_SCRATCH_BYTES = 16 << 20
@@ -51,7 +52,7 @@ class Config(ctypes.Structure):
                 ("ffn_pre_gain", ctypes.c_void_p), ("ffn_pre_eps", ctypes.c_float),
                 ("ffn_post_gain", ctypes.c_void_p), ("ffn_post_eps", ctypes.c_float),
                 ("residual_gate", ctypes.c_void_p), ("residual_gate_temperature", ctypes.c_float),
-                ("residual_gate_eps", ctypes.c_float)]
+                ("residual_gate_eps", ctypes.c_float), ("act_format", ctypes.c_int32)]
 
 
 class Nvfp4Weight(ctypes.Structure):
@@ -61,7 +62,8 @@ class Nvfp4Weight(ctypes.Structure):
 class WorkspaceLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in ("status", "expert_count", "expert_offset", "logits", "topk_idx",
                                               "topk_w", "inv", "row_token", "z", "zp", "h", "y", "ss", "c",
-                                              "xn", "ss_out", "total")] + [("rows", ctypes.c_int64)]
+                                              "xn", "ss_out", "zq_codes", "zq_scales", "hq_codes", "hq_scales",
+                                              "total")] + [("rows", ctypes.c_int64)]
 
 
 _lib: Optional[ctypes.CDLL] = None
@@ -93,6 +95,8 @@ def lib() -> ctypes.CDLL:
         L.muse_latent_moe_forward_static_scratch.restype = ctypes.c_int
         L.muse_selftest_bounded_wait.argtypes = [ctypes.c_uint64, vp, vp]
         L.muse_selftest_bounded_wait.restype = ctypes.c_int
+        L.muse_quantize_nvfp4_rows.argtypes = [vp, ctypes.c_int64, ctypes.c_int64, vp, vp, vp]
+        L.muse_quantize_nvfp4_rows.restype = ctypes.c_int
         L.muse_latent_moe_launch_count.argtypes = [cp]
         L.muse_latent_moe_launch_count.restype = ctypes.c_int32
         _lib = L
@@ -112,7 +116,7 @@ def make_config(T: int, D: int, L: int, I: int, E: int, k: int, dtype: str = "bf
                 router_mode: int = ROUTER_SOFTMAX, router_logit_scale: float = 1.0, routed_scaling: float = 1.0,
                 norm_mode: int = NORM_CENTRED, gamma_shared: bool = False, pre_norm_eps: float = 1e-5,
                 ffn_pre_eps: float = 1e-5, ffn_post_eps: float = 1e-8, residual_gate_temperature: float = 0.3,
-                residual_gate_eps: float = 1e-3) -> Config:
+                residual_gate_eps: float = 1e-3, act_format: int = ACT_BF16) -> Config:
     c = Config()
     lib().muse_moe_config_init(ctypes.byref(c))
     c.T, c.D, c.L, c.I, c.E, c.top_k = T, D, L, I, E, k
@@ -123,6 +127,7 @@ def make_config(T: int, D: int, L: int, I: int, E: int, k: int, dtype: str = "bf
     c.pre_norm_eps = pre_norm_eps
     c.ffn_pre_eps, c.ffn_post_eps = ffn_pre_eps, ffn_post_eps
     c.residual_gate_temperature, c.residual_gate_eps = residual_gate_temperature, residual_gate_eps
+    c.act_format = act_format
     return c
 
 
@@ -196,6 +201,9 @@ def stages(cfg: Config):
     names = list(STAGES)
     if cfg.pre_norm_gain:
         names.insert(names.index("gather"), "pre_expert_norm")
+    if cfg.act_format == ACT_NVFP4:
+        names[names.index("gather")] = "gather_quant"
+        names.insert(names.index("gate_up_swiglu") + 1, "quant_h")
     if cfg.ffn_pre_gain:
         names.insert(0, "ffn_pre_norm")
     if cfg.ffn_post_gain or cfg.residual_gate:
@@ -212,10 +220,18 @@ def event_handles(events) -> "ctypes.Array":
     return arr
 
 
+def quantize_nvfp4_rows(src, codes, scales, stream=None) -> None:
+    """NVFP4 activation quantiser: src bf16 [rows, K] -> codes uint8 [rows, K/2], scales
+    uint8 [rows, K/16] (CUDA tensors)."""
+    rows, K = src.shape
+    _check(lib().muse_quantize_nvfp4_rows(_ptr(src), int(rows), int(K), _ptr(codes), _ptr(scales),
+                                          _stream_handle(stream)), "muse_quantize_nvfp4_rows")
+
+
 def selftest_bounded_wait(limit_ns: int, status_dev, stream=None) -> None:
     """Run the device-side bounded-wait self-test (status_dev: zeroed CUDA int32[2])."""
     _check(lib().muse_selftest_bounded_wait(int(limit_ns), _ptr(status_dev), _stream_handle(stream)),
-           "muse_selftest_bounded_wait")
+           "muse_selftest_bounded_wait", "muse_quantize_nvfp4_rows")
 
 
 def last_device_status(cfg: Config, stream=None):

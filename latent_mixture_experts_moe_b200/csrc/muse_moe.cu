@@ -20,6 +20,8 @@
 #include "gemm_umma.cuh"
 #include "gemm_umma_2sm.cuh"
 #include "gemm_umma_fp4.cuh"
+#include "gemm_umma_w4a4.cuh"
+#include "nvfp4_act.cuh"
 #include "route_kernels.cuh"
 
 using namespace muse;
@@ -32,8 +34,10 @@ int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // ---------------------------------------------------------------------- tile sizing
 // tokens per grouped-GEMM tile: small tiles when experts see few tokens (decode)
+bool w4a4(const muse_moe_config& c) { return c.act_format == MUSE_ACT_NVFP4; }
 int grouped_bn(const muse_moe_config& c) {
   if ((c.T * c.top_k) <= 32 * c.E) return 32;
+  if (w4a4(c)) return 128;                                    // W4A4: accumulators leave TMEM room for scales
   return c.expert_weights == MUSE_EXPERTS_NVFP4 ? 192 : 256;  // NVFP4: accumulators leave TMEM room for weights
 }
 int dense_bn(const muse_moe_config& c) { return c.T <= 32 ? 32 : 256; }
@@ -81,6 +85,12 @@ Layout make_layout(const muse_moe_config& c) {
   l.pub.c = take(as * T * c.L);
   l.pub.xn = c.ffn_pre_gain != nullptr ? take(as * T * c.D) : 0;
   l.pub.ss_out = c.ffn_post_gain != nullptr ? take(sizeof(float) * T * (c.D / 32)) : 0;
+  if (w4a4(c)) {
+    l.pub.zq_codes = take(rows * (c.L / 2));
+    l.pub.zq_scales = take(rows * (c.L / 16));
+    l.pub.hq_codes = take(rows * (c.I / 2));
+    l.pub.hq_scales = take(rows * (c.I / 16));
+  }
   l.pub.total = o;
   l.pub.rows = rows;
   return l;
@@ -105,6 +115,10 @@ muse_status validate_sizes(const muse_moe_config* c) {
   if (c->T > (int64_t(1) << 24)) return MUSE_ERR_UNSUPPORTED;
   if (c->expert_weights != MUSE_EXPERTS_DENSE && c->expert_weights != MUSE_EXPERTS_NVFP4) return MUSE_ERR_INVALID_ARG;
   if (c->expert_weights == MUSE_EXPERTS_NVFP4 && c->dtype != MUSE_BF16) return MUSE_ERR_UNSUPPORTED;
+  if (c->act_format != MUSE_ACT_BF16 && c->act_format != MUSE_ACT_NVFP4) return MUSE_ERR_INVALID_ARG;
+  if (c->act_format == MUSE_ACT_NVFP4 &&
+      (c->expert_weights != MUSE_EXPERTS_NVFP4 || c->L % 256 != 0 || c->I % 256 != 0))
+    return MUSE_ERR_UNSUPPORTED;
   return MUSE_OK;
 }
 
@@ -161,6 +175,21 @@ bool make_code_map(CUtensorMap* m, const void* base, int64_t rows, int64_t K) {
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Byte matrix rows x cols (uint8: packed codes or E4M3 scales), boxes of box_rows rows x
+// box_cols bytes, 128-byte swizzle for code tiles the UMMA reads, none for scale boxes.
+bool make_u8_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_cols, int box_rows,
+                 bool swizzle) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Output map for TMA stores: rows x cols bf16 row-major, boxes of 16 rows x 128 columns,
@@ -230,6 +259,37 @@ cudaError_t launch_gemm_fp4(int bn, int mt, const TmaMaps& maps, const GemmArgs&
     return mt == 2 ? launch_gemm_fp4_t<192, EPI, 2>(maps, args, q4, grid, st)
                    : launch_gemm_fp4_t<192, EPI, 1>(maps, args, q4, grid, st);
   }
+}
+
+template <int BN, int EPI>
+cudaError_t launch_gemm_w4a4_t(const W4A4Maps& maps, const GemmArgs& args, const W4A4Args& q, int grid,
+                               cudaStream_t st) {
+  auto kern = k_umma_gemm_w4a4<BN, EPI, 2>;
+  const size_t smem = W4A4Shape<BN, EPI, 2>::kSmemBytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kW4A4Threads, smem, st>>>(maps, args, q);
+  return cudaGetLastError();
+}
+
+template <int EPI>
+cudaError_t launch_gemm_w4a4(int bn, const W4A4Maps& maps, const GemmArgs& args, const W4A4Args& q, int grid,
+                             cudaStream_t st) {
+  return bn == 32 ? launch_gemm_w4a4_t<32, EPI>(maps, args, q, grid, st)
+                  : launch_gemm_w4a4_t<128, EPI>(maps, args, q, grid, st);
+}
+
+// W4A4 maps: weight codes and scales of one or two matrices ([rows_w, K/2], [rows_w, K/16]),
+// token codes and scales ([R, K/2], [R, K/16]) in boxes of bn rows.
+bool make_w4a4_maps(W4A4Maps* m, const muse_nvfp4_weight* w, const muse_nvfp4_weight* w2, int64_t rows_w,
+                    const void* codes, const void* scales, int64_t R, int64_t K, int bn) {
+  std::memset(m, 0, sizeof(*m));
+  return make_u8_map(&m->a, w->codes, rows_w, K / 2, 128, 128, true) &&
+         make_u8_map(&m->a2, w2->codes, rows_w, K / 2, 128, 128, true) &&
+         make_u8_map(&m->b, codes, R, K / 2, 128, bn, true) &&
+         make_u8_map(&m->sfa, w->block_scales, rows_w, K / 16, 16, 128, false) &&
+         make_u8_map(&m->sfa2, w2->block_scales, rows_w, K / 16, 16, 128, false) &&
+         make_u8_map(&m->sfb, scales, R, K / 16, 16, bn, false);
 }
 
 template <typename TOut, int EPI, int MT>
@@ -322,6 +382,7 @@ GemmPlan plan_gate_up(const muse_moe_config& c, int bn_g) {
   return {false, 2, 128};
 }
 GemmPlan plan_down(const muse_moe_config& c, int bn_g) {
+  if (w4a4(c)) return {false, 2, 256};
   if (c.expert_weights == MUSE_EXPERTS_NVFP4) return c.L % 256 == 0 ? GemmPlan{false, 2, 256} : GemmPlan{false, 1, 128};
   if (c.dtype == MUSE_BF16 && bn_g == 256 && c.L % 512 == 0) return {true, 2, 512};
   if (c.dtype == MUSE_BF16 && bn_g == 256 && c.L % 256 == 0) return {true, 1, 256};
@@ -432,8 +493,19 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
     MUSE_CK(cudaGetLastError());
     MUSE_CK(mark());
   }
-  // (a5) gather into expert order
-  {
+  // (a5) gather into expert order (W4A4: gather and quantise to NVFP4 in one pass)
+  const bool q4a = w4a4(c);
+  uint8_t* zq_codes = at(lay.pub.zq_codes);
+  uint8_t* zq_scales = at(lay.pub.zq_scales);
+  uint8_t* hq_codes = at(lay.pub.hq_codes);
+  uint8_t* hq_scales = at(lay.pub.hq_scales);
+  const int quant_grid = static_cast<int>(std::min<int64_t>(lay.pub.rows, 16 * nsm));
+  if (q4a) {
+    k_quant_rows_nvfp4<<<quant_grid, 256, 0, st>>>(row_token, offsets + E, 0, reinterpret_cast<const __nv_bfloat16*>(z),
+                                                   static_cast<int>(L), 1, zq_codes, zq_scales);
+    MUSE_CK(cudaGetLastError());
+    MUSE_CK(mark());
+  } else {
     const int vpr = static_cast<int>(L * sizeof(T) / 16);
     const int rows_grid = static_cast<int>(std::min<int64_t>(lay.pub.rows, 16 * nsm));
     k_gather_rows<<<rows_grid, 128, 0, st>>>(row_token, offsets + E, reinterpret_cast<const uint4*>(z),
@@ -447,7 +519,9 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
     const bool fp4 = c.expert_weights == MUSE_EXPERTS_NVFP4;
     TmaMaps maps;
     Fp4Args q4{};
-    if (fp4) {
+    if (q4a) {
+      // W4A4: its maps are built at the launch below
+    } else if (fp4) {
       const muse_nvfp4_weight* wg = static_cast<const muse_nvfp4_weight*>(W_gate);
       const muse_nvfp4_weight* wu = static_cast<const muse_nvfp4_weight*>(W_up);
       std::memset(&maps, 0, sizeof(maps));
@@ -468,7 +542,15 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
     g.k_blocks = static_cast<int>(L * sizeof(T) / 128);
     g.out = h;
     g.ld_out = I;
-    if (fp4) {
+    if (q4a) {
+      W4A4Maps wm;
+      const muse_nvfp4_weight* wg = static_cast<const muse_nvfp4_weight*>(W_gate);
+      const muse_nvfp4_weight* wu = static_cast<const muse_nvfp4_weight*>(W_up);
+      if (!make_w4a4_maps(&wm, wg, wu, E * I, zq_codes, zq_scales, R, L, bn_g)) return MUSE_ERR_CUDA;
+      const W4A4Args wq{wg->matrix_scale, wu->matrix_scale};
+      g.k_blocks = static_cast<int>(L / 256);
+      MUSE_CK(launch_gemm_w4a4<EPI_SWIGLU>(bn_g, wm, g, wq, nsm, st));
+    } else if (fp4) {
       MUSE_CK(launch_gemm_fp4<EPI_SWIGLU>(bn_g, 2, maps, g, q4, nsm, st));
     } else if (pgu.pair) {
       if (!make_out_map(&maps.out, h, R, I)) return MUSE_ERR_CUDA;
@@ -478,12 +560,21 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
     }
     MUSE_CK(mark());
   }
+  // W4A4: quantise h (already in expert order) for the down projection
+  if (q4a) {
+    k_quant_rows_nvfp4<<<quant_grid, 256, 0, st>>>(row_token, offsets + E, 0, reinterpret_cast<const __nv_bfloat16*>(h),
+                                                   static_cast<int>(I), 0, hq_codes, hq_scales);
+    MUSE_CK(cudaGetLastError());
+    MUSE_CK(mark());
+  }
   // (a7) down projection + sum-of-squares partials
   {
     const bool fp4 = c.expert_weights == MUSE_EXPERTS_NVFP4;
     TmaMaps maps;
     Fp4Args q4{};
-    if (fp4) {
+    if (q4a) {
+      // W4A4: its maps are built at the launch below
+    } else if (fp4) {
       const muse_nvfp4_weight* wd = static_cast<const muse_nvfp4_weight*>(W_down);
       std::memset(&maps, 0, sizeof(maps));
       if (!make_code_map(&maps.a, wd->codes, E * L, I) || !make_code_map(&maps.a2, wd->codes, E * L, I)) return MUSE_ERR_CUDA;
@@ -510,7 +601,14 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
       g.ss_gain_group_stride = c.gamma_shared ? 0 : L;
     }
     if (pdn.pair && !make_out_map(&maps.out, y, R, L)) return MUSE_ERR_CUDA;
-    if (fp4) {
+    if (q4a) {
+      W4A4Maps wm;
+      const muse_nvfp4_weight* wd = static_cast<const muse_nvfp4_weight*>(W_down);
+      if (!make_w4a4_maps(&wm, wd, wd, E * L, hq_codes, hq_scales, R, I, bn_g)) return MUSE_ERR_CUDA;
+      const W4A4Args wq{wd->matrix_scale, wd->matrix_scale};
+      g.k_blocks = static_cast<int>(I / 256);
+      MUSE_CK(launch_gemm_w4a4<EPI_STORE_SS>(bn_g, wm, g, wq, nsm, st));
+    } else if (fp4) {
       MUSE_CK(launch_gemm_fp4<EPI_STORE_SS>(bn_g, pdn.mt, maps, g, q4, nsm, st));
     } else if (pdn.pair && pdn.mt == 2) {
       MUSE_CK((launch_gemm_2sm<T, EPI_STORE_SS, 2>(maps, g, nsm / 2, st)));
@@ -709,6 +807,17 @@ muse_status muse_latent_moe_last_device_status(const muse_moe_config* cfg, void*
   return static_cast<muse_status>(word[0]);
 }
 
+muse_status muse_quantize_nvfp4_rows(const void* src, int64_t rows, int64_t K, void* codes, void* scales,
+                                     void* stream) {
+  if (src == nullptr || codes == nullptr || scales == nullptr || !aligned16(src) || !aligned16(codes)) return MUSE_ERR_INVALID_ARG;
+  if (rows < 1 || K < 16 || K % 16 != 0 || rows > (int64_t(1) << 30) || K > (int64_t(1) << 20)) return MUSE_ERR_INVALID_ARG;
+  const int grid = static_cast<int>(std::min<int64_t>(rows, 16 * sm_count()));
+  k_quant_rows_nvfp4<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      nullptr, nullptr, static_cast<int>(rows), static_cast<const __nv_bfloat16*>(src), static_cast<int>(K), 0,
+      static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales));
+  return cudaGetLastError() == cudaSuccess ? MUSE_OK : MUSE_ERR_CUDA;
+}
+
 muse_status muse_selftest_bounded_wait(uint64_t limit_ns, uint32_t* status_dev, void* stream) {
   if (status_dev == nullptr || limit_ns < 1 || limit_ns > 10000000000ull) return MUSE_ERR_INVALID_ARG;
   k_selftest_wait<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns, status_dev);
@@ -734,7 +843,7 @@ int32_t muse_latent_moe_launch_count(const muse_moe_config* cfg) {
   // and the optional sublayer pre-norm (first), pre-expert norm (between pooler and
   // gather) and sublayer post-norm / residual gate (last)
   return 11 + (cfg->pre_norm_gain != nullptr) + (cfg->ffn_pre_gain != nullptr) +
-         (cfg->ffn_post_gain != nullptr || cfg->residual_gate != nullptr);
+         (cfg->ffn_post_gain != nullptr || cfg->residual_gate != nullptr) + (cfg->act_format == MUSE_ACT_NVFP4);
 }
 
 }  // extern "C"

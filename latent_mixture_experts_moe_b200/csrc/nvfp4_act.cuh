@@ -1,0 +1,97 @@
+// nvfp4_act.cuh -- NVFP4 quantisation of the expert GEMMs' activation operands (W4A4 mode).
+//
+// The released checkpoint quantises both operands of the expert GEMMs (Muse Spark Open deep
+// dive §7.4): per block of 16 consecutive values of a row, one E4M3 scale and sixteen 4-bit
+// E2M1 codes (OCP Microscaling formats v1.0). Here, with no tensor-wide scale:
+//   scale = E4M3(amax / 6), code_i = E2M1(v_i / decoded scale)
+// both rounded to nearest with ties to even, E2M1 saturating at +-6; amax, the division by
+// 6 and v_i / scale are IEEE float32 operations on the float32 value of the stored bfloat16
+// activation. Codes are packed two per byte, the low nibble holding the even element, the
+// same packing as the NVFP4 expert weights.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+
+namespace muse {
+
+// Exact value of an E4M3 byte (bias 7, subnormal when the exponent field is 0; the NaN
+// pattern S.1111.111 decodes to NaN).
+__device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
+  const uint32_t e = (b >> 3) & 15u, m = b & 7u;
+  float v;
+  if (e == 15u && m == 7u) {
+    v = __int_as_float(0x7FC00000);
+  } else if (e == 0u) {
+    v = static_cast<float>(m) * 0.001953125f;  // m * 2^-9
+  } else {
+    v = __int_as_float(static_cast<int>(((e + 120u) << 23) | (m << 20)));
+  }
+  return (b & 0x80u) ? -v : v;
+}
+
+// 4-bit E2M1 code of q: the magnitude index counts the rounding boundaries below |q| (the
+// midpoints 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5 between the magnitudes 0, 0.5, 1, 1.5, 2, 3,
+// 4, 6), each midpoint going to the neighbour with an even index; the sign bit only on a
+// nonzero magnitude. NaN compares false everywhere and gives 0.
+__device__ __forceinline__ uint32_t e2m1_rne(float q) {
+  const float a = fabsf(q);
+  const uint32_t m = static_cast<uint32_t>(a > 0.25f) + static_cast<uint32_t>(a >= 0.75f) +
+                     static_cast<uint32_t>(a > 1.25f) + static_cast<uint32_t>(a >= 1.75f) +
+                     static_cast<uint32_t>(a > 2.5f) + static_cast<uint32_t>(a >= 3.5f) +
+                     static_cast<uint32_t>(a > 5.0f);
+  return (q < 0.0f && m != 0u) ? (m | 8u) : m;
+}
+
+// One block of 16 values -> 8 code bytes (two words, element 2i in the low nibble of byte i)
+// and the E4M3 scale byte.
+__device__ __forceinline__ void quant_block16(const float (&v)[16], uint2& codes, uint32_t& sbyte) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  sbyte = f32_to_e4m3_rn_satfinite(amax / 6.0f);
+  const float s = e4m3_to_f32(sbyte);
+  uint32_t w[2] = {0u, 0u};
+  if (s > 0.0f) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) w[i >> 3] |= e2m1_rne(v[i] / s) << (4 * (i & 7));
+  }
+  codes = make_uint2(w[0], w[1]);
+}
+
+// Quantise rows of bf16 activations of K values (K a multiple of 16) into codes
+// [rows, K/2] and scales [rows, K/16]. Row r of the output reads source row row_token[r]
+// when `gather` (z in token order, dispatched into expert order on the way) or row r itself
+// (h, already in expert order); rows whose row_token is negative (an expert's padding) get
+// zero codes and scales. One block per row, grid-strided over the device row count; one
+// thread per block of 16 values (two 16-byte loads, one 8-byte and one 1-byte store).
+// Without row_token every row is quantised from itself, and total_rows may be NULL, rows_host
+// giving the count.
+__global__ void k_quant_rows_nvfp4(const int* __restrict__ row_token, const int* __restrict__ total_rows,
+                                   int rows_host, const __nv_bfloat16* __restrict__ src, int K, int gather,
+                                   uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+  const int R = total_rows != nullptr ? *total_rows : rows_host;
+  const int nb = K / 16;
+  for (int r = blockIdx.x; r < R; r += gridDim.x) {
+    const int tok = row_token != nullptr ? row_token[r] : r;
+    const int64_t srow = gather ? tok : r;
+    for (int b = threadIdx.x; b < nb; b += blockDim.x) {
+      uint2 c = make_uint2(0u, 0u);
+      uint32_t sb = 0u;
+      if (tok >= 0) {
+        const uint4* p = reinterpret_cast<const uint4*>(src + srow * K + b * 16);
+        const uint4 u[2] = {p[0], p[1]};
+        const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(u);
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = __bfloat162float(h[i]);
+        quant_block16(v, c, sb);
+      }
+      *reinterpret_cast<uint2*>(codes + static_cast<int64_t>(r) * (K / 2) + b * 8) = c;
+      scales[static_cast<int64_t>(r) * nb + b] = static_cast<uint8_t>(sb);
+    }
+  }
+}
+
+}  // namespace muse

@@ -194,6 +194,44 @@ __device__ __forceinline__ void umma_ts_bf16(uint32_t d_tmem, uint32_t a_tmem, u
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(z), "r"(z), "r"(z), "r"(z));
 }
 
+// Block-scaled FP4 UMMA (kind::mxf4nvf4, one E4M3 scale per 16 elements of K): A and B are
+// E2M1 codes in shared memory, K-major, 64 elements (32 bytes) per row per MMA; the scale
+// factors are read from TMEM at sfa_tmem / sfb_tmem. Scale layout (per MMA): the 4 scale
+// bytes of A row m (K sub-blocks 0..3, low byte first) at lane m, column sfa + m / 32; those
+// of B row n at column sfb + n / 32, lane n % 32 of EVERY lane quadrant (each quadrant's
+// datapath reads its own copy).
+__device__ __forceinline__ void umma_mxf4nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem));
+}
+// Instruction descriptor of the block-scaled kinds: A and B format E2M1 (1) at bits 7-9 and
+// 10-12, both K-major, N >> 3 at bits 17-22, scale format UE4M3 (bit 23 = 0), M >> 4 at bits
+// 24-28, scale-factor byte ids 0 (bits 4-5, 29-30), K = 64 (bit 31 = 0); FP32 accumulation.
+__device__ __forceinline__ uint32_t idesc_mxf4nvf4(uint32_t M, uint32_t N) {
+  return (1u << 7) | (1u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+// Thread i of the warp writes one / four 32-bit values to lane (quadrant * 32 + i) at
+// column col / columns [col, col + 4).
+__device__ __forceinline__ void tmem_st_x1(uint32_t taddr, uint32_t a) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(a) : "memory");
+}
+__device__ __forceinline__ void tmem_st_x4(uint32_t taddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+// Nearest E4M3 byte of a float (ties to even, saturating at +-448): the hardware conversion
+// of two floats to an E4M3 pair, given v twice, low byte taken.
+__device__ __forceinline__ uint32_t f32_to_e4m3_rn_satfinite(float v) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %1;" : "=h"(r) : "f"(v));
+  return static_cast<uint32_t>(r) & 0xFFu;
+}
+
 // Thread i of the warp writes r[0..31] to lane (warp quadrant * 32 + i), columns [col, col+32).
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(

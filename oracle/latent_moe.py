@@ -174,20 +174,21 @@ def expert_ffn(z: Array, W_gate: Array, W_up: Array, W_down: Array,
     given, maps each GEMM's activation operand (z, then the SwiGLU output h) to the values
     the GEMM multiplies (the W4A4 mode's quantise-dequantise)."""
     if act is not None:
-        z = act(z)
+        z = act(z, 0)
     a = z @ W_gate.T
     u = z @ W_up.T
     h = silu(a) * u
     if act is not None:
-        h = act(h)
+        h = act(h, 1)
     return h @ W_down.T
 
 
-def nvfp4_activation(v: Array) -> Array:
+def nvfp4_activation(v: Array, ref=None, adopted=None) -> Array:
     """W4A4 operand of an expert GEMM: the activation as the kernels store it (bfloat16),
-    quantised per 16 to E2M1 codes with E4M3 scales, and dequantised (oracle.nvfp4)."""
+    quantised per 16 to E2M1 codes with E4M3 scales, and dequantised (oracle.nvfp4); ref /
+    adopted as in quantize_activations_nvfp4."""
     from .nvfp4 import dequantize_activations_nvfp4, quantize_activations_nvfp4
-    codes, scales = quantize_activations_nvfp4(round_bf16(v))
+    codes, scales = quantize_activations_nvfp4(round_bf16(v), ref=ref, adopted=adopted)
     return dequantize_activations_nvfp4(codes, scales)
 
 
@@ -259,7 +260,8 @@ def latent_moe_forward(x: Array, W_router: Array, W_pool: Array, experts: Expert
                        ffn_pre_gain: Optional[Array] = None, ffn_pre_eps: float = 1e-5,
                        ffn_post_gain: Optional[Array] = None, ffn_post_eps: float = 1e-8,
                        gate: Optional[Array] = None, gate_temperature: float = 0.3, gate_floor: float = 1e-3,
-                       xn_round: Optional[str] = None, act_format: str = "bf16") -> Dict[str, Array]:
+                       xn_round: Optional[str] = None, act_format: str = "bf16",
+                       act_ref: Optional[Callable] = None) -> Dict[str, Array]:
     """Forward pass of the latent-MoE block for every row of x, in float64.
 
     experts: (W_gate [E,I,L], W_up [E,I,L], W_down [E,L,I]) or a callable e -> the three
@@ -272,7 +274,10 @@ def latent_moe_forward(x: Array, W_router: Array, W_pool: Array, experts: Expert
     xn_round="bf16" rounds xn to bfloat16 before the router and the pooler read it, as the
     pages' implementation stores it (the routing decision is then taken on the same values
     the bfloat16 kernels see). act_format="nvfp4" runs the expert GEMMs W4A4: their
-    activation operands (z rows, SwiGLU outputs) go through nvfp4_activation.
+    activation operands (z rows, SwiGLU outputs) go through nvfp4_activation. act_ref, for
+    W4A4: a callable (token rows, slots) -> ((z codes, z scales), (h codes, h scales)) of
+    those assignments from another implementation, whose decisions are adopted where they
+    sit at a rounding boundary (quantize_activations_nvfp4); "act_adopted" counts them.
 
     Returns every intermediate: xn, logits, keys, idx, g, z, y [T,k,L], ss [T,k], n, c,
     f (the block's output), out.
@@ -294,10 +299,14 @@ def latent_moe_forward(x: Array, W_router: Array, W_pool: Array, experts: Expert
     L = z.shape[1]
     y = np.zeros((T, k, L))
     get = experts if callable(experts) else (lambda e: (experts[0][e], experts[1][e], experts[2][e]))
+    adopted = [0]
     for e in np.unique(idx):                                             # (a3) dispatch
         tok, slot = np.nonzero(idx == e)
         Wg, Wu, Wd = get(int(e))
-        act = nvfp4_activation if act_format == "nvfp4" else None
+        act = None
+        if act_format == "nvfp4":
+            refs = act_ref(tok, slot) if act_ref is not None else (None, None)
+            act = (lambda v, stage, refs=refs: nvfp4_activation(v, refs[stage], adopted))
         y[tok, slot, :] = expert_ffn(z[tok], as_f64(Wg), as_f64(Wu), as_f64(Wd), act)  # (a6, a7)
     gam = gamma[idx] if gamma.ndim == 2 else np.broadcast_to(gamma, (T, k, L))
     if norm_mode == "centred":                                           # (a8)
@@ -313,7 +322,7 @@ def latent_moe_forward(x: Array, W_router: Array, W_pool: Array, experts: Expert
     if gate is not None:
         out = residual_gate(x_res, out, gate, gate_temperature, gate_floor)
     return {"xn": xn, "logits": logits, "keys": keys, "idx": idx, "g": g, "z": z, "y": y, "ss": ss,
-            "n": n, "c": c, "f": f, "out": out}
+            "n": n, "c": c, "f": f, "out": out, "act_adopted": adopted[0]}
 
 
 # ---------------------------------------------------------------------------------------

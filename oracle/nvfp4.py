@@ -102,18 +102,53 @@ def round_e2m1(q) -> np.ndarray:
     return np.where((q < 0) & (mag > 0), mag | 8, mag).astype(np.uint8)
 
 
-def quantize_activations_nvfp4(x):
+def quantize_activations_nvfp4(x, ref=None, rel_tol: float = 2.0 ** -7, adopted=None):
     """Rows [..., n] (n a multiple of 16; values exactly representable in float32) ->
-    (codes uint8 [..., n/2] low nibble first, scales uint8 E4M3 [..., n/16])."""
+    (codes uint8 [..., n/2] low nibble first, scales uint8 E4M3 [..., n/16]).
+
+    ref: optional (codes, scales) of the same rows from another implementation whose input
+    may differ from x by accumulation-order rounding. Where a decision of ref differs from
+    this one, it is adopted only if this input lies within rel_tol (relative) of the rounding
+    boundary between the two neighbouring values -- for a scale, amax / 6 near the midpoint of
+    two adjacent E4M3 values; for a code, value / scale near the midpoint of two adjacent E2M1
+    values of the same sign -- since then both decisions are correct for inputs that close;
+    any other difference raises ValueError. adopted (a one-element list) counts adoptions."""
     x32 = np.asarray(x, dtype=np.float32)
     blocks = x32.reshape(x32.shape[:-1] + (x32.shape[-1] // 16, 16))
     amax = np.max(np.abs(blocks), axis=-1)                          # exact
     s = (amax / np.float32(6.0)).astype(np.float32)                  # one float32 division
     sbyte = round_e4m3(s.astype(np.float64))
+    if ref is not None:
+        rs = np.asarray(ref[1], dtype=np.uint8).reshape(sbyte.shape)
+        diff = rs != sbyte
+        if diff.any():
+            mid = (decode_e4m3(rs[diff]) + decode_e4m3(sbyte[diff])) / 2.0
+            sv = s[diff].astype(np.float64)
+            near = (np.abs(rs[diff].astype(int) - sbyte[diff].astype(int)) == 1) & (np.abs(sv - mid) <= rel_tol * sv)
+            if not near.all():
+                raise ValueError(f"{int((~near).sum())} scale bytes differ away from a rounding boundary")
+            sbyte = np.where(diff, rs, sbyte)
+            if adopted is not None:
+                adopted[0] += int(diff.sum())
     sdec = decode_e4m3(sbyte).astype(np.float32)                     # exact in float32
     with np.errstate(divide="ignore", invalid="ignore"):
         q = np.where(sdec[..., None] > 0, blocks / sdec[..., None], np.float32(0.0)).astype(np.float32)
     codes = round_e2m1(q.astype(np.float64)).reshape(x32.shape)
+    if ref is not None:
+        rc = unpack_nibbles(np.asarray(ref[0], dtype=np.uint8)).reshape(codes.shape)
+        diff = rc != codes
+        if diff.any():
+            qd = q.reshape(codes.shape)[diff].astype(np.float64)
+            a, b = codes[diff].astype(int), rc[diff].astype(int)
+            same_side = ((a & 8) == (b & 8)) | ((a & 7) == 0) | ((b & 7) == 0)
+            adjacent = same_side & (np.abs((a & 7) - (b & 7)) == 1)
+            mid = (np.abs(decode_e2m1(a)) + np.abs(decode_e2m1(b))) / 2.0
+            near = adjacent & (np.abs(np.abs(qd) - mid) <= rel_tol * np.abs(qd))
+            if not near.all():
+                raise ValueError(f"{int((~near).sum())} codes differ away from a rounding boundary")
+            codes = np.where(diff, rc, codes)
+            if adopted is not None:
+                adopted[0] += int(diff.sum())
     packed = (codes[..., 0::2] | (codes[..., 1::2] << 4)).astype(np.uint8)
     return packed, sbyte
 

@@ -56,6 +56,8 @@ class Run:
         T = T or w.T
         self.w, self.T = w, T
         weights = {k: v for k, v in inp.items() if k != "x"}
+        if w.act == "nvfp4":
+            modes = dict(modes, act_format=moe.ACT_NVFP4)
         self.model = moe.LatentMoE(weights, T_max=T, k=w.k, eps=w.eps, **modes)
         dev = inp["x"].device
         self.idx = torch.full((T, w.k), -1, dtype=torch.int32, device=dev)
@@ -88,8 +90,27 @@ def expert_source(inp: Dict[str, torch.Tensor]):
     return lambda e: (inp["W_gate"][e], inp["W_up"][e], inp["W_down"][e])
 
 
-def oracle_block(w: W.Workload, inp: Dict[str, torch.Tensor], rows: np.ndarray, **kw) -> Dict[str, np.ndarray]:
-    """The oracle on token rows `rows` of x (tokens are independent)."""
+def w4a4_reference(run: "Run", rows: np.ndarray):
+    """For the W4A4 oracle: the CUDA path's quantised activation rows of each assignment, as
+    candidate decisions that the oracle adopts only where its own input sits at a rounding
+    boundary (oracle.quantize_activations_nvfp4 raises on any other difference)."""
+    k, L, I, R = run.w.k, run.w.L, run.w.I, run.layout["rows"]
+    ginv = run.inter("inv", torch.int32, (run.T * k,)).cpu().numpy()
+    zc = run.inter("zq_codes", torch.uint8, (R, L // 2)).cpu().numpy()
+    zs = run.inter("zq_scales", torch.uint8, (R, L // 16)).cpu().numpy()
+    hc = run.inter("hq_codes", torch.uint8, (R, I // 2)).cpu().numpy()
+    hs = run.inter("hq_scales", torch.uint8, (R, I // 16)).cpu().numpy()
+
+    def ref(tok, slot):
+        r = ginv[np.asarray(rows)[tok] * k + slot]
+        return (zc[r], zs[r]), (hc[r], hs[r])
+    return ref
+
+
+def oracle_block(w: W.Workload, inp: Dict[str, torch.Tensor], rows: np.ndarray, run: Optional["Run"] = None,
+                 **kw) -> Dict[str, np.ndarray]:
+    """The oracle on token rows `rows` of x (tokens are independent). For W4A4 workloads,
+    `run` supplies the candidate quantisation decisions (w4a4_reference)."""
     x = host(inp["x"][torch.as_tensor(rows, device=inp["x"].device)])
     bias = host(inp["router_bias"]) if "router_bias" in inp else None
     if "pre_norm_gain" in inp:
@@ -99,6 +120,10 @@ def oracle_block(w: W.Workload, inp: Dict[str, torch.Tensor], rows: np.ndarray, 
             kw = dict(kw, **{key: host(inp[name])})
     if "ffn_pre_gain" in inp and w.dtype == "bf16":
         kw = dict(kw, xn_round="bf16")
+    if w.act == "nvfp4":
+        kw = dict(kw, act_format="nvfp4")
+        if run is not None:
+            kw = dict(kw, act_ref=w4a4_reference(run, rows))
     return oracle.latent_moe_forward(x, host(inp["W_router"]), host(inp["W_pool"]), expert_source(inp),
                                      host(inp["gamma"]), host(inp["W_unpool"]), w.k, w.eps, router_bias=bias,
                                      **kw)
@@ -128,7 +153,7 @@ def check_routing(ref: Dict[str, np.ndarray], gpu_idx: np.ndarray, gpu_g: np.nda
     return alt_tokens
 
 
-def oracle_on_gpu_alternatives(w, inp, rows, ref, gpu_idx, alt_tokens, **kw):
+def oracle_on_gpu_alternatives(w, inp, rows, ref, gpu_idx, alt_tokens, run=None, **kw):
     """For near-tie tokens, the oracle output under the oracle's alternative routing that
     the GPU chose (found in oracle.topk_alternatives), with the oracle's own weights."""
     out = ref["out"].copy()
@@ -139,7 +164,7 @@ def oracle_on_gpu_alternatives(w, inp, rows, ref, gpu_idx, alt_tokens, **kw):
                                        kw.get("routed_scaling", 1.0))
         else:
             g = oracle.softmax_weights(ref["logits"][t:t + 1], sel)
-        r1 = oracle_block(w, inp, rows[t:t + 1], routing=(sel, g), **kw)
+        r1 = oracle_block(w, inp, rows[t:t + 1], run=run, routing=(sel, g), **kw)
         out[t] = r1["out"][0]
     return out
 

@@ -94,6 +94,83 @@ def test_host_io_entry_point_matches_device_entry_point(mid):
     assert torch.equal(out_host, run.out.cpu())
 
 
+# ------------------------------------------------------------- W4A4 (NVFP4 activations)
+def test_nvfp4_activation_quantiser_bit_exact():
+    """The C-ABI quantiser against the oracle's on the same seeded bf16 rows: every code and
+    scale byte equal (rows of N(0, 1) values, of tiny values near the E4M3 subnormals, of
+    large values, and all-zero blocks)."""
+    w = W.Workload("quant", T=64, D=256, L=256, I=256, E=2, k=1, dtype="bf16", seed=21)
+    x = W.make_tensor(w, "x", "cuda")                           # [64, 256] bf16
+    x[8:16] *= 1e-3
+    x[16:24] *= 60.0
+    x[24, :16] = 0.0
+    x[25] = 0.0
+    codes = torch.empty((64, 128), dtype=torch.uint8, device="cuda")
+    scales = torch.empty((64, 16), dtype=torch.uint8, device="cuda")
+    moe.quantize_nvfp4_rows(x, codes, scales)
+    torch.cuda.synchronize()
+    ref_c, ref_s = oracle.quantize_activations_nvfp4(host(x))
+    np.testing.assert_array_equal(scales.cpu().numpy(), ref_s)
+    np.testing.assert_array_equal(codes.cpu().numpy(), ref_c)
+
+
+W4A4 = [
+    # name, T, D, L, I, E, k
+    ("w4a4_tiles128", 256, 1024, 512, 512, 16, 4),
+    ("w4a4_tiles32", 16, 1024, 512, 512, 32, 2),
+    ("w4a4_ragged", 300, 512, 256, 768, 8, 3),
+    # several tiles per CTA and K = 2048: the stage and scale-slot rings wrap many times
+    ("w4a4_many_tiles", 2048, 512, 2048, 2048, 64, 4),
+]
+
+
+@pytest.mark.parametrize("case", W4A4, ids=[c[0] for c in W4A4])
+def test_w4a4_experts(case):
+    """NVFP4 weights and activations (tcgen05 kind::mxf4nvf4) against the oracle running the
+    same quantiser on its own activations and the dequantised weight codes."""
+    name, T, D, L, I, E, k = case
+    w = W.Workload(name, T=T, D=D, L=L, I=I, E=E, k=k, dtype="bf16", seed=13, experts="nvfp4", act="nvfp4")
+    inp = W.make_inputs(w, "cuda")
+    run = Run(w, inp)
+    assert moe.stages(run.model.config(T))[6] == "gather_quant"
+    rows = np.arange(T)
+    ref = oracle_block(w, inp, rows, run=run)
+    gidx = run.idx.cpu().numpy()
+    alts = check_routing(ref, gidx, run.g.cpu().numpy(), w.k)
+    ref_out = oracle_on_gpu_alternatives(w, inp, rows, ref, gidx, alts, run=run)
+    r, _ = assert_close(host(run.out), ref_out, f"{name} out", rel=NVFP4_REL_L2)
+    decisions = T * k * (L + I) * 17 // 16          # codes and block scales of z and h
+    print(f"{name}: rel-L2 {r:.2e}; boundary decisions adopted {ref['act_adopted']} of {decisions}")
+    assert ref["act_adopted"] <= 1e-3 * decisions
+    if not alts:
+        R = run.layout["rows"]
+        ginv = run.inter("inv", torch.int32, (T * k,)).cpu().numpy()
+        y = host(run.inter("y", torch.bfloat16, (R, L)))[ginv].reshape(T, k, L)
+        assert_close(y, ref["y"], f"{name} expert outputs", rel=NVFP4_REL_L2)
+        # the quantised latent rows in expert order: every scale byte equal to the oracle's
+        # quantisation of its own bf16-rounded z, codes equal except where the two bf16 values
+        # of z differ (a float32 vs float64 accumulation crossing a bf16 rounding boundary)
+        zq_s = run.inter("zq_scales", torch.uint8, (R, L // 16)).cpu().numpy()[ginv]
+        ref_c, ref_s = oracle.quantize_activations_nvfp4(oracle.round_bf16(np.repeat(ref["z"], k, axis=0)))
+        assert np.mean(zq_s != ref_s) < 1e-3
+
+
+@pytest.mark.slow
+def test_full_size_w4a4_layer_sampled_tokens():
+    w = W.WORKLOADS["nvfp4_w4a4"]
+    inp = W.make_inputs(w, "cuda")
+    run = Run(w, inp)
+    rows = np.sort(np.random.default_rng(4).choice(w.T, size=10, replace=False))
+    ref = oracle_block(w, inp, rows, run=run)
+    gidx = run.idx.cpu().numpy()[rows]
+    alts = check_routing(ref, gidx, run.g.cpu().numpy()[rows], w.k)
+    ref_out = oracle_on_gpu_alternatives(w, inp, rows, ref, gidx, alts, run=run)
+    r, _ = assert_close(host(run.out)[rows], ref_out, "w4a4 layer out", rel=NVFP4_REL_L2)
+    decisions = len(rows) * w.k * (w.L + w.I) * 17 // 16
+    print(f"w4a4 full layer: rel-L2 {r:.2e}; boundary decisions adopted {ref['act_adopted']} of {decisions}")
+    assert ref["act_adopted"] <= 1e-3 * decisions
+
+
 # ------------------------------------------------------------------------- CUDA graphs
 GRAPH = [
     # name, T, D, L, I, E, k: decode-sized tiles (one-CTA kernels), and CTA-pair tiles whose

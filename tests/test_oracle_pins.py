@@ -554,3 +554,47 @@ def test_w4a4_expert_matches_dequantised_operands():
     a = zq @ b["W_gate"][e].T
     h = oracle.nvfp4_activation(a / (1 + np.exp(-a)) * (zq @ b["W_up"][e].T))
     np.testing.assert_allclose(got["y"][0, 0], (h @ b["W_down"][e].T)[0], rtol=1e-12, atol=1e-12)
+
+
+def test_activation_quantiser_adopts_only_boundary_decisions():
+    """Another implementation's decision is adopted only where the input sits within 2^-7 of
+    the rounding boundary between two adjacent values; any other difference is an error."""
+    base = np.zeros((1, 16), np.float32)
+    base[0, 0] = 3.0                            # amax 3 -> scale E4M3(0.5) = 0x30, exact
+    own_c, own_s = oracle.quantize_activations_nvfp4(base)
+    n = [0]
+    c, s = oracle.quantize_activations_nvfp4(base, ref=(own_c, own_s), adopted=n)
+    assert n[0] == 0 and np.array_equal(c, own_c) and np.array_equal(s, own_s)
+
+    def with_code(x, i, code):
+        c0, s0 = oracle.quantize_activations_nvfp4(x)
+        u = oracle.unpack_nibbles(c0)
+        u[0, i] = code
+        return (u[:, 0::2] | (u[:, 1::2] << 4)).astype(np.uint8), s0
+
+    near = base.copy()
+    near[0, 1] = np.float32(0.5 * 1.2501)       # q = 1.2501: just above the 1 / 1.5 midpoint -> 1.5
+    assert oracle.unpack_nibbles(oracle.quantize_activations_nvfp4(near)[0])[0, 1] == 3
+    n = [0]
+    c, _ = oracle.quantize_activations_nvfp4(near, ref=with_code(near, 1, 2), adopted=n)
+    assert n[0] == 1 and oracle.unpack_nibbles(c)[0, 1] == 2
+    far = base.copy()
+    far[0, 1] = np.float32(0.5 * 1.4)           # q = 1.4: well inside the 1.5 interval
+    with pytest.raises(ValueError):
+        oracle.quantize_activations_nvfp4(far, ref=with_code(far, 1, 2))
+    with pytest.raises(ValueError):             # code 5 (value 3) is not a neighbour of 3 (value 1.5)
+        oracle.quantize_activations_nvfp4(near, ref=with_code(near, 1, 5))
+    # a scale near the midpoint of E4M3 0.5 (0x30) and 0.5625 (0x31): amax / 6 = 0.53126
+    sc = np.zeros((1, 16), np.float32)
+    sc[0, 0] = np.float32(6 * 0.53126)
+    _, s_own = oracle.quantize_activations_nvfp4(sc)
+    assert s_own[0, 0] == 0x31
+    forced = sc.copy()
+    n = [0]
+    ref_c = oracle.quantize_activations_nvfp4(forced)[0]
+    # the other implementation chose 0x30 and coded the block with it (6.37 -> saturates at 6)
+    q_other = np.array([[0x7] + [0] * 7], np.uint8)
+    c, s = oracle.quantize_activations_nvfp4(sc, ref=(q_other, np.array([[0x30]], np.uint8)), adopted=n)
+    assert s[0, 0] == 0x30 and n[0] == 1
+    with pytest.raises(ValueError):             # a scale two steps away is never adopted
+        oracle.quantize_activations_nvfp4(sc, ref=(ref_c, np.array([[0x2F]], np.uint8)))

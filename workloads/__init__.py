@@ -46,6 +46,7 @@ class Workload:
     routing: str = "uniform"   # "uniform" (no bias) or "zipf" (selection bias, s=1.2)
     seed: int = 0
     experts: str = "bf16"      # expert weight storage: "bf16" (the dtype) or "nvfp4"
+    act: str = "bf16"          # expert GEMM activations: "bf16" or "nvfp4" (W4A4)
 
     def with_tokens(self, T: int) -> "Workload":
         return dataclasses.replace(self, T=T)
@@ -68,6 +69,11 @@ WORKLOADS: Dict[str, Workload] = {
     # decode-like NVFP4 case on ~1 GB of weights (2-3 tokens per expert; profiling captures)
     "nvfp4_decode_e32": Workload("nvfp4_decode_e32", T=32, D=8192, L=4096, I=4096, E=32, k=2, dtype="bf16",
                                  experts="nvfp4"),
+    # the same NVFP4 layers with both operands of the expert GEMMs in NVFP4 (W4A4)
+    "nvfp4_w4a4": Workload("nvfp4_w4a4", T=4096, D=8192, L=4096, I=4096, E=256, k=8, dtype="bf16",
+                           experts="nvfp4", act="nvfp4"),
+    "nvfp4_w4a4_decode": Workload("nvfp4_w4a4_decode", T=64, D=8192, L=4096, I=4096, E=256, k=8, dtype="bf16",
+                                  experts="nvfp4", act="nvfp4"),
 }
 
 # tensor ids of the generator (fixed, part of the workload definition)
