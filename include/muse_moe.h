@@ -86,10 +86,10 @@ typedef struct muse_nvfp4_weight {
 typedef enum muse_act_format {
   MUSE_ACT_BF16 = 0,          /* W4A16: activations stay bf16                           */
   MUSE_ACT_NVFP4 = 1          /* W4A4 (deep dive §7.4): the latent rows and the SwiGLU
-                                 output are quantised per 16 values to E2M1 codes with an
-                                 E4M3 scale E4M3(amax / 6) (nearest, ties to even, float32
-                                 arithmetic, no tensor scale) and the tensor core reads
-                                 both operands as 4-bit codes; requires NVFP4 experts and
+                                 output are quantised per 16 values: scale E4M3(amax / 6),
+                                 codes the E2M1 values nearest to value / scale (ties to
+                                 even, no tensor scale); the tensor core reads both
+                                 operands as 4-bit codes; requires NVFP4 experts and
                                  L, I multiples of 256                                   */
 } muse_act_format;
 
@@ -255,8 +255,9 @@ MUSE_API muse_status muse_selftest_bounded_wait(uint64_t limit_ns, uint32_t* sta
  * and to h, muse_act_format): rows x K bf16 values (device, row-major, 16-byte aligned, K a
  * multiple of 16) -> codes uint8 [rows, K/2] (two E2M1 codes per byte, low nibble = even
  * element; 16-byte aligned) and scales uint8 [rows, K/16] (E4M3), per block of 16 values
- * scale = E4M3(amax / 6), code = E2M1(value / scale), nearest with ties to even, float32
- * arithmetic. Enqueued on `stream`; INVALID_ARG for null / misaligned pointers or sizes. */
+ * scale = E4M3(amax / 6) (amax / 6 in float32), code = the E2M1 value nearest to the exact
+ * quotient value / scale, ties to even. Enqueued on `stream`; INVALID_ARG for null /
+ * misaligned pointers or sizes. */
 MUSE_API muse_status muse_quantize_nvfp4_rows(const void* src, int64_t rows, int64_t K, void* codes,
                                               void* scales, void* stream);
 

@@ -14,8 +14,10 @@
 // warp of m's lane quadrant; token row n's word at column sfb + 4 kk + n / 32 in every lane
 // quadrant (each scale warp writes the same words into its own quadrant).
 //
-// Roles (320 threads, one CTA per SM): warp 0 TMA producer, warp 1 TMEM owner + UMMA
-// issuer, warps 2..5 epilogue, warps 6..9 scale warps (warp w serves lane quadrant w % 4).
+// Roles (448 threads, one CTA per SM): warp 0 TMA producer, warp 1 TMEM owner + UMMA
+// issuer, warps 2..5 scale warps (warp w serves lane quadrant w % 4), warps 6..13 epilogue
+// in two groups of four taking alternate 32-token chunks (the 4-bit main loop is short, so
+// the single-buffered accumulator's drain must be too).
 // Barriers: per TMA stage full (bytes) / empty (UMMA commit -- after the scale warps have
 // read the stage, since the UMMA waits for them); per TMEM scale slot sfull (4 scale
 // warps) / sfree (UMMA commit); accumulator full / empty. Every wait is bounded (ptx.cuh).
@@ -67,7 +69,7 @@ struct W4A4Shape {
   static_assert(8 * (2 * kStages + 2 * kSlots + 4) + 8 <= 512, "barrier area");
 };
 
-constexpr int kW4A4Threads = 320;
+constexpr int kW4A4Threads = 448;
 
 template <int BN, int EPI, int MT>
 __global__ void __launch_bounds__(kW4A4Threads, 1)
@@ -114,7 +116,7 @@ __global__ void __launch_bounds__(kW4A4Threads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(accf_bar(a), 1);
-      mbar_init(acce_bar(a), 4);
+      mbar_init(acce_bar(a), 8);  // 8 epilogue warps
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -242,8 +244,8 @@ __global__ void __launch_bounds__(kW4A4Threads, 1)
       }
     }
     __syncwarp();
-  } else if (warp >= 6) {
-    // ---------------------------------------------------------------- scale warps
+  } else if (warp < 6) {
+    // ---------------------------------------------------------------- scale warps (2..5)
     const int quad = warp & 3;
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
     int stage = 0, cs = 0;
@@ -301,8 +303,9 @@ __global__ void __launch_bounds__(kW4A4Threads, 1)
       }
     }
   } else {
-    // ---------------------------------------------------------------- epilogue
+    // ---------------------------------------------------------------- epilogue (6..13)
     const int qd = warp & 3;
+    const int grp = (warp - 6) >> 2;  // chunks c with c % 2 == grp
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
@@ -320,7 +323,7 @@ __global__ void __launch_bounds__(kW4A4Threads, 1)
         const float ms_u = q.mscale_a2[g];
         const int f = m0 + qd * 32 + lane;
         const bool f_ok = f < p.m_valid;
-        for (int c = 0; c < nchunks; ++c) {
+        for (int c = grp; c < nchunks; c += 2) {
           uint32_t v[32], u[32];
           tmem_ld32(taddr + 32u * c, v);
           tmem_ld32(taddr + BN + 32u * c, u);
@@ -329,7 +332,7 @@ __global__ void __launch_bounds__(kW4A4Threads, 1)
           for (int i = 0; i < 32; ++i) {
             const int tok = c * 32 + i;
             const float a = __uint_as_float(v[i]) * ms_a;
-            const float h = a / (1.0f + expf(-a)) * (__uint_as_float(u[i]) * ms_u);  // SiLU(gate) * up
+            const float h = __fdividef(a, 1.0f + __expf(-a)) * (__uint_as_float(u[i]) * ms_u);  // SiLU(gate) * up
             if (tok < n && f_ok) out[(static_cast<int64_t>(row0) + tok) * p.ld_out + f] = from_f32<TOut>(h);
           }
         }
@@ -342,7 +345,7 @@ __global__ void __launch_bounds__(kW4A4Threads, 1)
           float gain1 = 1.0f;
           if (EPI == EPI_STORE_SS && p.ss_gain != nullptr && f_ok)
             gain1 = 1.0f + to_f32(reinterpret_cast<const __nv_bfloat16*>(p.ss_gain)[g * p.ss_gain_group_stride + f]);
-          for (int c = 0; c < nchunks; ++c) {
+          for (int c = grp; c < nchunks; c += 2) {
             uint32_t v[32];
             tmem_ld32(taddr + static_cast<uint32_t>(half * BN) + 32u * c, v);
             tmem_ld_wait();

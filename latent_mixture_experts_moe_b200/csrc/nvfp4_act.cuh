@@ -3,11 +3,13 @@
 // The released checkpoint quantises both operands of the expert GEMMs (Muse Spark Open deep
 // dive §7.4): per block of 16 consecutive values of a row, one E4M3 scale and sixteen 4-bit
 // E2M1 codes (OCP Microscaling formats v1.0). Here, with no tensor-wide scale:
-//   scale = E4M3(amax / 6), code_i = E2M1(v_i / decoded scale)
-// both rounded to nearest with ties to even, E2M1 saturating at +-6; amax, the division by
-// 6 and v_i / scale are IEEE float32 operations on the float32 value of the stored bfloat16
-// activation. Codes are packed two per byte, the low nibble holding the even element, the
-// same packing as the NVFP4 expert weights.
+//   scale = E4M3(amax / 6), code_i = the E2M1 value nearest to the exact quotient v_i / scale
+// both with ties to even, E2M1 saturating at +-6; amax / 6 is one IEEE float32 division on
+// the float32 values of the stored bfloat16 activation. The code needs no division: the
+// rounding boundaries of v / scale are the E2M1 midpoints t times scale, products of at most
+// 3 and 4 significant bits and so exact in float32, and |v| is compared with them. Codes
+// are packed two per byte, the low nibble holding the even element, the same packing as the
+// NVFP4 expert weights.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -31,17 +33,17 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
   return (b & 0x80u) ? -v : v;
 }
 
-// 4-bit E2M1 code of q: the magnitude index counts the rounding boundaries below |q| (the
-// midpoints 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5 between the magnitudes 0, 0.5, 1, 1.5, 2, 3,
-// 4, 6), each midpoint going to the neighbour with an even index; the sign bit only on a
-// nonzero magnitude. NaN compares false everywhere and gives 0.
-__device__ __forceinline__ uint32_t e2m1_rne(float q) {
-  const float a = fabsf(q);
-  const uint32_t m = static_cast<uint32_t>(a > 0.25f) + static_cast<uint32_t>(a >= 0.75f) +
-                     static_cast<uint32_t>(a > 1.25f) + static_cast<uint32_t>(a >= 1.75f) +
-                     static_cast<uint32_t>(a > 2.5f) + static_cast<uint32_t>(a >= 3.5f) +
-                     static_cast<uint32_t>(a > 5.0f);
-  return (q < 0.0f && m != 0u) ? (m | 8u) : m;
+// 4-bit E2M1 code of v / s given the boundaries b[i] = t_i * s: the magnitude index counts
+// the midpoints t = 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5 (between the magnitudes 0, 0.5, 1,
+// 1.5, 2, 3, 4, 6) below |v| / s, a value exactly on a midpoint going to the neighbour with
+// an even index; the sign bit only on a nonzero magnitude. NaN compares false and gives 0.
+__device__ __forceinline__ uint32_t e2m1_code(float v, const float (&b)[7]) {
+  const float a = fabsf(v);
+  const uint32_t m = static_cast<uint32_t>(a > b[0]) + static_cast<uint32_t>(a >= b[1]) +
+                     static_cast<uint32_t>(a > b[2]) + static_cast<uint32_t>(a >= b[3]) +
+                     static_cast<uint32_t>(a > b[4]) + static_cast<uint32_t>(a >= b[5]) +
+                     static_cast<uint32_t>(a > b[6]);
+  return (v < 0.0f && m != 0u) ? (m | 8u) : m;
 }
 
 // One block of 16 values -> 8 code bytes (two words, element 2i in the low nibble of byte i)
@@ -54,8 +56,9 @@ __device__ __forceinline__ void quant_block16(const float (&v)[16], uint2& codes
   const float s = e4m3_to_f32(sbyte);
   uint32_t w[2] = {0u, 0u};
   if (s > 0.0f) {
+    const float b[7] = {0.25f * s, 0.75f * s, 1.25f * s, 1.75f * s, 2.5f * s, 3.5f * s, 5.0f * s};  // exact
 #pragma unroll
-    for (int i = 0; i < 16; ++i) w[i >> 3] |= e2m1_rne(v[i] / s) << (4 * (i & 7));
+    for (int i = 0; i < 16; ++i) w[i >> 3] |= e2m1_code(v[i], b) << (4 * (i & 7));
   }
   codes = make_uint2(w[0], w[1]);
 }

@@ -18,11 +18,12 @@ infinities, largest value 448.
 
 Activations of the W4A4 mode (deep dive §7.4: the released checkpoint quantises both
 operands of the expert GEMMs) use the same element and block formats without a tensor
-scale: per block of 16 consecutive values of a row, scale = E4M3(amax / 6) and code =
-E2M1(value / scale), both rounded to nearest with ties to even, E2M1 saturating at 6. The
-arithmetic is single precision, as the kernels do it (the rounding decisions are then taken
-in the same precision on both sides): amax and value / scale are float32 operations on the
-float32 value of the stored bfloat16 activation.
+scale: per block of 16 consecutive values of a row, scale = E4M3(amax / 6) (amax / 6 one
+float32 division, as the kernels do it) and code = the E2M1 value nearest to the exact
+quotient value / scale, both with ties to even, E2M1 saturating at 6. The quotient is taken
+in float64, which orders it exactly against the E2M1 midpoints: scale has 4 significant
+bits, so a value that is not exactly a midpoint times scale differs from it by at least one
+float32 unit, far more than float64 rounding.
 """
 from __future__ import annotations
 
@@ -130,15 +131,15 @@ def quantize_activations_nvfp4(x, ref=None, rel_tol: float = 2.0 ** -7, adopted=
             sbyte = np.where(diff, rs, sbyte)
             if adopted is not None:
                 adopted[0] += int(diff.sum())
-    sdec = decode_e4m3(sbyte).astype(np.float32)                     # exact in float32
+    sdec = decode_e4m3(sbyte)                                        # exact
     with np.errstate(divide="ignore", invalid="ignore"):
-        q = np.where(sdec[..., None] > 0, blocks / sdec[..., None], np.float32(0.0)).astype(np.float32)
-    codes = round_e2m1(q.astype(np.float64)).reshape(x32.shape)
+        q = np.where(sdec[..., None] > 0, blocks.astype(np.float64) / sdec[..., None], 0.0)
+    codes = round_e2m1(q).reshape(x32.shape)
     if ref is not None:
         rc = unpack_nibbles(np.asarray(ref[0], dtype=np.uint8)).reshape(codes.shape)
         diff = rc != codes
         if diff.any():
-            qd = q.reshape(codes.shape)[diff].astype(np.float64)
+            qd = q.reshape(codes.shape)[diff]
             a, b = codes[diff].astype(int), rc[diff].astype(int)
             same_side = ((a & 8) == (b & 8)) | ((a & 7) == 0) | ((b & 7) == 0)
             adjacent = same_side & (np.abs((a & 7) - (b & 7)) == 1)
