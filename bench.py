@@ -132,7 +132,8 @@ def stage_work(w: W.Workload, n_touched: int):
         "ffn_pre_norm": (0, 2 * T * D * a + D * a),
         "ffn_post_norm_gate": (0, 3 * T * D * a + T * (D // 32) * 4 + D * (a + 4)),
         # W4A4: latent rows gathered and quantised (0.5625 B per value out), h quantised
-        "gather_quant": (0, T * L * a + A * L * 0.5625),
+        "quant_z": (0, T * L * a + T * L * 0.5625),
+        "gather_codes": (0, T * L * 0.5625 + A * L * 0.5625),
         "quant_h": (0, A * I * a + A * I * 0.5625),
     }
 

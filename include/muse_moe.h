@@ -266,10 +266,10 @@ MUSE_API const char* muse_status_string(muse_status s);
 
 /* Number of kernel launches one forward call makes for cfg: 11, plus one each for the
  * pre-expert norm, the pre-FFN norm, the post-FFN norm / residual gate (one kernel
- * finishes both) and the W4A4 quantisation of h. In launch order: [ffn pre norm], router,
- * top-k, histogram, tiles, assign rows, pooler, [pre-expert norm], gather (W4A4: gather and
- * quantise), gate/up, [quantise h], down, norm + combine, unpooler, [post norm / gate].
- * stage_events must hold this many + 1 events. */
+ * finishes both) and two for W4A4. In launch order: [ffn pre norm], router, top-k,
+ * histogram, tiles, assign rows, pooler, [pre-expert norm], [W4A4: quantise z], gather (W4A4:
+ * of the quantised bytes), gate/up, [W4A4: quantise h], down, norm + combine, unpooler,
+ * [post norm / gate]. stage_events must hold this many + 1 events. */
 MUSE_API int32_t muse_latent_moe_launch_count(const muse_moe_config* cfg);
 
 #ifdef __cplusplus

@@ -202,7 +202,8 @@ def stages(cfg: Config):
     if cfg.pre_norm_gain:
         names.insert(names.index("gather"), "pre_expert_norm")
     if cfg.act_format == ACT_NVFP4:
-        names[names.index("gather")] = "gather_quant"
+        names[names.index("gather")] = "gather_codes"
+        names.insert(names.index("gather_codes"), "quant_z")
         names.insert(names.index("gate_up_swiglu") + 1, "quant_h")
     if cfg.ffn_pre_gain:
         names.insert(0, "ffn_pre_norm")

@@ -45,6 +45,7 @@ int dense_bn(const muse_moe_config& c) { return c.T <= 32 ? 32 : 256; }
 struct Layout {
   muse_moe_workspace_layout pub;
   size_t tiles_gu, tiles_dn, ntiles;  // int4 lists; int[8]: tile counts [0..1], tile counters [4..7]
+  size_t zt_codes, zt_scales;         // W4A4: the latent quantised in token order [T, L/2], [T, L/16]
   int64_t max_tiles_gu, max_tiles_dn;
 };
 
@@ -85,7 +86,10 @@ Layout make_layout(const muse_moe_config& c) {
   l.pub.c = take(as * T * c.L);
   l.pub.xn = c.ffn_pre_gain != nullptr ? take(as * T * c.D) : 0;
   l.pub.ss_out = c.ffn_post_gain != nullptr ? take(sizeof(float) * T * (c.D / 32)) : 0;
+  l.zt_codes = l.zt_scales = 0;
   if (w4a4(c)) {
+    l.zt_codes = take(T * (c.L / 2));
+    l.zt_scales = take(T * (c.L / 16));
     l.pub.zq_codes = take(rows * (c.L / 2));
     l.pub.zq_scales = take(rows * (c.L / 16));
     l.pub.hq_codes = take(rows * (c.I / 2));
@@ -501,8 +505,17 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
   uint8_t* hq_scales = at(lay.pub.hq_scales);
   const int quant_grid = static_cast<int>(std::min<int64_t>(lay.pub.rows, 16 * nsm));
   if (q4a) {
-    k_quant_rows_nvfp4<<<quant_grid, 256, 0, st>>>(row_token, offsets + E, 0, reinterpret_cast<const __nv_bfloat16*>(z),
-                                                   static_cast<int>(L), 1, zq_codes, zq_scales);
+    uint8_t* zt_codes = at(lay.zt_codes);
+    uint8_t* zt_scales = at(lay.zt_scales);
+    k_quant_rows_nvfp4<<<static_cast<unsigned>(std::min<int64_t>(Tn, 16 * nsm)), 256, 0, st>>>(
+        nullptr, nullptr, static_cast<int>(Tn), reinterpret_cast<const __nv_bfloat16*>(z), static_cast<int>(L),
+        zt_codes, zt_scales);
+    MUSE_CK(cudaGetLastError());
+    MUSE_CK(mark());
+    k_gather_nvfp4_rows<<<quant_grid, 128, 0, st>>>(row_token, offsets + E, reinterpret_cast<const uint4*>(zt_codes),
+                                                    reinterpret_cast<const uint4*>(zt_scales),
+                                                    reinterpret_cast<uint4*>(zq_codes),
+                                                    reinterpret_cast<uint4*>(zq_scales), static_cast<int>(L));
     MUSE_CK(cudaGetLastError());
     MUSE_CK(mark());
   } else {
@@ -563,7 +576,7 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
   // W4A4: quantise h (already in expert order) for the down projection
   if (q4a) {
     k_quant_rows_nvfp4<<<quant_grid, 256, 0, st>>>(row_token, offsets + E, 0, reinterpret_cast<const __nv_bfloat16*>(h),
-                                                   static_cast<int>(I), 0, hq_codes, hq_scales);
+                                                   static_cast<int>(I), hq_codes, hq_scales);
     MUSE_CK(cudaGetLastError());
     MUSE_CK(mark());
   }
@@ -813,7 +826,7 @@ muse_status muse_quantize_nvfp4_rows(const void* src, int64_t rows, int64_t K, v
   if (rows < 1 || K < 16 || K % 16 != 0 || rows > (int64_t(1) << 30) || K > (int64_t(1) << 20)) return MUSE_ERR_INVALID_ARG;
   const int grid = static_cast<int>(std::min<int64_t>(rows, 16 * sm_count()));
   k_quant_rows_nvfp4<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      nullptr, nullptr, static_cast<int>(rows), static_cast<const __nv_bfloat16*>(src), static_cast<int>(K), 0,
+      nullptr, nullptr, static_cast<int>(rows), static_cast<const __nv_bfloat16*>(src), static_cast<int>(K),
       static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales));
   return cudaGetLastError() == cudaSuccess ? MUSE_OK : MUSE_ERR_CUDA;
 }
@@ -843,7 +856,7 @@ int32_t muse_latent_moe_launch_count(const muse_moe_config* cfg) {
   // and the optional sublayer pre-norm (first), pre-expert norm (between pooler and
   // gather) and sublayer post-norm / residual gate (last)
   return 11 + (cfg->pre_norm_gain != nullptr) + (cfg->ffn_pre_gain != nullptr) +
-         (cfg->ffn_post_gain != nullptr || cfg->residual_gate != nullptr) + (cfg->act_format == MUSE_ACT_NVFP4);
+         (cfg->ffn_post_gain != nullptr || cfg->residual_gate != nullptr) + 2 * (cfg->act_format == MUSE_ACT_NVFP4);
 }
 
 }  // extern "C"
