@@ -21,6 +21,11 @@
 // Barriers: per TMA stage full (bytes) / empty (UMMA commit -- after the scale warps have
 // read the stage, since the UMMA waits for them); per TMEM scale slot sfull (4 scale
 // warps) / sfree (UMMA commit); accumulator full / empty. Every wait is bounded (ptx.cuh).
+// Tiles: with a tile counter the producer claims the CTA's next tile from it (atomicAdd)
+// and hands the index to the other roles through a 4-slot ring in shared memory, so CTAs
+// that free up one after the other take consecutive tiles -- the token chunks of one
+// expert's weight tile start together and DRAM delivers the tile once; without a counter,
+// static round robin.
 #pragma once
 
 #include "gemm_umma.cuh"
@@ -66,7 +71,9 @@ struct W4A4Shape {
   static constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes + 512;
   static_assert(kStages >= 2, "tile too large for the shared-memory ring");
   static_assert(kSlots >= 2, "no TMEM room for the scale slots");
-  static_assert(8 * (2 * kStages + 2 * kSlots + 4) + 8 <= 512, "barrier area");
+  static constexpr int kSched = 4;
+  static constexpr int kSchedReaders = 1 + 4 + 8;  // UMMA thread, scale warps, epilogue warps
+  static_assert(8 * (2 * kStages + 2 * kSlots + 4 + 2 * kSched) + 8 + 4 * kSched <= 512, "barrier area");
 };
 
 constexpr int kW4A4Threads = 448;
@@ -83,9 +90,11 @@ __global__ void __launch_bounds__(kW4A4Threads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * S::kStageBytes);
-  // bars: full[kStages], empty[kStages], sfull[kSlots], sfree[kSlots], accf[2], acce[2]
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 2 * kSlots + 4);
+  // bars: full[kStages], empty[kStages], sfull[kSlots], sfree[kSlots], accf[2], acce[2],
+  // tfull[kSched], tempty[kSched]
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 2 * kSlots + 4 + 2 * S::kSched);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  volatile int* tile_ring = reinterpret_cast<volatile int*>(tmem_holder + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -96,6 +105,8 @@ __global__ void __launch_bounds__(kW4A4Threads, 1)
   auto sfree_bar = [&](int c) { return bar0 + 8u * (2 * kStages + kSlots + c); };
   auto accf_bar = [&](int a) { return bar0 + 8u * (2 * kStages + 2 * kSlots + a); };
   auto acce_bar = [&](int a) { return bar0 + 8u * (2 * kStages + 2 * kSlots + 2 + a); };
+  auto tfull_bar = [&](int i) { return bar0 + 8u * (2 * kStages + 2 * kSlots + 4 + i); };
+  auto tempty_bar = [&](int i) { return bar0 + 8u * (2 * kStages + 2 * kSlots + 4 + S::kSched + i); };
   // stage layout: weight codes (MT x 16 KB), token codes, weight scales (MT x 2 KB), token scales
   auto code_tile = [&](int s, int m) { return smem + s * S::kStageBytes + m * S::kCodeBytes; };
   auto b_tile = [&](int s) { return smem + s * S::kStageBytes + MT * S::kCodeBytes; };
@@ -118,6 +129,10 @@ __global__ void __launch_bounds__(kW4A4Threads, 1)
       mbar_init(accf_bar(a), 1);
       mbar_init(acce_bar(a), 8);  // 8 epilogue warps
     }
+    for (int i = 0; i < S::kSched; ++i) {
+      mbar_init(tfull_bar(i), 1);
+      mbar_init(tempty_bar(i), S::kSchedReaders);
+    }
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&maps.a);
@@ -138,6 +153,35 @@ __global__ void __launch_bounds__(kW4A4Threads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const int num_tiles = *p.num_tiles_dev;
+  const bool dyn = p.tile_counter != nullptr;
+
+  // The CTA's i-th tile: -1 past the end, -2 when a wait gave up. The producer claims and
+  // publishes it; the other roles receive it (one thread or a whole warp) and free the slot
+  // (one arrival per thread or warp).
+  auto claim_publish = [&](int i) -> int {
+    int t = dyn ? atomicAdd(p.tile_counter, 1) : static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
+    if (t >= num_tiles) t = -1;
+    if (!dyn) return t;
+    const int sl = i % S::kSched;
+    const uint32_t ph = static_cast<uint32_t>(i / S::kSched) & 1u;
+    if (!mbar_wait(tempty_bar(sl), ph ^ 1u, abort_flag, p.status, 0x1700u + sl)) return -2;
+    tile_ring[sl] = t;
+    mbar_arrive(tfull_bar(sl));
+    return t;
+  };
+  auto receive = [&](int i, uint32_t code) -> int {
+    if (!dyn) {
+      const int t = static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
+      return t < num_tiles ? t : -1;
+    }
+    const int sl = i % S::kSched;
+    const uint32_t ph = static_cast<uint32_t>(i / S::kSched) & 1u;
+    if (!mbar_wait(tfull_bar(sl), ph, abort_flag, p.status, code + sl)) return -2;
+    return tile_ring[sl];
+  };
+  auto release = [&](int i) {
+    if (dyn) mbar_arrive(tempty_bar(i % S::kSched));
+  };
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
@@ -146,7 +190,13 @@ __global__ void __launch_bounds__(kW4A4Threads, 1)
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_phase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+      for (int i = 0; ok; ++i) {
+        const int t = claim_publish(i);
+        if (t == -2) {
+          ok = false;
+          break;
+        }
+        if (t < 0) break;
         int g, m0, row0, n;
         gemm_tile(p, t, BN, g, m0, row0, n);
         const int a_row = g * p.rows_per_group + m0;
@@ -187,7 +237,14 @@ __global__ void __launch_bounds__(kW4A4Threads, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       bool issued_any = false;
-      for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+      for (int i = 0; ok; ++i) {
+        const int t = receive(i, 0x1800u);
+        if (t == -2) {
+          ok = false;
+          break;
+        }
+        release(i);
+        if (t < 0) break;
         int g, m0, row0, n;
         gemm_tile(p, t, BN, g, m0, row0, n);
         const uint32_t N = static_cast<uint32_t>((n + 15) & ~15);
@@ -251,7 +308,13 @@ __global__ void __launch_bounds__(kW4A4Threads, 1)
     int stage = 0, cs = 0;
     uint32_t phase = 0, cphase = 0;
     bool ok = true;
-    for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+    for (int i = 0; ok; ++i) {
+      int t = receive(i, 0x1900u);
+      if (!__all_sync(0xffffffffu, t != -2)) break;
+      t = __shfl_sync(0xffffffffu, t, 0);
+      __syncwarp();
+      if (lane == 0) release(i);
+      if (t < 0) break;
       for (int kb = 0; kb < p.k_blocks; ++kb) {
         const bool ready = mbar_wait(full_bar(stage), phase, abort_flag, p.status, 0x1400u + stage) &&
                            mbar_wait(sfree_bar(cs), cphase ^ 1u, abort_flag, p.status, 0x1500u + cs);
@@ -308,7 +371,13 @@ __global__ void __launch_bounds__(kW4A4Threads, 1)
     const int grp = (warp - 6) >> 2;  // chunks c with c % 2 == grp
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+    for (int i = 0;; ++i) {
+      int t = receive(i, 0x1A00u);
+      if (!__all_sync(0xffffffffu, t != -2)) break;
+      t = __shfl_sync(0xffffffffu, t, 0);
+      __syncwarp();
+      if (lane == 0) release(i);
+      if (t < 0) break;
       int g, m0, row0, n;
       gemm_tile(p, t, BN, g, m0, row0, n);
       const bool ready = mbar_wait(accf_bar(acc), acc_phase, abort_flag, p.status, 0x1600u + acc);

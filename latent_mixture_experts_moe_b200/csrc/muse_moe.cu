@@ -562,6 +562,7 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
       if (!make_w4a4_maps(&wm, wg, wu, E * I, zq_codes, zq_scales, R, L, bn_g)) return MUSE_ERR_CUDA;
       const W4A4Args wq{wg->matrix_scale, wu->matrix_scale};
       g.k_blocks = static_cast<int>(L / 256);
+      g.tile_counter = ntiles + 4;
       MUSE_CK(launch_gemm_w4a4<EPI_SWIGLU>(bn_g, wm, g, wq, nsm, st));
     } else if (fp4) {
       MUSE_CK(launch_gemm_fp4<EPI_SWIGLU>(bn_g, 2, maps, g, q4, nsm, st));
@@ -620,6 +621,7 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
       if (!make_w4a4_maps(&wm, wd, wd, E * L, hq_codes, hq_scales, R, I, bn_g)) return MUSE_ERR_CUDA;
       const W4A4Args wq{wd->matrix_scale, wd->matrix_scale};
       g.k_blocks = static_cast<int>(I / 256);
+      g.tile_counter = ntiles + 5;
       MUSE_CK(launch_gemm_w4a4<EPI_STORE_SS>(bn_g, wm, g, wq, nsm, st));
     } else if (fp4) {
       MUSE_CK(launch_gemm_fp4<EPI_STORE_SS>(bn_g, pdn.mt, maps, g, q4, nsm, st));
