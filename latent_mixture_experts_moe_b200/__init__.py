@@ -232,7 +232,7 @@ def quantize_nvfp4_rows(src, codes, scales, stream=None) -> None:
 def selftest_bounded_wait(limit_ns: int, status_dev, stream=None) -> None:
     """Run the device-side bounded-wait self-test (status_dev: zeroed CUDA int32[2])."""
     _check(lib().muse_selftest_bounded_wait(int(limit_ns), _ptr(status_dev), _stream_handle(stream)),
-           "muse_selftest_bounded_wait", "muse_quantize_nvfp4_rows")
+           "muse_selftest_bounded_wait")
 
 
 def last_device_status(cfg: Config, stream=None):
