@@ -456,7 +456,7 @@ def main():
     ap.add_argument("--no-side", action="store_true", help="skip the decode / skewed side workloads")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle cpu_baseline")
     ap.add_argument("--no-nvfp4", action="store_true", help="skip the NVFP4-expert side workloads")
-    ap.add_argument("--cpu-tokens", type=int, default=4)
+    ap.add_argument("--cpu-tokens", type=int, default=16)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world = int(os.environ.get("WORLD_SIZE", "1"))
