@@ -462,6 +462,13 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        # the FP64 oracle on the host cores: rank 0 alone, no process group; the seeded
+        # inputs are generated on the GPU when there is one (same bytes either way)
+        if rank == 0:
+            dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
+            print(json.dumps(run_reference(W.WORKLOADS[args.workload], args, dev)), flush=True)
+        return
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
@@ -469,10 +476,6 @@ def main():
                                              device_id=dev)
     w = W.WORKLOADS[args.workload]
     try:
-        if args.impl == "reference":
-            if rank == 0:
-                print(json.dumps(run_reference(w, args, dev)), flush=True)
-            return
         peaks, peak_kind = load_peaks()
         inp = make_rank_inputs(w, rank, dev)
         main_res = run_ours(w, inp, args.steps, args.warmup, rank, world, peaks, peak_kind, True,
