@@ -211,6 +211,25 @@ MUSE_API muse_status muse_latent_moe_forward_host_io(const muse_moe_config* cfg,
                                             const void* gamma, const void* W_unpool,
                                             void* out_dev, void* out_host, void* stream);
 
+/* A sequence of batches through the forward with host buffers, the copies overlapped with
+ * the compute. Batch b (of n_batches, each cfg->T tokens): x_host[b] (pinned host memory)
+ * is copied into x_dev[b % 2] on h2d_stream, its forward runs on `stream` into
+ * out_dev[b % 2], and out_dev[b % 2] is copied into out_host[b] on d2h_stream, so that while
+ * batch b computes, batch b + 1 uploads and batch b - 1 downloads. Events (created and
+ * released inside) order every reuse of the two device buffers; the batches' forwards share
+ * cfg->workspace, serialised on `stream`. x_host / out_host: host arrays of n_batches
+ * pointers; x_dev / out_dev: host arrays of 2 device pointers (16-byte aligned); the three
+ * streams must differ. Returns after enqueueing; synchronise d2h_stream before reading the
+ * last out_host. */
+MUSE_API muse_status muse_latent_moe_forward_host_batches(const muse_moe_config* cfg, int64_t n_batches,
+                                                 const void* const* x_host, void* const* out_host,
+                                                 void* const* x_dev, void* const* out_dev,
+                                                 const void* W_router, const void* W_pool,
+                                                 const void* W_gate, const void* W_up,
+                                                 const void* W_down, const void* gamma,
+                                                 const void* W_unpool, void* stream,
+                                                 void* h2d_stream, void* d2h_stream);
+
 /* Synchronises `stream` and returns the status word the last forward on this
  * workspace recorded on the device (MUSE_OK, MUSE_ERR_TIMEOUT or MUSE_ERR_DEVICE);
  * *detail (may be NULL) receives the kernel-specific detail code. */

@@ -27,7 +27,7 @@ STATUS = {0: "MUSE_OK", 1: "MUSE_ERR_INVALID_ARG", 2: "MUSE_ERR_UNSUPPORTED", 3:
 EXPORTS = ("muse_moe_config_init", "muse_latent_moe_workspace_size", "muse_latent_moe_workspace_layout",
            "muse_latent_moe_forward", "muse_latent_moe_forward_host_io", "muse_latent_moe_last_device_status",
            "muse_status_string", "muse_latent_moe_launch_count", "muse_latent_moe_forward_static_scratch",
-           "muse_selftest_bounded_wait", "muse_quantize_nvfp4_rows")
+           "muse_selftest_bounded_wait", "muse_quantize_nvfp4_rows", "muse_latent_moe_forward_host_batches")
 
 # size of the library's built-in scratch array (MUSE_STATIC_SCRATCH_BYTES)
 STATIC_SCRATCH_BYTES = 16 << 20
@@ -97,6 +97,8 @@ def lib() -> ctypes.CDLL:
         L.muse_selftest_bounded_wait.restype = ctypes.c_int
         L.muse_quantize_nvfp4_rows.argtypes = [vp, ctypes.c_int64, ctypes.c_int64, vp, vp, vp]
         L.muse_quantize_nvfp4_rows.restype = ctypes.c_int
+        L.muse_latent_moe_forward_host_batches.argtypes = [cp, ctypes.c_int64, vp, vp, vp, vp] + [vp] * 7 + [vp] * 3
+        L.muse_latent_moe_forward_host_batches.restype = ctypes.c_int
         L.muse_latent_moe_launch_count.argtypes = [cp]
         L.muse_latent_moe_launch_count.restype = ctypes.c_int32
         _lib = L
@@ -189,6 +191,23 @@ def forward_host_io(cfg: Config, x_host, x_dev, W_router, W_pool, W_gate, W_up, 
                                                  _ptr(gamma), _ptr(W_unpool), _ptr(out_dev), _ptr(out_host),
                                                  _stream_handle(stream))
     _check(code, "muse_latent_moe_forward_host_io")
+
+
+def forward_host_batches(cfg: Config, x_hosts, out_hosts, x_devs, out_devs, W_router, W_pool, W_gate, W_up, W_down,
+                         gamma, W_unpool, stream, h2d_stream, d2h_stream) -> None:
+    """Batches through the forward with host buffers, copies overlapped with compute (two
+    device buffers each for x and out; three distinct torch.cuda.Stream objects)."""
+    n = len(x_hosts)
+    xh = (ctypes.c_void_p * n)(*[_ptr(t) for t in x_hosts])
+    oh = (ctypes.c_void_p * n)(*[_ptr(t) for t in out_hosts])
+    xd = (ctypes.c_void_p * 2)(*[_ptr(t) for t in x_devs])
+    od = (ctypes.c_void_p * 2)(*[_ptr(t) for t in out_devs])
+    code = lib().muse_latent_moe_forward_host_batches(
+        ctypes.byref(cfg), n, ctypes.cast(xh, ctypes.c_void_p), ctypes.cast(oh, ctypes.c_void_p),
+        ctypes.cast(xd, ctypes.c_void_p), ctypes.cast(od, ctypes.c_void_p), _ptr(W_router), _ptr(W_pool),
+        _ptr(W_gate), _ptr(W_up), _ptr(W_down), _ptr(gamma), _ptr(W_unpool), _stream_handle(stream),
+        _stream_handle(h2d_stream), _stream_handle(d2h_stream))
+    _check(code, "muse_latent_moe_forward_host_batches")
 
 
 STAGES = ("router", "topk", "expert_hist", "tiles", "assign_rows", "pooler", "gather", "gate_up_swiglu",

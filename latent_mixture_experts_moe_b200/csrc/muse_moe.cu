@@ -791,6 +791,61 @@ muse_status muse_latent_moe_forward_host_io(const muse_moe_config* cfg, const vo
   return MUSE_OK;
 }
 
+muse_status muse_latent_moe_forward_host_batches(const muse_moe_config* cfg, int64_t n_batches,
+                                                 const void* const* x_host, void* const* out_host,
+                                                 void* const* x_dev, void* const* out_dev, const void* W_router,
+                                                 const void* W_pool, const void* W_gate, const void* W_up,
+                                                 const void* W_down, const void* gamma, const void* W_unpool,
+                                                 void* stream, void* h2d_stream, void* d2h_stream) {
+  muse_status s = validate_sizes(cfg);
+  if (s != MUSE_OK) return s;
+  if (n_batches < 1 || x_host == nullptr || out_host == nullptr || x_dev == nullptr || out_dev == nullptr)
+    return MUSE_ERR_INVALID_ARG;
+  if (stream == h2d_stream || stream == d2h_stream || h2d_stream == d2h_stream) return MUSE_ERR_INVALID_ARG;
+  for (int64_t b = 0; b < n_batches; ++b)
+    if (x_host[b] == nullptr || out_host[b] == nullptr) return MUSE_ERR_INVALID_ARG;
+  for (int i = 0; i < 2; ++i)
+    if (x_dev[i] == nullptr || out_dev[i] == nullptr || !aligned16(x_dev[i]) || !aligned16(out_dev[i]))
+      return MUSE_ERR_INVALID_ARG;
+  cudaStream_t sc = static_cast<cudaStream_t>(stream), su = static_cast<cudaStream_t>(h2d_stream),
+               sd = static_cast<cudaStream_t>(d2h_stream);
+  const size_t bytes = static_cast<size_t>(cfg->T) * cfg->D * act_size(*cfg);
+  // per device buffer: uploaded, computed, downloaded
+  cudaEvent_t up[2] = {nullptr, nullptr}, comp[2] = {nullptr, nullptr}, down[2] = {nullptr, nullptr};
+  muse_status rc = MUSE_OK;
+  for (int i = 0; i < 2 && rc == MUSE_OK; ++i)
+    if (cudaEventCreateWithFlags(&up[i], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&comp[i], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&down[i], cudaEventDisableTiming) != cudaSuccess)
+      rc = MUSE_ERR_CUDA;
+  for (int64_t b = 0; b < n_batches && rc == MUSE_OK; ++b) {
+    const int i = static_cast<int>(b & 1);
+    // upload batch b once the forward of batch b - 2 has read x_dev[i]
+    if (b >= 2 && cudaStreamWaitEvent(su, comp[i], 0) != cudaSuccess) rc = MUSE_ERR_CUDA;
+    if (rc == MUSE_OK && (cudaMemcpyAsync(x_dev[i], x_host[b], bytes, cudaMemcpyHostToDevice, su) != cudaSuccess ||
+                          cudaEventRecord(up[i], su) != cudaSuccess))
+      rc = MUSE_ERR_CUDA;
+    // compute once uploaded and once batch b - 2's output has left out_dev[i]
+    if (rc == MUSE_OK && cudaStreamWaitEvent(sc, up[i], 0) != cudaSuccess) rc = MUSE_ERR_CUDA;
+    if (rc == MUSE_OK && b >= 2 && cudaStreamWaitEvent(sc, down[i], 0) != cudaSuccess) rc = MUSE_ERR_CUDA;
+    if (rc == MUSE_OK)
+      rc = muse_latent_moe_forward(cfg, x_dev[i], W_router, W_pool, W_gate, W_up, W_down, gamma, W_unpool,
+                                   out_dev[i], stream);
+    if (rc == MUSE_OK && cudaEventRecord(comp[i], sc) != cudaSuccess) rc = MUSE_ERR_CUDA;
+    // download once computed
+    if (rc == MUSE_OK && (cudaStreamWaitEvent(sd, comp[i], 0) != cudaSuccess ||
+                          cudaMemcpyAsync(out_host[b], out_dev[i], bytes, cudaMemcpyDeviceToHost, sd) != cudaSuccess ||
+                          cudaEventRecord(down[i], sd) != cudaSuccess))
+      rc = MUSE_ERR_CUDA;
+  }
+  for (int i = 0; i < 2; ++i) {  // released once the work recorded on them completes
+    if (up[i]) cudaEventDestroy(up[i]);
+    if (comp[i]) cudaEventDestroy(comp[i]);
+    if (down[i]) cudaEventDestroy(down[i]);
+  }
+  return rc;
+}
+
 muse_status muse_latent_moe_forward_static_scratch(const muse_moe_config* cfg, const void* x, const void* W_router,
                                                   const void* W_pool, const void* W_gate, const void* W_up,
                                                   const void* W_down, const void* gamma, const void* W_unpool,

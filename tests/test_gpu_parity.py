@@ -171,6 +171,32 @@ def test_full_size_w4a4_layer_sampled_tokens():
     assert ref["act_adopted"] <= 1e-3 * decisions
 
 
+def test_host_batches_entry_point_matches_device_forwards(mid):
+    """Three different batches through the overlapped host-buffer call give, bit for bit,
+    the outputs of three device forwards."""
+    w, inp = mid
+    import dataclasses
+    model = moe.LatentMoE({n: v for n, v in inp.items() if n != "x"}, T_max=w.T, k=w.k, eps=w.eps)
+    xs = [W.make_inputs(dataclasses.replace(w, seed=s), "cuda", names=["x"])["x"] for s in (31, 32, 33)]
+    want = [model(x.clone()) for x in xs]
+    torch.cuda.synchronize()
+    x_hosts = [x.cpu().pin_memory() for x in xs]
+    out_hosts = [torch.empty((w.T, w.D), dtype=torch.bfloat16).pin_memory() for _ in xs]
+    x_devs = [torch.empty_like(xs[0]) for _ in range(2)]
+    out_devs = [torch.empty((w.T, w.D), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    cfg = model.config(w.T, model.workspace)
+    wt = model.w
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    moe.forward_host_batches(cfg, x_hosts, out_hosts, x_devs, out_devs, wt["W_router"], wt["W_pool"], wt["W_gate"],
+                             wt["W_up"], wt["W_down"], wt["gamma"], wt["W_unpool"], torch.cuda.current_stream(), up,
+                             down)
+    torch.cuda.synchronize()
+    for got, ref in zip(out_hosts, want):
+        assert torch.equal(got, ref.cpu())
+    code, detail = moe.last_device_status(cfg)
+    assert code == 0
+
+
 # ------------------------------------------------------------------------- CUDA graphs
 GRAPH = [
     # name, T, D, L, I, E, k: decode-sized tiles (one-CTA kernels), and CTA-pair tiles whose
