@@ -30,6 +30,7 @@ import datetime
 import json
 import math
 import os
+import platform
 import statistics
 import subprocess
 import sys
@@ -268,6 +269,8 @@ def run_ours(w: W.Workload, inp, steps: int, warmup: int, rank: int, world: int,
     else:
         roof = {"bound": "hbm", "achieved": by / t_dom / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
+    # against the datasheet figures too: 8 TB/s HBM3e, 2.25 PFLOP/s dense bf16 (x 4 for FP4)
+    roof["frac_of_spec"] = roof["achieved"] / (8000.0 if roof["bound"] == "hbm" else 2250.0 * ratio)
     roof["kernel"] = dname
     roof["peak_source"] = f"{peak_kind} ({'sustained' if roof['bound'] == 'tensor' else 'copy'})" + \
         (" x 4 (nominal FP4 / BF16 dense ratio)" if fp4_gemm and roof["bound"] == "tensor" else "")
@@ -400,10 +403,23 @@ def host_cores():
         return os.cpu_count()
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or "unknown"
+
+
 def cpu_baseline(w: W.Workload, dev, n_tokens: int):
     x, shared, bias, experts = oracle_sample(w, n_tokens, dev, widen=False)
     dt = time_oracle(w, x, shared, bias, experts)
+    flops_per_token = 2 * (w.E * w.D + w.L * w.D + w.k * 3 * w.L * w.I + w.D * w.L)
     return {"value": n_tokens / dt, "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
+            "gflops_fp64": n_tokens * flops_per_token / dt / 1e9, "cpu_model": cpu_model(),
             "sample": f"first {n_tokens} tokens of the {w.name} workload (T={w.T}) through the FP64 numpy "
                       f"oracle, widening bf16 weights to f64 included; {len(experts)} distinct experts; {dt:.1f} s"}
 
