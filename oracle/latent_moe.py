@@ -21,7 +21,7 @@ Sources (page title, then section / equation):
     the lower index, weights renormalised over the selected set, a zero-centred-gain
     RMSNorm y/rms(y)*(1+gamma_e) per expert.
 
-Readings where the pages are open or disagree (each is listed in the design doc):
+Readings where the pages are open or disagree:
   * router score: softmax (default); the pages' released router (sigmoid of the logit
     times 1/sqrt(32), selection-only bias, s/(sum s + 1e-15) * routed_scaling_factor)
     is `router_mode="sigmoid"`;
