@@ -50,7 +50,7 @@ extern "C" {
 typedef enum muse_status {
   MUSE_OK = 0,
   MUSE_ERR_INVALID_ARG = 1,   /* null / misaligned pointer, inconsistent sizes */
-  MUSE_ERR_UNSUPPORTED = 2,   /* shape or mode this build does not implement */
+  MUSE_ERR_UNSUPPORTED = 2,   /* shape or mode the library does not implement   */
   MUSE_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required */
   MUSE_ERR_CUDA = 4,          /* a CUDA runtime / driver call failed */
   MUSE_ERR_TIMEOUT = 5,       /* a bounded device-side wait ran out */
