@@ -203,6 +203,8 @@ GRAPH = [
     # tile counters must be re-zeroed inside every replay
     ("graph_small_tiles", 96, 1024, 512, 512, 32, 4),
     ("graph_pair_tiles", 1024, 1024, 512, 512, 4, 2),
+    # NVFP4 weights and activations (W4A4): its GEMMs claim tiles from counters too
+    ("graph_w4a4", 512, 1024, 512, 512, 8, 2),
 ]
 
 
@@ -212,9 +214,12 @@ def test_cuda_graph_replay_matches_eager(case):
     bit, also after new tokens are written into the captured input buffer."""
     import dataclasses
     name, T, D, L, I, E, k = case
-    w = W.Workload(name, T=T, D=D, L=L, I=I, E=E, k=k, dtype="bf16", seed=11)
+    w4a4 = name.endswith("w4a4")
+    w = W.Workload(name, T=T, D=D, L=L, I=I, E=E, k=k, dtype="bf16", seed=11,
+                   experts="nvfp4" if w4a4 else "bf16", act="nvfp4" if w4a4 else "bf16")
     inp = W.make_inputs(w, "cuda")
-    model = moe.LatentMoE({n: v for n, v in inp.items() if n != "x"}, T_max=T, k=k, eps=w.eps)
+    modes = {"act_format": moe.ACT_NVFP4} if w4a4 else {}
+    model = moe.LatentMoE({n: v for n, v in inp.items() if n != "x"}, T_max=T, k=k, eps=w.eps, **modes)
     x = inp["x"].clone()
     out_g = torch.empty((T, D), dtype=torch.bfloat16, device="cuda")
     side = torch.cuda.Stream()
