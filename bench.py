@@ -250,6 +250,8 @@ def run_ours(w: W.Workload, inp, steps: int, warmup: int, rank: int, world: int,
     if code != 0:
         raise RuntimeError(f"device status {code} detail {detail:#x}")
     stage_ms = [sum(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(steps)) / steps for i in range(nst)]
+    # each step's own duration (its first to its last library event): median, min, max
+    per_step = sorted(ev[s][0].elapsed_time(ev[s][nst]) for s in range(steps))
     n_touched = int(torch.unique(idx).numel())
     work = stage_work(w, n_touched)
     dom = max(range(nst), key=lambda i: stage_ms[i])
@@ -285,6 +287,7 @@ def run_ours(w: W.Workload, inp, steps: int, warmup: int, rank: int, world: int,
         "value": job_tokens_per_s(world, w.T, steps, ms_max),
         "ms_per_step": ms_max / steps,
         "stage_ms": {stage_names[i]: round(stage_ms[i], 4) for i in range(nst)},
+        "step_ms": {"median": per_step[len(per_step) // 2], "min": per_step[0], "max": per_step[-1]},
         "roofline": roof,
         "step": {"tflops": sf / t_step / 1e12, "gbs": sb / t_step / 1e9, "roofline_ms": step_roof * 1e3,
                  "frac_of_step_roofline": step_roof / t_step, "distinct_experts": n_touched},
@@ -418,8 +421,18 @@ def cpu_baseline(w: W.Workload, dev, n_tokens: int):
     x, shared, bias, experts = oracle_sample(w, n_tokens, dev, widen=False)
     dt = time_oracle(w, x, shared, bias, experts)
     flops_per_token = 2 * (w.E * w.D + w.L * w.D + w.k * 3 * w.L * w.I + w.D * w.L)
+    # the same oracle on one core (BLAS limited to one thread), one token, widening included
+    one_core = None
+    try:
+        from threadpoolctl import threadpool_limits
+        x1, shared1, bias1, experts1 = oracle_sample(w, 1, dev, widen=False)
+        with threadpool_limits(limits=1):
+            one_core = 1.0 / time_oracle(w, x1, shared1, bias1, experts1)
+    except ImportError:
+        pass
     return {"value": n_tokens / dt, "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
             "gflops_fp64": n_tokens * flops_per_token / dt / 1e9, "cpu_model": cpu_model(),
+            "one_core_tokens_per_s": one_core,
             "sample": f"first {n_tokens} tokens of the {w.name} workload (T={w.T}) through the FP64 numpy "
                       f"oracle, widening bf16 weights to f64 included; {len(experts)} distinct experts; {dt:.1f} s"}
 
@@ -546,7 +559,8 @@ def main():
                 "data": "synthetic (seeded counter-based N(0,1) inputs, N(0,1/fan_in) weights)",
                 "config": dict(config_dict(w), parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
                 "roofline": main_res["roofline"], "step_roofline": main_res["step"],
-                "stage_ms": main_res["stage_ms"], "gpu_launches": main_res["gpu_launches"],
+                "stage_ms": main_res["stage_ms"], "step_ms": main_res["step_ms"],
+                "gpu_launches": main_res["gpu_launches"],
                 "clocks": main_res.get("clocks"), "e2e": main_res.get("e2e"),
             }
             if "graph" in main_res:
