@@ -33,37 +33,11 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
   return (b & 0x80u) ? -v : v;
 }
 
-// 4-bit E2M1 code of v / s given the boundaries b[i] = t_i * s: the magnitude index counts
-// the midpoints t = 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5 (between the magnitudes 0, 0.5, 1,
-// 1.5, 2, 3, 4, 6) below |v| / s, a value exactly on a midpoint going to the neighbour with
-// an even index; the sign bit only on a nonzero magnitude. NaN compares false and gives 0.
-__device__ __forceinline__ uint32_t e2m1_code(float v, const float (&b)[7]) {
-  const float a = fabsf(v);
-  const uint32_t m = static_cast<uint32_t>(a > b[0]) + static_cast<uint32_t>(a >= b[1]) +
-                     static_cast<uint32_t>(a > b[2]) + static_cast<uint32_t>(a >= b[3]) +
-                     static_cast<uint32_t>(a > b[4]) + static_cast<uint32_t>(a >= b[5]) +
-                     static_cast<uint32_t>(a > b[6]);
-  return (v < 0.0f && m != 0u) ? (m | 8u) : m;
-}
-
-// One block of 16 values -> 8 code bytes (two words, element 2i in the low nibble of byte i)
-// and the E4M3 scale byte.
-__device__ __forceinline__ void quant_block16(const float (&v)[16], uint2& codes, uint32_t& sbyte) {
-  float amax = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
-  sbyte = f32_to_e4m3_rn_satfinite(amax / 6.0f);
-  const float s = e4m3_to_f32(sbyte);
-  uint32_t w[2] = {0u, 0u};
-  if (s > 0.0f) {
-    const float b[7] = {0.25f * s, 0.75f * s, 1.25f * s, 1.75f * s, 2.5f * s, 3.5f * s, 5.0f * s};  // exact
-#pragma unroll
-    for (int i = 0; i < 16; ++i) w[i >> 3] |= e2m1_code(v[i], b) << (4 * (i & 7));
-  }
-  codes = make_uint2(w[0], w[1]);
-}
-
-// The same for 16 bf16 values given as 8 packed pairs, two values per instruction: |v| and
+// One block of 16 bf16 values, given as 8 packed pairs, -> 8 code bytes (two words, element
+// 2i in the low nibble of byte i) and the E4M3 scale byte. A code's magnitude index counts the
+// E2M1 midpoints t = 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5 (between the magnitudes 0, 0.5, 1,
+// 1.5, 2, 3, 4, 6) below |v| / s, a value exactly on a midpoint going to the neighbour with an
+// even index; the sign bit is set only on a nonzero magnitude. Two values per instruction: |v| and
 // the boundaries t * s are compared as bf16 pairs (exact: v is bf16, and t * s has at most
 // 3 + 4 significant bits), the comparison results (1.0 or 0.0) summed as bf16 pairs, and
 // each count k (0..7) read from the bits of k + 128.0 (= 2^7 (1 + k / 128): k is the low
