@@ -280,6 +280,80 @@ MUSE_API muse_status muse_selftest_bounded_wait(uint64_t limit_ns, uint32_t* sta
 MUSE_API muse_status muse_quantize_nvfp4_rows(const void* src, int64_t rows, int64_t K, void* codes,
                                               void* scales, void* stream);
 
+/* ---------------------------------------------------------------------------------
+ * Expert parallelism (EP) over G ranks (Muse Spark Open deep dive, §4.3: the two expert
+ * tensors split along the expert dimension, the latent rows moved to the experts' ranks
+ * and back, the norm weights replicated; on each rank the local experts see every row
+ * with top-1 routing and unit weight, and the routing weights are applied after the
+ * rows return, so the per-expert norm still precedes the weighting). Rank r owns the
+ * experts [r * E / G, (r + 1) * E / G); E must be a multiple of G. One forward is three
+ * calls around two exchanges that the caller performs (an all-to-all, e.g. NCCL):
+ *
+ *   1. muse_ep_dispatch on every rank, for its own cfg->T tokens: routing, pooler, and
+ *      the send buffer of its T * k (token, expert) rows, grouped by destination rank
+ *      (rank_counts[r] rows for rank r, in rank order).
+ *   2. exchange: rank r receives the rows every rank sent to it, concatenated in source
+ *      rank order, with their local expert indices.
+ *   3. muse_ep_experts on every rank over the rows it received: gate/up + SwiGLU, down
+ *      projection and the partial sums of squares, returned in the order received.
+ *   4. exchange back: the inverse of step 2, so that each rank's results land in the
+ *      rows of its own send buffer.
+ *   5. muse_ep_combine on every rank: per-expert norm, weighted combine, unpooler (and
+ *      the optional feed-forward sublayer steps), into out.
+ *
+ * cfg is the whole block's configuration (E = all experts) on every call. Calls 1 and 5
+ * of one forward use the same cfg->workspace (the token rank's workspace, role
+ * MUSE_EP_HOME); call 3 uses an expert workspace (role MUSE_EP_EXPERTS) in
+ * cfg->workspace. The result equals muse_latent_moe_forward on the same tokens up to
+ * the rounding of the GEMMs (a GEMM of other row counts may tile differently). Calls are
+ * enqueued on `stream` without synchronising; the host reads rank_counts (a device
+ * array) to size the exchange. stage_events is ignored. Status word: calls 1 and 3 reset
+ * their workspace's word, call 5 adds to the word of call 1.
+ * --------------------------------------------------------------------------------- */
+typedef enum muse_ep_role {
+  MUSE_EP_HOME = 1,    /* routing, pooler, send plan, combine, unpooler of cfg->T tokens */
+  MUSE_EP_EXPERTS = 2  /* grouped GEMMs over up to `rows` received rows                  */
+} muse_ep_role;
+
+/* Offsets of the buffers of a role's workspace (total = bytes to allocate, 256-byte
+ * aligned base). For MUSE_EP_EXPERTS, rows = the most rows one call will receive (at
+ * most the sum over ranks of T_rank * min(k, E / G)); buffers a role does not use have
+ * offset 0 and no bytes. INVALID_ARG if E is not a multiple of ep_size or the role is
+ * unknown. */
+MUSE_API muse_status muse_ep_workspace_layout(const muse_moe_config* cfg, int32_t ep_size, int32_t role,
+                                              int64_t rows, muse_moe_workspace_layout* layout);
+
+/* EP step 1 on the tokens' rank. x [T, D] -> send_z [T * k, L] (dtype cfg->dtype): row
+ * p is the latent z of the token of the p-th (token, expert) pair in destination order
+ * -- experts ascending, then tokens ascending, then slot -- so the rows for rank r form
+ * the contiguous block [sum_{q<r} rank_counts[q], + rank_counts[r]); send_expert
+ * int32 [T * k]: each row's expert index on its owning rank (0 .. E/G - 1);
+ * rank_counts int32 [ep_size]. All device memory (send_z 16-byte aligned). */
+MUSE_API muse_status muse_ep_dispatch(const muse_moe_config* cfg, int32_t ep_size, const void* x,
+                                      const void* W_router, const void* W_pool, void* send_z,
+                                      int32_t* send_expert, int32_t* rank_counts, void* stream);
+
+/* EP step 3 on an expert rank. recv_z [rows, L] and recv_expert int32 [rows] (local
+ * expert indices) -> ret_y [rows, L] (dtype cfg->dtype), the expert outputs before the
+ * norm, and ret_ss float [rows, L/32], their partial sums of squares per 32 columns,
+ * both in the order received. W_gate / W_up / W_down: this rank's E/G experts, laid out
+ * as in muse_latent_moe_forward with E/G in place of E (NVFP4: descriptors of them);
+ * gamma: this rank's slice [E/G, L] (or the shared [L]), read only in
+ * MUSE_NORM_INPUT_SCALED mode. rows = 0 launches nothing. A local index outside
+ * 0 .. E/G - 1 is recorded as MUSE_ERR_DEVICE in the status word and its row returns
+ * zeros. */
+MUSE_API muse_status muse_ep_experts(const muse_moe_config* cfg, int32_t ep_size, int64_t rows,
+                                     const void* recv_z, const int32_t* recv_expert, const void* W_gate,
+                                     const void* W_up, const void* W_down, const void* gamma, void* ret_y,
+                                     float* ret_ss, void* stream);
+
+/* EP step 5 on the tokens' rank, after the exchange back: back_y [T * k, L] and back_ss
+ * float [T * k, L/32] in the rows of this rank's send buffer -> out [T, D]. gamma: all
+ * E experts' gains (replicated), x: this rank's input (read by the residual gate). */
+MUSE_API muse_status muse_ep_combine(const muse_moe_config* cfg, int32_t ep_size, const void* x,
+                                     const void* back_y, const float* back_ss, const void* gamma,
+                                     const void* W_unpool, void* out, void* stream);
+
 /* Static string for a status code. */
 MUSE_API const char* muse_status_string(muse_status s);
 

@@ -27,7 +27,11 @@ STATUS = {0: "MUSE_OK", 1: "MUSE_ERR_INVALID_ARG", 2: "MUSE_ERR_UNSUPPORTED", 3:
 EXPORTS = ("muse_moe_config_init", "muse_latent_moe_workspace_size", "muse_latent_moe_workspace_layout",
            "muse_latent_moe_forward", "muse_latent_moe_forward_host_io", "muse_latent_moe_last_device_status",
            "muse_status_string", "muse_latent_moe_launch_count", "muse_latent_moe_forward_static_scratch",
-           "muse_selftest_bounded_wait", "muse_quantize_nvfp4_rows", "muse_latent_moe_forward_host_batches")
+           "muse_selftest_bounded_wait", "muse_quantize_nvfp4_rows", "muse_latent_moe_forward_host_batches",
+           "muse_ep_workspace_layout", "muse_ep_dispatch", "muse_ep_experts", "muse_ep_combine")
+
+# roles of an expert-parallel workspace (muse_ep_role)
+EP_HOME, EP_EXPERTS = 1, 2
 
 # size of the library's built-in scratch array (MUSE_STATIC_SCRATCH_BYTES)
 STATIC_SCRATCH_BYTES = 16 << 20
@@ -99,6 +103,15 @@ def lib() -> ctypes.CDLL:
         L.muse_quantize_nvfp4_rows.restype = ctypes.c_int
         L.muse_latent_moe_forward_host_batches.argtypes = [cp, ctypes.c_int64, vp, vp, vp, vp] + [vp] * 7 + [vp] * 3
         L.muse_latent_moe_forward_host_batches.restype = ctypes.c_int
+        i32, i64 = ctypes.c_int32, ctypes.c_int64
+        L.muse_ep_workspace_layout.argtypes = [cp, i32, i32, i64, ctypes.POINTER(WorkspaceLayout)]
+        L.muse_ep_workspace_layout.restype = ctypes.c_int
+        L.muse_ep_dispatch.argtypes = [cp, i32] + [vp] * 7
+        L.muse_ep_dispatch.restype = ctypes.c_int
+        L.muse_ep_experts.argtypes = [cp, i32, i64] + [vp] * 9
+        L.muse_ep_experts.restype = ctypes.c_int
+        L.muse_ep_combine.argtypes = [cp, i32] + [vp] * 7
+        L.muse_ep_combine.restype = ctypes.c_int
         L.muse_latent_moe_launch_count.argtypes = [cp]
         L.muse_latent_moe_launch_count.restype = ctypes.c_int32
         _lib = L
@@ -210,6 +223,35 @@ def forward_host_batches(cfg: Config, x_hosts, out_hosts, x_devs, out_devs, W_ro
     _check(code, "muse_latent_moe_forward_host_batches")
 
 
+def ep_workspace_layout(cfg: Config, ep_size: int, role: int, rows: int = 0) -> Dict[str, int]:
+    """Buffer offsets (and "total" bytes) of an expert-parallel workspace: role EP_HOME for
+    cfg.T tokens, EP_EXPERTS for up to `rows` received rows."""
+    lay = WorkspaceLayout()
+    _check(lib().muse_ep_workspace_layout(ctypes.byref(cfg), int(ep_size), int(role), int(rows), ctypes.byref(lay)),
+           "muse_ep_workspace_layout")
+    return {name: int(getattr(lay, name)) for name, _ in WorkspaceLayout._fields_}
+
+
+def ep_dispatch(cfg: Config, ep_size: int, x, W_router, W_pool, send_z, send_expert, rank_counts, stream=None) -> None:
+    """Expert-parallel step 1 (cfg.workspace: an EP_HOME workspace)."""
+    _check(lib().muse_ep_dispatch(ctypes.byref(cfg), int(ep_size), _ptr(x), _ptr(W_router), _ptr(W_pool), _ptr(send_z),
+                                  _ptr(send_expert), _ptr(rank_counts), _stream_handle(stream)), "muse_ep_dispatch")
+
+
+def ep_experts(cfg: Config, ep_size: int, rows: int, recv_z, recv_expert, W_gate, W_up, W_down, gamma, ret_y, ret_ss,
+               stream=None) -> None:
+    """Expert-parallel step 3 (cfg.workspace: an EP_EXPERTS workspace)."""
+    _check(lib().muse_ep_experts(ctypes.byref(cfg), int(ep_size), int(rows), _ptr(recv_z), _ptr(recv_expert),
+                                 _ptr(W_gate), _ptr(W_up), _ptr(W_down), _ptr(gamma), _ptr(ret_y), _ptr(ret_ss),
+                                 _stream_handle(stream)), "muse_ep_experts")
+
+
+def ep_combine(cfg: Config, ep_size: int, x, back_y, back_ss, gamma, W_unpool, out, stream=None) -> None:
+    """Expert-parallel step 5 (cfg.workspace: the EP_HOME workspace of step 1)."""
+    _check(lib().muse_ep_combine(ctypes.byref(cfg), int(ep_size), _ptr(x), _ptr(back_y), _ptr(back_ss), _ptr(gamma),
+                                 _ptr(W_unpool), _ptr(out), _stream_handle(stream)), "muse_ep_combine")
+
+
 STAGES = ("router", "topk", "expert_hist", "tiles", "assign_rows", "pooler", "gather", "gate_up_swiglu",
           "down_sumsq", "norm_combine", "unpooler")
 
@@ -260,6 +302,45 @@ def last_device_status(cfg: Config, stream=None):
     return int(code), int(detail.value)
 
 
+def expert_weight_dims(weights: Dict):
+    """(I, L, nvfp4) from the expert weights: dense W_gate [E, I, L], or NVFP4 codes
+    W_gate_codes [E, I, L/2]."""
+    if "W_gate_codes" in weights:
+        _, I, L2 = weights["W_gate_codes"].shape
+        return int(I), int(2 * L2), True
+    _, I, L = weights["W_gate"].shape
+    return int(I), int(L), False
+
+
+def expert_operands(weights: Dict, nvfp4: bool):
+    """The W_gate, W_up, W_down arguments of the C ABI: the dense tensors, or Nvfp4Weight
+    descriptors of <name>_codes [E, out, in/2], <name>_scales [E, out, in/16] and
+    <name>_mscale [E]."""
+    if not nvfp4:
+        return tuple(weights[n] for n in ("W_gate", "W_up", "W_down"))
+    return tuple(Nvfp4Weight(_ptr(weights[n + "_codes"]), _ptr(weights[n + "_scales"]), _ptr(weights[n + "_mscale"]))
+                 for n in ("W_gate", "W_up", "W_down"))
+
+
+def block_config(T: int, dims: Dict, dtype: str, modes: Dict, weights: Dict, nvfp4: bool, workspace=None) -> Config:
+    """Config of the block for T tokens: sizes, modes, the optional pointers found in
+    weights (router_bias, pre_norm_gain, ffn_pre_gain, ffn_post_gain, residual_gate) and
+    the workspace (a uint8 CUDA tensor) if given."""
+    d = dims
+    c = make_config(T, d["D"], d["L"], d["I"], d["E"], d["k"], dtype, d["eps"], **modes)
+    if nvfp4:
+        c.expert_weights = EXPERTS_NVFP4
+    if weights.get("router_bias") is not None:
+        c.router_bias = _ptr(weights["router_bias"])
+    for name in ("pre_norm_gain", "ffn_pre_gain", "ffn_post_gain", "residual_gate"):
+        if weights.get(name) is not None:
+            setattr(c, name, _ptr(weights[name]))
+    if workspace is not None:
+        c.workspace = _ptr(workspace)
+        c.workspace_bytes = workspace.numel()
+    return c
+
+
 class LatentMoE:
     """Holds the block's device weights and a workspace; calling it runs the forward.
 
@@ -273,37 +354,17 @@ class LatentMoE:
         import torch
         self.w = dict(weights)
         E, D = weights["W_router"].shape
-        self.nvfp4 = "W_gate_codes" in weights
-        if self.nvfp4:
-            # NVFP4 experts: <name>_codes [E, out, in/2], <name>_scales [E, out, in/16], <name>_mscale [E]
-            _, I, L2 = weights["W_gate_codes"].shape
-            L = 2 * L2
-            for n in ("W_gate", "W_up", "W_down"):
-                self.w[n] = Nvfp4Weight(_ptr(weights[n + "_codes"]), _ptr(weights[n + "_scales"]),
-                                        _ptr(weights[n + "_mscale"]))
-        else:
-            _, I, L = weights["W_gate"].shape
+        I, L, self.nvfp4 = expert_weight_dims(weights)
+        self.w["W_gate"], self.w["W_up"], self.w["W_down"] = expert_operands(weights, self.nvfp4)
         self.dtype = {torch.float32: "f32", torch.bfloat16: "bf16"}[weights["W_router"].dtype]
-        self.dims = dict(D=int(D), L=int(L), I=int(I), E=int(E), k=k, eps=eps)
+        self.dims = dict(D=int(D), L=L, I=I, E=int(E), k=k, eps=eps)
         self.modes = modes
         cfg = self.config(T_max)
         self.workspace = torch.empty(workspace_size(cfg), dtype=torch.uint8, device=weights["W_router"].device)
         self.T_max = T_max
 
     def config(self, T: int, workspace=None) -> Config:
-        d = self.dims
-        c = make_config(T, d["D"], d["L"], d["I"], d["E"], d["k"], self.dtype, d["eps"], **self.modes)
-        if self.nvfp4:
-            c.expert_weights = EXPERTS_NVFP4
-        if self.w.get("router_bias") is not None:
-            c.router_bias = _ptr(self.w["router_bias"])
-        for name in ("pre_norm_gain", "ffn_pre_gain", "ffn_post_gain", "residual_gate"):
-            if self.w.get(name) is not None:
-                setattr(c, name, _ptr(self.w[name]))
-        if workspace is not None:
-            c.workspace = _ptr(workspace)
-            c.workspace_bytes = workspace.numel()
-        return c
+        return block_config(T, self.dims, self.dtype, self.modes, self.w, self.nvfp4, workspace)
 
     def __call__(self, x, out=None, stream=None, topk_idx=None, topk_w=None, stage_events=None):
         """stage_events: optional ctypes array of launch_count + 1 cudaEvent_t handles."""

@@ -51,50 +51,60 @@ struct Layout {
 
 size_t act_size(const muse_moe_config& c) { return c.dtype == MUSE_BF16 ? 2 : 4; }
 
-Layout make_layout(const muse_moe_config& c) {
+// Which buffers a workspace holds: those of the whole forward, or of one side of the
+// expert-parallel split -- the token's own rank (routing, send plan, pooler, combine,
+// unpooler) or an expert shard (grouped GEMMs over the rows it received; c.T = rows).
+// Buffers a role does not use have offset 0 and no bytes.
+enum class Role { kFull, kHome, kExperts };
+
+Layout make_layout(const muse_moe_config& c, Role role = Role::kFull) {
   Layout l{};
+  const bool home = role != Role::kExperts, grouped = role != Role::kHome;
   const int64_t T = c.T, E = c.E, k = c.top_k;
   const int64_t assign = T * k;
-  const int64_t rows = align_up(static_cast<size_t>(assign + 15 * std::min<int64_t>(E, assign)), 16);
+  // rows of the expert-ordered buffers: each expert's rows padded to 16 (home: the send
+  // plan, unpadded)
+  const int64_t rows =
+      grouped ? static_cast<int64_t>(align_up(static_cast<size_t>(assign + 15 * std::min<int64_t>(E, assign)), 16))
+              : assign;
   const int bn = grouped_bn(c);
   const int64_t chunks = cdiv(assign, bn) + std::min<int64_t>(E, assign);
-  l.max_tiles_gu = chunks * (c.I / 128);
-  l.max_tiles_dn = chunks * (c.L / 128);
+  l.max_tiles_gu = grouped ? chunks * (c.I / 128) : 0;
+  l.max_tiles_dn = grouped ? chunks * (c.L / 128) : 0;
   const size_t as = act_size(c);
   size_t o = 0;
-  auto take = [&](size_t bytes) {
+  auto take = [&](bool used, size_t bytes) -> size_t {
+    if (!used) return 0;
     const size_t at = o;
     o = align_up(o + bytes, kAlign);
     return at;
   };
-  l.pub.status = take(16);
-  l.pub.expert_count = take(sizeof(int32_t) * E);
-  l.pub.expert_offset = take(sizeof(int32_t) * (E + 1));
-  l.ntiles = take(sizeof(int32_t) * 8);
-  l.pub.logits = take(sizeof(float) * T * E);
-  l.pub.topk_idx = take(sizeof(int32_t) * assign);
-  l.pub.topk_w = take(sizeof(float) * assign);
-  l.pub.inv = take(sizeof(int32_t) * assign);
-  l.pub.row_token = take(sizeof(int32_t) * rows);
-  l.tiles_gu = take(sizeof(int4) * l.max_tiles_gu);
-  l.tiles_dn = take(sizeof(int4) * l.max_tiles_dn);
-  l.pub.z = take(as * T * c.L);
-  l.pub.zp = take(as * rows * c.L);
-  l.pub.h = take(as * rows * c.I);
-  l.pub.y = take(as * rows * c.L);
-  l.pub.ss = take(sizeof(float) * rows * (c.L / 32));
-  l.pub.c = take(as * T * c.L);
-  l.pub.xn = c.ffn_pre_gain != nullptr ? take(as * T * c.D) : 0;
-  l.pub.ss_out = c.ffn_post_gain != nullptr ? take(sizeof(float) * T * (c.D / 32)) : 0;
-  l.zt_codes = l.zt_scales = 0;
-  if (w4a4(c)) {
-    l.zt_codes = take(T * (c.L / 2));
-    l.zt_scales = take(T * (c.L / 16));
-    l.pub.zq_codes = take(rows * (c.L / 2));
-    l.pub.zq_scales = take(rows * (c.L / 16));
-    l.pub.hq_codes = take(rows * (c.I / 2));
-    l.pub.hq_scales = take(rows * (c.I / 16));
-  }
+  l.pub.status = take(true, 16);
+  l.pub.expert_count = take(true, sizeof(int32_t) * E);
+  l.pub.expert_offset = take(true, sizeof(int32_t) * (E + 1));
+  l.ntiles = take(true, sizeof(int32_t) * 8);
+  l.pub.logits = take(home, sizeof(float) * T * E);
+  l.pub.topk_idx = take(home, sizeof(int32_t) * assign);
+  l.pub.topk_w = take(home, sizeof(float) * assign);
+  l.pub.inv = take(true, sizeof(int32_t) * assign);
+  l.pub.row_token = take(true, sizeof(int32_t) * rows);
+  l.tiles_gu = take(grouped, sizeof(int4) * l.max_tiles_gu);
+  l.tiles_dn = take(grouped, sizeof(int4) * l.max_tiles_dn);
+  l.pub.z = take(home, as * T * c.L);
+  l.pub.zp = take(grouped, as * rows * c.L);
+  l.pub.h = take(grouped, as * rows * c.I);
+  l.pub.y = take(grouped, as * rows * c.L);
+  l.pub.ss = take(grouped, sizeof(float) * rows * (c.L / 32));
+  l.pub.c = take(home, as * T * c.L);
+  l.pub.xn = take(home && c.ffn_pre_gain != nullptr, as * T * c.D);
+  l.pub.ss_out = take(home && c.ffn_post_gain != nullptr, sizeof(float) * T * (c.D / 32));
+  const bool q = grouped && w4a4(c);
+  l.zt_codes = take(q, T * (c.L / 2));
+  l.zt_scales = take(q, T * (c.L / 16));
+  l.pub.zq_codes = take(q, rows * (c.L / 2));
+  l.pub.zq_scales = take(q, rows * (c.L / 16));
+  l.pub.hq_codes = take(q, rows * (c.I / 2));
+  l.pub.hq_scales = take(q, rows * (c.I / 16));
   l.pub.total = o;
   l.pub.rows = rows;
   return l;
@@ -399,137 +409,191 @@ GemmPlan plan_down(const muse_moe_config& c, int bn_g) {
     if ((x) != cudaSuccess) return MUSE_ERR_CUDA;  \
   } while (0)
 
+#define MUSE_TRY(x)                     \
+  do {                                  \
+    const muse_status s_ = (x);         \
+    if (s_ != MUSE_OK) return s_;       \
+  } while (0)
+
+// One pass of kernels over a workspace: its buffers, the stream and the optional stage
+// events (recorded after each launch of the full forward; null on the expert-parallel
+// entry points).
 template <typename T>
-muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void* x, const void* W_router,
-                         const void* W_pool, const void* W_gate, const void* W_up, const void* W_down,
-                         const void* gamma, const void* W_unpool, void* out, cudaStream_t st) {
-  uint8_t* ws = static_cast<uint8_t*>(c.workspace);
-  auto at = [&](size_t off) { return ws + off; };
-  uint32_t* status = reinterpret_cast<uint32_t*>(at(lay.pub.status));
-  int* counts = reinterpret_cast<int*>(at(lay.pub.expert_count));
-  int* offsets = reinterpret_cast<int*>(at(lay.pub.expert_offset));
-  int* ntiles = reinterpret_cast<int*>(at(lay.ntiles));
-  float* logits = reinterpret_cast<float*>(at(lay.pub.logits));
-  int* topk_idx = reinterpret_cast<int*>(at(lay.pub.topk_idx));
-  float* topk_w = reinterpret_cast<float*>(at(lay.pub.topk_w));
-  int* inv = reinterpret_cast<int*>(at(lay.pub.inv));
-  int* row_token = reinterpret_cast<int*>(at(lay.pub.row_token));
-  int4* tiles_gu = reinterpret_cast<int4*>(at(lay.tiles_gu));
-  int4* tiles_dn = reinterpret_cast<int4*>(at(lay.tiles_dn));
-  T* z = reinterpret_cast<T*>(at(lay.pub.z));
-  T* zp = reinterpret_cast<T*>(at(lay.pub.zp));
-  T* h = reinterpret_cast<T*>(at(lay.pub.h));
-  T* y = reinterpret_cast<T*>(at(lay.pub.y));
-  float* ss = reinterpret_cast<float*>(at(lay.pub.ss));
-  T* cbuf = reinterpret_cast<T*>(at(lay.pub.c));
-  const bool bf = sizeof(T) == 2;
-  const int64_t Tn = c.T, D = c.D, L = c.L, I = c.I, E = c.E, k = c.top_k;
-  const int64_t assign = Tn * k;
-  const int nsm = sm_count();
-  const int bn_d = dense_bn(c), bn_g = grouped_bn(c);
-  const GemmPlan pgu = plan_gate_up(c, bn_g), pdn = plan_down(c, bn_g);
-
-  MUSE_CK(cudaMemsetAsync(status, 0, 16, st));
-  MUSE_CK(cudaMemsetAsync(counts, 0, sizeof(int) * E, st));
+struct Pass {
+  const muse_moe_config& c;
+  const Layout& lay;
+  cudaStream_t st;
+  void* const* events;
   int stage = 0;
-  auto mark = [&]() -> cudaError_t {
-    if (c.stage_events == nullptr) return cudaSuccess;
-    return cudaEventRecord(static_cast<cudaEvent_t>(c.stage_events[stage++]), st);
-  };
-  MUSE_CK(mark());
+  int nsm;
+  uint8_t* ws;
+  uint32_t* status;
+  int *counts, *offsets, *ntiles, *topk_idx, *inv, *row_token;
+  float* topk_w;
+  Pass(const muse_moe_config& c_, const Layout& l, cudaStream_t s, void* const* ev)
+      : c(c_), lay(l), st(s), events(ev), nsm(sm_count()), ws(static_cast<uint8_t*>(c_.workspace)) {
+    status = ptr<uint32_t>(l.pub.status);
+    counts = ptr<int>(l.pub.expert_count);
+    offsets = ptr<int>(l.pub.expert_offset);
+    ntiles = ptr<int>(l.ntiles);
+    topk_idx = ptr<int>(l.pub.topk_idx);
+    topk_w = ptr<float>(l.pub.topk_w);
+    inv = ptr<int>(l.pub.inv);
+    row_token = ptr<int>(l.pub.row_token);
+  }
+  uint8_t* at(size_t off) const { return ws + off; }
+  template <typename U>
+  U* ptr(size_t off) const { return reinterpret_cast<U*>(ws + off); }
+  cudaError_t mark() {
+    if (events == nullptr) return cudaSuccess;
+    return cudaEventRecord(static_cast<cudaEvent_t>(events[stage++]), st);
+  }
+};
 
-  // feed-forward sublayer pre-norm (optional): the router and the pooler read xn
-  const void* xin = x;
+// status word and expert histogram zeroed; the first stage event
+template <typename T>
+muse_status begin(Pass<T>& p) {
+  MUSE_CK(cudaMemsetAsync(p.status, 0, 16, p.st));
+  MUSE_CK(cudaMemsetAsync(p.counts, 0, sizeof(int) * p.c.E, p.st));
+  MUSE_CK(p.mark());
+  return MUSE_OK;
+}
+
+// feed-forward sublayer pre-norm (optional), (a1) router logits, (a2) top-k and weights;
+// *xin: the rows the router and the pooler read (x, or its normalisation)
+template <typename T>
+muse_status route(Pass<T>& p, const void* x, const void* W_router, const void** xin) {
+  const muse_moe_config& c = p.c;
+  const int64_t Tn = c.T, D = c.D, E = c.E, k = c.top_k;
+  *xin = x;
   if (c.ffn_pre_gain != nullptr) {
-    T* xn = reinterpret_cast<T*>(at(lay.pub.xn));
-    k_rmsnorm_rows<T><<<static_cast<unsigned>(Tn), 256, 0, st>>>(reinterpret_cast<const T*>(x), xn,
-                                                                 reinterpret_cast<const T*>(c.ffn_pre_gain),
-                                                                 static_cast<int>(D), c.ffn_pre_eps);
+    T* xn = p.template ptr<T>(p.lay.pub.xn);
+    k_rmsnorm_rows<T><<<static_cast<unsigned>(Tn), 256, 0, p.st>>>(reinterpret_cast<const T*>(x), xn,
+                                                                   reinterpret_cast<const T*>(c.ffn_pre_gain),
+                                                                   static_cast<int>(D), c.ffn_pre_eps);
     MUSE_CK(cudaGetLastError());
-    MUSE_CK(mark());
-    xin = xn;
+    MUSE_CK(p.mark());
+    *xin = xn;
   }
-  // (a1) router logits
-  if (bf) {
-    muse_status s = dense_gemm<T, float>(W_router, E, xin, Tn, D, logits, bn_d, status, nullptr, st);
-    if (s != MUSE_OK) return s;
+  float* logits = p.template ptr<float>(p.lay.pub.logits);
+  if (sizeof(T) == 2) {
+    MUSE_TRY((dense_gemm<T, float>(W_router, E, *xin, Tn, D, logits, dense_bn(c), p.status, nullptr, p.st)));
   } else {
-    k_router_logits_f32<<<static_cast<unsigned>(Tn), 256, 0, st>>>(reinterpret_cast<const float*>(xin),
-                                                                  reinterpret_cast<const float*>(W_router),
-                                                                  static_cast<int>(D), static_cast<int>(E), logits);
+    k_router_logits_f32<<<static_cast<unsigned>(Tn), 256, 0, p.st>>>(reinterpret_cast<const float*>(*xin),
+                                                                    reinterpret_cast<const float*>(W_router),
+                                                                    static_cast<int>(D), static_cast<int>(E), logits);
     MUSE_CK(cudaGetLastError());
   }
-  MUSE_CK(mark());
-  // (a2) top-k and weights
-  k_topk<<<static_cast<unsigned>(cdiv(Tn * 32, 256)), 256, 0, st>>>(
+  MUSE_CK(p.mark());
+  k_topk<<<static_cast<unsigned>(cdiv(Tn * 32, 256)), 256, 0, p.st>>>(
       logits, static_cast<int>(Tn), static_cast<int>(E), static_cast<int>(k), c.router_bias, c.router_mode,
-      c.router_logit_scale, c.routed_scaling, topk_idx, topk_w, c.topk_idx_out, c.topk_w_out);
+      c.router_logit_scale, c.routed_scaling, p.topk_idx, p.topk_w, c.topk_idx_out, c.topk_w_out);
   MUSE_CK(cudaGetLastError());
-  MUSE_CK(mark());
-  // (a3) permutation
-  {
-    const int grid = static_cast<int>(std::min<int64_t>(cdiv(assign, 256), 4 * nsm));
-    k_expert_hist<<<grid, 256, sizeof(int) * E, st>>>(topk_idx, static_cast<int>(assign), static_cast<int>(E),
-                                                      counts, status);
-    MUSE_CK(cudaGetLastError());
-    MUSE_CK(mark());
-    const int threads = static_cast<int>(align_up(static_cast<size_t>(E), 32));
-    k_build_tiles<<<1, threads, 0, st>>>(counts, static_cast<int>(E), bn_g, static_cast<int>(I / pgu.step), pgu.step,
-                                         static_cast<int>(L / pdn.step), pdn.step, offsets, tiles_gu, ntiles,
-                                         tiles_dn, ntiles + 1, ntiles + 4, row_token);
-    MUSE_CK(cudaGetLastError());
-    MUSE_CK(mark());
-    k_assign_rows<<<static_cast<unsigned>(E), 1024, 0, st>>>(topk_idx, static_cast<int>(assign), static_cast<int>(k),
-                                                            counts, offsets, inv, row_token);
-    MUSE_CK(cudaGetLastError());
-    MUSE_CK(mark());
-  }
-  // (a4) pooler
-  {
-    muse_status s = dense_gemm<T, T>(W_pool, L, xin, Tn, D, z, bn_d, status, ntiles + 6, st);
-    if (s != MUSE_OK) return s;
-    MUSE_CK(mark());
-  }
-  // pages' pre_expert_norm on z (optional)
+  MUSE_CK(p.mark());
+  return MUSE_OK;
+}
+
+// (a3) expert histogram of n assignments (out-of-range indices are counted nowhere and
+// recorded in the status word)
+template <typename T>
+muse_status hist(Pass<T>& p, const int* idx, int64_t n) {
+  const int grid = static_cast<int>(std::min<int64_t>(cdiv(n, 256), 4 * p.nsm));
+  k_expert_hist<<<grid, 256, sizeof(int) * p.c.E, p.st>>>(idx, static_cast<int>(n), static_cast<int>(p.c.E), p.counts,
+                                                            p.status);
+  MUSE_CK(cudaGetLastError());
+  MUSE_CK(p.mark());
+  return MUSE_OK;
+}
+
+// (a3) padded expert offsets, grouped-GEMM tile lists and the stable row of each of the n
+// assignments idx (k per token)
+template <typename T>
+muse_status permute(Pass<T>& p, const int* idx, int64_t n, int k) {
+  const muse_moe_config& c = p.c;
+  const int bn_g = grouped_bn(c);
+  const GemmPlan pgu = plan_gate_up(c, bn_g), pdn = plan_down(c, bn_g);
+  const int threads = static_cast<int>(align_up(static_cast<size_t>(c.E), 32));
+  k_build_tiles<<<1, threads, 0, p.st>>>(p.counts, static_cast<int>(c.E), bn_g, static_cast<int>(c.I / pgu.step),
+                                         pgu.step, static_cast<int>(c.L / pdn.step), pdn.step, p.offsets,
+                                         p.template ptr<int4>(p.lay.tiles_gu), p.ntiles,
+                                         p.template ptr<int4>(p.lay.tiles_dn), p.ntiles + 1, p.ntiles + 4,
+                                         p.row_token);
+  MUSE_CK(cudaGetLastError());
+  MUSE_CK(p.mark());
+  k_assign_rows<<<static_cast<unsigned>(c.E), 1024, 0, p.st>>>(idx, static_cast<int>(n), k, p.counts, p.offsets,
+                                                               p.inv, p.row_token);
+  MUSE_CK(cudaGetLastError());
+  MUSE_CK(p.mark());
+  return MUSE_OK;
+}
+
+// (a4) pooler, then the pages' pre_expert_norm on z (optional)
+template <typename T>
+muse_status pool(Pass<T>& p, const void* xin, const void* W_pool) {
+  const muse_moe_config& c = p.c;
+  T* z = p.template ptr<T>(p.lay.pub.z);
+  MUSE_TRY((dense_gemm<T, T>(W_pool, c.L, xin, c.T, c.D, z, dense_bn(c), p.status, p.ntiles + 6, p.st)));
+  MUSE_CK(p.mark());
   if (c.pre_norm_gain != nullptr) {
-    k_rmsnorm_rows<T><<<static_cast<unsigned>(Tn), 256, 0, st>>>(z, z, reinterpret_cast<const T*>(c.pre_norm_gain),
-                                                                 static_cast<int>(L), c.pre_norm_eps);
+    k_rmsnorm_rows<T><<<static_cast<unsigned>(c.T), 256, 0, p.st>>>(
+        z, z, reinterpret_cast<const T*>(c.pre_norm_gain), static_cast<int>(c.L), c.pre_norm_eps);
     MUSE_CK(cudaGetLastError());
-    MUSE_CK(mark());
+    MUSE_CK(p.mark());
   }
-  // (a5) gather into expert order (W4A4: gather and quantise to NVFP4 in one pass)
+  return MUSE_OK;
+}
+
+// (a5) gather of the latent rows zsrc [nsrc, L] into expert order (W4A4: quantised to
+// NVFP4 once per source row, then the codes gathered), (a6) gate/up + SwiGLU, (a7) down
+// projection + sum-of-squares partials, over the tiles permute() listed
+template <typename T>
+muse_status experts(Pass<T>& p, const T* zsrc, int64_t nsrc, const void* W_gate, const void* W_up,
+                    const void* W_down, const void* gamma) {
+  const muse_moe_config& c = p.c;
+  const Layout& lay = p.lay;
+  cudaStream_t st = p.st;
+  const bool bf = sizeof(T) == 2;
+  const int64_t L = c.L, I = c.I, E = c.E;
+  const int nsm = p.nsm;
+  const int bn_g = grouped_bn(c);
+  const GemmPlan pdn = plan_down(c, bn_g), pgu = plan_gate_up(c, bn_g);
+  T* zp = p.template ptr<T>(lay.pub.zp);
+  T* h = p.template ptr<T>(lay.pub.h);
+  T* y = p.template ptr<T>(lay.pub.y);
+  float* ss = p.template ptr<float>(lay.pub.ss);
   const bool q4a = w4a4(c);
-  uint8_t* zq_codes = at(lay.pub.zq_codes);
-  uint8_t* zq_scales = at(lay.pub.zq_scales);
-  uint8_t* hq_codes = at(lay.pub.hq_codes);
-  uint8_t* hq_scales = at(lay.pub.hq_scales);
+  uint8_t* zq_codes = p.at(lay.pub.zq_codes);
+  uint8_t* zq_scales = p.at(lay.pub.zq_scales);
+  uint8_t* hq_codes = p.at(lay.pub.hq_codes);
+  uint8_t* hq_scales = p.at(lay.pub.hq_scales);
   const int quant_grid = static_cast<int>(std::min<int64_t>(lay.pub.rows, 16 * nsm));
   if (q4a) {
-    uint8_t* zt_codes = at(lay.zt_codes);
-    uint8_t* zt_scales = at(lay.zt_scales);
-    k_quant_rows_nvfp4<<<static_cast<unsigned>(std::min<int64_t>(Tn, 16 * nsm)), 256, 0, st>>>(
-        nullptr, nullptr, static_cast<int>(Tn), reinterpret_cast<const __nv_bfloat16*>(z), static_cast<int>(L),
+    uint8_t* zt_codes = p.at(lay.zt_codes);
+    uint8_t* zt_scales = p.at(lay.zt_scales);
+    k_quant_rows_nvfp4<<<static_cast<unsigned>(std::min<int64_t>(nsrc, 16 * nsm)), 256, 0, st>>>(
+        nullptr, nullptr, static_cast<int>(nsrc), reinterpret_cast<const __nv_bfloat16*>(zsrc), static_cast<int>(L),
         zt_codes, zt_scales);
     MUSE_CK(cudaGetLastError());
-    MUSE_CK(mark());
-    k_gather_nvfp4_rows<<<quant_grid, 128, 0, st>>>(row_token, offsets + E, reinterpret_cast<const uint4*>(zt_codes),
+    MUSE_CK(p.mark());
+    k_gather_nvfp4_rows<<<quant_grid, 128, 0, st>>>(p.row_token, p.offsets + E,
+                                                    reinterpret_cast<const uint4*>(zt_codes),
                                                     reinterpret_cast<const uint4*>(zt_scales),
                                                     reinterpret_cast<uint4*>(zq_codes),
                                                     reinterpret_cast<uint4*>(zq_scales), static_cast<int>(L));
     MUSE_CK(cudaGetLastError());
-    MUSE_CK(mark());
+    MUSE_CK(p.mark());
   } else {
     const int vpr = static_cast<int>(L * sizeof(T) / 16);
     const int rows_grid = static_cast<int>(std::min<int64_t>(lay.pub.rows, 16 * nsm));
-    k_gather_rows<<<rows_grid, 128, 0, st>>>(row_token, offsets + E, reinterpret_cast<const uint4*>(z),
+    k_gather_rows<<<rows_grid, 128, 0, st>>>(p.row_token, p.offsets + E, reinterpret_cast<const uint4*>(zsrc),
                                             reinterpret_cast<uint4*>(zp), vpr);
     MUSE_CK(cudaGetLastError());
-    MUSE_CK(mark());
+    MUSE_CK(p.mark());
   }
   const int64_t R = lay.pub.rows;
+  const bool fp4 = c.expert_weights == MUSE_EXPERTS_NVFP4;
   // (a6) gate/up + SwiGLU
   {
-    const bool fp4 = c.expert_weights == MUSE_EXPERTS_NVFP4;
     TmaMaps maps;
     Fp4Args q4{};
     if (q4a) {
@@ -546,10 +610,10 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
     } else if (!make_maps(&maps, W_gate, W_up, E * I, zp, R, L, bf)) {
       return MUSE_ERR_CUDA;
     }
-    GemmArgs g = base_args(status);
-    g.tiles = tiles_gu;
-    g.num_tiles_dev = ntiles;
-    g.tile_counter = ntiles + 4;
+    GemmArgs g = base_args(p.status);
+    g.tiles = p.template ptr<int4>(lay.tiles_gu);
+    g.num_tiles_dev = p.ntiles;
+    g.tile_counter = p.ntiles + 4;
     g.rows_per_group = static_cast<int>(I);
     g.m_valid = static_cast<int>(I);
     g.k_blocks = static_cast<int>(L * sizeof(T) / 128);
@@ -562,7 +626,6 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
       if (!make_w4a4_maps(&wm, wg, wu, E * I, zq_codes, zq_scales, R, L, bn_g)) return MUSE_ERR_CUDA;
       const W4A4Args wq{wg->matrix_scale, wu->matrix_scale};
       g.k_blocks = static_cast<int>(L / 256);
-      g.tile_counter = ntiles + 4;
       MUSE_CK(launch_gemm_w4a4<EPI_SWIGLU>(bn_g, wm, g, wq, nsm, st));
     } else if (fp4) {
       MUSE_CK(launch_gemm_fp4<EPI_SWIGLU>(bn_g, 2, maps, g, q4, nsm, st));
@@ -572,18 +635,18 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
     } else {
       MUSE_CK((launch_gemm_bn<T, T, EPI_SWIGLU>(bn_g, 2, maps, g, nsm, st)));
     }
-    MUSE_CK(mark());
+    MUSE_CK(p.mark());
   }
   // W4A4: quantise h (already in expert order) for the down projection
   if (q4a) {
-    k_quant_rows_nvfp4<<<quant_grid, 256, 0, st>>>(row_token, offsets + E, 0, reinterpret_cast<const __nv_bfloat16*>(h),
-                                                   static_cast<int>(I), hq_codes, hq_scales);
+    k_quant_rows_nvfp4<<<quant_grid, 256, 0, st>>>(p.row_token, p.offsets + E, 0,
+                                                   reinterpret_cast<const __nv_bfloat16*>(h), static_cast<int>(I),
+                                                   hq_codes, hq_scales);
     MUSE_CK(cudaGetLastError());
-    MUSE_CK(mark());
+    MUSE_CK(p.mark());
   }
   // (a7) down projection + sum-of-squares partials
   {
-    const bool fp4 = c.expert_weights == MUSE_EXPERTS_NVFP4;
     TmaMaps maps;
     Fp4Args q4{};
     if (q4a) {
@@ -599,10 +662,10 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
     } else if (!make_maps(&maps, W_down, nullptr, E * L, h, R, I, bf)) {
       return MUSE_ERR_CUDA;
     }
-    GemmArgs g = base_args(status);
-    g.tiles = tiles_dn;
-    g.num_tiles_dev = ntiles + 1;
-    g.tile_counter = ntiles + 5;
+    GemmArgs g = base_args(p.status);
+    g.tiles = p.template ptr<int4>(lay.tiles_dn);
+    g.num_tiles_dev = p.ntiles + 1;
+    g.tile_counter = p.ntiles + 5;
     g.rows_per_group = static_cast<int>(L);
     g.m_valid = static_cast<int>(L);
     g.k_blocks = static_cast<int>(I * sizeof(T) / 128);
@@ -621,7 +684,6 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
       if (!make_w4a4_maps(&wm, wd, wd, E * L, hq_codes, hq_scales, R, I, bn_g)) return MUSE_ERR_CUDA;
       const W4A4Args wq{wd->matrix_scale, wd->matrix_scale};
       g.k_blocks = static_cast<int>(I / 256);
-      g.tile_counter = ntiles + 5;
       MUSE_CK(launch_gemm_w4a4<EPI_STORE_SS>(bn_g, wm, g, wq, nsm, st));
     } else if (fp4) {
       MUSE_CK(launch_gemm_fp4<EPI_STORE_SS>(bn_g, pdn.mt, maps, g, q4, nsm, st));
@@ -632,50 +694,189 @@ muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void
     } else {
       MUSE_CK((launch_gemm_bn<T, T, EPI_STORE_SS>(bn_g, pdn.mt, maps, g, nsm, st)));
     }
-    MUSE_CK(mark());
+    MUSE_CK(p.mark());
   }
-  // (a8 + a9) per-expert RMSNorm and weighted combine
+  return MUSE_OK;
+}
+
+// (a8 + a9) per-expert RMSNorm and weighted combine of the expert outputs y (row inv[t*k+j]
+// for token t's j-th expert) with their sum-of-squares partials ss, (a10) unpooler, and the
+// feed-forward sublayer's post-norm and residual gate (optional)
+template <typename T>
+muse_status combine(Pass<T>& p, const T* y, const float* ss, const void* x, const void* gamma, const void* W_unpool,
+                    void* out) {
+  const muse_moe_config& c = p.c;
+  const int64_t Tn = c.T, D = c.D, L = c.L, k = c.top_k;
+  T* cbuf = p.template ptr<T>(p.lay.pub.c);
   {
     const int vec = 16 / static_cast<int>(sizeof(T));
     // a vector per thread up to 256 threads; one warp per selected row for the scales
     const int threads = static_cast<int>(
         std::max<int64_t>(32 * std::min<int64_t>(k, 8), std::min<int64_t>(256, align_up(static_cast<size_t>(L / vec), 32))));
-    k_combine<T><<<static_cast<unsigned>(Tn), threads, 0, st>>>(
-        topk_idx, topk_w, inv, ss, static_cast<int>(L / 32), y, reinterpret_cast<const T*>(gamma),
+    k_combine<T><<<static_cast<unsigned>(Tn), threads, 0, p.st>>>(
+        p.topk_idx, p.topk_w, p.inv, ss, static_cast<int>(L / 32), y, reinterpret_cast<const T*>(gamma),
         c.gamma_shared ? 0 : L, static_cast<int>(L), static_cast<int>(k), c.eps, cbuf);
     MUSE_CK(cudaGetLastError());
-    MUSE_CK(mark());
+    MUSE_CK(p.mark());
   }
   // (a10) unpooler; with the sublayer post-norm its epilogue also writes the partial sums
   // of (f * (1 + w))^2
   const bool post = c.ffn_post_gain != nullptr;
-  {
-    muse_status s;
-    if (post) {
-      DenseSS sq;
-      sq.ss = reinterpret_cast<float*>(at(lay.pub.ss_out));
-      sq.ld = static_cast<int>(D / 32);
-      sq.gain = c.ffn_post_gain;
-      s = dense_gemm<T, T, EPI_STORE_SS>(W_unpool, D, cbuf, Tn, L, out, bn_d, status, ntiles + 7, st, sq);
-    } else {
-      s = dense_gemm<T, T>(W_unpool, D, cbuf, Tn, L, out, bn_d, status, ntiles + 7, st);
-    }
-    if (s != MUSE_OK) return s;
+  if (post) {
+    DenseSS sq;
+    sq.ss = p.template ptr<float>(p.lay.pub.ss_out);
+    sq.ld = static_cast<int>(D / 32);
+    sq.gain = c.ffn_post_gain;
+    MUSE_TRY((dense_gemm<T, T, EPI_STORE_SS>(W_unpool, D, cbuf, Tn, L, out, dense_bn(c), p.status, p.ntiles + 7,
+                                             p.st, sq)));
+  } else {
+    MUSE_TRY((dense_gemm<T, T>(W_unpool, D, cbuf, Tn, L, out, dense_bn(c), p.status, p.ntiles + 7, p.st)));
   }
-  MUSE_CK(mark());
+  MUSE_CK(p.mark());
   // feed-forward sublayer post-norm and residual gate (optional), in place on out
   if (post || c.residual_gate != nullptr) {
     const int vec = 16 / static_cast<int>(sizeof(T));
     const dim3 grid(static_cast<unsigned>(cdiv(Tn, kFinishRows)),
                     static_cast<unsigned>(cdiv(D, static_cast<int64_t>(kFinishThreads) * vec)));
-    k_ffn_finish<T><<<grid, kFinishThreads, 0, st>>>(
-        reinterpret_cast<T*>(out), reinterpret_cast<const T*>(x), reinterpret_cast<const float*>(at(lay.pub.ss_out)),
+    k_ffn_finish<T><<<grid, kFinishThreads, 0, p.st>>>(
+        reinterpret_cast<T*>(out), reinterpret_cast<const T*>(x), p.template ptr<const float>(p.lay.pub.ss_out),
         static_cast<int>(D / 32), reinterpret_cast<const T*>(c.ffn_post_gain), c.ffn_post_eps, c.residual_gate,
         1.0f / c.residual_gate_temperature, c.residual_gate_eps, static_cast<int>(D), static_cast<int>(Tn));
     MUSE_CK(cudaGetLastError());
-    MUSE_CK(mark());
+    MUSE_CK(p.mark());
   }
   return MUSE_OK;
+}
+
+template <typename T>
+muse_status forward_impl(const muse_moe_config& c, const Layout& lay, const void* x, const void* W_router,
+                         const void* W_pool, const void* W_gate, const void* W_up, const void* W_down,
+                         const void* gamma, const void* W_unpool, void* out, cudaStream_t st) {
+  Pass<T> p(c, lay, st, c.stage_events);
+  const int64_t assign = c.T * c.top_k;
+  const void* xin = nullptr;
+  MUSE_TRY(begin(p));
+  MUSE_TRY(route(p, x, W_router, &xin));
+  MUSE_TRY(hist(p, p.topk_idx, assign));
+  MUSE_TRY(permute(p, p.topk_idx, assign, c.top_k));
+  MUSE_TRY(pool(p, xin, W_pool));
+  MUSE_TRY(experts(p, p.template ptr<const T>(lay.pub.z), c.T, W_gate, W_up, W_down, gamma));
+  return combine(p, p.template ptr<const T>(lay.pub.y), p.template ptr<const float>(lay.pub.ss), x, gamma, W_unpool,
+                 out);
+}
+
+// Expert parallelism, the token's own rank before the exchange: routing, the send plan,
+// the pooler and the send buffer.
+template <typename T>
+muse_status ep_dispatch_impl(const muse_moe_config& c, const Layout& lay, int G, const void* x, const void* W_router,
+                             const void* W_pool, void* send_z, int32_t* send_expert, int32_t* rank_counts,
+                             cudaStream_t st) {
+  Pass<T> p(c, lay, st, nullptr);
+  const int64_t assign = c.T * c.top_k;
+  const int E_loc = static_cast<int>(c.E / G);
+  const void* xin = nullptr;
+  MUSE_TRY(begin(p));
+  MUSE_TRY(route(p, x, W_router, &xin));
+  MUSE_TRY(hist(p, p.topk_idx, assign));
+  const int threads = static_cast<int>(align_up(static_cast<size_t>(c.E), 32));
+  k_ep_plan<<<1, threads, 0, st>>>(p.counts, static_cast<int>(c.E), E_loc, G, p.offsets, rank_counts, p.ntiles + 4);
+  MUSE_CK(cudaGetLastError());
+  k_assign_rows<<<static_cast<unsigned>(c.E), 1024, 0, st>>>(p.topk_idx, static_cast<int>(assign), c.top_k, p.counts,
+                                                             p.offsets, p.inv, p.row_token);
+  MUSE_CK(cudaGetLastError());
+  MUSE_TRY(pool(p, xin, W_pool));
+  const int vpr = static_cast<int>(c.L * sizeof(T) / 16);
+  const int grid = static_cast<int>(std::min<int64_t>(assign, 16 * p.nsm));
+  k_ep_pack<<<grid, 128, 0, st>>>(p.topk_idx, p.inv, static_cast<int>(assign), c.top_k, E_loc,
+                                  p.template ptr<const uint4>(lay.pub.z), vpr, static_cast<uint4*>(send_z),
+                                  send_expert);
+  MUSE_CK(cudaGetLastError());
+  return MUSE_OK;
+}
+
+// Expert parallelism, an expert shard: the received rows through this rank's experts
+// (cl: the local configuration, cl.T = rows received, cl.top_k = 1, cl.E = E / G), the
+// results put back in the order received.
+template <typename T>
+muse_status ep_experts_impl(const muse_moe_config& cl, const Layout& lay, const void* recv_z,
+                            const int32_t* recv_expert, const void* W_gate, const void* W_up, const void* W_down,
+                            const void* gamma, void* ret_y, float* ret_ss, cudaStream_t st) {
+  Pass<T> p(cl, lay, st, nullptr);
+  const int64_t R = cl.T;
+  MUSE_TRY(begin(p));
+  MUSE_CK(cudaMemsetAsync(p.inv, 0xFF, sizeof(int) * R, st));  // rows with no slot stay -1
+  MUSE_TRY(hist(p, recv_expert, R));
+  MUSE_TRY(permute(p, recv_expert, R, 1));
+  MUSE_TRY(experts(p, static_cast<const T*>(recv_z), R, W_gate, W_up, W_down, gamma));
+  const int grid = static_cast<int>(std::min<int64_t>(R, 16 * p.nsm));
+  k_ep_unpermute<<<grid, 128, 0, st>>>(p.inv, static_cast<int>(R), p.template ptr<const uint4>(lay.pub.y),
+                                       p.template ptr<const uint4>(lay.pub.ss),
+                                       static_cast<int>(cl.L * sizeof(T) / 16), static_cast<int>(cl.L / 128),
+                                       static_cast<uint4*>(ret_y), reinterpret_cast<uint4*>(ret_ss));
+  MUSE_CK(cudaGetLastError());
+  return MUSE_OK;
+}
+
+// weight operands of the expert GEMMs: dense (16-byte aligned) or NVFP4 descriptors
+muse_status validate_experts(const muse_moe_config* cfg, const void* W_gate, const void* W_up, const void* W_down) {
+  const void* experts[] = {W_gate, W_up, W_down};
+  for (const void* p : experts) {
+    if (cfg->expert_weights == MUSE_EXPERTS_NVFP4) {
+      if (!valid_nvfp4(p)) return MUSE_ERR_INVALID_ARG;
+    } else if (p == nullptr || !aligned16(p)) {
+      return MUSE_ERR_INVALID_ARG;
+    }
+  }
+  return MUSE_OK;
+}
+
+// the configuration's optional pointers and their parameters
+muse_status validate_options(const muse_moe_config* cfg) {
+  if (cfg->router_bias != nullptr && (reinterpret_cast<uintptr_t>(cfg->router_bias) & 3u)) return MUSE_ERR_INVALID_ARG;
+  if (cfg->pre_norm_gain != nullptr && !aligned16(cfg->pre_norm_gain)) return MUSE_ERR_INVALID_ARG;
+  if (cfg->pre_norm_gain != nullptr && !(cfg->pre_norm_eps >= 0.0f)) return MUSE_ERR_INVALID_ARG;
+  if (cfg->ffn_pre_gain != nullptr && (!aligned16(cfg->ffn_pre_gain) || !(cfg->ffn_pre_eps >= 0.0f)))
+    return MUSE_ERR_INVALID_ARG;
+  if (cfg->ffn_post_gain != nullptr && (!aligned16(cfg->ffn_post_gain) || !(cfg->ffn_post_eps >= 0.0f)))
+    return MUSE_ERR_INVALID_ARG;
+  if (cfg->residual_gate != nullptr &&
+      (!aligned16(cfg->residual_gate) || !(cfg->residual_gate_temperature > 0.0f) || !(cfg->residual_gate_eps >= 0.0f)))
+    return MUSE_ERR_INVALID_ARG;
+  return MUSE_OK;
+}
+
+// workspace present, aligned and large enough for the layout; the driver entry point
+// the tensor maps need
+muse_status check_workspace(const muse_moe_config* cfg, const Layout& lay) {
+  if (cfg->workspace == nullptr || (reinterpret_cast<uintptr_t>(cfg->workspace) & (kAlign - 1)))
+    return MUSE_ERR_WORKSPACE;
+  if (cfg->workspace_bytes < lay.pub.total) return MUSE_ERR_WORKSPACE;
+  if (encode_fn() == nullptr) return MUSE_ERR_CUDA;
+  return MUSE_OK;
+}
+
+// model configuration valid and its experts divisible among ep_size ranks
+muse_status validate_ep(const muse_moe_config* cfg, int32_t ep_size) {
+  MUSE_TRY(validate_sizes(cfg));
+  if (ep_size < 1 || cfg->E % ep_size != 0) return MUSE_ERR_INVALID_ARG;
+  return MUSE_OK;
+}
+
+// An expert shard's configuration: its E / G experts, the rows it received as tokens with
+// one expert each; the steps before and after the experts belong to the tokens' ranks.
+muse_moe_config expert_shard_config(const muse_moe_config& c, int32_t G, int64_t rows) {
+  muse_moe_config l = c;
+  l.E = c.E / G;
+  l.top_k = 1;
+  l.T = rows;
+  l.router_bias = nullptr;
+  l.pre_norm_gain = nullptr;
+  l.ffn_pre_gain = l.ffn_post_gain = nullptr;
+  l.residual_gate = nullptr;
+  l.topk_idx_out = nullptr;
+  l.topk_w_out = nullptr;
+  l.stage_events = nullptr;
+  return l;
 }
 
 // Scratch for muse_latent_moe_forward_static_scratch: a fixed array in device global
@@ -741,38 +942,95 @@ muse_status muse_latent_moe_workspace_layout(const muse_moe_config* cfg, muse_mo
 muse_status muse_latent_moe_forward(const muse_moe_config* cfg, const void* x, const void* W_router,
                                     const void* W_pool, const void* W_gate, const void* W_up, const void* W_down,
                                     const void* gamma, const void* W_unpool, void* out, void* stream) {
-  muse_status s = validate_sizes(cfg);
-  if (s != MUSE_OK) return s;
+  MUSE_TRY(validate_sizes(cfg));
   const void* ptrs[] = {x, W_router, W_pool, gamma, W_unpool, out};
   for (const void* p : ptrs)
     if (p == nullptr || !aligned16(p)) return MUSE_ERR_INVALID_ARG;
-  const void* experts[] = {W_gate, W_up, W_down};
-  for (const void* p : experts) {
-    if (cfg->expert_weights == MUSE_EXPERTS_NVFP4) {
-      if (!valid_nvfp4(p)) return MUSE_ERR_INVALID_ARG;
-    } else if (p == nullptr || !aligned16(p)) {
-      return MUSE_ERR_INVALID_ARG;
-    }
-  }
-  if (cfg->router_bias != nullptr && (reinterpret_cast<uintptr_t>(cfg->router_bias) & 3u)) return MUSE_ERR_INVALID_ARG;
-  if (cfg->pre_norm_gain != nullptr && !aligned16(cfg->pre_norm_gain)) return MUSE_ERR_INVALID_ARG;
-  if (cfg->pre_norm_gain != nullptr && !(cfg->pre_norm_eps >= 0.0f)) return MUSE_ERR_INVALID_ARG;
-  if (cfg->ffn_pre_gain != nullptr && (!aligned16(cfg->ffn_pre_gain) || !(cfg->ffn_pre_eps >= 0.0f)))
-    return MUSE_ERR_INVALID_ARG;
-  if (cfg->ffn_post_gain != nullptr && (!aligned16(cfg->ffn_post_gain) || !(cfg->ffn_post_eps >= 0.0f)))
-    return MUSE_ERR_INVALID_ARG;
-  if (cfg->residual_gate != nullptr &&
-      (!aligned16(cfg->residual_gate) || !(cfg->residual_gate_temperature > 0.0f) || !(cfg->residual_gate_eps >= 0.0f)))
-    return MUSE_ERR_INVALID_ARG;
+  MUSE_TRY(validate_experts(cfg, W_gate, W_up, W_down));
+  MUSE_TRY(validate_options(cfg));
   const Layout lay = make_layout(*cfg);
-  if (cfg->workspace == nullptr || (reinterpret_cast<uintptr_t>(cfg->workspace) & (kAlign - 1)))
-    return MUSE_ERR_WORKSPACE;
-  if (cfg->workspace_bytes < lay.pub.total) return MUSE_ERR_WORKSPACE;
-  if (encode_fn() == nullptr) return MUSE_ERR_CUDA;
+  MUSE_TRY(check_workspace(cfg, lay));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cfg->dtype == MUSE_BF16)
     return forward_impl<__nv_bfloat16>(*cfg, lay, x, W_router, W_pool, W_gate, W_up, W_down, gamma, W_unpool, out, st);
   return forward_impl<float>(*cfg, lay, x, W_router, W_pool, W_gate, W_up, W_down, gamma, W_unpool, out, st);
+}
+
+muse_status muse_ep_workspace_layout(const muse_moe_config* cfg, int32_t ep_size, int32_t role, int64_t rows,
+                                     muse_moe_workspace_layout* layout) {
+  if (layout == nullptr) return MUSE_ERR_INVALID_ARG;
+  MUSE_TRY(validate_ep(cfg, ep_size));
+  if (role == MUSE_EP_HOME) {
+    *layout = make_layout(*cfg, Role::kHome).pub;
+  } else if (role == MUSE_EP_EXPERTS) {
+    if (rows < 0) return MUSE_ERR_INVALID_ARG;
+    const muse_moe_config cl = expert_shard_config(*cfg, ep_size, std::max<int64_t>(rows, 1));
+    MUSE_TRY(validate_sizes(&cl));
+    *layout = make_layout(cl, Role::kExperts).pub;
+  } else {
+    return MUSE_ERR_INVALID_ARG;
+  }
+  return MUSE_OK;
+}
+
+muse_status muse_ep_dispatch(const muse_moe_config* cfg, int32_t ep_size, const void* x, const void* W_router,
+                             const void* W_pool, void* send_z, int32_t* send_expert, int32_t* rank_counts,
+                             void* stream) {
+  MUSE_TRY(validate_ep(cfg, ep_size));
+  const void* ptrs[] = {x, W_router, W_pool, send_z};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return MUSE_ERR_INVALID_ARG;
+  if (send_expert == nullptr || rank_counts == nullptr || (reinterpret_cast<uintptr_t>(send_expert) & 3u) ||
+      (reinterpret_cast<uintptr_t>(rank_counts) & 3u))
+    return MUSE_ERR_INVALID_ARG;
+  MUSE_TRY(validate_options(cfg));
+  const Layout lay = make_layout(*cfg, Role::kHome);
+  MUSE_TRY(check_workspace(cfg, lay));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cfg->dtype == MUSE_BF16)
+    return ep_dispatch_impl<__nv_bfloat16>(*cfg, lay, ep_size, x, W_router, W_pool, send_z, send_expert, rank_counts,
+                                           st);
+  return ep_dispatch_impl<float>(*cfg, lay, ep_size, x, W_router, W_pool, send_z, send_expert, rank_counts, st);
+}
+
+muse_status muse_ep_experts(const muse_moe_config* cfg, int32_t ep_size, int64_t rows, const void* recv_z,
+                            const int32_t* recv_expert, const void* W_gate, const void* W_up, const void* W_down,
+                            const void* gamma, void* ret_y, float* ret_ss, void* stream) {
+  MUSE_TRY(validate_ep(cfg, ep_size));
+  if (rows < 0) return MUSE_ERR_INVALID_ARG;
+  if (rows == 0) return MUSE_OK;  // nothing received: nothing to launch
+  const void* ptrs[] = {recv_z, gamma, ret_y, ret_ss};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return MUSE_ERR_INVALID_ARG;
+  if (recv_expert == nullptr || (reinterpret_cast<uintptr_t>(recv_expert) & 3u)) return MUSE_ERR_INVALID_ARG;
+  const muse_moe_config cl = expert_shard_config(*cfg, ep_size, rows);
+  MUSE_TRY(validate_sizes(&cl));
+  MUSE_TRY(validate_experts(&cl, W_gate, W_up, W_down));
+  const Layout lay = make_layout(cl, Role::kExperts);
+  MUSE_TRY(check_workspace(&cl, lay));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cl.dtype == MUSE_BF16)
+    return ep_experts_impl<__nv_bfloat16>(cl, lay, recv_z, recv_expert, W_gate, W_up, W_down, gamma, ret_y, ret_ss,
+                                          st);
+  return ep_experts_impl<float>(cl, lay, recv_z, recv_expert, W_gate, W_up, W_down, gamma, ret_y, ret_ss, st);
+}
+
+muse_status muse_ep_combine(const muse_moe_config* cfg, int32_t ep_size, const void* x, const void* back_y,
+                            const float* back_ss, const void* gamma, const void* W_unpool, void* out, void* stream) {
+  MUSE_TRY(validate_ep(cfg, ep_size));
+  const void* ptrs[] = {x, back_y, back_ss, gamma, W_unpool, out};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return MUSE_ERR_INVALID_ARG;
+  MUSE_TRY(validate_options(cfg));
+  const Layout lay = make_layout(*cfg, Role::kHome);
+  MUSE_TRY(check_workspace(cfg, lay));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cfg->dtype == MUSE_BF16) {
+    Pass<__nv_bfloat16> p(*cfg, lay, st, nullptr);
+    return combine(p, static_cast<const __nv_bfloat16*>(back_y), back_ss, x, gamma, W_unpool, out);
+  }
+  Pass<float> p(*cfg, lay, st, nullptr);
+  return combine(p, static_cast<const float*>(back_y), back_ss, x, gamma, W_unpool, out);
 }
 
 muse_status muse_latent_moe_forward_host_io(const muse_moe_config* cfg, const void* x_host, void* x_dev,

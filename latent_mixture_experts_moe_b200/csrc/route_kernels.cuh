@@ -455,6 +455,69 @@ __global__ void k_combine(const int* __restrict__ topk_idx, const float* __restr
 }
 
 // --------------------------------------------------------------------------------------
+// Expert parallelism over G ranks, rank r owning experts [r * E_loc, (r + 1) * E_loc).
+// The latent of a token crosses to each rank that owns one of its experts (one row per
+// selected expert, 2 L bytes); the expert outputs and their partial sums of squares
+// come back; the per-expert norm and the weighted combine run on the token's own rank.
+// --------------------------------------------------------------------------------------
+
+// Send plan (one block, a thread per expert): the T*k assignments in expert-major order
+// without padding, offsets[e] = number of assignments to experts below e. Because the
+// owners' expert ranges are contiguous and ascending, that order is also rank-major:
+// rank r's rows are [offsets[r * E_loc], offsets[(r + 1) * E_loc]), rank_counts[r] of
+// them. Also zeroes the tile counters of the pooler and unpooler GEMMs, as k_build_tiles
+// does in the single-GPU forward.
+__global__ void k_ep_plan(const int* __restrict__ counts, int E, int E_loc, int G, int* __restrict__ offsets,
+                          int* __restrict__ rank_counts, int* __restrict__ tile_counters) {
+  const int e = threadIdx.x;
+  const int n = (e < E) ? counts[e] : 0;
+  int total;
+  const int off = block_exclusive_scan(n, &total);
+  if (e < E) offsets[e] = off;
+  if (threadIdx.x == 0) {
+    offsets[E] = total;
+    for (int i = 0; i < 4; ++i) tile_counters[i] = 0;
+  }
+  __syncthreads();  // offsets visible to the whole block
+  for (int r = threadIdx.x; r < G; r += blockDim.x) rank_counts[r] = offsets[(r + 1) * E_loc] - offsets[r * E_loc];
+}
+
+// Send buffer: assignment a = t*k + j to expert e = idx[a] goes to row inv[a] (its place
+// in the send plan) as a copy of z's row t, tagged with e's index on its owning rank,
+// e - E_loc * (e / E_loc). One block per assignment, grid-strided; 16-byte vectors.
+__global__ void k_ep_pack(const int* __restrict__ idx, const int* __restrict__ inv, int n, int k, int E_loc,
+                          const uint4* __restrict__ z, int vec_per_row, uint4* __restrict__ send_z,
+                          int* __restrict__ send_expert) {
+  for (int a = blockIdx.x; a < n; a += gridDim.x) {
+    const int pos = inv[a];
+    const uint4* src = z + static_cast<int64_t>(a / k) * vec_per_row;
+    uint4* dst = send_z + static_cast<int64_t>(pos) * vec_per_row;
+    for (int c = threadIdx.x; c < vec_per_row; c += blockDim.x) dst[c] = src[c];
+    if (threadIdx.x == 0) send_expert[pos] = idx[a] % E_loc;
+  }
+}
+
+// An expert shard's results in the order its rows were received: ret_y[r] = y[inv[r]]
+// and ret_ss[r] = ss[inv[r]] (the L/32 partial sums of squares). A row whose expert
+// index was out of range has no slot (inv[r] < 0, the histogram recorded the error) and
+// gets zeros. One block per row, grid-strided; 16-byte vectors.
+__global__ void k_ep_unpermute(const int* __restrict__ inv, int R, const uint4* __restrict__ y,
+                               const uint4* __restrict__ ss, int vec_y, int vec_ss, uint4* __restrict__ ret_y,
+                               uint4* __restrict__ ret_ss) {
+  for (int r = blockIdx.x; r < R; r += gridDim.x) {
+    const int row = inv[r];
+    for (int c = threadIdx.x; c < vec_y + vec_ss; c += blockDim.x) {
+      const bool is_y = c < vec_y;
+      const int j = is_y ? c : c - vec_y;
+      const int vpr = is_y ? vec_y : vec_ss;
+      const uint4* src = (is_y ? y : ss) + static_cast<int64_t>(row) * vpr;
+      uint4* dst = (is_y ? ret_y : ret_ss) + static_cast<int64_t>(r) * vpr;
+      dst[j] = row >= 0 ? src[j] : make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+}
+
+// --------------------------------------------------------------------------------------
 // Self-test of the bounded waits: one thread waits on an mbarrier that nothing will ever
 // complete, through the same mbar_wait the GEMMs use, with a short limit; the timeout is
 // recorded in status (a completed wait would be recorded as a device error).

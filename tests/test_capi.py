@@ -111,3 +111,59 @@ def test_forward_rejects_null_and_misaligned_pointers_before_any_launch():
     cfg.workspace_bytes = 16
     assert lib.muse_latent_moe_forward(ctypes.byref(cfg), *args, None) == 3
     assert lib.muse_latent_moe_forward(None, *args, None) == 1
+
+
+@pytest.mark.parametrize("name", ["mid", "prefill", "nvfp4_w4a4"])
+@pytest.mark.parametrize("G", [1, 2, 8])
+def test_expert_parallel_workspaces_hold_only_their_roles_buffers(name, G):
+    w = W.WORKLOADS[name]
+    cfg = moe.make_config(w.T, w.D, w.L, w.I, w.E, w.k, w.dtype, w.eps,
+                          act_format=moe.ACT_NVFP4 if w.act == "nvfp4" else moe.ACT_BF16)
+    if w.experts == "nvfp4":
+        cfg.expert_weights = moe.EXPERTS_NVFP4
+    full = moe.workspace_layout(cfg)
+    home = moe.ep_workspace_layout(cfg, G, moe.EP_HOME)
+    rows = G * w.T * min(w.k, w.E // G)
+    shard = moe.ep_workspace_layout(cfg, G, moe.EP_EXPERTS, rows)
+    for n in ("zp", "h", "y", "ss", "zq_codes", "hq_codes"):
+        assert home[n] == 0, n
+    for n in ("logits", "topk_idx", "topk_w", "z", "c"):
+        assert shard[n] == 0, n
+        assert home[n] > 0 or n == "logits", n
+    assert home["rows"] == w.T * w.k  # the send plan has no padding
+    assert shard["rows"] >= rows and shard["rows"] <= rows + 16 * min(w.E // G, rows)
+    assert home["total"] < full["total"]
+    if G == 1:
+        assert shard["total"] < full["total"]
+    assert all(v % 256 == 0 for k, v in shard.items() if k not in ("total", "rows"))
+
+
+def test_expert_parallel_arguments_are_rejected_before_any_launch():
+    lib = moe.lib()
+    cfg = moe.make_config(16, 256, 128, 128, 8, 2, "f32")
+    lay = moe.WorkspaceLayout()
+    assert lib.muse_ep_workspace_layout(ctypes.byref(cfg), 3, moe.EP_HOME, 0, ctypes.byref(lay)) == 1  # 8 % 3
+    assert lib.muse_ep_workspace_layout(ctypes.byref(cfg), 0, moe.EP_HOME, 0, ctypes.byref(lay)) == 1
+    assert lib.muse_ep_workspace_layout(ctypes.byref(cfg), 2, 7, 0, ctypes.byref(lay)) == 1  # unknown role
+    assert lib.muse_ep_workspace_layout(ctypes.byref(cfg), 2, moe.EP_EXPERTS, -1, ctypes.byref(lay)) == 1
+    p = [ctypes.c_void_p(4096 * (i + 1)) for i in range(9)]
+    # dispatch: x, W_router, W_pool, send_z, send_expert, rank_counts
+    for bad in range(6):
+        a = list(p[:6])
+        a[bad] = ctypes.c_void_p(0)
+        assert lib.muse_ep_dispatch(ctypes.byref(cfg), 2, *a, None) == 1
+    assert lib.muse_ep_dispatch(ctypes.byref(cfg), 2, *p[:6], None) == 3  # no workspace
+    # experts: nothing received launches nothing, whatever the pointers
+    assert lib.muse_ep_experts(ctypes.byref(cfg), 2, 0, *([None] * 8), None) == 0
+    for bad in range(8):
+        a = list(p[:8])
+        a[bad] = ctypes.c_void_p(0)
+        assert lib.muse_ep_experts(ctypes.byref(cfg), 2, 5, *a, None) == 1
+    assert lib.muse_ep_experts(ctypes.byref(cfg), 2, 5, *p[:8], None) == 3
+    # combine: x, back_y, back_ss, gamma, W_unpool, out
+    for bad in range(6):
+        a = list(p[:6])
+        a[bad] = ctypes.c_void_p(4096 * (bad + 1) + 4)
+        assert lib.muse_ep_combine(ctypes.byref(cfg), 2, *a, None) == 1
+    assert lib.muse_ep_combine(ctypes.byref(cfg), 2, *p[:6], None) == 3
+    assert lib.muse_ep_combine(ctypes.byref(cfg), 3, *p[:6], None) == 1

@@ -1,0 +1,201 @@
+"""Expert parallelism: the exchange orchestration of latent_mixture_experts_moe_b200.ep on
+CPU ranks (gloo, uneven token counts, a rank with no tokens), and the library's three EP
+entry points on one GPU with the ranks' exchanges done by slicing (no kernel waits on
+another). Both compare with the FP64 oracle's single-device forward of the same tokens.
+
+The CPU ranks' compute is a test stand-in written here from the EP contract of
+include/muse_moe.h (send rows in expert, token, slot order; expert outputs and per-32-column
+partial sums of squares back in the order received; norm and combine on the token's rank),
+built from the oracle's steps; it checks that ep_forward routes every row to the rank that
+owns its expert and every result back to the row it came from.
+"""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+class OracleShard:
+    """Rank `rank` of G in float64 on the CPU, following the EP contract step by step."""
+
+    def __init__(self, inp, rank, G, k, eps):
+        f = oracle.as_f64
+        self.Wr, self.Wp, self.Wu = f(inp["W_router"]), f(inp["W_pool"]), f(inp["W_unpool"])
+        self.gamma = f(inp["gamma"])
+        self.E = self.Wr.shape[0]
+        self.E_loc = self.E // G
+        lo = rank * self.E_loc
+        # this rank holds only its own experts
+        self.Wg = f(inp["W_gate"][lo:lo + self.E_loc])
+        self.Wup = f(inp["W_up"][lo:lo + self.E_loc])
+        self.Wd = f(inp["W_down"][lo:lo + self.E_loc])
+        self.G, self.k, self.eps = G, k, eps
+        self.L = self.Wp.shape[0]
+
+    def dispatch(self, x):
+        x = x.numpy()
+        T, k = x.shape[0], self.k
+        if T == 0:
+            self.pos, self.idx, self.g = {}, np.zeros((0, k), np.int64), np.zeros((0, k))
+            return (torch.zeros((0, self.L), dtype=torch.float64), torch.zeros(0, dtype=torch.int32), [0] * self.G)
+        self.idx, self.g, _ = oracle.route(oracle.router_logits(x, self.Wr), k)
+        z = oracle.pooler(x, self.Wp)
+        pairs = sorted((int(self.idx[t, j]), t, j) for t in range(T) for j in range(k))
+        self.pos = {(t, j): p for p, (_, t, j) in enumerate(pairs)}
+        send_z = np.stack([z[t] for _, t, _ in pairs])
+        send_e = np.array([e % self.E_loc for e, _, _ in pairs], dtype=np.int32)
+        counts = [sum(1 for e, _, _ in pairs if e // self.E_loc == r) for r in range(self.G)]
+        return torch.from_numpy(send_z), torch.from_numpy(send_e), counts
+
+    def experts(self, recv_z, recv_e):
+        z, e = recv_z.numpy(), recv_e.numpy()
+        y = np.zeros((z.shape[0], self.L))
+        for i in range(z.shape[0]):
+            y[i] = oracle.expert_ffn(z[i:i + 1], self.Wg[e[i]], self.Wup[e[i]], self.Wd[e[i]])[0]
+        ss = (y * y).reshape(y.shape[0], self.L // 32, 32).sum(axis=2)
+        return torch.from_numpy(y), torch.from_numpy(ss)
+
+    def combine(self, x, back_y, back_ss):
+        T, k = x.shape[0], self.k
+        y, ss = back_y.numpy(), back_ss.numpy()
+        n = np.zeros((T, k, self.L))
+        for t in range(T):
+            for j in range(k):
+                p = self.pos[(t, j)]
+                n[t, j] = oracle.centred_rmsnorm(y[p], self.gamma[self.idx[t, j]], self.eps)
+                assert abs(ss[p].sum() - (y[p] ** 2).sum()) <= 1e-9 * max(1.0, ss[p].sum())
+        return torch.from_numpy(oracle.unpooler(oracle.combine(n, self.g), self.Wu))
+
+
+def _tokens(w, counts):
+    whole = torch.empty((sum(counts), w.D), dtype=torch.float32)
+    W.fill(whole, w.seed, W.TID["x"], 1.0)
+    starts = np.concatenate([[0], np.cumsum(counts)])
+    return whole, [whole[starts[r]:starts[r + 1]] for r in range(len(counts))]
+
+
+def _worker(rank, world, port, counts, q):
+    import sys
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from latent_mixture_experts_moe_b200 import ep
+        w = W.WORKLOADS["tiny"]
+        inp = W.make_inputs(w, "cpu", names=["W_router", "W_pool", "W_gate", "W_up", "W_down", "gamma", "W_unpool"])
+        _, xs = _tokens(w, counts)
+        shard = OracleShard(inp, rank, world, w.k, w.eps)
+        out = ep.ep_forward(shard, xs[rank].to(torch.float64))
+        f = oracle.as_f64
+        err, n_remote = 0.0, 0
+        if counts[rank]:
+            ref = oracle.latent_moe_forward(f(xs[rank]), f(inp["W_router"]), f(inp["W_pool"]),
+                                            (f(inp["W_gate"]), f(inp["W_up"]), f(inp["W_down"])), f(inp["gamma"]),
+                                            f(inp["W_unpool"]), w.k, w.eps)
+            err = float(np.abs(out.numpy() - ref["out"]).max())
+            n_remote = int(np.sum(ref["idx"] // shard.E_loc != rank))
+        q.put((rank, tuple(out.shape), err, n_remote))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("counts", [(5, 11), (3, 0, 7, 5)], ids=["2ranks", "4ranks_one_empty"])
+def test_ep_forward_over_gloo_ranks_matches_the_single_device_block(counts):
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    world = len(counts)
+    procs = [ctx.Process(target=_worker, args=(r, world, port, counts, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=300) for _ in range(world))
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    w = W.WORKLOADS["tiny"]
+    for r, shape, err, _ in res:
+        assert shape == (counts[r], w.D)
+        assert err < 1e-12, f"rank {r}: max error {err}"
+    assert sum(n for *_, n in res) > 0  # rows did cross between ranks
+
+
+# ---------------------------------------------------------------------------------- GPU
+@pytest.mark.gpu
+@pytest.mark.parametrize("G,counts", [(1, (96,)), (2, (100, 156)), (4, (64, 0, 97, 95))],
+                         ids=["1rank", "2ranks", "4ranks_one_empty"])
+def test_ep_entry_points_on_one_gpu_match_the_oracle_and_the_fused_forward(G, counts):
+    import latent_mixture_experts_moe_b200 as moe
+    from latent_mixture_experts_moe_b200 import ep
+    import parity_util as P
+    w = W.WORKLOADS["mid"]
+    dev = torch.device("cuda")
+    inp = W.make_inputs(w, dev)
+    T = sum(counts)
+    x = inp["x"][:T]
+    starts = np.concatenate([[0], np.cumsum(counts)])
+    xs = [x[starts[r]:starts[r + 1]] for r in range(G)]
+    E_loc = w.E // G
+    shards = []
+    for r in range(G):
+        wts = {n: v for n, v in inp.items() if n not in ("x", "W_gate", "W_up", "W_down")}
+        for n in ("W_gate", "W_up", "W_down"):
+            wts[n] = inp[n][r * E_loc:(r + 1) * E_loc].contiguous()
+        shards.append(ep.ExpertShard(wts, r, G, T_max=max(counts), k=w.k, eps=w.eps))
+    outs = ep.ep_forward_one_device(shards, xs)
+    torch.cuda.synchronize()
+    for s in shards:
+        code, detail = moe.last_device_status(s.config(1, s.ws_home))
+        assert code == 0, f"home status {code} {detail:#x}"
+        code, detail = moe.last_device_status(s.config(1, s.ws_experts))
+        assert code == 0, f"expert status {code} {detail:#x}"
+    got = torch.cat(outs)
+    assert got.shape == (T, w.D)
+    # the fused single-GPU forward of the same tokens: same kernels, other tilings
+    fused = P.Run(w, inp, T=T)
+    d = (got.float() - fused.out.float()).abs()
+    assert P.rel_l2(got.float().cpu().numpy(), fused.out.float().cpu().numpy()) < 2e-3
+    # the oracle, with the routing rule of the parity tests
+    rows = np.arange(T)
+    ref = P.oracle_block(w, inp, rows)
+    alt = P.check_routing(ref, fused.idx.cpu().numpy(), fused.g.cpu().numpy(), w.k)
+    want = P.oracle_on_gpu_alternatives(w, inp, rows, ref, fused.idx.cpu().numpy(), alt)
+    P.assert_close(got.float().cpu().numpy(), want, f"EP over {G} ranks")
+    print(f"G={G}: max |EP - fused| = {float(d.max()):.3e}, equal elements {float((d == 0).float().mean()):.4f}")
+
+
+@pytest.mark.gpu
+def test_ep_experts_records_an_out_of_range_local_expert_and_zeroes_its_row():
+    import latent_mixture_experts_moe_b200 as moe
+    from latent_mixture_experts_moe_b200 import ep
+    w = W.WORKLOADS["mid"]
+    dev = torch.device("cuda")
+    inp = W.make_inputs(w, dev)
+    G = 2
+    E_loc = w.E // G
+    wts = {n: v for n, v in inp.items() if n not in ("x", "W_gate", "W_up", "W_down")}
+    for n in ("W_gate", "W_up", "W_down"):
+        wts[n] = inp[n][:E_loc].contiguous()
+    s = ep.ExpertShard(wts, 0, G, T_max=16, k=w.k, eps=w.eps)
+    recv_z = torch.randn((5, w.L), device=dev).to(torch.bfloat16)
+    recv_e = torch.tensor([0, 3, E_loc, 7, 1], dtype=torch.int32, device=dev)  # row 2 out of range
+    y, ss = s.experts(recv_z, recv_e)
+    torch.cuda.synchronize()
+    code, _ = moe.last_device_status(s.config(1, s.ws_experts))
+    assert moe.STATUS[code] == "MUSE_ERR_DEVICE"
+    assert torch.count_nonzero(y[2]) == 0 and torch.count_nonzero(ss[2]) == 0
+    assert torch.count_nonzero(y[0]) > 0 and torch.count_nonzero(y[4]) > 0
