@@ -61,8 +61,10 @@ class ExpertShard:
         self.rows_max = rows_max if rows_max is not None else ep_size * T_max * min(k, self.E_loc)
         home = ep_workspace_layout(self.config(T_max), ep_size, EP_HOME)["total"]
         shard = ep_workspace_layout(self.config(T_max), ep_size, EP_EXPERTS, max(self.rows_max, 1))["total"]
-        self.ws_home = torch.empty(home, dtype=torch.uint8, device=dev)
-        self.ws_experts = torch.empty(shard, dtype=torch.uint8, device=dev)
+        # zeroed once, so that a status read before a side has run (a rank with no tokens, a
+        # shard that received no rows) reads MUSE_OK
+        self.ws_home = torch.zeros(home, dtype=torch.uint8, device=dev)
+        self.ws_experts = torch.zeros(shard, dtype=torch.uint8, device=dev)
         self.send_z = torch.empty((T_max * k, L), dtype=self.act, device=dev)
         self.send_expert = torch.empty(T_max * k, dtype=torch.int32, device=dev)
         self.rank_counts = torch.empty(ep_size, dtype=torch.int32, device=dev)
