@@ -368,14 +368,20 @@ muse_status dense_gemm(const void* W, int64_t M, const void* X, int64_t T, int64
   g.ss_ld = sq.ld;
   g.ss_gain = sq.gain;
   g.ss_gain_group_stride = 0;
-  // a CTA pair per 256 features x 256 tokens when that fills at least one wave of pairs
+  // a CTA pair per 256 features x 256 tokens when that fills at least one wave of pairs;
+  // 512 features (two weight tiles per CTA, so each staged token tile feeds twice the
+  // MMAs) when the width allows
   if (bf && bn == 256 && cdiv(M, 256) * cdiv(T, 256) >= nsm / 2) {
     if (sizeof(TOut) == 2 && !make_out_map(&maps.out, out, T, M)) return MUSE_ERR_CUDA;
-    g.m_step = 256;
-    g.m_tiles = static_cast<int>(cdiv(M, 256));
+    const bool wide = sizeof(TOut) == 2 && M % 512 == 0;
+    g.m_step = wide ? 512 : 256;
+    g.m_tiles = static_cast<int>(cdiv(M, g.m_step));
     g.num_tiles = static_cast<int>(g.m_tiles * cdiv(T, 256));
     g.tile_counter = tile_counter;
     const int pairs = std::min(g.num_tiles, nsm / 2);
+    if constexpr (sizeof(TOut) == 2) {
+      if (wide) return launch_gemm_2sm<TOut, EPI, 2>(maps, g, pairs, st) == cudaSuccess ? MUSE_OK : MUSE_ERR_CUDA;
+    }
     return launch_gemm_2sm<TOut, EPI, 1>(maps, g, pairs, st) == cudaSuccess ? MUSE_OK : MUSE_ERR_CUDA;
   }
   // two 128-row weight tiles per CTA when that still leaves at least a full wave of tiles
