@@ -135,47 +135,76 @@ def test_ep_forward_over_gloo_ranks_matches_the_single_device_block(counts):
 
 
 # ---------------------------------------------------------------------------------- GPU
+EXPERT_KEYS = ("W_gate", "W_up", "W_down")  # dense tensors or their NVFP4 _codes / _scales / _mscale
+
+EP_CASES = [
+    # name, workload, ranks, tokens per rank, with the feed-forward sublayer steps
+    ("mid_1rank", W.WORKLOADS["mid"], 1, (96,), False),
+    ("mid_2ranks", W.WORKLOADS["mid"], 2, (100, 156), False),
+    ("mid_4ranks_one_empty", W.WORKLOADS["mid"], 4, (64, 0, 97, 95), False),
+    ("sublayer_2ranks", W.Workload("ep_sublayer", T=256, D=2048, L=1024, I=1024, E=64, k=4, dtype="bf16", seed=5),
+     2, (120, 136), True),
+    ("f32_2ranks", W.Workload("ep_f32", T=37, D=256, L=256, I=128, E=8, k=3, dtype="f32", seed=7), 2, (17, 20),
+     False),
+    ("nvfp4_w4a16_2ranks", W.Workload("ep_nvfp4", T=200, D=1024, L=512, I=512, E=16, k=4, dtype="bf16", seed=13,
+                                      experts="nvfp4"), 2, (90, 110), False),
+    ("nvfp4_w4a4_4ranks", W.Workload("ep_w4a4", T=256, D=1024, L=512, I=512, E=16, k=4, dtype="bf16", seed=13,
+                                     experts="nvfp4", act="nvfp4"), 4, (70, 58, 64, 64), False),
+]
+
+
+def _shard_weights(inp, r, E_loc):
+    """Rank r's weights: everything replicated except its slice of the expert tensors."""
+    wts = {}
+    for n, v in inp.items():
+        if n == "x":
+            continue
+        if n.startswith(EXPERT_KEYS):
+            wts[n] = v[r * E_loc:(r + 1) * E_loc].contiguous()
+        else:
+            wts[n] = v
+    return wts
+
+
 @pytest.mark.gpu
-@pytest.mark.parametrize("G,counts", [(1, (96,)), (2, (100, 156)), (4, (64, 0, 97, 95))],
-                         ids=["1rank", "2ranks", "4ranks_one_empty"])
-def test_ep_entry_points_on_one_gpu_match_the_oracle_and_the_fused_forward(G, counts):
+@pytest.mark.parametrize("case", EP_CASES, ids=[c[0] for c in EP_CASES])
+def test_ep_entry_points_on_one_gpu_match_the_oracle_and_the_fused_forward(case):
     import latent_mixture_experts_moe_b200 as moe
     from latent_mixture_experts_moe_b200 import ep
     import parity_util as P
-    w = W.WORKLOADS["mid"]
+    name, w, G, counts, sublayer = case
     dev = torch.device("cuda")
     inp = W.make_inputs(w, dev)
+    if sublayer:
+        inp.update(W.sublayer_inputs(w, dev))
     T = sum(counts)
     x = inp["x"][:T]
     starts = np.concatenate([[0], np.cumsum(counts)])
     xs = [x[starts[r]:starts[r + 1]] for r in range(G)]
     E_loc = w.E // G
-    shards = []
-    for r in range(G):
-        wts = {n: v for n, v in inp.items() if n not in ("x", "W_gate", "W_up", "W_down")}
-        for n in ("W_gate", "W_up", "W_down"):
-            wts[n] = inp[n][r * E_loc:(r + 1) * E_loc].contiguous()
-        shards.append(ep.ExpertShard(wts, r, G, T_max=max(counts), k=w.k, eps=w.eps))
+    modes = dict(act_format=moe.ACT_NVFP4) if w.act == "nvfp4" else {}
+    shards = [ep.ExpertShard(_shard_weights(inp, r, E_loc), r, G, T_max=max(counts), k=w.k, eps=w.eps, **modes)
+              for r in range(G)]
     outs = ep.ep_forward_one_device(shards, xs)
     torch.cuda.synchronize()
     for s in shards:
-        code, detail = moe.last_device_status(s.config(1, s.ws_home))
-        assert code == 0, f"home status {code} {detail:#x}"
-        code, detail = moe.last_device_status(s.config(1, s.ws_experts))
-        assert code == 0, f"expert status {code} {detail:#x}"
+        for ws in (s.ws_home, s.ws_experts):
+            code, detail = moe.last_device_status(s.config(1, ws))
+            assert code == 0, f"status {code} {detail:#x}"
     got = torch.cat(outs)
     assert got.shape == (T, w.D)
-    # the fused single-GPU forward of the same tokens: same kernels, other tilings
+    # the fused single-GPU forward of the same tokens: the same kernels over other row counts
     fused = P.Run(w, inp, T=T)
     d = (got.float() - fused.out.float()).abs()
-    assert P.rel_l2(got.float().cpu().numpy(), fused.out.float().cpu().numpy()) < 2e-3
-    # the oracle, with the routing rule of the parity tests
+    assert P.rel_l2(got.double().cpu().numpy(), fused.out.double().cpu().numpy()) < 2e-3
+    # the oracle, with the routing rule of the parity tests (W4A4: the fused run's activation
+    # codes are the candidate decisions at rounding boundaries)
     rows = np.arange(T)
-    ref = P.oracle_block(w, inp, rows)
+    ref = P.oracle_block(w, inp, rows, run=fused)
     alt = P.check_routing(ref, fused.idx.cpu().numpy(), fused.g.cpu().numpy(), w.k)
-    want = P.oracle_on_gpu_alternatives(w, inp, rows, ref, fused.idx.cpu().numpy(), alt)
-    P.assert_close(got.float().cpu().numpy(), want, f"EP over {G} ranks")
-    print(f"G={G}: max |EP - fused| = {float(d.max()):.3e}, equal elements {float((d == 0).float().mean()):.4f}")
+    want = P.oracle_on_gpu_alternatives(w, inp, rows, ref, fused.idx.cpu().numpy(), alt, run=fused)
+    P.assert_close(got.double().cpu().numpy(), want, f"EP {name}", rel=2e-2 if w.experts == "nvfp4" else P.REL_L2)
+    print(f"{name}: max |EP - fused| = {float(d.max()):.3e}, equal elements {float((d == 0).float().mean()):.4f}")
 
 
 @pytest.mark.gpu
