@@ -114,6 +114,7 @@ def stage_work(w: W.Workload, n_touched: int):
     T, D, L, I, E, k = w.T, w.D, w.L, w.I, w.E, w.k
     a = 2 if w.dtype == "bf16" else 4
     ab = 0.5625 if w.experts == "nvfp4" else a      # bytes per expert weight
+    aa = 0.5625 if w.act == "nvfp4" else a          # bytes per activation value the expert GEMMs read
     A = T * k
     return {
         "router": (2 * T * E * D, T * D * a + E * D * a + T * E * 4),
@@ -123,8 +124,9 @@ def stage_work(w: W.Workload, n_touched: int):
         "assign_rows": (0, A * 8),
         "pooler": (2 * T * L * D, T * D * a + L * D * a + T * L * a),
         "gather": (0, T * L * a + A * L * a),
-        "gate_up_swiglu": (2 * A * L * 2 * I, n_touched * 2 * I * L * ab + A * L * a + A * I * a),
-        "down_sumsq": (2 * A * I * L, n_touched * L * I * ab + A * I * a + A * L * a + A * (L // 32) * 4),
+        # W4A4: the GEMMs read their activation operands as codes (0.5625 B per value)
+        "gate_up_swiglu": (2 * A * L * 2 * I, n_touched * 2 * I * L * ab + A * L * aa + A * I * a),
+        "down_sumsq": (2 * A * I * L, n_touched * L * I * ab + A * I * aa + A * L * a + A * (L // 32) * 4),
         "norm_combine": (0, A * L * a + A * (L // 32) * 4 + T * L * a + n_touched * L * a),
         "unpooler": (2 * T * D * L, T * L * a + D * L * a + T * D * a),
         # optional steps: pre-expert norm on z; the feed-forward sublayer's pre-norm on x
@@ -132,7 +134,8 @@ def stage_work(w: W.Workload, n_touched: int):
         "pre_expert_norm": (0, 2 * T * L * a + L * a),
         "ffn_pre_norm": (0, 2 * T * D * a + D * a),
         "ffn_post_norm_gate": (0, 3 * T * D * a + T * (D // 32) * 4 + D * (a + 4)),
-        # W4A4: latent rows gathered and quantised (0.5625 B per value out), h quantised
+        # W4A4: latent rows quantised once per token (0.5625 B per value out), then gathered;
+        # h quantised
         "quant_z": (0, T * L * a + T * L * 0.5625),
         "gather_codes": (0, T * L * 0.5625 + A * L * 0.5625),
         "quant_h": (0, A * I * a + A * I * 0.5625),

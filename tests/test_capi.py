@@ -167,3 +167,20 @@ def test_expert_parallel_arguments_are_rejected_before_any_launch():
         assert lib.muse_ep_combine(ctypes.byref(cfg), 2, *a, None) == 1
     assert lib.muse_ep_combine(ctypes.byref(cfg), 2, *p[:6], None) == 3
     assert lib.muse_ep_combine(ctypes.byref(cfg), 3, *p[:6], None) == 1
+
+
+@pytest.mark.parametrize("w4a4", [False, True])
+@pytest.mark.parametrize("pre_expert,ffn_pre,ffn_post", [(0, 0, 0), (1, 0, 0), (0, 1, 1), (1, 1, 0), (0, 0, 1)])
+def test_stage_names_match_the_library_launch_count(w4a4, pre_expert, ffn_pre, ffn_post):
+    cfg = moe.make_config(64, 1024, 512, 512, 16, 2, "bf16", act_format=moe.ACT_NVFP4 if w4a4 else moe.ACT_BF16)
+    if w4a4:
+        cfg.expert_weights = moe.EXPERTS_NVFP4
+    # any non-null pointer switches a step on; launch_count reads no memory
+    cfg.pre_norm_gain = 4096 if pre_expert else None
+    cfg.ffn_pre_gain = 4096 if ffn_pre else None
+    cfg.ffn_post_gain = 4096 if ffn_post else None
+    names = moe.stages(cfg)
+    assert len(names) == moe.launch_count(cfg)
+    assert len(set(names)) == len(names)
+    assert ("quant_z" in names) == w4a4 and ("gather_codes" in names) == w4a4
+    assert names.index("pooler") < names.index("gather_codes" if w4a4 else "gather") < names.index("gate_up_swiglu")
