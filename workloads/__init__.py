@@ -69,6 +69,9 @@ WORKLOADS: Dict[str, Workload] = {
     # decode-like NVFP4 case on ~1 GB of weights (2-3 tokens per expert; profiling captures)
     "nvfp4_decode_e32": Workload("nvfp4_decode_e32", T=32, D=8192, L=4096, I=4096, E=32, k=2, dtype="bf16",
                                  experts="nvfp4"),
+    # NVFP4 experts on prefill-sized tiles (256 tokens per expert) at a few GB: the small case
+    # the W4A16 kernel is profiled on
+    "nvfp4_e16": Workload("nvfp4_e16", T=2048, D=8192, L=4096, I=4096, E=16, k=2, dtype="bf16", experts="nvfp4"),
     # the same NVFP4 layers with both operands of the expert GEMMs in NVFP4 (W4A4)
     "nvfp4_w4a4": Workload("nvfp4_w4a4", T=4096, D=8192, L=4096, I=4096, E=256, k=8, dtype="bf16",
                            experts="nvfp4", act="nvfp4"),
