@@ -63,7 +63,28 @@ struct GemmArgs {
   uint32_t* status;          // workspace status word
   int* tile_counter;         // CTA-pair kernel: tiles are claimed from this counter (zero
                              // before the launch); nullptr: static round robin over pairs
+  int k_splits;              // one-CTA dense GEMM: K divided into this many equal ranges of
+                             // k-blocks (0 or 1: none); range s writes its FP32 partial
+                             // product to (float*)out + s * split_stride
+  int64_t split_stride;
 };
+
+// Split-K decode of launch tile t (dense tiling): range s = t / base of base tile t % base,
+// base = num_tiles / k_splits, over k-blocks [kb0, kb1). Without splits: the whole K.
+__device__ __forceinline__ void split_range(const GemmArgs& p, int num_tiles, int& t, int& s, int& kb0, int& kb1) {
+  if (p.k_splits > 1) {
+    const int base = num_tiles / p.k_splits;
+    const int per = p.k_blocks / p.k_splits;  // the host splits only evenly
+    s = t / base;
+    t -= s * base;
+    kb0 = s * per;
+    kb1 = kb0 + per;
+  } else {
+    s = 0;
+    kb0 = 0;
+    kb1 = p.k_blocks;
+  }
+}
 
 template <typename TIn>
 struct ElemTraits;
@@ -211,12 +232,13 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ Tm
       uint32_t issued_mask = 0, issued_phase = 0;  // per stage, for the abort drain
       bool ok = true;
       for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
-        int g, m0, row0, n;
-        gemm_tile(p, t, BN, g, m0, row0, n);
+        int g, m0, row0, n, tb = t, ks, kb0, kb1;
+        split_range(p, num_tiles, tb, ks, kb0, kb1);
+        gemm_tile(p, tb, BN, g, m0, row0, n);
         const int nb16 = (n + 15) >> 4;
         const uint32_t bytes = S::kABytes * (kDual ? 2u : 1u) + static_cast<uint32_t>(nb16) * 2048u;
         const int a_row = g * p.rows_per_group + m0;
-        for (int kb = 0; kb < p.k_blocks; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.status, 0x100u + stage)) {
             ok = false;
             break;
@@ -262,8 +284,9 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ Tm
       bool ok = true;
       bool issued_any = false;
       for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
-        int g, m0, row0, n;
-        gemm_tile(p, t, BN, g, m0, row0, n);
+        int g, m0, row0, n, tb = t, ks, kb0, kb1;
+        split_range(p, num_tiles, tb, ks, kb0, kb1);
+        gemm_tile(p, tb, BN, g, m0, row0, n);
         const uint32_t N = static_cast<uint32_t>((n + 15) & ~15);
         const uint32_t idesc = idesc_f32acc(ElemTraits<TIn>::kFmt, 128u, N);
         if (!mbar_wait(acce_bar(acc), acc_phase ^ 1u, abort_flag, p.status, 0x200u + acc)) {
@@ -272,7 +295,7 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ Tm
         }
         tc_fence_after();
         const uint32_t d = tmem_base + static_cast<uint32_t>(acc) * S::kAccCols;
-        for (int kb = 0; kb < p.k_blocks; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(full_bar(stage), phase, abort_flag, p.status, 0x300u + stage)) {
             ok = false;
             break;
@@ -282,7 +305,7 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ Tm
           const uint32_t sB = sA + S::kABytes * (kDual ? 2u : 1u);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
+            const uint32_t accum = (kb > kb0 || kk > 0) ? 1u : 0u;
             const uint64_t db = sdesc_k_sw128(sB + 32u * kk);
             umma<kTF32>(d, sdesc_k_sw128(sA + 32u * kk), db, idesc, accum);
             if (kDual) umma<kTF32>(d + BN, sdesc_k_sw128(sA + S::kABytes + 32u * kk), db, idesc, accum);
@@ -316,15 +339,16 @@ __global__ void __launch_bounds__(192, 1) k_umma_gemm(const __grid_constant__ Tm
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
-      int g, m0, row0, n;
-      gemm_tile(p, t, BN, g, m0, row0, n);
+      int g, m0, row0, n, tb = t, ks, kb0, kb1;
+      split_range(p, num_tiles, tb, ks, kb0, kb1);
+      gemm_tile(p, tb, BN, g, m0, row0, n);
       // every lane waits; the vote keeps the warp converged for the .sync.aligned loads
       const bool ready = mbar_wait(accf_bar(acc), acc_phase, abort_flag, p.status, 0x400u + acc);
       if (!__all_sync(0xffffffffu, ready)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc) * S::kAccCols;
-      TOut* out = reinterpret_cast<TOut*>(p.out);
+      TOut* out = reinterpret_cast<TOut*>(p.out) + static_cast<int64_t>(ks) * p.split_stride;
       const int nchunks = (n + 31) >> 5;
       if constexpr (EPI == EPI_SWIGLU) {
         const int f = m0 + q * 32 + lane;  // output feature of this thread (within group)

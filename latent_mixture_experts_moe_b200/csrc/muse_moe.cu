@@ -12,6 +12,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -46,6 +47,7 @@ struct Layout {
   muse_moe_workspace_layout pub;
   size_t tiles_gu, tiles_dn, ntiles;  // int4 lists; int[8]: tile counts [0..1], tile counters [4..7]
   size_t zt_codes, zt_scales;         // W4A4: the latent quantised in token order [T, L/2], [T, L/16]
+  size_t splitk, splitk_bytes;        // FP32 partial products of split-K dense GEMMs (0 bytes: none)
   int64_t max_tiles_gu, max_tiles_dn;
 };
 
@@ -105,6 +107,14 @@ Layout make_layout(const muse_moe_config& c, Role role = Role::kFull) {
   l.pub.zq_scales = take(q, rows * (c.L / 16));
   l.pub.hq_codes = take(q, rows * (c.I / 2));
   l.pub.hq_scales = take(q, rows * (c.I / 16));
+  // split-K partials of the dense GEMMs (router, pooler, unpooler) when one of them has a K
+  // of 64 k-blocks or more: up to 32 ranges of T x M floats, at most 8 MiB -- decode-sized
+  // outputs; larger ones cost more in partial traffic than the extra CTAs win
+  const int64_t kb_max = std::max(c.D, c.L) * static_cast<int64_t>(as) / 128;
+  l.splitk_bytes = (home && kb_max >= 64)
+                       ? std::min<size_t>(size_t(8) << 20, sizeof(float) * 32 * T * std::max({c.D, c.L, c.E}))
+                       : 0;
+  l.splitk = take(l.splitk_bytes > 0, l.splitk_bytes);
   l.pub.total = o;
   l.pub.rows = rows;
   return l;
@@ -349,10 +359,17 @@ struct DenseSS {
   const void* gain = nullptr;
 };
 
+// Scratch for split-K partial products (null: K is never split).
+struct SplitK {
+  float* buf = nullptr;
+  size_t bytes = 0;
+};
+
 // dense C[T, M] = X[T, K] W[M, K]^T
 template <typename TIn, typename TOut, int EPI = EPI_STORE>
 muse_status dense_gemm(const void* W, int64_t M, const void* X, int64_t T, int64_t K, void* out, int bn,
-                       uint32_t* status, int* tile_counter, cudaStream_t st, DenseSS sq = DenseSS{}) {
+                       uint32_t* status, int* tile_counter, cudaStream_t st, DenseSS sq = DenseSS{},
+                       SplitK sk = SplitK{}) {
   TmaMaps maps;
   const bool bf = sizeof(TIn) == 2;
   if (!make_maps(&maps, W, nullptr, M, X, T, K, bf)) return MUSE_ERR_CUDA;
@@ -389,6 +406,28 @@ muse_status dense_gemm(const void* W, int64_t M, const void* X, int64_t T, int64
   g.m_step = 128 * mt;
   g.m_tiles = static_cast<int>(cdiv(M, g.m_step));
   g.num_tiles = static_cast<int>(g.m_tiles * cdiv(T, bn));
+  // K split into S equal ranges while the tiles of all ranges still fit one wave: each
+  // range writes its FP32 partial product, k_splitk_reduce sums them in range order
+  int S = 1;
+  if (EPI == EPI_STORE && sk.buf != nullptr && M % 4 == 0) {
+    while (2 * S * g.num_tiles <= nsm && g.k_blocks % (2 * S) == 0 && g.k_blocks / (2 * S) >= 4 &&
+           sizeof(float) * static_cast<size_t>(2 * S) * T * M <= sk.bytes)
+      S *= 2;
+  }
+  if (S > 1) {
+    g.k_splits = S;
+    g.split_stride = T * M;
+    g.out = sk.buf;
+    g.ld_out = M;
+    g.num_tiles *= S;
+    if (launch_gemm_bn<TIn, float, EPI_STORE>(bn, mt, maps, g, std::min(g.num_tiles, nsm), st) != cudaSuccess)
+      return MUSE_ERR_CUDA;
+    const int64_t n4 = T * M / 4;
+    const int rgrid = static_cast<int>(std::min<int64_t>(cdiv(n4, 256), 4 * nsm));
+    k_splitk_reduce<TOut><<<rgrid, 256, 0, st>>>(reinterpret_cast<const float4*>(sk.buf), n4, S,
+                                                 static_cast<TOut*>(out));
+    return cudaGetLastError() == cudaSuccess ? MUSE_OK : MUSE_ERR_CUDA;
+  }
   const int grid = std::min(g.num_tiles, nsm);
   return launch_gemm_bn<TIn, TOut, EPI>(bn, mt, maps, g, grid, st) == cudaSuccess ? MUSE_OK : MUSE_ERR_CUDA;
 }
@@ -448,6 +487,14 @@ struct Pass {
     row_token = ptr<int>(l.pub.row_token);
   }
   uint8_t* at(size_t off) const { return ws + off; }
+  SplitK splitk() const {
+    SplitK k;
+    if (lay.splitk_bytes > 0) {
+      k.buf = reinterpret_cast<float*>(ws + lay.splitk);
+      k.bytes = lay.splitk_bytes;
+    }
+    return k;
+  }
   template <typename U>
   U* ptr(size_t off) const { return reinterpret_cast<U*>(ws + off); }
   cudaError_t mark() {
@@ -483,7 +530,8 @@ muse_status route(Pass<T>& p, const void* x, const void* W_router, const void** 
   }
   float* logits = p.template ptr<float>(p.lay.pub.logits);
   if (sizeof(T) == 2) {
-    MUSE_TRY((dense_gemm<T, float>(W_router, E, *xin, Tn, D, logits, dense_bn(c), p.status, nullptr, p.st)));
+    MUSE_TRY((dense_gemm<T, float>(W_router, E, *xin, Tn, D, logits, dense_bn(c), p.status, nullptr, p.st, DenseSS{},
+                                   p.splitk())));
   } else {
     k_router_logits_f32<<<static_cast<unsigned>(Tn), 256, 0, p.st>>>(reinterpret_cast<const float*>(*xin),
                                                                     reinterpret_cast<const float*>(W_router),
@@ -538,7 +586,8 @@ template <typename T>
 muse_status pool(Pass<T>& p, const void* xin, const void* W_pool) {
   const muse_moe_config& c = p.c;
   T* z = p.template ptr<T>(p.lay.pub.z);
-  MUSE_TRY((dense_gemm<T, T>(W_pool, c.L, xin, c.T, c.D, z, dense_bn(c), p.status, p.ntiles + 6, p.st)));
+  MUSE_TRY((dense_gemm<T, T>(W_pool, c.L, xin, c.T, c.D, z, dense_bn(c), p.status, p.ntiles + 6, p.st, DenseSS{},
+                             p.splitk())));
   MUSE_CK(p.mark());
   if (c.pre_norm_gain != nullptr) {
     k_rmsnorm_rows<T><<<static_cast<unsigned>(c.T), 256, 0, p.st>>>(
@@ -736,7 +785,8 @@ muse_status combine(Pass<T>& p, const T* y, const float* ss, const void* x, cons
     MUSE_TRY((dense_gemm<T, T, EPI_STORE_SS>(W_unpool, D, cbuf, Tn, L, out, dense_bn(c), p.status, p.ntiles + 7,
                                              p.st, sq)));
   } else {
-    MUSE_TRY((dense_gemm<T, T>(W_unpool, D, cbuf, Tn, L, out, dense_bn(c), p.status, p.ntiles + 7, p.st)));
+    MUSE_TRY((dense_gemm<T, T>(W_unpool, D, cbuf, Tn, L, out, dense_bn(c), p.status, p.ntiles + 7, p.st, DenseSS{},
+                               p.splitk())));
   }
   MUSE_CK(p.mark());
   // feed-forward sublayer post-norm and residual gate (optional), in place on out

@@ -455,6 +455,35 @@ __global__ void k_combine(const int* __restrict__ topk_idx, const float* __restr
 }
 
 // --------------------------------------------------------------------------------------
+// Split-K GEMM: out[i] = sum over the S K-ranges of part[s * n + i] (i < n = T * M), summed
+// in range order so that equal inputs give equal bits, converted to the output type.
+// Grid-strided over groups of 4 elements (n is a multiple of 4: M is a multiple of 128).
+// --------------------------------------------------------------------------------------
+template <typename TOut>
+__global__ void k_splitk_reduce(const float4* __restrict__ part, int64_t n4, int S, TOut* __restrict__ out) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float4 acc = part[i];
+    for (int s = 1; s < S; ++s) {
+      const float4 v = part[static_cast<int64_t>(s) * n4 + i];
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    if constexpr (sizeof(TOut) == 4) {
+      reinterpret_cast<float4*>(out)[i] = acc;
+    } else {
+      __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
+      uint2 w;
+      w.x = *reinterpret_cast<uint32_t*>(&lo);
+      w.y = *reinterpret_cast<uint32_t*>(&hi);
+      reinterpret_cast<uint2*>(out)[i] = w;
+    }
+  }
+}
+
+// --------------------------------------------------------------------------------------
 // Expert parallelism over G ranks, rank r owning experts [r * E_loc, (r + 1) * E_loc).
 // The latent of a token crosses to each rank that owns one of its experts (one row per
 // selected expert, 2 L bytes); the expert outputs and their partial sums of squares
