@@ -9,6 +9,7 @@ partial sums of squares back in the order received; norm and combine on the toke
 built from the oracle's steps; it checks that ep_forward routes every row to the rank that
 owns its expert and every result back to the row it came from.
 """
+import math
 import os
 import socket
 
@@ -138,18 +139,21 @@ def test_ep_forward_over_gloo_ranks_matches_the_single_device_block(counts):
 EXPERT_KEYS = ("W_gate", "W_up", "W_down")  # dense tensors or their NVFP4 _codes / _scales / _mscale
 
 EP_CASES = [
-    # name, workload, ranks, tokens per rank, with the feed-forward sublayer steps
-    ("mid_1rank", W.WORKLOADS["mid"], 1, (96,), False),
-    ("mid_2ranks", W.WORKLOADS["mid"], 2, (100, 156), False),
-    ("mid_4ranks_one_empty", W.WORKLOADS["mid"], 4, (64, 0, 97, 95), False),
+    # name, workload, ranks, tokens per rank, extra steps ("sublayer": the feed-forward
+    # sublayer around the block; "pages": the released model's router and norms)
+    ("mid_1rank", W.WORKLOADS["mid"], 1, (96,), None),
+    ("mid_2ranks", W.WORKLOADS["mid"], 2, (100, 156), None),
+    ("mid_4ranks_one_empty", W.WORKLOADS["mid"], 4, (64, 0, 97, 95), None),
     ("sublayer_2ranks", W.Workload("ep_sublayer", T=256, D=2048, L=1024, I=1024, E=64, k=4, dtype="bf16", seed=5),
-     2, (120, 136), True),
+     2, (120, 136), "sublayer"),
+    ("pages_mode_2ranks", W.Workload("ep_pages", T=256, D=2048, L=1024, I=1024, E=64, k=4, dtype="bf16", eps=1e-8,
+                                     seed=5), 2, (140, 116), "pages"),
     ("f32_2ranks", W.Workload("ep_f32", T=37, D=256, L=256, I=128, E=8, k=3, dtype="f32", seed=7), 2, (17, 20),
-     False),
+     None),
     ("nvfp4_w4a16_2ranks", W.Workload("ep_nvfp4", T=200, D=1024, L=512, I=512, E=16, k=4, dtype="bf16", seed=13,
-                                      experts="nvfp4"), 2, (90, 110), False),
+                                      experts="nvfp4"), 2, (90, 110), None),
     ("nvfp4_w4a4_4ranks", W.Workload("ep_w4a4", T=256, D=1024, L=512, I=512, E=16, k=4, dtype="bf16", seed=13,
-                                     experts="nvfp4", act="nvfp4"), 4, (70, 58, 64, 64), False),
+                                     experts="nvfp4", act="nvfp4"), 4, (70, 58, 64, 64), None),
 ]
 
 
@@ -172,17 +176,31 @@ def test_ep_entry_points_on_one_gpu_match_the_oracle_and_the_fused_forward(case)
     import latent_mixture_experts_moe_b200 as moe
     from latent_mixture_experts_moe_b200 import ep
     import parity_util as P
-    name, w, G, counts, sublayer = case
+    name, w, G, counts, extra = case
     dev = torch.device("cuda")
     inp = W.make_inputs(w, dev)
-    if sublayer:
+    modes, oracle_modes = {}, {}
+    if extra == "sublayer":
         inp.update(W.sublayer_inputs(w, dev))
+    elif extra == "pages":
+        # sigmoid router on logits x 1/sqrt(D/256) with a selection-only bias, centred
+        # pre-expert norm, one input-scaled post-expert gain shared by every expert
+        inp["gamma"] = inp["gamma"][0].contiguous()
+        pre = torch.empty(w.L, dtype=torch.bfloat16, device=dev)
+        inp["pre_norm_gain"] = W.fill(pre, w.seed, 11, 0.3)
+        inp["router_bias"] = (W.normal_f64(w.seed, 12, 0, w.E) * 0.05).to(torch.float32).to(dev)
+        scale = 1.0 / math.sqrt(w.D / 256)
+        modes = dict(router_mode=moe.ROUTER_SIGMOID, router_logit_scale=scale, routed_scaling=1.0,
+                     norm_mode=moe.NORM_INPUT_SCALED, gamma_shared=True, pre_norm_eps=1e-5)
+        oracle_modes = dict(router_mode="sigmoid", logit_scale=scale, routed_scaling=1.0, norm_mode="input_scaled",
+                            pre_norm_eps=1e-5)
     T = sum(counts)
     x = inp["x"][:T]
     starts = np.concatenate([[0], np.cumsum(counts)])
     xs = [x[starts[r]:starts[r + 1]] for r in range(G)]
     E_loc = w.E // G
-    modes = dict(act_format=moe.ACT_NVFP4) if w.act == "nvfp4" else {}
+    if w.act == "nvfp4":
+        modes = dict(modes, act_format=moe.ACT_NVFP4)
     shards = [ep.ExpertShard(_shard_weights(inp, r, E_loc), r, G, T_max=max(counts), k=w.k, eps=w.eps, **modes)
               for r in range(G)]
     outs = ep.ep_forward_one_device(shards, xs)
@@ -194,15 +212,15 @@ def test_ep_entry_points_on_one_gpu_match_the_oracle_and_the_fused_forward(case)
     got = torch.cat(outs)
     assert got.shape == (T, w.D)
     # the fused single-GPU forward of the same tokens: the same kernels over other row counts
-    fused = P.Run(w, inp, T=T)
+    fused = P.Run(w, inp, T=T, **{k: v for k, v in modes.items() if k != "act_format"})
     d = (got.float() - fused.out.float()).abs()
     assert P.rel_l2(got.double().cpu().numpy(), fused.out.double().cpu().numpy()) < 2e-3
     # the oracle, with the routing rule of the parity tests (W4A4: the fused run's activation
     # codes are the candidate decisions at rounding boundaries)
     rows = np.arange(T)
-    ref = P.oracle_block(w, inp, rows, run=fused)
+    ref = P.oracle_block(w, inp, rows, run=fused, **oracle_modes)
     alt = P.check_routing(ref, fused.idx.cpu().numpy(), fused.g.cpu().numpy(), w.k)
-    want = P.oracle_on_gpu_alternatives(w, inp, rows, ref, fused.idx.cpu().numpy(), alt, run=fused)
+    want = P.oracle_on_gpu_alternatives(w, inp, rows, ref, fused.idx.cpu().numpy(), alt, run=fused, **oracle_modes)
     P.assert_close(got.double().cpu().numpy(), want, f"EP {name}", rel=2e-2 if w.experts == "nvfp4" else P.REL_L2)
     print(f"{name}: max |EP - fused| = {float(d.max()):.3e}, equal elements {float((d == 0).float().mean()):.4f}")
 
