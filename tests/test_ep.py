@@ -246,3 +246,39 @@ def test_ep_experts_records_an_out_of_range_local_expert_and_zeroes_its_row():
     assert moe.STATUS[code] == "MUSE_ERR_DEVICE"
     assert torch.count_nonzero(y[2]) == 0 and torch.count_nonzero(ss[2]) == 0
     assert torch.count_nonzero(y[0]) > 0 and torch.count_nonzero(y[4]) > 0
+
+
+# --------------------------------------------------------------------- host-only checks
+def _tiny_weights(E_loc):
+    w = W.WORKLOADS["tiny"]
+    inp = W.make_inputs(w, "cpu", names=["W_router", "W_pool", "W_gate", "W_up", "W_down", "gamma", "W_unpool"])
+    for n in ("W_gate", "W_up", "W_down"):
+        inp[n] = inp[n][:E_loc].contiguous()
+    return w, inp
+
+
+def test_expert_shard_rejects_a_split_that_does_not_divide_or_match():
+    from latent_mixture_experts_moe_b200 import ep
+    w, inp = _tiny_weights(4)
+    with pytest.raises(ValueError, match="do not split"):
+        ep.ExpertShard(inp, 0, 3, T_max=16, k=w.k)          # 8 experts over 3 ranks
+    with pytest.raises(ValueError, match="this rank owns"):
+        ep.ExpertShard(inp, 0, 4, T_max=16, k=w.k)          # holds 4, owns 2
+
+
+def test_expert_shard_sizes_its_buffers_for_the_worst_case_receive():
+    from latent_mixture_experts_moe_b200 import ep
+    import latent_mixture_experts_moe_b200 as moe
+    w, inp = _tiny_weights(4)
+    s = ep.ExpertShard(inp, 1, 2, T_max=16, k=w.k)
+    assert s.rows_max == 2 * 16 * min(w.k, 4)
+    assert s.send_z.shape == (16 * w.k, w.L) and s.send_expert.shape == (16 * w.k,)
+    cfg = s.config(16)
+    assert s.ws_home.numel() == moe.ep_workspace_layout(cfg, 2, moe.EP_HOME)["total"]
+    assert s.ws_experts.numel() == moe.ep_workspace_layout(cfg, 2, moe.EP_EXPERTS, s.rows_max)["total"]
+    assert int(s.ws_home.abs().sum()) == 0 and int(s.ws_experts.abs().sum()) == 0  # start zeroed
+    assert s.gamma_local.shape == (4, w.L)
+    assert torch.equal(s.gamma_local, inp["gamma"][4:8])   # rank 1's experts 4..7
+    # a rank with no tokens sends nothing and never calls the library
+    z, e, counts = s.dispatch(torch.empty((0, w.D)))
+    assert z.shape[0] == 0 and e.shape[0] == 0 and counts == [0, 0]
