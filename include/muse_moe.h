@@ -357,12 +357,14 @@ MUSE_API muse_status muse_ep_combine(const muse_moe_config* cfg, int32_t ep_size
 /* Static string for a status code. */
 MUSE_API const char* muse_status_string(muse_status s);
 
-/* Number of kernel launches one forward call makes for cfg: 11, plus one each for the
- * pre-expert norm, the pre-FFN norm, the post-FFN norm / residual gate (one kernel
- * finishes both) and two for W4A4. In launch order: [ffn pre norm], router, top-k,
- * histogram, tiles, assign rows, pooler, [pre-expert norm], [W4A4: quantise z], gather (W4A4:
- * of the quantised bytes), gate/up, [W4A4: quantise h], down, norm + combine, unpooler,
- * [post norm / gate]. stage_events must hold this many + 1 events. */
+/* Number of stages one forward call runs for cfg -- the positions of stage_events: 11, plus
+ * one each for the pre-expert norm, the pre-FFN norm, the post-FFN norm / residual gate (one
+ * kernel finishes both) and two for W4A4. In order: [ffn pre norm], router, top-k, histogram,
+ * tiles, assign rows, pooler, [pre-expert norm], [W4A4: quantise z], gather (W4A4: of the
+ * quantised bytes), gate/up, [W4A4: quantise h], down, norm + combine, unpooler, [post norm /
+ * gate]. Each stage is one kernel, except that a dense GEMM (router, pooler, unpooler) whose
+ * tiles would fill less than half the SMs splits K and adds a partial-sum kernel inside its
+ * stage (decode-sized token counts). stage_events must hold this many + 1 events. */
 MUSE_API int32_t muse_latent_moe_launch_count(const muse_moe_config* cfg);
 
 #ifdef __cplusplus
