@@ -50,8 +50,12 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
-        d = json.load(open(p))
-        return {k: float(d[k]) for k in PEAKS_FALLBACK}, "measured"
+        try:
+            d = json.load(open(p))
+            if all(k in d for k in PEAKS_FALLBACK):
+                return {k: float(d[k]) for k in PEAKS_FALLBACK}, "measured"
+        except (ValueError, TypeError):
+            pass
     return dict(PEAKS_FALLBACK), "fallback"
 
 
