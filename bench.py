@@ -157,6 +157,39 @@ def step_work(w: W.Workload, n_touched: int):
     return flops, byts, fp4_flops
 
 
+def at_full_clock(clk) -> bool:
+    """True when the timed region ran at the GPU's maximum SM clock (median of the samples
+    taken during it within 3%, no power-cap reason): the burst GEMM peak, measured at that
+    clock, is then the tensor roofline; otherwise the sustained (power-capped) peak is."""
+    if not clk or not clk.get("sm_mhz") or not clk.get("sm_max_mhz"):
+        return False
+    return clk["sm_mhz"] >= 0.97 * clk["sm_max_mhz"]
+
+
+def roofline(w: W.Workload, kernel: str, fl: float, by: float, t: float, peaks, tensor_peak: float, burst: bool):
+    """Roofline of one kernel: algorithmic FLOPs fl and bytes by over its time t (s), against
+    the measured tensor peak (W4A4 expert GEMMs run on the FP4 path: the bf16 peak times the
+    nominal dense FP4 / BF16 ratio, 9 / 2.25 PFLOP/s) or the measured copy bandwidth,
+    whichever bounds it."""
+    fp4_gemm = w.act == "nvfp4" and kernel in ("gate_up_swiglu", "down_sumsq")
+    ratio = 4.0 if fp4_gemm else 1.0
+    t_tensor = fl / (ratio * tensor_peak * 1e12)
+    t_hbm = by / (peaks["hbm_gbs"] * 1e9)
+    if t_tensor >= t_hbm:
+        roof = {"bound": "tensor", "achieved": fl / t / 1e12, "peak": ratio * tensor_peak, "unit": "TFLOP/s"}
+        kind = ("burst, timed region at max SM clock" if burst else "sustained, timed region below max clock")
+        roof["peak_source"] = f"measured bf16 GEMM ({kind})" + (" x 4 (FP4 / BF16 nominal)" if fp4_gemm else "")
+    else:
+        roof = {"bound": "hbm", "achieved": by / t / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "peak_source": "measured copy bandwidth"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["kernel"] = kernel
+    roof["algorithmic_flops"] = fl
+    roof["algorithmic_bytes"] = by
+    roof["traffic"] = measured_traffic(kernel, w)
+    return roof
+
+
 # ------------------------------------------------------------------------------ our arm
 def rank_tokens(w: W.Workload, rank: int, dev) -> torch.Tensor:
     """Rank r's batch: tokens [rT, (r+1)T) of the workload's one seeded token stream, so N
@@ -211,7 +244,10 @@ def time_graph(w: W.Workload, model, inp, out, idx, steps: int, warmup: int, wor
 
 
 def run_ours(w: W.Workload, inp, steps: int, warmup: int, rank: int, world: int, peaks, peak_kind,
-             sample_clocks: bool, e2e_steps: int, graph_steps: int = 0):
+             sample_clocks: bool, e2e_steps: int, graph_steps: int = 0, flush_bytes: int = 0):
+    """Times `steps` forwards of workload w. flush_bytes > 0: between steps a buffer of that
+    many bytes (larger than L2) is overwritten, outside each step's own events, and the step
+    time is the sum of the steps' own durations (first to last library event)."""
     import latent_mixture_experts_moe_b200 as moe
     dev = inp["x"].device
     weights = {k: v for k, v in inp.items() if k != "x"}
@@ -239,10 +275,13 @@ def run_ours(w: W.Workload, inp, steps: int, warmup: int, rank: int, world: int,
         time.sleep(0.3)
     barrier(world)
     torch.cuda.synchronize()
+    flush = torch.empty(flush_bytes // 4, dtype=torch.int32, device=dev) if flush_bytes else None
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     wall0 = time.time()
     t_start.record(stream)
     for s in range(steps):
+        if flush is not None:
+            flush.fill_(s)
         model(inp["x"], out=out, topk_idx=idx, stage_events=handles[s])
     t_end.record(stream)
     torch.cuda.synchronize()
@@ -252,6 +291,8 @@ def run_ours(w: W.Workload, inp, steps: int, warmup: int, rank: int, world: int,
         time.sleep(0.2)
         clocks.stop()
     ms = t_start.elapsed_time(t_end)
+    if flush is not None:
+        ms = sum(ev[s][0].elapsed_time(ev[s][nst]) for s in range(steps))
     ms_max = all_max(ms, world, dev)
     code, detail = moe.last_device_status(model.config(w.T, model.workspace))
     if code != 0:
@@ -265,30 +306,15 @@ def run_ours(w: W.Workload, inp, steps: int, warmup: int, rank: int, world: int,
     dname = stage_names[dom]
     fl, by = work[dname]
     t_dom = stage_ms[dom] * 1e-3
-    # W4A4 expert GEMMs run on the FP4 tensor path: its peak is the measured bf16 peak times
-    # the nominal dense FP4 / BF16 ratio (9 / 2.25 PFLOP/s)
-    fp4_gemm = w.act == "nvfp4" and dname in ("gate_up_swiglu", "down_sumsq")
-    ratio = 4.0 if fp4_gemm else 1.0
-    t_tensor = fl / (ratio * peaks["bf16_tflops_sustained"] * 1e12)
-    t_hbm = by / (peaks["hbm_gbs"] * 1e9)
-    if t_tensor >= t_hbm:
-        roof = {"bound": "tensor", "achieved": fl / t_dom / 1e12, "peak": ratio * peaks["bf16_tflops_sustained"],
-                "unit": "TFLOP/s"}
-        roof["frac_of_burst_peak"] = fl / t_dom / 1e12 / (ratio * peaks["bf16_tflops"])
-    else:
-        roof = {"bound": "hbm", "achieved": by / t_dom / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
-    # against the datasheet figures too: 8 TB/s HBM3e, 2.25 PFLOP/s dense bf16 (x 4 for FP4)
-    roof["frac_of_spec"] = roof["achieved"] / (8000.0 if roof["bound"] == "hbm" else 2250.0 * ratio)
-    roof["kernel"] = dname
-    roof["peak_source"] = f"{peak_kind} ({'sustained' if roof['bound'] == 'tensor' else 'copy'})" + \
-        (" x 4 (nominal FP4 / BF16 dense ratio)" if fp4_gemm and roof["bound"] == "tensor" else "")
-    roof["algorithmic_flops"] = fl
-    roof["algorithmic_bytes"] = by
-    roof["traffic"] = measured_traffic(dname, w)
+    clk = clocks.summary(wall0, wall1) if clocks else None
+    burst = at_full_clock(clk)
+    tensor_peak = peaks["bf16_tflops"] if burst else peaks["bf16_tflops_sustained"]
+    roof = roofline(w, dname, fl, by, t_dom, peaks, tensor_peak, burst)
+    if peak_kind != "measured":
+        roof["peak_source"] += " (recipe fallback figures)"
     sf, sb, sf4 = step_work(w, n_touched)
     t_step = ms_max / steps * 1e-3
-    bf16_peak = peaks["bf16_tflops_sustained"] * 1e12
+    bf16_peak = tensor_peak * 1e12
     step_roof = max((sf - sf4) / bf16_peak + sf4 / (4.0 * bf16_peak), sb / (peaks["hbm_gbs"] * 1e9))
     res = {
         "value": job_tokens_per_s(world, w.T, steps, ms_max),
@@ -301,8 +327,8 @@ def run_ours(w: W.Workload, inp, steps: int, warmup: int, rank: int, world: int,
         "wall_s": wall1 - wall0,
         "gpu_launches": steps * moe.launch_count(model.config(w.T)),
     }
-    if clocks:
-        res["clocks"] = clocks.summary(wall0, wall1)
+    if clk:
+        res["clocks"] = clk
     if e2e_steps > 0:
         res["e2e"] = run_e2e(w, model, inp, e2e_steps, world, dev)
     if graph_steps > 0:
@@ -372,38 +398,71 @@ def kernel_source_sha():
 
 
 # ------------------------------------------------------------------------------ oracle arm
-def oracle_sample(w: W.Workload, n_tokens: int, dev, widen: bool):
-    """Host copies of what the oracle needs for tokens [0, n) of the workload: those x
-    rows, the shared weights and the experts their routing touches (generated on `dev`
-    with the shared seeded generator). widen=True converts them to float64 up front."""
-    import oracle
-    xr = torch.empty((n_tokens, w.D), dtype=W.TORCH_DTYPE[w.dtype], device=dev)
-    W.fill(xr, w.seed, W.TID["x"], 1.0)
-    shared = {n: W.make_tensor(w, n, dev).cpu() for n in ("W_router", "W_pool", "gamma", "W_unpool")}
-    x = xr.cpu()
-    bias = W.zipf_router_bias(w) if w.routing == "zipf" else None
-    logits = oracle.router_logits(oracle.as_f64(x), oracle.as_f64(shared["W_router"]))
-    idx, _, _ = oracle.route(logits, w.k, None if bias is None else oracle.as_f64(bias))
-    experts = {}
-    for e in np.unique(idx):
-        experts[int(e)] = tuple(W.expert_slab(w, n, int(e), dev).cpu() for n in ("W_gate", "W_up", "W_down"))
-    if widen:
-        x = oracle.as_f64(x)
-        shared = {n: oracle.as_f64(v) for n, v in shared.items()}
-        experts = {e: tuple(oracle.as_f64(m) for m in v) for e, v in experts.items()}
-        bias = None if bias is None else oracle.as_f64(bias)
-    return x, shared, bias, experts
+CPU_TOKENS = 1024
 
 
-def time_oracle(w, x, shared, bias, experts):
-    """Wall time of one oracle forward (as_f64 is a no-op on pre-widened arrays)."""
-    import oracle
-    f = oracle.as_f64
-    t0 = time.perf_counter()
-    oracle.latent_moe_forward(f(x), f(shared["W_router"]), f(shared["W_pool"]), lambda e: experts[e],
-                              f(shared["gamma"]), f(shared["W_unpool"]), w.k, w.eps,
-                              router_bias=None if bias is None else f(bias))
-    return time.perf_counter() - t0
+class OracleSample:
+    """What the FP64 oracle needs for tokens [0, n) of a workload, generated with the shared
+    seeded generator (on the GPU when there is one: the same bytes either way): those x
+    rows and the shared weights widened to float64, the routing bias, and the expert
+    weights of the experts that routing touches, widened to float64 one expert at a time
+    when the oracle asks for them (widen time recorded, so that the timed figure is the
+    oracle's arithmetic and not the conversion of 2-byte weights to 8-byte ones)."""
+
+    def __init__(self, w: W.Workload, n_tokens: int, dev):
+        import oracle
+        self.w, self.n, self.dev = w, n_tokens, dev
+        xr = torch.empty((n_tokens, w.D), dtype=W.TORCH_DTYPE[w.dtype], device=dev)
+        self.x = oracle.as_f64(W.fill(xr, w.seed, W.TID["x"], 1.0))
+        self.shared = {n: oracle.as_f64(W.make_tensor(w, n, dev)) for n in ("W_router", "W_pool", "gamma", "W_unpool")}
+        bias = W.zipf_router_bias(w) if w.routing == "zipf" else None
+        self.bias = None if bias is None else oracle.as_f64(bias)
+        logits = oracle.router_logits(self.x, self.shared["W_router"])
+        idx, _, _ = oracle.route(logits, w.k, self.bias)
+        self.experts_touched = len(np.unique(idx))
+        self.widen_s = 0.0
+        self.cache = {}
+
+    def expert(self, e: int):
+        if e in self.cache:
+            return self.cache[e]
+        t0 = time.perf_counter()
+        mats = tuple(W.expert_slab(self.w, n, e, self.dev).to(torch.float64).cpu().numpy()
+                     for n in ("W_gate", "W_up", "W_down"))
+        self.widen_s += time.perf_counter() - t0
+        return mats
+
+    def keep_widened(self):
+        """Hold every touched expert's float64 weights (for repeated runs), if they fit in
+        70% of the host's available memory (the full layer: 103 GB)."""
+        need = self.experts_touched * 3 * self.w.L * self.w.I * 8
+        try:
+            import psutil
+            avail = psutil.virtual_memory().available
+        except ImportError:
+            avail = 0
+        if need > 0.7 * avail:
+            return False
+        import oracle
+        logits = oracle.router_logits(self.x, self.shared["W_router"])
+        idx, _, _ = oracle.route(logits, self.w.k, self.bias)
+        for e in np.unique(idx):
+            self.cache[int(e)] = self.expert(int(e))
+        return True
+
+    def run(self) -> float:
+        """One oracle forward over the sample; returns its time without the widening."""
+        import oracle
+        w0 = self.widen_s
+        t0 = time.perf_counter()
+        oracle.latent_moe_forward(self.x, self.shared["W_router"], self.shared["W_pool"], self.expert,
+                                  self.shared["gamma"], self.shared["W_unpool"], self.w.k, self.w.eps,
+                                  router_bias=self.bias)
+        return time.perf_counter() - t0 - (self.widen_s - w0)
+
+    def describe(self) -> str:
+        return (f"tokens 0-{self.n - 1} of the {self.w.name} batch ({self.experts_touched} experts touched), "
+                f"FP64 numpy oracle, expert-major; weights widened to f64 outside the timed region")
 
 
 def host_cores():
@@ -411,6 +470,18 @@ def host_cores():
         return len(os.sched_getaffinity(0))
     except AttributeError:
         return os.cpu_count()
+
+
+def blas_threads() -> int:
+    """Threads the host BLAS runs the oracle's matrix products on."""
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except ImportError:
+        pass
+    return host_cores()
 
 
 def cpu_model() -> str:
@@ -425,40 +496,30 @@ def cpu_model() -> str:
 
 
 def cpu_baseline(w: W.Workload, dev, n_tokens: int):
-    x, shared, bias, experts = oracle_sample(w, n_tokens, dev, widen=False)
-    dt = time_oracle(w, x, shared, bias, experts)
+    sample = OracleSample(w, n_tokens, dev)
+    dt = sample.run()
     flops_per_token = 2 * (w.E * w.D + w.L * w.D + w.k * 3 * w.L * w.I + w.D * w.L)
-    # the same oracle on one core (BLAS limited to one thread), one token, widening included
-    one_core = None
-    try:
-        from threadpoolctl import threadpool_limits
-        x1, shared1, bias1, experts1 = oracle_sample(w, 1, dev, widen=False)
-        with threadpool_limits(limits=1):
-            one_core = 1.0 / time_oracle(w, x1, shared1, bias1, experts1)
-    except ImportError:
-        pass
-    return {"value": n_tokens / dt, "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
-            "gflops_fp64": n_tokens * flops_per_token / dt / 1e9, "cpu_model": cpu_model(),
-            "one_core_tokens_per_s": one_core,
-            "sample": f"first {n_tokens} tokens of the {w.name} workload (T={w.T}) through the FP64 numpy "
-                      f"oracle, widening bf16 weights to f64 included; {len(experts)} distinct experts; {dt:.1f} s"}
+    return {"value": n_tokens / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": sample.describe() + f"; {dt:.1f} s, {n_tokens * flops_per_token / dt / 1e9:.0f} GFLOP/s FP64"}
 
 
 def run_reference(w: W.Workload, args, dev):
-    """The FP64 oracle as the reference arm: every step runs the workload's first token
-    through the whole block, on weights widened to float64 before timing."""
-    x, shared, bias, experts = oracle_sample(w, 1, dev, widen=True)
-    times = [time_oracle(w, x, shared, bias, experts) for _ in range(args.warmup + args.steps)][args.warmup:]
+    """The FP64 oracle as the reference arm, on the same basis as cpu_baseline: every step
+    runs the block on tokens 0..CPU_TOKENS-1 of the workload, expert-major, with the expert
+    weights widened to float64 outside the timed region (held across steps when they fit in
+    host memory, else widened again each step, untimed)."""
+    sample = OracleSample(w, args.cpu_tokens, dev)
+    sample.keep_widened()
+    times = [sample.run() for _ in range(args.warmup + args.steps)][args.warmup:]
     total = sum(times)
-    value = args.steps / total
+    value = args.steps * sample.n / total
     return {
         "metric": metric_name(), "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_dict(w), "impl": "reference",
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
-                         "sample": f"token 0 of the {w.name} workload per step, FP64 numpy oracle, "
-                                   f"weights pre-widened to f64"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": sample.describe() + " (each step)"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -469,10 +530,10 @@ def metric_name():
 
 
 def config_dict(w: W.Workload):
+    """The workload named by what it is; the same dict in both arms."""
     return {"workload": f"{w.name}: latent-MoE layer T={w.T} D={w.D} L={w.L} I={w.I} E={w.E} top-{w.k} "
                         f"{w.dtype} {w.routing} routing",
-            "T": w.T, "D": w.D, "L": w.L, "I": w.I, "E": w.E, "top_k": w.k, "routing": w.routing,
-            "l2": "inputs larger than L2: each step streams the touched experts' weights (up to 25.8 GB)"}
+            "l2": "inputs larger than L2 (each step streams the touched experts' weights)"}
 
 
 _DIST = {"on": False}
@@ -491,6 +552,23 @@ def all_max(v: float, world: int, dev) -> float:
     return float(t.item())
 
 
+def sig(v, n=4):
+    """v rounded to n significant digits (keeps the JSON line short)."""
+    if v is None or v == 0 or not math.isfinite(v):
+        return v
+    return round(v, n - 1 - int(math.floor(math.log10(abs(v)))))
+
+
+def side_entry(r):
+    """One side workload in the JSON line: tokens/s, ms per step, the dominant kernel's
+    roofline fraction and bound, and the whole step's fraction of its roofline."""
+    e = {"v": sig(r["value"]), "ms": sig(r["ms_per_step"]), "frac": sig(r["roofline"]["frac"], 3),
+         "bound": r["roofline"]["bound"], "step_frac": sig(r["step"]["frac_of_step_roofline"], 3)}
+    if "graph" in r:
+        e["graph_ms"] = sig(r["graph"]["ms_per_step"])
+    return e
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -498,10 +576,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="prefill", choices=list(W.WORKLOADS))
-    ap.add_argument("--no-side", action="store_true", help="skip the decode / skewed side workloads")
+    ap.add_argument("--no-side", action="store_true", help="skip the side workloads")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle cpu_baseline")
     ap.add_argument("--no-nvfp4", action="store_true", help="skip the NVFP4-expert side workloads")
-    ap.add_argument("--cpu-tokens", type=int, default=16)
+    ap.add_argument("--cpu-tokens", type=int, default=CPU_TOKENS)
+    ap.add_argument("--detail", default=None, help="also write every measurement (per-kernel times, "
+                                                   "rooflines of every workload) to this JSON file")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -523,62 +603,75 @@ def main():
     try:
         peaks, peak_kind = load_peaks()
         inp = make_rank_inputs(w, rank, dev)
-        main_res = run_ours(w, inp, args.steps, args.warmup, rank, world, peaks, peak_kind, True,
-                            e2e_steps=min(args.steps, 20),
-                            graph_steps=args.steps if w.name.endswith("decode") else 0)
+
+        def run(wl, inputs, steps, **kw):
+            return run_ours(wl, inputs, steps, args.warmup, rank, world, peaks, peak_kind, True, **kw)
+        main_res = run(w, inp, args.steps, e2e_steps=min(args.steps, 20),
+                       graph_steps=args.steps if w.name.endswith("decode") else 0)
         side = {}
         if not args.no_side and w.name == "prefill":
             wd = W.WORKLOADS["decode"]
             inp_d = dict(inp, x=rank_tokens(wd, rank, dev))
-            side["decode"] = run_ours(wd, inp_d, max(args.steps, 50), args.warmup, rank, world, peaks, peak_kind,
-                                      False, e2e_steps=0, graph_steps=max(args.steps, 50))
+            side["decode"] = run(wd, inp_d, max(args.steps, 50), e2e_steps=0, graph_steps=max(args.steps, 50))
             wz = W.WORKLOADS["prefill_zipf"]
-            inp_z = dict(inp, router_bias=W.zipf_router_bias(wz).to(dev))
-            side["prefill_zipf"] = run_ours(wz, inp_z, args.steps, args.warmup, rank, world, peaks, peak_kind,
-                                            False, e2e_steps=0)
+            side["prefill_zipf"] = run(wz, dict(inp, router_bias=W.zipf_router_bias(wz).to(dev)), args.steps,
+                                       e2e_steps=0)
             # the whole feed-forward sublayer: pre-norm, the block, post-norm, residual gate
-            inp_s = dict(inp, **W.sublayer_inputs(w, dev))
-            side["prefill_sublayer"] = run_ours(w, inp_s, args.steps, args.warmup, rank, world, peaks, peak_kind,
-                                                False, e2e_steps=0)
+            side["prefill_sublayer"] = run(w, dict(inp, **W.sublayer_inputs(w, dev)), args.steps, e2e_steps=0)
             if not args.no_nvfp4:
                 # NVFP4 experts (quantised from the same bf16 weights): T=4096 and a T=64 decode
                 wq = W.WORKLOADS["nvfp4"]
                 q = W.make_inputs(wq, dev, names=["W_gate", "W_up", "W_down"])
                 inp_q = dict({k: v for k, v in inp.items() if k not in ("W_gate", "W_up", "W_down")}, **q)
                 inp_q["x"] = rank_tokens(wq, rank, dev)
-                side["nvfp4"] = run_ours(wq, inp_q, args.steps, args.warmup, rank, world, peaks, peak_kind,
-                                         False, e2e_steps=0)
+                side["nvfp4"] = run(wq, inp_q, args.steps, e2e_steps=0)
                 wqd = W.WORKLOADS["nvfp4_decode"]
                 inp_qd = dict(inp_q, x=rank_tokens(wqd, rank, dev))
-                side["nvfp4_decode"] = run_ours(wqd, inp_qd, max(args.steps, 50), args.warmup, rank, world, peaks,
-                                                peak_kind, False, e2e_steps=0)
+                side["nvfp4_decode"] = run(wqd, inp_qd, max(args.steps, 50), e2e_steps=0,
+                                           graph_steps=max(args.steps, 50))
                 # the same weights with NVFP4 activations (W4A4, tcgen05 kind::mxf4nvf4)
-                side["nvfp4_w4a4"] = run_ours(W.WORKLOADS["nvfp4_w4a4"], inp_q, args.steps, args.warmup, rank, world,
-                                              peaks, peak_kind, False, e2e_steps=0)
-                side["nvfp4_w4a4_decode"] = run_ours(W.WORKLOADS["nvfp4_w4a4_decode"], inp_qd, max(args.steps, 50),
-                                                     args.warmup, rank, world, peaks, peak_kind, False, e2e_steps=0,
-                                                     graph_steps=max(args.steps, 50))
+                side["nvfp4_w4a4"] = run(W.WORKLOADS["nvfp4_w4a4"], inp_q, args.steps, e2e_steps=0)
+                side["nvfp4_w4a4_decode"] = run(W.WORKLOADS["nvfp4_w4a4_decode"], inp_qd, max(args.steps, 50),
+                                                e2e_steps=0, graph_steps=max(args.steps, 50))
+                del q, inp_q, inp_qd
+            # the mid layer (0.41 GB of weights): a 256 MiB buffer is overwritten between steps
+            # so that no step finds the previous one's weights in L2
+            del inp_d
+            wm = W.WORKLOADS["mid"]
+            inp_m = make_rank_inputs(wm, rank, dev)
+            side["mid"] = run(wm, inp_m, max(args.steps, 50), e2e_steps=0, flush_bytes=256 << 20)
         if rank == 0:
+            roof = {k: main_res["roofline"][k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic",
+                                                          "kernel", "peak_source")}
+            for k in ("achieved", "peak", "frac"):
+                roof[k] = sig(roof[k])
+            clk = main_res.get("clocks") or {}
             line = {
-                "metric": metric_name(), "value": main_res["value"], "unit": "tokens/s", "n_gpus": world,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": main_res["ms_per_step"],
+                "metric": metric_name(), "value": sig(main_res["value"], 6), "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": sig(main_res["ms_per_step"], 5),
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
-                "data": "synthetic (seeded counter-based N(0,1) inputs, N(0,1/fan_in) weights)",
-                "config": dict(config_dict(w), parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
-                "roofline": main_res["roofline"], "step_roofline": main_res["step"],
-                "stage_ms": main_res["stage_ms"], "step_ms": main_res["step_ms"],
+                "data": "synthetic (seeded N(0,1) x, N(0,1/fan_in) weights)",
+                "config": config_dict(w), "roofline": roof,
+                "step_roofline_frac": sig(main_res["step"]["frac_of_step_roofline"], 3),
                 "gpu_launches": main_res["gpu_launches"],
-                "clocks": main_res.get("clocks"), "e2e": main_res.get("e2e"),
+                "clocks": {"sm_mhz": clk.get("sm_mhz"), "sm_max_mhz": clk.get("sm_max_mhz"),
+                           "reasons": clk.get("reasons", [])},
             }
+            e2e = main_res.get("e2e")
+            if e2e:
+                line["e2e"] = {"value": sig(e2e["value"], 6), "unit": e2e["unit"],
+                               "h2d_bytes_per_step": e2e["h2d_bytes_per_step"],
+                               "d2h_bytes_per_step": e2e["d2h_bytes_per_step"]}
             if "graph" in main_res:
-                line["graph_replay"] = main_res["graph"]
-            for name, r in side.items():
-                line[name] = {"value": r["value"], "unit": "tokens/s", "ms_per_step": r["ms_per_step"],
-                              "roofline": r["roofline"], "step_roofline": r["step"], "stage_ms": r["stage_ms"]}
-                if "graph" in r:
-                    line[name]["graph_replay"] = r["graph"]
+                line["graph_replay_ms"] = sig(main_res["graph"]["ms_per_step"])
+            if side:
+                line["side"] = {name: side_entry(r) for name, r in side.items()}
             if world == 1 and not args.no_cpu:
                 line["cpu_baseline"] = cpu_baseline(w, dev, args.cpu_tokens)
+            if args.detail:
+                detail = {"line": line, "main": main_res, "side": side, "cpu_model": cpu_model()}
+                with open(args.detail, "w") as f:
+                    json.dump(detail, f, indent=1, default=float)
             print(json.dumps(line), flush=True)
     finally:
         if world > 1:

@@ -232,7 +232,9 @@ MUSE_API muse_status muse_latent_moe_forward_host_batches(const muse_moe_config*
 
 /* Synchronises `stream` and returns the status word the last forward on this
  * workspace recorded on the device (MUSE_OK, MUSE_ERR_TIMEOUT or MUSE_ERR_DEVICE);
- * *detail (may be NULL) receives the kernel-specific detail code. */
+ * *detail (may be NULL) receives the kernel-specific detail code. With cfg->workspace ==
+ * NULL it reads the word of the built-in scratch array that
+ * muse_latent_moe_forward_static_scratch uses on the current device. */
 MUSE_API muse_status muse_latent_moe_last_device_status(const muse_moe_config* cfg, void* stream,
                                                uint32_t* detail);
 
@@ -247,14 +249,17 @@ MUSE_API muse_status muse_latent_moe_last_device_status(const muse_moe_config* c
  *   - Sizes whose workspace (muse_latent_moe_workspace_size) exceeds
  *     MUSE_STATIC_SCRATCH_BYTES are rejected with MUSE_ERR_WORKSPACE before any launch.
  *   - It allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
- *   - The first call on each device looks up the array's device address with that
- *     device current; make that first call before any stream capture.
+ *   - Each call made outside stream capture looks up the array's device address on the
+ *     current device (so an address from before a cudaDeviceReset, which frees the array,
+ *     is never reused); a call made during capture uses the address of the last uncaptured
+ *     call on that device, so make the first call on each device before any capture.
  *   - All calls share the one array and it keeps the last call's contents (each call
  *     clears what must start at zero). Calls whose work overlaps on the GPU -- on two
  *     streams, or on one device from two threads without ordering -- race on it: order
  *     them on one stream or serialise them.
- *   - The device-side status word lives in that shared array and is not readable
- *     through muse_latent_moe_last_device_status. */
+ *   - The device-side status word (bounded-wait timeouts, index checks) lives in that
+ *     shared array: muse_latent_moe_last_device_status with cfg->workspace == NULL reads
+ *     it (the last call's word on the current device). */
 #define MUSE_STATIC_SCRATCH_BYTES (16u << 20)
 MUSE_API muse_status muse_latent_moe_forward_static_scratch(const muse_moe_config* cfg, const void* x,
                                                             const void* W_router, const void* W_pool,

@@ -944,16 +944,23 @@ constexpr int kMaxDevices = 64;
 std::mutex g_static_scratch_mu;
 void* g_static_scratch_ptr[kMaxDevices] = {};
 
-// Device address of g_static_scratch on the current device, looked up once per device.
-muse_status static_scratch_address(void** ptr) {
+// Device address of g_static_scratch on the current device. It is looked up again on every
+// call made outside stream capture (a cheap lookup once the module is loaded), so that an
+// address cached before a cudaDeviceReset -- which unloads the module and frees the array --
+// is never used afterwards; during capture the address of the last uncaptured call on this
+// device is used, so the first call on a device must come before any capture.
+muse_status static_scratch_address(cudaStream_t st, void** ptr) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MUSE_ERR_CUDA;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) return MUSE_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_static_scratch_mu);
-  if (g_static_scratch_ptr[dev] == nullptr) {
+  if (cap == cudaStreamCaptureStatusNone) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return MUSE_ERR_CUDA;
     g_static_scratch_ptr[dev] = p;
   }
+  if (g_static_scratch_ptr[dev] == nullptr) return MUSE_ERR_CUDA;  // first call made under capture
   *ptr = g_static_scratch_ptr[dev];
   return MUSE_OK;
 }
@@ -1168,7 +1175,7 @@ muse_status muse_latent_moe_forward_static_scratch(const muse_moe_config* cfg, c
   if (s != MUSE_OK) return s;
   if (make_layout(*cfg).pub.total > MUSE_STATIC_SCRATCH_BYTES) return MUSE_ERR_WORKSPACE;
   void* scratch = nullptr;
-  const muse_status a = static_scratch_address(&scratch);
+  const muse_status a = static_scratch_address(static_cast<cudaStream_t>(stream), &scratch);
   if (a != MUSE_OK) return a;
   muse_moe_config c = *cfg;
   c.workspace = scratch;
@@ -1179,13 +1186,15 @@ muse_status muse_latent_moe_forward_static_scratch(const muse_moe_config* cfg, c
 muse_status muse_latent_moe_last_device_status(const muse_moe_config* cfg, void* stream, uint32_t* detail) {
   muse_status s = validate_sizes(cfg);
   if (s != MUSE_OK) return s;
-  if (cfg->workspace == nullptr) return MUSE_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // no workspace: the word of the built-in scratch array (muse_latent_moe_forward_static_scratch)
+  void* ws = cfg->workspace;
+  if (ws == nullptr && static_scratch_address(st, &ws) != MUSE_OK) return MUSE_ERR_CUDA;
   if (cudaStreamSynchronize(st) != cudaSuccess) return MUSE_ERR_CUDA;
   uint32_t word[2] = {0, 0};
   const Layout lay = make_layout(*cfg);
-  if (cudaMemcpy(word, static_cast<uint8_t*>(cfg->workspace) + lay.pub.status, sizeof(word),
-                 cudaMemcpyDeviceToHost) != cudaSuccess)
+  if (cudaMemcpy(word, static_cast<uint8_t*>(ws) + lay.pub.status, sizeof(word), cudaMemcpyDeviceToHost) !=
+      cudaSuccess)
     return MUSE_ERR_CUDA;
   if (detail != nullptr) *detail = word[1];
   return static_cast<muse_status>(word[0]);

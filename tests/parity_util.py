@@ -43,6 +43,27 @@ def assert_close(got: np.ndarray, ref: np.ndarray, what: str, rel=REL_L2, max_ab
     return r, ma / rms
 
 
+def assert_close_stored(got: np.ndarray, ref: np.ndarray, what: str, rel=REL_L2, max_abs_rms=MAX_ABS_RMS,
+                        stored_bits: int = 8):
+    """For an intermediate the CUDA path stores in a narrow type (bf16: 8 significant bits)
+    and the oracle never rounds: rel-L2 <= rel, and elementwise |got - ref| <= max_abs_rms *
+    rms(ref) + 2^-stored_bits * |ref| -- the block-output bound plus one unit in the last
+    place of the stored value itself (its own rounding, and the neighbour a value within
+    the computational error of a rounding boundary may round to). Large elements of an
+    intermediate (a latent row dominated by one expert's normalised output reaches |c| ~ 10,
+    where a bf16 unit is 2^-4) would otherwise fail a bound meant for the block output."""
+    got = np.asarray(got, dtype=np.float64)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
+    r = rel_l2(got, ref)
+    rms = math.sqrt(float(np.mean(ref * ref)))
+    excess = np.abs(got - ref) - (max_abs_rms * rms + np.ldexp(np.abs(ref), -stored_bits))
+    assert r <= rel, f"{what}: rel-L2 {r:.3e} > {rel}"
+    worst = int(np.argmax(excess))
+    assert excess.flat[worst] <= 0, (f"{what}: element {np.unravel_index(worst, ref.shape)} got "
+                                     f"{got.flat[worst]:.6g} ref {ref.flat[worst]:.6g} (rms {rms:.3e})")
+    return r, float(np.abs(got - ref).max()) / rms
+
+
 def ws_view(ws: torch.Tensor, off: int, dtype: torch.dtype, shape: Sequence[int]) -> torch.Tensor:
     n = int(np.prod(shape)) * torch.tensor([], dtype=dtype).element_size()
     return ws[off:off + n].view(dtype).view(*shape)
@@ -167,6 +188,78 @@ def oracle_on_gpu_alternatives(w, inp, rows, ref, gpu_idx, alt_tokens, run=None,
         r1 = oracle_block(w, inp, rows[t:t + 1], run=run, routing=(sel, g), **kw)
         out[t] = r1["out"][0]
     return out
+
+
+def forced_weights(logits: np.ndarray, idx: np.ndarray, router_mode: str = "softmax", logit_scale: float = 1.0,
+                   routed_scaling: float = 1.0, **_) -> np.ndarray:
+    """The oracle's routing weights for the experts idx[t, :] of every token (any valid
+    set and order): its own weights where idx is its own choice, the weights of the
+    alternative set where a near tie let the CUDA path pick another valid set."""
+    if router_mode == "sigmoid":
+        return oracle.sigmoid_weights(logits, idx, logit_scale, routed_scaling)
+    return oracle.softmax_weights(logits, idx)
+
+
+def check_every_token(w: W.Workload, inp: Dict[str, torch.Tensor], run: "Run", rel: float = REL_L2,
+                      **oracle_modes) -> Dict[str, float]:
+    """Whole-output parity of one forward at any size (the benchmark spec tolerances):
+
+    * routing: every token's set, order and weights against the oracle's router on all
+      tokens (check_routing: a differing set only at a near tie, and then one of the
+      oracle's valid alternatives);
+    * the oracle then runs the whole block on every token under the CUDA path's validated
+      routing (its sets and slot order, the oracle's weights for them), so that every
+      assignment row has a reference: out [T, D], the pooler's z, the expert outputs y and
+      their sums of squares on every one of the T*k rows, and the combined latent c;
+    * the permutation (counts, padded offsets, inv, row_token) bit for bit against its
+      integer definition on the CUDA path's (validated) expert indices.
+    The output is held to assert_close (the block's tolerance); the intermediates the CUDA
+    path stores in the activation dtype (z, y, c) to assert_close_stored, and the sums of
+    squares (float32 partials) to twice the relative tolerance.
+    Returns the measured errors and the near-tie count."""
+    T, k, L, E = run.T, w.k, w.L, w.E
+    rows = np.arange(T)
+    x = host(inp["x"][:T])
+    logits = oracle.router_logits(x, host(inp["W_router"]))
+    del x
+    bias = host(inp["router_bias"]) if "router_bias" in inp else None
+    ro = {n: oracle_modes[n] for n in ("router_mode", "logit_scale", "routed_scaling") if n in oracle_modes}
+    idx, g, keys = oracle.route(logits, k, bias, **ro)
+    gidx = run.idx.cpu().numpy()
+    alts = check_routing({"keys": keys, "idx": idx, "g": g}, gidx, run.g.cpu().numpy(), k)
+    routing = (gidx.astype(np.int64), forced_weights(logits, gidx, **ro))
+    del logits, keys
+    ref = oracle_block(w, inp, rows, run=run, routing=routing, **oracle_modes)
+    res = {"near_ties": len(alts)}
+    res["out"], _ = assert_close(host(run.out), ref.pop("out"), f"{w.name} out (all {T} tokens)", rel=rel)
+    act = run.act()
+    bits = 8 if act == torch.bfloat16 else 24
+    res["z"], _ = assert_close_stored(host(run.inter("z", act, (T, L))), ref.pop("z"), f"{w.name} z", rel=rel,
+                                      stored_bits=bits)
+    res["c"], _ = assert_close_stored(host(run.inter("c", act, (T, L))), ref.pop("c"), f"{w.name} c", rel=rel,
+                                      stored_bits=bits)
+    # the permutation, from the validated indices
+    counts, offsets, inv = expected_permutation(gidx, E)
+    R = run.layout["rows"]
+    assert np.array_equal(run.inter("expert_count", torch.int32, (E,)).cpu().numpy(), counts)
+    assert np.array_equal(run.inter("expert_offset", torch.int32, (E + 1,)).cpu().numpy(), offsets)
+    ginv = run.inter("inv", torch.int32, (T * k,)).cpu().numpy()
+    assert np.array_equal(ginv, inv)
+    rtok = run.inter("row_token", torch.int32, (R,)).cpu().numpy()
+    assert np.array_equal(rtok[inv], np.arange(T * k) // k)
+    pad = np.ones(R, dtype=bool)
+    pad[inv] = False
+    pad[offsets[-1]:] = False                      # rows past the last expert are never written
+    assert np.all(rtok[pad] == -1)
+    # every assignment row of y and of its sum of squares (padding rows excluded)
+    sel = torch.as_tensor(ginv.astype(np.int64), device=run.out.device)
+    y = host(run.inter("y", act, (R, L))[sel]).reshape(T, k, L)
+    res["y"], _ = assert_close_stored(y, ref.pop("y"), f"{w.name} y (all {T * k} rows)", rel=rel, stored_bits=bits)
+    del y
+    ss = run.inter("ss", torch.float32, (R, L // 32))[sel].double().sum(1).cpu().numpy().reshape(T, k)
+    res["ss"], _ = assert_close(ss, ref.pop("ss"), f"{w.name} sum of squares", rel=2 * rel)
+    res["act_adopted"] = ref.get("act_adopted", 0)
+    return res
 
 
 def expected_permutation(idx: np.ndarray, E: int):

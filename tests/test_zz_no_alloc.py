@@ -18,7 +18,6 @@ import torch
 
 import latent_mixture_experts_moe_b200 as moe
 import workloads as W
-from parity_util import assert_close, host
 
 
 def _weights(inp):
@@ -28,6 +27,10 @@ def _weights(inp):
 @pytest.mark.gpu
 @pytest.mark.parametrize("name", ["tiny", "mid"])
 def test_static_scratch_forward_matches_workspace_forward_on_two_calls(name):
+    """Same kernels, same sizes: the output equals the regular entry point's bit for bit,
+    on two calls in a row with different tokens; the status word of the built-in array
+    (read with a config that names no workspace) reports success; and a call after the
+    first allocates no device memory (free memory unchanged across it)."""
     w = W.WORKLOADS[name]
     inp = W.make_inputs(w, "cuda")
     x2 = torch.empty_like(inp["x"])
@@ -38,9 +41,16 @@ def test_static_scratch_forward_matches_workspace_forward_on_two_calls(name):
     for call, x in enumerate((inp["x"], x2)):
         ref = model(x)                                            # regular entry point
         out = torch.full_like(ref, float("nan"))
+        torch.cuda.synchronize()
+        free0 = torch.cuda.mem_get_info()[0]
         moe.forward_static_scratch(cfg, x, *_weights(inp), out)
         torch.cuda.synchronize()
-        assert_close(host(out), host(ref), f"{name}: static-scratch call {call}")
+        free1 = torch.cuda.mem_get_info()[0]
+        assert torch.equal(out, ref), f"{name}: static-scratch call {call} differs"
+        code, detail = moe.last_device_status(cfg)                # cfg.workspace is NULL
+        assert code == 0, (moe.STATUS.get(code), hex(detail))
+        if call > 0:                                              # kernels loaded by the first
+            assert free1 == free0, f"device memory changed by {free0 - free1} bytes"
 
 
 def test_static_scratch_rejects_sizes_beyond_the_array():
