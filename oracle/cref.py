@@ -21,6 +21,12 @@ CFLAGS = ["-O2", "-std=c99", "-ffp-contract=off", "-fno-fast-math", "-shared", "
 _lib: Optional[ctypes.CDLL] = None
 
 
+class RefNvfp4(ctypes.Structure):
+    """One NVFP4 expert tensor [E, out, in]: codes [E, out, in/2] (low nibble = even
+    element), E4M3 block scales [E, out, in/16], float32 matrix scales [E]."""
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("matrix_scale", ctypes.c_void_p)]
+
+
 class RefCfg(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int), ("D", ctypes.c_int), ("L", ctypes.c_int), ("I", ctypes.c_int),
                 ("E", ctypes.c_int), ("k", ctypes.c_int), ("eps", ctypes.c_double),
@@ -43,6 +49,12 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(LIB)
         L.ref_latent_moe_forward.argtypes = [ctypes.POINTER(RefCfg)] + [ctypes.c_void_p] * 11
         L.ref_latent_moe_forward.restype = ctypes.c_int
+        L.ref_latent_moe_forward_nvfp4.argtypes = [ctypes.POINTER(RefCfg)] + [ctypes.c_void_p] * 11
+        L.ref_latent_moe_forward_nvfp4.restype = ctypes.c_int
+        L.ref_e2m1_value.argtypes = [ctypes.c_uint]
+        L.ref_e2m1_value.restype = ctypes.c_double
+        L.ref_e4m3_value.argtypes = [ctypes.c_uint]
+        L.ref_e4m3_value.restype = ctypes.c_double
         _lib = L
     return _lib
 
@@ -53,21 +65,54 @@ def _f64(a) -> np.ndarray:
     return np.ascontiguousarray(a, dtype=np.float64)
 
 
+def e2m1_value(code: int) -> float:
+    return float(lib().ref_e2m1_value(int(code)))
+
+
+def e4m3_value(byte: int) -> float:
+    return float(lib().ref_e4m3_value(int(byte)))
+
+
+def _u8(a) -> np.ndarray:
+    if hasattr(a, "detach"):
+        a = a.detach().cpu().numpy()
+    return np.ascontiguousarray(a, dtype=np.uint8)
+
+
+def _f32(a) -> np.ndarray:
+    if hasattr(a, "detach"):
+        a = a.detach().cpu().float().numpy()
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
 def latent_moe_forward_c(x, W_router, W_pool, experts, gamma, W_unpool, k: int, eps: float,
                          router_bias=None, router_mode: str = "softmax", logit_scale: float = 1.0,
                          routed_scaling: float = 1.0, norm_mode: str = "centred", pre_norm_gain=None,
-                         pre_norm_eps: float = 1e-5) -> Dict[str, np.ndarray]:
+                         pre_norm_eps: float = 1e-5, nvfp4: bool = False) -> Dict[str, np.ndarray]:
     """The block on every row of x [T, D]; experts = (W_gate [E, I, L], W_up [E, I, L],
-    W_down [E, L, I]); gamma [E, L] or [L]. Returns out [T, D], idx [T, k], g [T, k]."""
+    W_down [E, L, I]), or with nvfp4=True three (codes, block scales, matrix scales) triples
+    that the C code decodes itself; gamma [E, L] or [L]. Returns out [T, D], idx [T, k],
+    g [T, k]."""
     x, Wr, Wp, Wu_ = _f64(x), _f64(W_router), _f64(W_pool), _f64(W_unpool)
-    Wg, Wup, Wd = (_f64(m) for m in experts)
     gam = _f64(gamma)
     T, D = x.shape
     E = Wr.shape[0]
     L = Wp.shape[0]
-    I = Wg.shape[1]
+    keep = []
+    if nvfp4:
+        mats = []
+        for codes, scales, ms in experts:
+            c8, s8, m32 = _u8(codes), _u8(scales), _f32(ms)
+            assert c8.shape[:2] == s8.shape[:2] and c8.shape[2] * 2 == s8.shape[2] * 16 and m32.shape == (E,)
+            keep += [c8, s8, m32]
+            mats.append(RefNvfp4(c8.ctypes.data, s8.ctypes.data, m32.ctypes.data))
+        I = experts[0][0].shape[1]
+        assert tuple(experts[0][0].shape) == (E, I, L // 2) and tuple(experts[2][0].shape) == (E, L, I // 2)
+    else:
+        Wg, Wup, Wd = (_f64(m) for m in experts)
+        I = Wg.shape[1]
+        assert Wg.shape == (E, I, L) and Wup.shape == (E, I, L) and Wd.shape == (E, L, I)
     assert Wr.shape == (E, D) and Wp.shape == (L, D) and Wu_.shape == (D, L)
-    assert Wg.shape == (E, I, L) and Wup.shape == (E, I, L) and Wd.shape == (E, L, I)
     assert gam.shape in ((E, L), (L,))
     bias = None if router_bias is None else _f64(router_bias)
     pre = None if pre_norm_gain is None else _f64(pre_norm_gain)
@@ -80,8 +125,12 @@ def latent_moe_forward_c(x, W_router, W_pool, experts, gamma, W_unpool, k: int, 
     idx = np.zeros((T, k), dtype=np.int32)
     g = np.zeros((T, k))
     p = lambda a: a.ctypes.data  # noqa: E731
-    rc = lib().ref_latent_moe_forward(ctypes.byref(c), p(x), p(Wr), p(Wp), p(Wg), p(Wup), p(Wd), p(gam), p(Wu_),
-                                      p(out), p(idx), p(g))
+    if nvfp4:
+        rc = lib().ref_latent_moe_forward_nvfp4(ctypes.byref(c), p(x), p(Wr), p(Wp), *[ctypes.addressof(m) for m in mats],
+                                                p(gam), p(Wu_), p(out), p(idx), p(g))
+    else:
+        rc = lib().ref_latent_moe_forward(ctypes.byref(c), p(x), p(Wr), p(Wp), p(Wg), p(Wup), p(Wd), p(gam), p(Wu_),
+                                          p(out), p(idx), p(g))
     if rc != 0:
-        raise ValueError("ref_latent_moe_forward rejected the configuration")
+        raise ValueError("the C reference rejected the configuration")
     return {"out": out, "idx": idx.astype(np.int64), "g": g}

@@ -22,6 +22,15 @@
  * The bias only selects (deep dive §4.2: weights come from the unbiased scores). All
  * matrices are row-major [out, in]; W_gate / W_up are [E, I, L], W_down [E, L, I]; gamma is
  * [E, L], or [L] when gamma_shared.
+ *
+ * NVFP4 expert weights (deep dive §7.3 bytes bullet, §7.4 NVFP4 paragraph: 4-bit values,
+ * one E4M3 scale per 16 consecutive weights of a row, one FP32 scale per matrix) are
+ * decoded element by element from the bit fields of the OCP MX v1.0 formats:
+ *   E2M1 code s.ee.m:  (-1)^s * (e == 0 ? m / 2 : 2^(e-1) * (1 + m / 2))
+ *   E4M3 byte s.eeee.mmm: (-1)^s * (e == 0 ? m / 8 * 2^-6 : 2^(e-7) * (1 + m / 8)),
+ *                         S.1111.111 is NaN
+ *   w[o, i] = e2m1(nibble i of row o) * e4m3(scale byte i / 16 of row o) * matrix_scale,
+ * the nibble of an even i being the low half of byte i / 2.
  */
 #include <math.h>
 #include <stdlib.h>
@@ -57,11 +66,84 @@ static double mean_square(const double* v, int n) {
   return s / n;
 }
 
+/* ---- NVFP4 expert weights ---------------------------------------------------------- */
+typedef struct {
+  const unsigned char* codes;   /* [E, out, in/2], low nibble = even element */
+  const unsigned char* scales;  /* [E, out, in/16] E4M3 bytes                */
+  const float* matrix_scale;    /* [E]                                       */
+} ref_nvfp4;
+
+double ref_e2m1_value(unsigned code) {
+  const unsigned s = (code >> 3) & 1u, e = (code >> 1) & 3u, m = code & 1u;
+  const double mag = e == 0 ? m * 0.5 : ldexp(1.0 + m * 0.5, (int)e - 1);
+  return s ? -mag : mag;
+}
+
+double ref_e4m3_value(unsigned byte) {
+  const unsigned s = (byte >> 7) & 1u, e = (byte >> 3) & 15u, m = byte & 7u;
+  if (e == 15u && m == 7u) return NAN;
+  const double mag = e == 0 ? ldexp(m / 8.0, -6) : ldexp(1.0 + m / 8.0, (int)e - 7);
+  return s ? -mag : mag;
+}
+
+/* y[r] = sum_c W_e[r, c] v[c] for expert e's R x C NVFP4 matrix, decoded per element */
+static void matvec_nvfp4(const ref_nvfp4* w, size_t e, int R, int C, const double* v, double* y) {
+  const double ms = (double)w->matrix_scale[e];
+  for (int r = 0; r < R; ++r) {
+    const unsigned char* crow = w->codes + (e * (size_t)R + r) * (size_t)(C / 2);
+    const unsigned char* srow = w->scales + (e * (size_t)R + r) * (size_t)(C / 16);
+    double s = 0.0;
+    for (int c = 0; c < C; ++c) {
+      const unsigned byte = crow[c / 2];
+      const unsigned code = (c % 2 == 0) ? (byte & 15u) : (byte >> 4);
+      s += ref_e2m1_value(code) * ref_e4m3_value(srow[c / 16]) * ms * v[c];
+    }
+    y[r] = s;
+  }
+}
+
+/* The expert weights of one forward: dense double matrices, or NVFP4 descriptions. */
+typedef struct {
+  const double *gate, *up, *down;
+  const ref_nvfp4 *qgate, *qup, *qdown;
+} ref_experts;
+
+static void expert_matvec(const ref_experts* x, int which, size_t e, int R, int C, const double* v, double* y) {
+  const double* dense = which == 0 ? x->gate : which == 1 ? x->up : x->down;
+  const ref_nvfp4* q = which == 0 ? x->qgate : which == 1 ? x->qup : x->qdown;
+  if (q != NULL)
+    matvec_nvfp4(q, e, R, C, v, y);
+  else
+    matvec(dense + e * (size_t)R * C, v, R, C, y);
+}
+
+static int forward(const ref_cfg* c, const double* x, const double* W_router, const double* W_pool,
+                   const ref_experts* ex, const double* gamma, const double* W_unpool, double* out, int* idx_out,
+                   double* g_out);
+
 /* Returns 0, or -1 for an invalid configuration or a failed allocation. idx_out [T, k] and
  * g_out [T, k] may be NULL. */
 int ref_latent_moe_forward(const ref_cfg* c, const double* x, const double* W_router, const double* W_pool,
                            const double* W_gate, const double* W_up, const double* W_down, const double* gamma,
                            const double* W_unpool, double* out, int* idx_out, double* g_out) {
+  const ref_experts ex = {W_gate, W_up, W_down, NULL, NULL, NULL};
+  return forward(c, x, W_router, W_pool, &ex, gamma, W_unpool, out, idx_out, g_out);
+}
+
+/* The same block with NVFP4 expert weights (in must be a multiple of 16 for every matrix:
+ * L for gate / up, I for down). */
+int ref_latent_moe_forward_nvfp4(const ref_cfg* c, const double* x, const double* W_router, const double* W_pool,
+                                 const ref_nvfp4* W_gate, const ref_nvfp4* W_up, const ref_nvfp4* W_down,
+                                 const double* gamma, const double* W_unpool, double* out, int* idx_out,
+                                 double* g_out) {
+  if (c == NULL || W_gate == NULL || W_up == NULL || W_down == NULL || c->L % 16 || c->I % 16) return -1;
+  const ref_experts ex = {NULL, NULL, NULL, W_gate, W_up, W_down};
+  return forward(c, x, W_router, W_pool, &ex, gamma, W_unpool, out, idx_out, g_out);
+}
+
+static int forward(const ref_cfg* c, const double* x, const double* W_router, const double* W_pool,
+                   const ref_experts* ex, const double* gamma, const double* W_unpool, double* out, int* idx_out,
+                   double* g_out) {
   if (c == NULL || c->T < 0 || c->D < 1 || c->L < 1 || c->I < 1 || c->E < 1 || c->k < 1 || c->k > c->E) return -1;
   const int D = c->D, L = c->L, I = c->I, E = c->E, k = c->k;
   double* l = malloc(sizeof(double) * E);
@@ -119,10 +201,10 @@ int ref_latent_moe_forward(const ref_cfg* c, const double* x, const double* W_ro
     for (int i = 0; i < L; ++i) cc[i] = 0.0;
     for (int j = 0; j < k; ++j) {
       const int e = sel[j];
-      matvec(W_gate + (size_t)e * I * L, z, I, L, a);
-      matvec(W_up + (size_t)e * I * L, z, I, L, u);
+      expert_matvec(ex, 0, (size_t)e, I, L, z, a);
+      expert_matvec(ex, 1, (size_t)e, I, L, z, u);
       for (int i = 0; i < I; ++i) a[i] = a[i] * sigmoid(a[i]) * u[i];
-      matvec(W_down + (size_t)e * L * I, a, L, I, y);
+      expert_matvec(ex, 2, (size_t)e, L, I, a, y);
       const double* gm = c->gamma_shared ? gamma : gamma + (size_t)e * L;
       if (c->norm_mode == 1) {
         for (int i = 0; i < L; ++i) y[i] *= 1.0 + gm[i];

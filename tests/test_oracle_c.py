@@ -7,6 +7,7 @@ fixed by construction, router rows that produce chosen logits). It is also compa
 numpy oracle -- an independent implementation of the same definition -- on seeded inputs in
 every mode both support.
 """
+import ctypes
 import functools
 import itertools
 import math
@@ -223,3 +224,62 @@ def test_c_reference_agrees_with_the_numpy_oracle(name, T, mode):
     assert np.allclose(c["g"], r["g"], rtol=1e-13, atol=1e-15)
     scale = np.abs(r["out"]).max()
     assert np.abs(c["out"] - r["out"]).max() <= 1e-12 * scale
+
+
+# ------------------------------------------------------------------- NVFP4 experts
+def test_c_decoders_match_the_ocp_tables_and_every_e4m3_byte():
+    """The C decoders of the 4-bit E2M1 values and the E4M3 block-scale bytes against the
+    OCP MX v1.0 tables (golden files) and, for E4M3, every byte against torch's float8."""
+    for s in lines("fp4_e2m1.txt"):
+        code, val = s.split()
+        got = cref.e2m1_value(int(code))
+        assert got == float(val) and math.copysign(1.0, got) == (-1.0 if val.startswith("-") else 1.0)
+    for s in lines("fp8_e4m3.txt"):
+        b, val = s.split()
+        got = cref.e4m3_value(int(b, 16))
+        assert (math.isnan(got) and val == "nan") or got == float(val)
+    import torch
+    ref = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = np.array([cref.e4m3_value(b) for b in range(256)])
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    assert np.array_equal(got[~np.isnan(got)], ref[~np.isnan(ref)])
+
+
+NVFP4_AGREE = [
+    W.Workload("c_nvfp4_tiny", T=12, D=256, L=128, I=128, E=8, k=2, dtype="bf16", seed=4, experts="nvfp4"),
+    # the NVFP4 parity workloads' expert count and top-k at a narrow width
+    W.Workload("c_nvfp4_mid", T=10, D=512, L=256, I=384, E=64, k=4, dtype="bf16", seed=9, experts="nvfp4"),
+]
+
+
+@pytest.mark.parametrize("w", NVFP4_AGREE, ids=lambda w: w.name)
+@pytest.mark.parametrize("mode", [0, 2])
+def test_c_reference_with_nvfp4_experts_agrees_with_the_numpy_oracle(w, mode):
+    """The C block decoding NVFP4 codes itself against the numpy oracle on the dequantised
+    weights (the same codes): routing identical, outputs to 1e-12 of their scale."""
+    m = dict(MODES[mode])
+    inp = W.make_inputs(w, "cpu")
+    f = oracle.as_f64
+    gamma = f(inp["gamma"])[0] if m.pop("shared_gamma", False) else f(inp["gamma"])
+    q = [(inp[n + "_codes"], inp[n + "_scales"], inp[n + "_mscale"]) for n in ("W_gate", "W_up", "W_down")]
+    c = cref.latent_moe_forward_c(inp["x"], inp["W_router"], inp["W_pool"], q, gamma, inp["W_unpool"], w.k, w.eps,
+                                  nvfp4=True, **m)
+
+    def deq(e):
+        return tuple(oracle.dequantize_nvfp4(cd[e].numpy(), sc[e].numpy(), float(ms[e])) for cd, sc, ms in q)
+    r = oracle.latent_moe_forward(f(inp["x"]), f(inp["W_router"]), f(inp["W_pool"]), deq, gamma, f(inp["W_unpool"]),
+                                  w.k, w.eps, **m)
+    assert np.array_equal(c["idx"], r["idx"])
+    assert np.abs(c["out"] - r["out"]).max() <= 1e-12 * np.abs(r["out"]).max()
+
+
+def test_c_reference_rejects_nvfp4_widths_that_are_not_whole_blocks():
+    w = NVFP4_AGREE[0]
+    inp = W.make_inputs(w, "cpu")
+    q = [(inp[n + "_codes"], inp[n + "_scales"], inp[n + "_mscale"]) for n in ("W_gate", "W_up", "W_down")]
+    c = cref.RefCfg(T=1, D=w.D, L=120, I=w.I, E=w.E, k=w.k, eps=w.eps)
+    mats = [cref.RefNvfp4(0, 0, 0) for _ in range(3)]
+    out = np.zeros((1, w.D))
+    rc = cref.lib().ref_latent_moe_forward_nvfp4(ctypes.byref(c), 0, 0, 0, *[ctypes.addressof(m) for m in mats], 0, 0,
+                                                 out.ctypes.data, 0, 0)
+    assert rc == -1
