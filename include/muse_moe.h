@@ -200,6 +200,38 @@ MUSE_API muse_status muse_latent_moe_forward(const muse_moe_config* cfg, const v
                                     const void* gamma, const void* W_unpool, void* out,
                                     void* stream);
 
+/* A tensor as muse_latent_moe_forward_checked receives it: a device pointer with its element
+ * type, rank, extents and strides (in elements, outermost first). The library reads
+ * row-major contiguous tensors only: strides must be the contiguous ones
+ * (stride[ndim-1] = 1, stride[i] = stride[i+1] * shape[i+1]). */
+typedef enum muse_elem_type { MUSE_ELEM_F32 = 0, MUSE_ELEM_BF16 = 1, MUSE_ELEM_U8 = 2 } muse_elem_type;
+typedef struct muse_tensor {
+  const void* data;           /* device memory, 16-byte aligned                        */
+  int32_t elem;               /* muse_elem_type (F32 / BF16 match muse_dtype)          */
+  int32_t ndim;               /* 1..3                                                  */
+  int64_t shape[3];
+  int64_t stride[3];
+} muse_tensor;
+
+/* muse_latent_moe_forward with every tensor described by its shape (Muse Spark Open deep
+ * dive, §4.3 implementation notes: the module's weights carry their shapes, e.g. the
+ * experts' gate/up projection [256, 8192, 4096] in the released code's fused layout). Before
+ * anything is launched, each tensor is checked against cfg:
+ *   x [T, D], W_router [E, D], W_pool [L, D], W_gate [E, I, L], W_up [E, I, L],
+ *   W_down [E, L, I], gamma [E, L] (or [L] with gamma_shared), W_unpool [D, L], out [T, D],
+ * all of element type cfg->dtype, contiguous, 16-byte aligned; out may not overlap any
+ * input. With cfg->expert_weights == MUSE_EXPERTS_NVFP4, W_gate / W_up / W_down each point
+ * to THREE consecutive descriptors -- codes u8 [E, out, in/2], block scales u8 [E, out,
+ * in/16], matrix scales f32 [E] -- and the forward receives them as muse_nvfp4_weight.
+ * Any mismatch returns MUSE_ERR_INVALID_ARG with nothing launched; otherwise the result
+ * is that of muse_latent_moe_forward on the same pointers. */
+MUSE_API muse_status muse_latent_moe_forward_checked(const muse_moe_config* cfg, const muse_tensor* x,
+                                                     const muse_tensor* W_router, const muse_tensor* W_pool,
+                                                     const muse_tensor* W_gate, const muse_tensor* W_up,
+                                                     const muse_tensor* W_down, const muse_tensor* gamma,
+                                                     const muse_tensor* W_unpool, const muse_tensor* out,
+                                                     void* stream);
+
 /* Same, with x and out in HOST memory (pinned for asynchronous copies): copies x into
  * the device buffer x_dev, runs the forward into out_dev, copies out_dev back to
  * out_host, all on `stream`. x_dev / out_dev are caller-owned device buffers. The

@@ -28,7 +28,8 @@ EXPORTS = ("muse_moe_config_init", "muse_latent_moe_workspace_size", "muse_laten
            "muse_latent_moe_forward", "muse_latent_moe_forward_host_io", "muse_latent_moe_last_device_status",
            "muse_status_string", "muse_latent_moe_launch_count", "muse_latent_moe_forward_static_scratch",
            "muse_selftest_bounded_wait", "muse_quantize_nvfp4_rows", "muse_latent_moe_forward_host_batches",
-           "muse_ep_workspace_layout", "muse_ep_dispatch", "muse_ep_experts", "muse_ep_combine")
+           "muse_ep_workspace_layout", "muse_ep_dispatch", "muse_ep_experts", "muse_ep_combine",
+           "muse_latent_moe_forward_checked")
 
 # roles of an expert-parallel workspace (muse_ep_role)
 EP_HOME, EP_EXPERTS = 1, 2
@@ -57,6 +58,27 @@ class Config(ctypes.Structure):
                 ("ffn_post_gain", ctypes.c_void_p), ("ffn_post_eps", ctypes.c_float),
                 ("residual_gate", ctypes.c_void_p), ("residual_gate_temperature", ctypes.c_float),
                 ("residual_gate_eps", ctypes.c_float), ("act_format", ctypes.c_int32)]
+
+
+class Tensor(ctypes.Structure):
+    """muse_tensor: device pointer, element type, rank, extents and strides (elements)."""
+    _fields_ = [("data", ctypes.c_void_p), ("elem", ctypes.c_int32), ("ndim", ctypes.c_int32),
+                ("shape", ctypes.c_int64 * 3), ("stride", ctypes.c_int64 * 3)]
+
+
+ELEM_F32, ELEM_BF16, ELEM_U8 = 0, 1, 2
+
+
+def tensor_desc(t) -> Tensor:
+    """The muse_tensor of a torch tensor (its own shape and strides: a non-contiguous view
+    is described as it is, and the library rejects it)."""
+    import torch
+    elem = {torch.float32: ELEM_F32, torch.bfloat16: ELEM_BF16, torch.uint8: ELEM_U8}.get(t.dtype, -1)
+    d = Tensor()
+    d.data, d.elem, d.ndim = int(t.data_ptr()), elem, t.dim()
+    for i in range(min(t.dim(), 3)):
+        d.shape[i], d.stride[i] = int(t.shape[i]), int(t.stride(i))
+    return d
 
 
 class Nvfp4Weight(ctypes.Structure):
@@ -112,6 +134,8 @@ def lib() -> ctypes.CDLL:
         L.muse_ep_experts.restype = ctypes.c_int
         L.muse_ep_combine.argtypes = [cp, i32] + [vp] * 7
         L.muse_ep_combine.restype = ctypes.c_int
+        L.muse_latent_moe_forward_checked.argtypes = [cp] + [ctypes.POINTER(Tensor)] * 9 + [vp]
+        L.muse_latent_moe_forward_checked.restype = ctypes.c_int
         L.muse_latent_moe_launch_count.argtypes = [cp]
         L.muse_latent_moe_launch_count.restype = ctypes.c_int32
         _lib = L
@@ -185,6 +209,26 @@ def forward(cfg: Config, x, W_router, W_pool, W_gate, W_up, W_down, gamma, W_unp
                                          _ptr(W_up), _ptr(W_down), _ptr(gamma), _ptr(W_unpool), _ptr(out),
                                          _stream_handle(stream))
     _check(code, "muse_latent_moe_forward")
+
+
+def forward_checked(cfg: Config, x, W_router, W_pool, W_gate, W_up, W_down, gamma, W_unpool, out,
+                    stream=None) -> None:
+    """Enqueue one forward through the shape-checked entry point: every argument is a torch
+    tensor (NVFP4 experts: a (codes, block scales, matrix scales) triple each) described by
+    its dtype, shape and strides; the library rejects a mismatch before launching anything."""
+    def one(t):
+        return ctypes.byref(tensor_desc(t))
+
+    def expert(t):
+        if isinstance(t, (tuple, list)):
+            arr = (Tensor * 3)(*[tensor_desc(p) for p in t])
+            return ctypes.cast(arr, ctypes.POINTER(Tensor)), arr
+        d = tensor_desc(t)
+        return ctypes.pointer(d), d
+    eg, eu, ed = expert(W_gate), expert(W_up), expert(W_down)
+    code = lib().muse_latent_moe_forward_checked(ctypes.byref(cfg), one(x), one(W_router), one(W_pool), eg[0], eu[0],
+                                                 ed[0], one(gamma), one(W_unpool), one(out), _stream_handle(stream))
+    _check(code, "muse_latent_moe_forward_checked")
 
 
 def forward_static_scratch(cfg: Config, x, W_router, W_pool, W_gate, W_up, W_down, gamma, W_unpool, out,
@@ -342,7 +386,8 @@ def block_config(T: int, dims: Dict, dtype: str, modes: Dict, weights: Dict, nvf
 
 
 class LatentMoE:
-    """Holds the block's device weights and a workspace; calling it runs the forward.
+    """Holds the block's device weights and a workspace; calling it runs the forward through
+    the shape-checked entry point (muse_latent_moe_forward_checked).
 
     weights: dict with W_router, W_pool, W_gate, W_up, W_down, gamma, W_unpool (torch
     CUDA tensors in the layouts of include/muse_moe.h); router_bias, pre_norm_gain and the
@@ -355,6 +400,9 @@ class LatentMoE:
         self.w = dict(weights)
         E, D = weights["W_router"].shape
         I, L, self.nvfp4 = expert_weight_dims(weights)
+        # the expert tensors as the shape-checked entry point takes them
+        self.experts = tuple((weights[n + "_codes"], weights[n + "_scales"], weights[n + "_mscale"]) if self.nvfp4
+                             else weights[n] for n in ("W_gate", "W_up", "W_down"))
         self.w["W_gate"], self.w["W_up"], self.w["W_down"] = expert_operands(weights, self.nvfp4)
         self.dtype = {torch.float32: "f32", torch.bfloat16: "bf16"}[weights["W_router"].dtype]
         self.dims = dict(D=int(D), L=L, I=I, E=int(E), k=k, eps=eps)
@@ -379,6 +427,5 @@ class LatentMoE:
         if out is None:
             out = torch.empty((T, self.dims["D"]), dtype=x.dtype, device=x.device)
         w = self.w
-        forward(cfg, x, w["W_router"], w["W_pool"], w["W_gate"], w["W_up"], w["W_down"], w["gamma"],
-                w["W_unpool"], out, stream)
+        forward_checked(cfg, x, w["W_router"], w["W_pool"], *self.experts, w["gamma"], w["W_unpool"], out, stream)
         return out

@@ -15,6 +15,7 @@
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
+#include <initializer_list>
 #include <mutex>
 
 #include "muse_moe.h"
@@ -935,6 +936,57 @@ muse_moe_config expert_shard_config(const muse_moe_config& c, int32_t G, int64_t
   return l;
 }
 
+// ---------------------------------------------------------------------- shape checks
+// A descriptor names a contiguous row-major tensor of element type `elem` and exactly the
+// extents `dims` (n of them), on a 16-byte boundary.
+bool tensor_is(const muse_tensor* t, int32_t elem, std::initializer_list<int64_t> dims) {
+  if (t == nullptr || t->data == nullptr || !aligned16(t->data) || t->elem != elem) return false;
+  if (t->ndim != static_cast<int32_t>(dims.size()) || t->ndim < 1 || t->ndim > 3) return false;
+  int i = 0;
+  for (int64_t d : dims)
+    if (t->shape[i++] != d) return false;
+  int64_t stride = 1;
+  for (int k = t->ndim - 1; k >= 0; --k) {
+    if (t->stride[k] != stride) return false;
+    stride *= t->shape[k];
+  }
+  return true;
+}
+
+size_t tensor_bytes(const muse_tensor* t) {
+  const size_t es = t->elem == MUSE_ELEM_F32 ? 4 : t->elem == MUSE_ELEM_BF16 ? 2 : 1;
+  size_t n = es;
+  for (int k = 0; k < t->ndim; ++k) n *= static_cast<size_t>(t->shape[k]);
+  return n;
+}
+
+bool overlaps(const muse_tensor* a, const muse_tensor* b) {
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a->data), b0 = reinterpret_cast<uintptr_t>(b->data);
+  return a0 < b0 + tensor_bytes(b) && b0 < a0 + tensor_bytes(a);
+}
+
+// An expert tensor [E, rows, cols]: one dense descriptor, or the three NVFP4 descriptors
+// (codes, block scales, matrix scales); fills the weight the forward takes.
+bool expert_tensor_is(const muse_moe_config& c, const muse_tensor* t, int64_t rows, int64_t cols,
+                      muse_nvfp4_weight* q, const void** dense) {
+  if (c.expert_weights == MUSE_EXPERTS_NVFP4) {
+    if (t == nullptr || cols % 16 != 0) return false;
+    if (!tensor_is(&t[0], MUSE_ELEM_U8, {c.E, rows, cols / 2}) || !tensor_is(&t[1], MUSE_ELEM_U8, {c.E, rows, cols / 16}))
+      return false;
+    // matrix scales: float [E], 4-byte aligned is enough for the kernels
+    const muse_tensor* m = &t[2];
+    if (m->data == nullptr || (reinterpret_cast<uintptr_t>(m->data) & 3u) || m->elem != MUSE_ELEM_F32 ||
+        m->ndim != 1 || m->shape[0] != c.E || m->stride[0] != 1)
+      return false;
+    *q = muse_nvfp4_weight{t[0].data, t[1].data, static_cast<const float*>(m->data)};
+    *dense = q;
+    return true;
+  }
+  if (!tensor_is(t, c.dtype, {c.E, rows, cols})) return false;
+  *dense = t->data;
+  return true;
+}
+
 // Scratch for muse_latent_moe_forward_static_scratch: a fixed array in device global
 // memory, so that entry point never allocates. In host code this name stands for the
 // symbol, not a device address; the address comes from cudaGetSymbolAddress.
@@ -1017,6 +1069,35 @@ muse_status muse_latent_moe_forward(const muse_moe_config* cfg, const void* x, c
   if (cfg->dtype == MUSE_BF16)
     return forward_impl<__nv_bfloat16>(*cfg, lay, x, W_router, W_pool, W_gate, W_up, W_down, gamma, W_unpool, out, st);
   return forward_impl<float>(*cfg, lay, x, W_router, W_pool, W_gate, W_up, W_down, gamma, W_unpool, out, st);
+}
+
+muse_status muse_latent_moe_forward_checked(const muse_moe_config* cfg, const muse_tensor* x,
+                                            const muse_tensor* W_router, const muse_tensor* W_pool,
+                                            const muse_tensor* W_gate, const muse_tensor* W_up,
+                                            const muse_tensor* W_down, const muse_tensor* gamma,
+                                            const muse_tensor* W_unpool, const muse_tensor* out, void* stream) {
+  MUSE_TRY(validate_sizes(cfg));
+  const muse_moe_config& c = *cfg;
+  const int32_t a = c.dtype;  // MUSE_F32 / MUSE_BF16 equal MUSE_ELEM_F32 / MUSE_ELEM_BF16
+  if (!tensor_is(x, a, {c.T, c.D}) || !tensor_is(W_router, a, {c.E, c.D}) || !tensor_is(W_pool, a, {c.L, c.D}) ||
+      !tensor_is(W_unpool, a, {c.D, c.L}) || !tensor_is(out, a, {c.T, c.D}))
+    return MUSE_ERR_INVALID_ARG;
+  if (!(c.gamma_shared ? tensor_is(gamma, a, {c.L}) : tensor_is(gamma, a, {c.E, c.L}))) return MUSE_ERR_INVALID_ARG;
+  muse_nvfp4_weight qg{}, qu{}, qd{};
+  const void *wg = nullptr, *wu = nullptr, *wd = nullptr;
+  if (!expert_tensor_is(c, W_gate, c.I, c.L, &qg, &wg) || !expert_tensor_is(c, W_up, c.I, c.L, &qu, &wu) ||
+      !expert_tensor_is(c, W_down, c.L, c.I, &qd, &wd))
+    return MUSE_ERR_INVALID_ARG;
+  const muse_tensor* inputs[] = {x, W_router, W_pool, gamma, W_unpool};
+  for (const muse_tensor* t : inputs)
+    if (overlaps(out, t)) return MUSE_ERR_INVALID_ARG;
+  const int n_exp = c.expert_weights == MUSE_EXPERTS_NVFP4 ? 3 : 1;
+  const muse_tensor* experts[] = {W_gate, W_up, W_down};
+  for (const muse_tensor* t : experts)
+    for (int i = 0; i < n_exp; ++i)
+      if (overlaps(out, &t[i])) return MUSE_ERR_INVALID_ARG;
+  return muse_latent_moe_forward(cfg, x->data, W_router->data, W_pool->data, wg, wu, wd, gamma->data,
+                                 W_unpool->data, const_cast<void*>(out->data), stream);
 }
 
 muse_status muse_ep_workspace_layout(const muse_moe_config* cfg, int32_t ep_size, int32_t role, int64_t rows,

@@ -184,3 +184,99 @@ def test_stage_names_match_the_library_launch_count(w4a4, pre_expert, ffn_pre, f
     assert len(set(names)) == len(names)
     assert ("quant_z" in names) == w4a4 and ("gather_codes" in names) == w4a4
     assert names.index("pooler") < names.index("gather_codes" if w4a4 else "gather") < names.index("gate_up_swiglu")
+
+
+# ------------------------------------------------------------ the shape-checked entry point
+def _desc(addr, elem, shape):
+    d = moe.Tensor()
+    d.data, d.elem, d.ndim = addr, elem, len(shape)
+    st = 1
+    for i in reversed(range(len(shape))):
+        d.shape[i], d.stride[i] = shape[i], st
+        st *= shape[i]
+    return d
+
+
+def _checked_args(cfg, nvfp4=False):
+    """Descriptors of every argument for cfg at non-overlapping (never dereferenced) addresses."""
+    T, D, L, I, E = cfg.T, cfg.D, cfg.L, cfg.I, cfg.E
+    a = cfg.dtype
+    base = iter(range(1 << 40, 1 << 50, 1 << 36))
+    args = {"x": _desc(next(base), a, (T, D)), "W_router": _desc(next(base), a, (E, D)),
+            "W_pool": _desc(next(base), a, (L, D)), "gamma": _desc(next(base), a, (E, L)),
+            "W_unpool": _desc(next(base), a, (D, L)), "out": _desc(next(base), a, (T, D))}
+    for n, (r, c) in (("W_gate", (I, L)), ("W_up", (I, L)), ("W_down", (L, I))):
+        if nvfp4:
+            args[n] = (moe.Tensor * 3)(_desc(next(base), moe.ELEM_U8, (E, r, c // 2)),
+                                       _desc(next(base), moe.ELEM_U8, (E, r, c // 16)),
+                                       _desc(next(base), moe.ELEM_F32, (E,)))
+        else:
+            args[n] = (moe.Tensor * 1)(_desc(next(base), a, (E, r, c)))
+    return args
+
+
+def _call_checked(cfg, args):
+    order = ("x", "W_router", "W_pool", "W_gate", "W_up", "W_down", "gamma", "W_unpool", "out")
+    ptrs = [ctypes.cast(args[n], ctypes.POINTER(moe.Tensor)) if isinstance(args[n], ctypes.Array)
+            else ctypes.pointer(args[n]) for n in order]
+    return moe.lib().muse_latent_moe_forward_checked(ctypes.byref(cfg), *ptrs, None)
+
+
+def test_tensor_descriptor_layout_matches_the_c_compiler(tmp_path):
+    fields = [f for f, _ in moe.Tensor._fields_]
+    src = ["#include <stdio.h>", "#include <stddef.h>", '#include "muse_moe.h"', "int main(void) {",
+           'printf("%zu\\n", sizeof(muse_tensor));']
+    src += [f'printf("%zu\\n", offsetof(muse_tensor, {f}));' for f in fields]
+    src += ["return 0; }"]
+    c = tmp_path / "probe_t.c"
+    c.write_text("\n".join(src))
+    exe = tmp_path / "probe_t"
+    subprocess.run(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), str(c), "-o", str(exe)], check=True)
+    vals = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
+    assert vals == [ctypes.sizeof(moe.Tensor)] + [getattr(moe.Tensor, f).offset for f in fields]
+
+
+@pytest.mark.parametrize("nvfp4", [False, True])
+def test_checked_forward_rejects_every_shape_mismatch_before_any_launch(nvfp4):
+    """Correct descriptors get past every shape check (and stop at the missing workspace);
+    a wrong extent, rank, element type, stride or alignment on any argument, or an output
+    overlapping an input, is MUSE_ERR_INVALID_ARG -- all without a GPU."""
+    cfg = moe.make_config(64, 1024, 512, 256, 16, 2, "bf16")
+    if nvfp4:
+        cfg.expert_weights = moe.EXPERTS_NVFP4
+    assert _call_checked(cfg, _checked_args(cfg, nvfp4)) == 3        # shapes fine: no workspace
+    names = ("x", "W_router", "W_pool", "W_gate", "W_up", "W_down", "gamma", "W_unpool", "out")
+    for n in names:
+        parts = 3 if (nvfp4 and n.startswith("W_") and n in ("W_gate", "W_up", "W_down")) else 1
+        for p in range(parts):
+            for corrupt in ("extent", "rank", "elem", "stride", "align", "null"):
+                args = _checked_args(cfg, nvfp4)
+                d = args[n][p] if isinstance(args[n], ctypes.Array) else args[n]
+                if corrupt == "extent":
+                    d.shape[0] += 1
+                elif corrupt == "rank":
+                    d.ndim = d.ndim + 1 if d.ndim < 3 else 1
+                elif corrupt == "elem":
+                    d.elem = moe.ELEM_F32 if d.elem != moe.ELEM_F32 else moe.ELEM_BF16
+                elif corrupt == "stride":
+                    d.stride[0] += 1
+                elif corrupt == "align":
+                    d.data += 8 if not (nvfp4 and p == 2) else 2
+                else:
+                    d.data = 0
+                assert _call_checked(cfg, args) == 1, (n, p, corrupt)
+    # the gain shared by all experts is [L]; a per-expert gain given as shared is rejected
+    cfg.gamma_shared = 1
+    assert _call_checked(cfg, _checked_args(cfg, nvfp4)) == 1
+    args = _checked_args(cfg, nvfp4)
+    args["gamma"] = _desc(args["gamma"].data, cfg.dtype, (cfg.L,))
+    assert _call_checked(cfg, args) == 3
+    # out may not overlap an input
+    cfg.gamma_shared = 0
+    args = _checked_args(cfg, nvfp4)
+    args["out"].data = args["x"].data
+    assert _call_checked(cfg, args) == 1
+    args = _checked_args(cfg, nvfp4)
+    w = args["W_down"][0]
+    args["out"].data = w.data + 4096
+    assert _call_checked(cfg, args) == 1
