@@ -177,11 +177,11 @@ def roofline(w: W.Workload, kernel: str, fl: float, by: float, t: float, peaks, 
     t_hbm = by / (peaks["hbm_gbs"] * 1e9)
     if t_tensor >= t_hbm:
         roof = {"bound": "tensor", "achieved": fl / t / 1e12, "peak": ratio * tensor_peak, "unit": "TFLOP/s"}
-        kind = ("burst, timed region at max SM clock" if burst else "sustained, timed region below max clock")
-        roof["peak_source"] = f"measured bf16 GEMM ({kind})" + (" x 4 (FP4 / BF16 nominal)" if fp4_gemm else "")
+        kind = "burst: max SM clock" if burst else "sustained: below max clock"
+        roof["peak_source"] = f"measured bf16 ({kind})" + (" x 4 (FP4 / BF16 nominal)" if fp4_gemm else "")
     else:
         roof = {"bound": "hbm", "achieved": by / t / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "peak_source": "measured copy bandwidth"}
+                "peak_source": "measured copy"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["kernel"] = kernel
     roof["algorithmic_flops"] = fl
@@ -461,8 +461,8 @@ class OracleSample:
         return time.perf_counter() - t0 - (self.widen_s - w0)
 
     def describe(self) -> str:
-        return (f"tokens 0-{self.n - 1} of the {self.w.name} batch ({self.experts_touched} experts touched), "
-                f"FP64 numpy oracle, expert-major; weights widened to f64 outside the timed region")
+        return (f"tokens 0-{self.n - 1} of {self.w.name} ({self.experts_touched} experts), FP64 numpy oracle "
+                f"expert-major, f64 widening untimed")
 
 
 def host_cores():
@@ -500,7 +500,7 @@ def cpu_baseline(w: W.Workload, dev, n_tokens: int):
     dt = sample.run()
     flops_per_token = 2 * (w.E * w.D + w.L * w.D + w.k * 3 * w.L * w.I + w.D * w.L)
     return {"value": n_tokens / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": sample.describe() + f"; {dt:.1f} s, {n_tokens * flops_per_token / dt / 1e9:.0f} GFLOP/s FP64"}
+            "sample": sample.describe() + f"; {dt:.1f} s, {n_tokens * flops_per_token / dt / 1e9:.0f} GFLOP/s"}
 
 
 def run_reference(w: W.Workload, args, dev):
@@ -532,8 +532,8 @@ def metric_name():
 def config_dict(w: W.Workload):
     """The workload named by what it is; the same dict in both arms."""
     return {"workload": f"{w.name}: latent-MoE layer T={w.T} D={w.D} L={w.L} I={w.I} E={w.E} top-{w.k} "
-                        f"{w.dtype} {w.routing} routing",
-            "l2": "inputs larger than L2 (each step streams the touched experts' weights)"}
+                        f"{w.dtype} {w.routing}",
+            "l2": "inputs > L2 (weights streamed)"}
 
 
 _DIST = {"on": False}
@@ -559,13 +559,15 @@ def sig(v, n=4):
     return round(v, n - 1 - int(math.floor(math.log10(abs(v)))))
 
 
+SIDE_FIELDS = ["tokens/s", "ms/step", "dominant kernel roofline frac", "graph ms/step"]
+
+
 def side_entry(r):
-    """One side workload in the JSON line: tokens/s, ms per step, the dominant kernel's
-    roofline fraction and bound, and the whole step's fraction of its roofline."""
-    e = {"v": sig(r["value"]), "ms": sig(r["ms_per_step"]), "frac": sig(r["roofline"]["frac"], 3),
-         "bound": r["roofline"]["bound"], "step_frac": sig(r["step"]["frac_of_step_roofline"], 3)}
+    """One side workload in the JSON line, as the list SIDE_FIELDS names (the graph-replay
+    time only where the workload is also timed that way)."""
+    e = [sig(r["value"]), sig(r["ms_per_step"]), sig(r["roofline"]["frac"], 3)]
     if "graph" in r:
-        e["graph_ms"] = sig(r["graph"]["ms_per_step"])
+        e.append(sig(r["graph"]["ms_per_step"]))
     return e
 
 
@@ -592,7 +594,7 @@ def main():
         # inputs are generated on the GPU when there is one (same bytes either way)
         if rank == 0:
             dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
-            print(json.dumps(run_reference(W.WORKLOADS[args.workload], args, dev)), flush=True)
+            print(json.dumps(run_reference(W.WORKLOADS[args.workload], args, dev), separators=(",", ":")), flush=True)
         return
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -650,7 +652,7 @@ def main():
                 "metric": metric_name(), "value": sig(main_res["value"], 6), "unit": "tokens/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": sig(main_res["ms_per_step"], 5),
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
-                "data": "synthetic (seeded N(0,1) x, N(0,1/fan_in) weights)",
+                "data": "synthetic",
                 "config": config_dict(w), "roofline": roof,
                 "step_roofline_frac": sig(main_res["step"]["frac_of_step_roofline"], 3),
                 "gpu_launches": main_res["gpu_launches"],
@@ -665,6 +667,7 @@ def main():
             if "graph" in main_res:
                 line["graph_replay_ms"] = sig(main_res["graph"]["ms_per_step"])
             if side:
+                line["side_fields"] = SIDE_FIELDS
                 line["side"] = {name: side_entry(r) for name, r in side.items()}
             if world == 1 and not args.no_cpu:
                 line["cpu_baseline"] = cpu_baseline(w, dev, args.cpu_tokens)
@@ -672,7 +675,7 @@ def main():
                 detail = {"line": line, "main": main_res, "side": side, "cpu_model": cpu_model()}
                 with open(args.detail, "w") as f:
                     json.dump(detail, f, indent=1, default=float)
-            print(json.dumps(line), flush=True)
+            print(json.dumps(line, separators=(",", ":")), flush=True)
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()

@@ -341,8 +341,9 @@ MUSE_API muse_status muse_quantize_nvfp4_rows(const void* src, int64_t rows, int
  * cfg is the whole block's configuration (E = all experts) on every call. Calls 1 and 5
  * of one forward use the same cfg->workspace (the token rank's workspace, role
  * MUSE_EP_HOME); call 3 uses an expert workspace (role MUSE_EP_EXPERTS) in
- * cfg->workspace. The result equals muse_latent_moe_forward on the same tokens up to
- * the rounding of the GEMMs (a GEMM of other row counts may tile differently). Calls are
+ * cfg->workspace. The result equals muse_latent_moe_forward on the same tokens bit for
+ * bit: the expert GEMMs see other row counts and may tile them differently, but every
+ * output element is accumulated over K in the same order whatever the tiling. Calls are
  * enqueued on `stream` without synchronising; the host reads rank_counts (a device
  * array) to size the exchange. stage_events is ignored. Status word: calls 1 and 3 reset
  * their workspace's word, call 5 adds to the word of call 1.
