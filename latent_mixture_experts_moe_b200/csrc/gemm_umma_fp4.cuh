@@ -4,20 +4,27 @@
 //
 // Weights stay 4-bit in HBM (0.5 B per weight + one E4M3 byte per 16 weights). TMA brings the
 // packed codes of a 128-row x 64-K tile (4 KB) and the token tile into shared memory; eight
-// converter warps expand each code row into 64 bf16 values (code x block scale is exact in
-// bf16: at most 2 + 4 significant bits) and write them straight into TENSOR MEMORY, where the
-// UMMA takes its A operand (kind::f16 with A in TMEM: 128 lanes x 32 columns per 64-K tile,
-// two K elements per column). The dequantised weights never touch shared memory, which
-// leaves its bandwidth to the TMA copies and the token operand. The per-matrix FP32 scale
-// multiplies the FP32 accumulator in the epilogue.
+// converter warps expand each code row into 64 f16 values and write them straight into
+// TENSOR MEMORY, where the UMMA takes its A operand (kind::f16 with A in TMEM: 128 lanes x 32
+// columns per 64-K tile, two K elements per column). The expansion is two hardware
+// conversions per pair of weights' worth of work: cvt.rn.f16x2.e2m1x2 turns a code byte into
+// two f16 values, cvt.rn.f16x2.e4m3x2 turns two block-scale bytes into f16, and one f16x2
+// multiply applies the scale -- exact, since a code value (2 significant bits) times an E4M3
+// scale (4 bits) is a normal f16 number (2^-10 .. 2688). The token operand is therefore f16
+// too (the gather converts the bf16 latent rows; this kernel's SwiGLU epilogue writes h as
+// f16 for the down projection), exact for activations of magnitude 2^-14 .. 65504. The
+// dequantised weights never touch shared memory. The per-matrix FP32 scale multiplies the
+// FP32 accumulator in the epilogue.
 //
 // Roles (448 threads, one CTA per SM): warp 0 TMA producer (codes + token tile, a deep ring:
 // 4-bit stages are small), warp 1 TMEM owner + UMMA issuer, warps 2..5 epilogue, warps 6..13
 // converters (warp w expands weight rows 32*(w%4) .. +31 -- the TMEM lanes it may write -- of
-// tile (w-6)/4; block scales read from global memory 8 k-blocks at a time). TMEM columns:
-// accumulators from 0, converted weight slots (2 or 3 of 32 * MT columns) after them.
-// Barriers: per TMA stage full (bytes) / empty (UMMA commit); per converted slot conv
-// (converter warps) / cfree (UMMA commit). Every wait is bounded (ptx.cuh).
+// tile (w-6)/4; block scales read from global memory 8 k-blocks at a time). A converter warp
+// issues the TMEM store of k-block j, expands k-block j+1 into registers, and only then waits
+// for the store and hands slot j to the UMMA, so each store's latency hides behind the next
+// expansion. TMEM columns: accumulators from 0, converted weight slots (32 * MT columns each)
+// after them. Barriers: per TMA stage full (bytes) / empty (UMMA commit); per converted slot
+// conv (converter warps) / cfree (UMMA commit). Every wait is bounded (ptx.cuh).
 #pragma once
 
 #include "gemm_umma.cuh"
@@ -38,18 +45,17 @@ struct Fp4Shape {
   static constexpr uint32_t kCodeBytes = 128u * 32u;  // packed codes of 128 rows x 64 K
   static constexpr uint32_t kBBytes = static_cast<uint32_t>(BN) * 128u;
   static constexpr uint32_t kStageBytes = kBBytes + kCodeBytes * MT;   // TMA ring stage
-  static constexpr int kSmemBudget = 227 * 1024 - 1024 - 1024;         // alignment, LUT + barriers
+  static constexpr int kSmemBudget = 227 * 1024 - 1024 - 1024;         // alignment, barriers
   static constexpr int kStagesFit = kSmemBudget / static_cast<int>(kStageBytes);
   static constexpr int kStages = kStagesFit > 16 ? 16 : kStagesFit;
   static constexpr int kAccStages = MT == 2 ? 1 : 2;
   static constexpr uint32_t kAccCols = static_cast<uint32_t>(BN) * MT;
   static constexpr uint32_t kTmemCols = 512;
-  // converted weight tiles in the TMEM columns the accumulators leave: 3 slots (measured
-  // best for decode-sized tiles; deeper did worse), or as many as fit
+  // converted weight tiles in the TMEM columns the accumulators leave, up to 4 slots
   static constexpr uint32_t kConvCols = 32u * MT;         // TMEM columns per slot
   static constexpr uint32_t kConvCol0 = kAccCols * kAccStages;
   static constexpr int kConvFit = static_cast<int>((kTmemCols - kConvCol0) / kConvCols);
-  static constexpr int kConvSlots = kConvFit > 3 ? 3 : kConvFit;
+  static constexpr int kConvSlots = kConvFit > 4 ? 4 : kConvFit;
   static constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes + 1024;
   static_assert(kConvSlots >= 2, "no TMEM room for converted weight tiles");
   static_assert(kStages >= 2, "tile too large for the shared-memory ring");
@@ -60,60 +66,61 @@ struct Fp4Shape {
 // warps 0 producer, 1 UMMA issuer, 2..5 epilogue, 6..13 converters (with MT = 1, 10..13 idle)
 constexpr int kFp4Threads = 448;
 
-// 4 codes (the low 16 bits of w: nibbles k0..k3) -> 4 bf16 in two words, low element
-// first, with byte-permute lookups: the magnitude (nibble bits 0-2) selects the high and low
-// byte of |value| from two 8-entry tables, the sign (nibble bit 3) selects 0x00 or 0x80 to
-// OR into the high byte.
-__device__ __forceinline__ void e2m1x4_to_bf16(uint32_t w, uint32_t& o0, uint32_t& o1) {
-  const uint32_t sel = w & 0x7777u;
-  // |value| as bf16: high bytes {00,3F,3F,3F,40,40,40,40}, low {00,00,80,C0,00,40,80,C0}
-  const uint32_t sgn = __byte_perm(0u, 0x80808080u, (w >> 1) & 0x4444u);
-  const uint32_t hi = __byte_perm(0x3F3F3F00u, 0x40404040u, sel) | sgn;
-  const uint32_t lo = __byte_perm(0xC0800000u, 0xC0804000u, sel);
-  o0 = __byte_perm(lo, hi, 0x5140u);
-  o1 = __byte_perm(lo, hi, 0x7362u);
+// 8 E2M1 codes (one 32-bit word; byte b holds K elements 2b (low nibble) and 2b + 1) -> 4
+// words of f16 pairs, the lower K element in the low half
+__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t& o0, uint32_t& o1, uint32_t& o2,
+                                                uint32_t& o3) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(o0), "=r"(o1), "=r"(o2), "=r"(o3)
+      : "r"(w));
 }
 
-__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
-  __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162*>(&a);
-  __nv_bfloat162 y = *reinterpret_cast<__nv_bfloat162*>(&b);
-  __nv_bfloat162 r = __hmul2(x, y);
-  return *reinterpret_cast<uint32_t*>(&r);
+// two E4M3 bytes (the low 16 bits of v, byte 0 first) -> f16 pair, byte 0 in the low half
+// (exact: E4M3 values have 4 significant bits and lie in 2^-9 .. 448; S.1111.111 -> NaN)
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t v) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, lo;\n\t}" : "=r"(r) : "r"(v));
+  return r;
 }
 
-// E4M3 byte -> bf16 bits (exact: at most 4 significant bits, 2^-9 .. 448), S.1111.111 -> NaN
-__device__ __forceinline__ uint32_t e4m3_to_bf16_bits(uint32_t b) {
-  const uint32_t s = (b >> 7) & 1u, e = (b >> 3) & 15u, m = b & 7u;
-  float v;
-  if (e == 15u && m == 7u) {
-    v = __int_as_float(0x7FC00000);
-  } else if (e == 0u) {
-    v = static_cast<float>(m) * 0.001953125f;  // m * 2^-9
-  } else {
-    v = __int_as_float(static_cast<int>(((e + 120u) << 23) | (m << 20)));
-  }
-  return __bfloat16_as_ushort(__float2bfloat16_rn(s ? -v : v));
+__device__ __forceinline__ uint32_t f16x2_mul(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
 }
 
-// One 64-weight row segment (32 code bytes at `codes`, 4 E4M3 scales in `s4`) -> 32 words of
-// bf16 pairs (K elements 2j, 2j+1 in word j), the TMEM column order of the A operand.
-__device__ __forceinline__ void expand_row(const uint8_t* codes, uint32_t s4, const uint16_t* lut,
-                                           uint32_t (&out)[32]) {
+// One 64-weight row segment (32 code bytes at `codes`, its 4 E4M3 block scales in s4, the
+// first in the low byte) -> 32 words of f16 pairs (K elements 2j, 2j+1 in word j), the TMEM
+// column order of the A operand.
+__device__ __forceinline__ void expand_row(const uint8_t* codes, uint32_t s4, uint32_t (&out)[32]) {
   const uint4 c0 = *reinterpret_cast<const uint4*>(codes);
   const uint4 c1 = *reinterpret_cast<const uint4*>(codes + 16);
   const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+  const uint32_t s01 = e4m3x2_to_f16x2(s4), s23 = e4m3x2_to_f16x2(s4 >> 16);
+  // each block scale in both halves of a word: blocks of 16 weights = 2 code words
+  const uint32_t sc[4] = {__byte_perm(s01, 0u, 0x1010u), __byte_perm(s01, 0u, 0x3232u), __byte_perm(s23, 0u, 0x1010u),
+                          __byte_perm(s23, 0u, 0x3232u)};
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const uint32_t sb = lut[(s4 >> (8 * (i >> 1))) & 0xFFu];   // one scale per 16 weights
-    const uint32_t s2 = sb | (sb << 16);
-    uint32_t a0, a1, b0, b1;
-    e2m1x4_to_bf16(words[i], a0, a1);
-    e2m1x4_to_bf16(words[i] >> 16, b0, b1);
-    out[4 * i + 0] = bf16x2_mul(a0, s2);
-    out[4 * i + 1] = bf16x2_mul(a1, s2);
-    out[4 * i + 2] = bf16x2_mul(b0, s2);
-    out[4 * i + 3] = bf16x2_mul(b1, s2);
+    uint32_t a0, a1, a2, a3;
+    e2m1x8_to_f16x2(words[i], a0, a1, a2, a3);
+    out[4 * i + 0] = f16x2_mul(a0, sc[i >> 1]);
+    out[4 * i + 1] = f16x2_mul(a1, sc[i >> 1]);
+    out[4 * i + 2] = f16x2_mul(a2, sc[i >> 1]);
+    out[4 * i + 3] = f16x2_mul(a3, sc[i >> 1]);
   }
+}
+
+// f32 -> f16, round to nearest even, saturating at +-65504 (the h the down projection reads)
+__device__ __forceinline__ __half f32_to_f16_sat(float v) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.f16.f32 %0, %1;" : "=h"(r) : "f"(v));
+  return __ushort_as_half(r);
 }
 
 template <int BN, int EPI, int MT>
@@ -127,8 +134,7 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr int kConv = S::kConvSlots;
-  uint16_t* lut = reinterpret_cast<uint16_t*>(smem + kStages * S::kStageBytes);  // 256 x bf16
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * S::kStageBytes + 512);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * S::kStageBytes);
   // bars: full[kStages], empty[kStages], conv[kConv], cfree[kConv], acc_full[2], acc_empty[2]
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 2 * kConv + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
@@ -147,7 +153,6 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
   // TMEM column of converted weight tile m of slot c
   auto conv_col = [&](int c, int m) { return S::kConvCol0 + static_cast<uint32_t>(c) * S::kConvCols + 32u * m; };
 
-  for (int i = threadIdx.x; i < 256; i += blockDim.x) lut[i] = static_cast<uint16_t>(e4m3_to_bf16_bits(i));
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(full_bar(s), 1);
@@ -236,7 +241,7 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
         int g, m0, row0, n;
         gemm_tile(p, t, BN, g, m0, row0, n);
         const uint32_t N = static_cast<uint32_t>((n + 15) & ~15);
-        const uint32_t idesc = idesc_f32acc(1u, 128u, N);
+        const uint32_t idesc = idesc_f32acc(0u, 128u, N);  // f16 A (TMEM) and B (shared memory)
         if (!mbar_wait(acce_bar(acc), acc_phase ^ 1u, abort_flag, p.status, 0xA00u + acc)) {
           ok = false;
           break;
@@ -317,6 +322,18 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
         };
         uint32_t cur[8], nxt[8];
         load8(0, cur);
+        // k-block j: expand into v, then finish k-block j - 1 (wait for its TMEM store, hand
+        // its slot to the UMMA), then store k-block j -- the store's latency overlaps the next
+        // expansion. pend: a store issued and not yet handed over, into slot pend_cs.
+        bool pend = false;
+        int pend_cs = 0;
+        auto hand_over = [&]() {
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(conv_bar(pend_cs));
+          pend = false;
+        };
         for (int kb0 = 0; ok && kb0 < p.k_blocks; kb0 += 8) {
           if (kb0 + 8 < p.k_blocks) load8(kb0 + 8, nxt);
 #pragma unroll
@@ -330,12 +347,11 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
               } else {
                 tc_fence_after();
                 uint32_t v[32];
-                expand_row(code_tile(stage, mat) + r * 32, cur[j], lut, v);
+                expand_row(code_tile(stage, mat) + r * 32, cur[j], v);
+                if (pend) hand_over();
                 tmem_st32(lane_base + conv_col(cs, mat), v);
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(conv_bar(cs));
+                pend = true;
+                pend_cs = cs;
                 if (++stage == kStages) {
                   stage = 0;
                   phase ^= 1u;
@@ -351,6 +367,7 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
 #pragma unroll
           for (int j = 0; j < 8; ++j) cur[j] = nxt[j];
         }
+        if (pend) hand_over();  // the tile's last k-block (also on the abort path: the store is in flight)
       }
     }
   } else {
@@ -370,9 +387,11 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
       const int nchunks = (n + 31) >> 5;
       const float ms_a = q4.mscale_a[g];
       if constexpr (EPI == EPI_SWIGLU) {
+        // h = SiLU(gate) * up, written as f16 (the down projection's f16 token operand)
         const float ms_u = q4.mscale_a2[g];
         const int f = m0 + q * 32 + lane;
         const bool f_ok = f < p.m_valid;
+        __half* hout = reinterpret_cast<__half*>(p.out);
         for (int c = 0; c < nchunks; ++c) {
           uint32_t v[32], u[32];
           tmem_ld32(taddr + 32u * c, v);
@@ -381,9 +400,8 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const int tok = c * 32 + i;
-            const float a = __uint_as_float(v[i]) * ms_a;
-            const float h = __fdividef(a, 1.0f + __expf(-a)) * (__uint_as_float(u[i]) * ms_u);
-            if (tok < n && f_ok) out[(static_cast<int64_t>(row0) + tok) * p.ld_out + f] = from_f32<TOut>(h);
+            const float h = silu_tanh(__uint_as_float(v[i]) * ms_a) * (__uint_as_float(u[i]) * ms_u);
+            if (tok < n && f_ok) hout[(static_cast<int64_t>(row0) + tok) * p.ld_out + f] = f32_to_f16_sat(h);
           }
         }
       } else {

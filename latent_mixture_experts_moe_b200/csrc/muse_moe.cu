@@ -37,10 +37,14 @@ int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // ---------------------------------------------------------------------- tile sizing
 // tokens per grouped-GEMM tile: small tiles when experts see few tokens (decode)
 bool w4a4(const muse_moe_config& c) { return c.act_format == MUSE_ACT_NVFP4; }
+#ifndef MUSE_NVFP4_TILE_TOKENS
+#define MUSE_NVFP4_TILE_TOKENS 192  // W4A16 prefill tiles: 128 or 192 tokens
+#endif
 int grouped_bn(const muse_moe_config& c) {
   if ((c.T * c.top_k) <= 32 * c.E) return 32;
-  if (w4a4(c)) return 128;                                    // W4A4: accumulators leave TMEM room for scales
-  return c.expert_weights == MUSE_EXPERTS_NVFP4 ? 192 : 256;  // NVFP4: accumulators leave TMEM room for weights
+  if (w4a4(c)) return 128;  // W4A4: accumulators leave TMEM room for scales
+  // NVFP4 weights: accumulators leave TMEM room for converted weight slots
+  return c.expert_weights == MUSE_EXPERTS_NVFP4 ? MUSE_NVFP4_TILE_TOKENS : 256;
 }
 int dense_bn(const muse_moe_config& c) { return c.T <= 32 ? 32 : 256; }
 
@@ -272,18 +276,23 @@ cudaError_t launch_gemm_fp4_t(const TmaMaps& maps, const GemmArgs& args, const F
   return cudaGetLastError();
 }
 
+template <int BN, int EPI>
+cudaError_t launch_gemm_fp4_bn(int mt, const TmaMaps& maps, const GemmArgs& args, const Fp4Args& q4, int grid,
+                               cudaStream_t st) {
+  if constexpr (EPI == EPI_SWIGLU) {
+    return launch_gemm_fp4_t<BN, EPI, 2>(maps, args, q4, grid, st);
+  } else {
+    return mt == 2 ? launch_gemm_fp4_t<BN, EPI, 2>(maps, args, q4, grid, st)
+                   : launch_gemm_fp4_t<BN, EPI, 1>(maps, args, q4, grid, st);
+  }
+}
+
 template <int EPI>
 cudaError_t launch_gemm_fp4(int bn, int mt, const TmaMaps& maps, const GemmArgs& args, const Fp4Args& q4, int grid,
                             cudaStream_t st) {
-  if constexpr (EPI == EPI_SWIGLU) {
-    return bn == 32 ? launch_gemm_fp4_t<32, EPI, 2>(maps, args, q4, grid, st)
-                    : launch_gemm_fp4_t<192, EPI, 2>(maps, args, q4, grid, st);
-  } else {
-    if (bn == 32) return mt == 2 ? launch_gemm_fp4_t<32, EPI, 2>(maps, args, q4, grid, st)
-                                 : launch_gemm_fp4_t<32, EPI, 1>(maps, args, q4, grid, st);
-    return mt == 2 ? launch_gemm_fp4_t<192, EPI, 2>(maps, args, q4, grid, st)
-                   : launch_gemm_fp4_t<192, EPI, 1>(maps, args, q4, grid, st);
-  }
+  if (bn == 32) return launch_gemm_fp4_bn<32, EPI>(mt, maps, args, q4, grid, st);
+  if (bn == 128) return launch_gemm_fp4_bn<128, EPI>(mt, maps, args, q4, grid, st);
+  return launch_gemm_fp4_bn<192, EPI>(mt, maps, args, q4, grid, st);
 }
 
 template <int BN, int EPI>
@@ -641,8 +650,14 @@ muse_status experts(Pass<T>& p, const T* zsrc, int64_t nsrc, const void* W_gate,
   } else {
     const int vpr = static_cast<int>(L * sizeof(T) / 16);
     const int rows_grid = static_cast<int>(std::min<int64_t>(lay.pub.rows, 16 * nsm));
-    k_gather_rows<<<rows_grid, 128, 0, st>>>(p.row_token, p.offsets + E, reinterpret_cast<const uint4*>(zsrc),
-                                            reinterpret_cast<uint4*>(zp), vpr);
+    // NVFP4 weights with bf16 activations (W4A16): the expert GEMMs' operands are f16, so the
+    // gathered rows are converted on the way (zp and h then hold f16)
+    if (c.expert_weights == MUSE_EXPERTS_NVFP4)
+      k_gather_rows<true><<<rows_grid, 128, 0, st>>>(p.row_token, p.offsets + E, reinterpret_cast<const uint4*>(zsrc),
+                                                     reinterpret_cast<uint4*>(zp), vpr);
+    else
+      k_gather_rows<false><<<rows_grid, 128, 0, st>>>(p.row_token, p.offsets + E, reinterpret_cast<const uint4*>(zsrc),
+                                                      reinterpret_cast<uint4*>(zp), vpr);
     MUSE_CK(cudaGetLastError());
     MUSE_CK(p.mark());
   }

@@ -381,10 +381,26 @@ __global__ void __launch_bounds__(kFinishThreads) k_ffn_finish(
   }
 }
 
+// bf16 -> f16, two or eight values at a time (round to nearest even, saturating): exact for
+// magnitudes 2^-14 .. 65504 (f16's normal range holds every 8-bit bf16 significand);
+// smaller values round to f16's subnormal grid of 2^-24, larger ones saturate at +-65504.
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
+  const float lo = __uint_as_float(v << 16), hi = __uint_as_float(v & 0xFFFF0000u);
+  uint32_t r;
+  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v) {
+  return make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z), bf16x2_to_f16x2(v.w));
+}
+
 // --------------------------------------------------------------------------------------
 // (a3) gather: Zp[row] = z[row_token[row]] (zeros for padding rows), 16-byte vectors;
 // one block per row (grid-strided), every thread moving several independent vectors.
+// kToF16: the rows are converted from bf16 to f16 on the way (the NVFP4-weight W4A16
+// path, whose tensor-core operands are f16).
 // --------------------------------------------------------------------------------------
+template <bool kToF16 = false>
 __global__ void k_gather_rows(const int* __restrict__ row_token, const int* __restrict__ total_rows,
                               const uint4* __restrict__ z, uint4* __restrict__ zp, int vec_per_row) {
   const int R = *total_rows;
@@ -393,7 +409,11 @@ __global__ void k_gather_rows(const int* __restrict__ row_token, const int* __re
     uint4* dst = zp + static_cast<int64_t>(r) * vec_per_row;
     if (tok >= 0) {
       const uint4* src = z + static_cast<int64_t>(tok) * vec_per_row;
-      for (int c = threadIdx.x; c < vec_per_row; c += blockDim.x) dst[c] = src[c];
+      for (int c = threadIdx.x; c < vec_per_row; c += blockDim.x) {
+        uint4 v = src[c];
+        if constexpr (kToF16) v = bf16x8_to_f16x8(v);
+        dst[c] = v;
+      }
     } else {
       for (int c = threadIdx.x; c < vec_per_row; c += blockDim.x) dst[c] = make_uint4(0, 0, 0, 0);
     }
