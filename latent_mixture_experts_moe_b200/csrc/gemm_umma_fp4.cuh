@@ -19,11 +19,12 @@
 // Roles (448 threads, one CTA per SM): warp 0 TMA producer (codes + token tile, a deep ring:
 // 4-bit stages are small), warp 1 TMEM owner + UMMA issuer, warps 2..5 epilogue, warps 6..13
 // converters (warp w expands weight rows 32*(w%4) .. +31 -- the TMEM lanes it may write -- of
-// tile (w-6)/4; block scales read from global memory 8 k-blocks at a time). A converter warp
-// issues the TMEM store of k-block j, expands k-block j+1 into registers, and only then waits
-// for the store and hands slot j to the UMMA, so each store's latency hides behind the next
-// expansion. TMEM columns: accumulators from 0, converted weight slots (32 * MT columns each)
-// after them. Barriers: per TMA stage full (bytes) / empty (UMMA commit); per converted slot
+// tile (w-6)/4; block scales read from global memory 8 k-blocks at a time). With four
+// converted slots (decode-sized tiles) a converter warp issues the TMEM store of k-block j,
+// expands k-block j+1, and only then waits for the store and hands slot j to the UMMA, so
+// each store's latency hides behind the next expansion; with two (prefill tiles) it hands
+// each slot over as soon as its store completes. TMEM columns: accumulators from 0,
+// converted weight slots (32 * MT columns each) after them. Barriers: per TMA stage full (bytes) / empty (UMMA commit); per converted slot
 // conv (converter warps) / cfree (UMMA commit). Every wait is bounded (ptx.cuh).
 #pragma once
 
@@ -56,6 +57,12 @@ struct Fp4Shape {
   static constexpr uint32_t kConvCol0 = kAccCols * kAccStages;
   static constexpr int kConvFit = static_cast<int>((kTmemCols - kConvCol0) / kConvCols);
   static constexpr int kConvSlots = kConvFit > 4 ? 4 : kConvFit;
+  // With 4 slots a converter warp hands slot j to the UMMA only after expanding k-block
+  // j + 1, so the TMEM store's latency hides behind that expansion. With 2 slots (192-token
+  // tiles) it hands each slot over as soon as its store completes: a late hand-over would
+  // leave the UMMA one expansion behind with no other slot to work on (measured: the T=4096
+  // NVFP4 step 5.37 -> 4.70 ms with the early hand-over there).
+  static constexpr bool kLateHandOver = kConvSlots >= 4;
   static constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes + 1024;
   static_assert(kConvSlots >= 2, "no TMEM room for converted weight tiles");
   static_assert(kStages >= 2, "tile too large for the shared-memory ring");
@@ -322,9 +329,9 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
         };
         uint32_t cur[8], nxt[8];
         load8(0, cur);
-        // k-block j: expand into v, then finish k-block j - 1 (wait for its TMEM store, hand
-        // its slot to the UMMA), then store k-block j -- the store's latency overlaps the next
-        // expansion. pend: a store issued and not yet handed over, into slot pend_cs.
+        // k-block j: expand into v, then (late hand-over) finish k-block j - 1 -- wait for its
+        // TMEM store, hand its slot to the UMMA -- then store k-block j; with the early
+        // hand-over the store is finished right away. pend: a store not yet handed over.
         bool pend = false;
         int pend_cs = 0;
         auto hand_over = [&]() {
@@ -352,6 +359,7 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
                 tmem_st32(lane_base + conv_col(cs, mat), v);
                 pend = true;
                 pend_cs = cs;
+                if (!S::kLateHandOver) hand_over();
                 if (++stage == kStages) {
                   stage = 0;
                   phase ^= 1u;
