@@ -158,12 +158,15 @@ def step_work(w: W.Workload, n_touched: int):
 
 
 def at_full_clock(clk) -> bool:
-    """True when the timed region ran at the GPU's maximum SM clock (median of the samples
-    taken during it within 3%, no power-cap reason): the burst GEMM peak, measured at that
-    clock, is then the tensor roofline; otherwise the sustained (power-capped) peak is."""
+    """True when the timed region ran at the GPU's maximum SM clock with no power-cap
+    throttling sampled (median within 3% of max, sw_power_cap never active): the burst GEMM
+    peak, measured at that clock, is then the tensor roofline. Otherwise the sustained peak
+    (measured under the 1 kW power cap) is: clock counters read inside the expert GEMMs show
+    that under the cap their SM clock falls to ~1.3 GHz even when 100 ms nvidia-smi samples
+    mostly report the maximum."""
     if not clk or not clk.get("sm_mhz") or not clk.get("sm_max_mhz"):
         return False
-    return clk["sm_mhz"] >= 0.97 * clk["sm_max_mhz"]
+    return clk["sm_mhz"] >= 0.97 * clk["sm_max_mhz"] and "sw_power_cap" not in clk.get("reasons", [])
 
 
 def roofline(w: W.Workload, kernel: str, fl: float, by: float, t: float, peaks, tensor_peak: float, burst: bool):
