@@ -261,6 +261,9 @@ cudaError_t launch_gemm_bn(int bn, int mt, const TmaMaps& maps, const GemmArgs& 
   } else {
     if (bn == 32) return mt == 2 ? launch_gemm<TIn, TOut, 32, EPI, 2>(maps, args, grid, st)
                                  : launch_gemm<TIn, TOut, 32, EPI, 1>(maps, args, grid, st);
+    if constexpr (EPI == EPI_STORE) {
+      if (bn == 128) return launch_gemm<TIn, TOut, 128, EPI, 1>(maps, args, grid, st);
+    }
     return mt == 2 ? launch_gemm<TIn, TOut, 256, EPI, 2>(maps, args, grid, st)
                    : launch_gemm<TIn, TOut, 256, EPI, 1>(maps, args, grid, st);
   }
@@ -415,6 +418,9 @@ muse_status dense_gemm(const void* W, int64_t M, const void* X, int64_t T, int64
   const int mt = (cdiv(M, 256) * cdiv(T, bn) >= nsm) ? 2 : 1;
   g.m_step = 128 * mt;
   g.m_tiles = static_cast<int>(cdiv(M, g.m_step));
+  // 128-token tiles when 256-token ones would fill at most half the SMs (the router: E = 256
+  // features x T / 256 token tiles)
+  if (EPI == EPI_STORE && bn == 256 && mt == 1 && 2 * g.m_tiles * cdiv(T, 256) <= nsm) bn = 128;
   g.num_tiles = static_cast<int>(g.m_tiles * cdiv(T, bn));
   // K split into S equal ranges while the tiles of all ranges still fit one wave: each
   // range writes its FP32 partial product, k_splitk_reduce sums them in range order
@@ -549,10 +555,16 @@ muse_status route(Pass<T>& p, const void* x, const void* W_router, const void** 
     MUSE_CK(cudaGetLastError());
   }
   MUSE_CK(p.mark());
-  k_topk<<<static_cast<unsigned>(cdiv(Tn * 32, 256)), 256, 0, p.st>>>(
-      logits, static_cast<int>(Tn), static_cast<int>(E), static_cast<int>(k), c.router_bias, c.router_mode,
-      c.router_logit_scale, c.routed_scaling, p.topk_idx, p.topk_w, c.topk_idx_out, c.topk_w_out);
-  MUSE_CK(cudaGetLastError());
+  {
+    // key slots per lane: E / 32 rounded up to a power of two (E <= 1024)
+    const int npl = E <= 32 ? 1 : E <= 64 ? 2 : E <= 128 ? 4 : E <= 256 ? 8 : E <= 512 ? 16 : 32;
+    auto kern = npl == 1 ? k_topk<1> : npl == 2 ? k_topk<2> : npl == 4 ? k_topk<4> : npl == 8 ? k_topk<8>
+              : npl == 16 ? k_topk<16> : k_topk<32>;
+    kern<<<static_cast<unsigned>(cdiv(Tn * 32, 256)), 256, 0, p.st>>>(
+        logits, static_cast<int>(Tn), static_cast<int>(E), static_cast<int>(k), c.router_bias, c.router_mode,
+        c.router_logit_scale, c.routed_scaling, p.topk_idx, p.topk_w, c.topk_idx_out, c.topk_w_out);
+    MUSE_CK(cudaGetLastError());
+  }
   MUSE_CK(p.mark());
   return MUSE_OK;
 }

@@ -81,6 +81,8 @@ __global__ void k_router_logits_f32(const float* __restrict__ x, const float* __
 //   softmax: g_j = exp(l_j - m) / sum_S exp(l - m)  (softmax over E renormalised on S)
 //   sigmoid: g_j = rsf * s_j / (sum_S s + 1e-15)
 // --------------------------------------------------------------------------------------
+// NPL: key slots per lane (E <= 32 * NPL; NPL a power of two up to 32).
+template <int NPL>
 __global__ void k_topk(const float* __restrict__ logits, int T, int E, int k,
                        const float* __restrict__ bias, int mode, float scale, float rsf,
                        int* __restrict__ idx_out, float* __restrict__ w_out,
@@ -89,22 +91,17 @@ __global__ void k_topk(const float* __restrict__ logits, int T, int E, int k,
   const int lane = threadIdx.x & 31;
   if (t >= T) return;  // warp-uniform
   const float* l = logits + static_cast<int64_t>(t) * E;
-  const int npl = (E + 31) >> 5;
-  float key[32];
+  float key[NPL];
   uint32_t taken = 0;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
+  for (int i = 0; i < NPL; ++i) {
     key[i] = neg_inf();
-    if (i < npl) {
-      const int e = lane + 32 * i;
-      if (e < E) {
-        const float li = l[e];
-        float kv = (mode == 0) ? li : 1.0f / (1.0f + expf(-scale * li));
-        if (bias != nullptr) kv += bias[e];
-        key[i] = (kv == kv) ? kv : neg_inf();  // a NaN key never wins over a number
-      } else {
-        taken |= 1u << i;
-      }
+    const int e = lane + 32 * i;
+    if (e < E) {
+      const float li = l[e];
+      float kv = (mode == 0) ? li : 1.0f / (1.0f + expf(-scale * li));
+      if (bias != nullptr) kv += bias[e];
+      key[i] = (kv == kv) ? kv : neg_inf();  // a NaN key never wins over a number
     } else {
       taken |= 1u << i;
     }
@@ -114,7 +111,7 @@ __global__ void k_topk(const float* __restrict__ logits, int T, int E, int k,
     float bk = neg_inf();
     int bi = 0x7fffffff;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
+    for (int i = 0; i < NPL; ++i) {
       const int e = lane + 32 * i;
       if (!((taken >> i) & 1u) && (key[i] > bk || (key[i] == bk && e < bi))) {
         bk = key[i];
@@ -222,22 +219,37 @@ __global__ void k_build_tiles(const int* __restrict__ counts, int E, int BN, int
 __global__ void k_assign_rows(const int* __restrict__ idx, int n, int k, const int* __restrict__ counts,
                               const int* __restrict__ offsets, int* __restrict__ inv,
                               int* __restrict__ row_token) {
+  // Warp w owns the contiguous segment [w * seg, (w + 1) * seg) of the assignments (seg a
+  // multiple of 32). Pass 1 counts the segment's assignments to this expert with ballots;
+  // an exclusive scan over the warps gives each segment's first rank; pass 2 walks the
+  // segment again and numbers the matches in order (rank = first + matches before it).
+  __shared__ int seg_count[32];
   const int e = blockIdx.x;
   const int cnt = counts[e];
   if (cnt == 0) return;  // block-uniform
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int seg = ((n + nw - 1) / nw + 31) & ~31;
+  const int a0 = w * seg, a1 = min(n, a0 + seg);
+  int mine = 0;
+  for (int a = a0 + lane; a - lane < a1; a += 32) {
+    const bool hit = a < a1 && idx[a] == e;
+    mine += __popc(__ballot_sync(0xffffffffu, hit));
+  }
+  if (lane == 0) seg_count[w] = mine;
+  __syncthreads();
+  int first = 0;
+  for (int i = 0; i < w; ++i) first += seg_count[i];
   const int base_row = offsets[e];
-  int found = 0;
-  for (int a0 = 0; a0 < n && found < cnt; a0 += blockDim.x) {
-    const int a = a0 + threadIdx.x;
-    const int flag = (a < n && idx[a] == e) ? 1 : 0;
-    int tot;
-    const int rank = found + block_exclusive_scan(flag, &tot);
-    if (flag) {
-      const int row = base_row + rank;
+  const unsigned below = (1u << lane) - 1u;
+  for (int a = a0 + lane; a - lane < a1; a += 32) {
+    const bool hit = a < a1 && idx[a] == e;
+    const unsigned b = __ballot_sync(0xffffffffu, hit);
+    if (hit) {
+      const int row = base_row + first + __popc(b & below);
       inv[a] = row;
       row_token[row] = a / k;
     }
-    found += tot;
+    first += __popc(b);
   }
 }
 
@@ -403,16 +415,29 @@ __device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v) {
 template <bool kToF16 = false>
 __global__ void k_gather_rows(const int* __restrict__ row_token, const int* __restrict__ total_rows,
                               const uint4* __restrict__ z, uint4* __restrict__ zp, int vec_per_row) {
+  // (z and zp never overlap)
   const int R = *total_rows;
   for (int r = blockIdx.x; r < R; r += gridDim.x) {
     const int tok = row_token[r];
     uint4* dst = zp + static_cast<int64_t>(r) * vec_per_row;
     if (tok >= 0) {
       const uint4* src = z + static_cast<int64_t>(tok) * vec_per_row;
-      for (int c = threadIdx.x; c < vec_per_row; c += blockDim.x) {
-        uint4 v = src[c];
-        if constexpr (kToF16) v = bf16x8_to_f16x8(v);
-        dst[c] = v;
+      // four vectors in flight per thread: all loads issued before the stores
+      for (int c0 = threadIdx.x; c0 < vec_per_row; c0 += 4 * blockDim.x) {
+        uint4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int c = c0 + u * blockDim.x;
+          if (c < vec_per_row) v[u] = src[c];
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int c = c0 + u * blockDim.x;
+          if (c < vec_per_row) {
+            if constexpr (kToF16) v[u] = bf16x8_to_f16x8(v[u]);
+            dst[c] = v[u];
+          }
+        }
       }
     } else {
       for (int c = threadIdx.x; c < vec_per_row; c += blockDim.x) dst[c] = make_uint4(0, 0, 0, 0);
