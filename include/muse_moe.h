@@ -395,14 +395,16 @@ MUSE_API muse_status muse_ep_combine(const muse_moe_config* cfg, int32_t ep_size
 /* Static string for a status code. */
 MUSE_API const char* muse_status_string(muse_status s);
 
-/* Number of stages one forward call runs for cfg -- the positions of stage_events: 11, plus
- * one each for the pre-expert norm, the pre-FFN norm, the post-FFN norm / residual gate (one
- * kernel finishes both) and two for W4A4. In order: [ffn pre norm], router, top-k, histogram,
- * tiles, assign rows, pooler, [pre-expert norm], [W4A4: quantise z], gather (W4A4: of the
- * quantised bytes), gate/up, [W4A4: quantise h], down, norm + combine, unpooler, [post norm /
- * gate]. Each stage is one kernel, except that a dense GEMM (router, pooler, unpooler) whose
- * tiles would fill less than half the SMs splits K and adds a partial-sum kernel inside its
- * stage (decode-sized token counts). stage_events must hold this many + 1 events. */
+/* Number of stages one forward call runs for cfg -- the positions of stage_events -- and
+ * the name of stage i (a static string; NULL past the last). In order: [ffn_pre_norm],
+ * router, topk, expert_hist, tiles, assign_rows, pooler, [pre_expert_norm], gather (with
+ * W4A4 activations: quant_z, gather_codes), gate_up_swiglu, [quant_h (W4A4)], down_sumsq,
+ * norm_combine, unpooler, [ffn_post_norm_gate]. Each stage is
+ * one kernel, except that a dense GEMM (router, pooler, unpooler) whose tiles would fill
+ * less than half the SMs splits K and adds a partial-sum kernel inside its stage
+ * (decode-sized token counts). stage_events must hold launch_count + 1 events. -1 / NULL
+ * for an invalid cfg. */
+MUSE_API const char* muse_latent_moe_stage_name(const muse_moe_config* cfg, int32_t i);
 MUSE_API int32_t muse_latent_moe_launch_count(const muse_moe_config* cfg);
 
 #ifdef __cplusplus

@@ -29,7 +29,7 @@ EXPORTS = ("muse_moe_config_init", "muse_latent_moe_workspace_size", "muse_laten
            "muse_status_string", "muse_latent_moe_launch_count", "muse_latent_moe_forward_static_scratch",
            "muse_selftest_bounded_wait", "muse_quantize_nvfp4_rows", "muse_latent_moe_forward_host_batches",
            "muse_ep_workspace_layout", "muse_ep_dispatch", "muse_ep_experts", "muse_ep_combine",
-           "muse_latent_moe_forward_checked")
+           "muse_latent_moe_forward_checked", "muse_latent_moe_stage_name")
 
 # roles of an expert-parallel workspace (muse_ep_role)
 EP_HOME, EP_EXPERTS = 1, 2
@@ -136,6 +136,8 @@ def lib() -> ctypes.CDLL:
         L.muse_ep_combine.restype = ctypes.c_int
         L.muse_latent_moe_forward_checked.argtypes = [cp] + [ctypes.POINTER(Tensor)] * 9 + [vp]
         L.muse_latent_moe_forward_checked.restype = ctypes.c_int
+        L.muse_latent_moe_stage_name.argtypes = [cp, ctypes.c_int32]
+        L.muse_latent_moe_stage_name.restype = ctypes.c_char_p
         L.muse_latent_moe_launch_count.argtypes = [cp]
         L.muse_latent_moe_launch_count.restype = ctypes.c_int32
         _lib = L
@@ -296,25 +298,15 @@ def ep_combine(cfg: Config, ep_size: int, x, back_y, back_ss, gamma, W_unpool, o
                                  _ptr(W_unpool), _ptr(out), _stream_handle(stream)), "muse_ep_combine")
 
 
-STAGES = ("router", "topk", "expert_hist", "tiles", "assign_rows", "pooler", "gather", "gate_up_swiglu",
-          "down_sumsq", "norm_combine", "unpooler")
-
-
 def stages(cfg: Config):
-    """Names of the kernels one forward launches for cfg, in launch order (STAGES plus the
-    optional sublayer pre-norm, pre-expert norm and sublayer post-norm / residual gate)."""
-    names = list(STAGES)
-    if cfg.pre_norm_gain:
-        names.insert(names.index("gather"), "pre_expert_norm")
-    if cfg.act_format == ACT_NVFP4:
-        names[names.index("gather")] = "gather_codes"
-        names.insert(names.index("gather_codes"), "quant_z")
-        names.insert(names.index("gate_up_swiglu") + 1, "quant_h")
-    if cfg.ffn_pre_gain:
-        names.insert(0, "ffn_pre_norm")
-    if cfg.ffn_post_gain or cfg.residual_gate:
-        names.append("ffn_post_norm_gate")
-    return tuple(names)
+    """Names of the stages one forward launches for cfg, in launch order (from the library:
+    muse_latent_moe_stage_name)."""
+    names = []
+    while True:
+        n = lib().muse_latent_moe_stage_name(ctypes.byref(cfg), len(names))
+        if n is None:
+            return tuple(names)
+        names.append(n.decode())
 
 
 def event_handles(events) -> "ctypes.Array":

@@ -1340,11 +1340,37 @@ const char* muse_status_string(muse_status s) {
 
 int32_t muse_latent_moe_launch_count(const muse_moe_config* cfg) {
   if (validate_sizes(cfg) != MUSE_OK) return -1;
-  // router, top-k, hist, tiles, rows, pooler, gather, gate/up, down, combine, unpooler,
-  // and the optional sublayer pre-norm (first), pre-expert norm (between pooler and
-  // gather) and sublayer post-norm / residual gate (last)
-  return 11 + (cfg->pre_norm_gain != nullptr) + (cfg->ffn_pre_gain != nullptr) +
-         (cfg->ffn_post_gain != nullptr || cfg->residual_gate != nullptr) + 2 * (cfg->act_format == MUSE_ACT_NVFP4);
+  int32_t n = 0;
+  while (muse_latent_moe_stage_name(cfg, n) != nullptr) ++n;
+  return n;
+}
+
+const char* muse_latent_moe_stage_name(const muse_moe_config* cfg, int32_t i) {
+  if (validate_sizes(cfg) != MUSE_OK || i < 0) return nullptr;
+  const muse_moe_config& c = *cfg;
+  const char* names[20];
+  int n = 0;
+  if (c.ffn_pre_gain != nullptr) names[n++] = "ffn_pre_norm";
+  names[n++] = "router";
+  names[n++] = "topk";
+  names[n++] = "expert_hist";
+  names[n++] = "tiles";
+  names[n++] = "assign_rows";
+  names[n++] = "pooler";
+  if (c.pre_norm_gain != nullptr) names[n++] = "pre_expert_norm";
+  if (w4a4(c)) {
+    names[n++] = "quant_z";
+    names[n++] = "gather_codes";
+  } else {
+    names[n++] = "gather";
+  }
+  names[n++] = "gate_up_swiglu";
+  if (w4a4(c)) names[n++] = "quant_h";
+  names[n++] = "down_sumsq";
+  names[n++] = "norm_combine";
+  names[n++] = "unpooler";
+  if (c.ffn_post_gain != nullptr || c.residual_gate != nullptr) names[n++] = "ffn_post_norm_gate";
+  return i < n ? names[i] : nullptr;
 }
 
 }  // extern "C"

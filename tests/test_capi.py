@@ -79,7 +79,7 @@ def test_workspace_size_and_layout(name):
     assert lay["rows"] >= w.T * w.k and lay["rows"] % 16 == 0
     assert lay["rows"] <= w.T * w.k + 16 * min(w.E, w.T * w.k)
     assert n >= lay["c"] + w.T * w.L * act
-    assert moe.launch_count(cfg) == 11
+    assert moe.launch_count(cfg) == 11 == len(moe.stages(cfg))
 
 
 @pytest.mark.parametrize("field,value,code", [
