@@ -104,9 +104,13 @@ __device__ __forceinline__ uint32_t f16x2_mul(uint32_t a, uint32_t b) {
 // One 64-weight row segment (32 code bytes at `codes`, its 4 E4M3 block scales in s4, the
 // first in the low byte) -> 32 words of f16 pairs (K elements 2j, 2j+1 in word j), the TMEM
 // column order of the A operand.
-__device__ __forceinline__ void expand_row(const uint8_t* codes, uint32_t s4, uint32_t (&out)[32]) {
-  const uint4 c0 = *reinterpret_cast<const uint4*>(codes);
-  const uint4 c1 = *reinterpret_cast<const uint4*>(codes + 16);
+// `flip` (bit 2 of the row): which 16-byte half of the row is read first. Rows are 32 bytes
+// apart, so the 8 lanes of a 16-byte load phase cover 4 rows' worth of banks twice unless
+// lanes 4..7 of each 8 start on the other half -- then every phase is conflict-free.
+__device__ __forceinline__ void expand_row(const uint8_t* codes, uint32_t s4, bool flip, uint32_t (&out)[32]) {
+  const uint4 p = *reinterpret_cast<const uint4*>(codes + (flip ? 16 : 0));
+  const uint4 q = *reinterpret_cast<const uint4*>(codes + (flip ? 0 : 16));
+  const uint4 c0 = flip ? q : p, c1 = flip ? p : q;
   const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
   const uint32_t s01 = e4m3x2_to_f16x2(s4), s23 = e4m3x2_to_f16x2(s4 >> 16);
   // each block scale in both halves of a word: blocks of 16 weights = 2 code words
@@ -354,7 +358,7 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
               } else {
                 tc_fence_after();
                 uint32_t v[32];
-                expand_row(code_tile(stage, mat) + r * 32, cur[j], v);
+                expand_row(code_tile(stage, mat) + r * 32, cur[j], (r & 4) != 0, v);
                 if (pend) hand_over();
                 tmem_st32(lane_base + conv_col(cs, mat), v);
                 pend = true;
