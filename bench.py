@@ -212,9 +212,11 @@ def make_rank_inputs(w: W.Workload, rank: int, dev):
     return inp
 
 
-def time_graph(w: W.Workload, model, inp, out, idx, steps: int, warmup: int, world: int, dev):
+def time_graph(w: W.Workload, model, inp, out, idx, steps: int, warmup: int, world: int, dev, flush_bytes: int = 0):
     """The same forward captured once in a CUDA graph and replayed: CUDA-event time of
-    `steps` replays (max over ranks), no host work between launches."""
+    `steps` replays (max over ranks), no host work between launches. flush_bytes > 0: a
+    buffer that large is overwritten between replays, outside each replay's own events, and
+    the time is the sum of the replays' own durations."""
     import latent_mixture_experts_moe_b200 as moe
     side = torch.cuda.Stream(device=dev)
     side.wait_stream(torch.cuda.current_stream())
@@ -230,14 +232,26 @@ def time_graph(w: W.Workload, model, inp, out, idx, steps: int, warmup: int, wor
     torch.cuda.synchronize()
     barrier(world)
     stream = torch.cuda.current_stream()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for _ in range(steps):
-        graph.replay()
-    t1.record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    ms = all_max(t0.elapsed_time(t1), world, dev)
+    if flush_bytes:
+        flush = torch.empty(flush_bytes // 4, dtype=torch.int32, device=dev)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for i, (a, b_) in enumerate(evs):
+            flush.fill_(i)
+            a.record(stream)
+            graph.replay()
+            b_.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        ms = all_max(sum(a.elapsed_time(b_) for a, b_ in evs), world, dev)
+    else:
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(steps):
+            graph.replay()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        ms = all_max(t0.elapsed_time(t1), world, dev)
     code, detail = moe.last_device_status(model.config(w.T, model.workspace))
     del graph
     if code != 0:
@@ -335,7 +349,7 @@ def run_ours(w: W.Workload, inp, steps: int, warmup: int, rank: int, world: int,
     if e2e_steps > 0:
         res["e2e"] = run_e2e(w, model, inp, e2e_steps, world, dev)
     if graph_steps > 0:
-        res["graph"] = time_graph(w, model, inp, out, idx, graph_steps, warmup, world, dev)
+        res["graph"] = time_graph(w, model, inp, out, idx, graph_steps, warmup, world, dev, flush_bytes)
     return res
 
 
@@ -644,7 +658,8 @@ def main():
             del inp_d
             wm = W.WORKLOADS["mid"]
             inp_m = make_rank_inputs(wm, rank, dev)
-            side["mid"] = run(wm, inp_m, max(args.steps, 50), e2e_steps=0, flush_bytes=256 << 20)
+            side["mid"] = run(wm, inp_m, max(args.steps, 50), e2e_steps=0, flush_bytes=256 << 20,
+                              graph_steps=max(args.steps, 50))
         if rank == 0:
             roof = {k: main_res["roofline"][k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic",
                                                           "kernel", "peak_source")}

@@ -67,6 +67,9 @@ struct GemmArgs {
                              // k-blocks (0 or 1: none); range s writes its FP32 partial
                              // product to (float*)out + s * split_stride
   int64_t split_stride;
+  int m_group;               // dense tiling: weight tiles per group (0: none). Tiles run group by
+                             // group, each group's m-tiles side by side for every token chunk,
+                             // so the weights a wave of CTAs streams stay within the group
 };
 
 // Split-K decode of launch tile t (dense tiling): range s = t / base of base tile t % base,
@@ -142,8 +145,16 @@ __device__ __forceinline__ void gemm_tile(const GemmArgs& p, int t, int BN, int&
     row0 = v.z;
     n = v.w;
   } else {
-    const int mt = t % p.m_tiles;
-    const int ch = t / p.m_tiles;
+    int mt = t % p.m_tiles;
+    int ch = t / p.m_tiles;
+    if (p.m_group > 0 && p.m_group < p.m_tiles) {
+      const int chunks = (p.T + BN - 1) / BN;
+      const int gi = t / (p.m_group * chunks);        // group (the last one may hold fewer m-tiles)
+      const int r = t - gi * p.m_group * chunks;
+      const int gsz = min(p.m_group, p.m_tiles - gi * p.m_group);
+      mt = gi * p.m_group + r % gsz;
+      ch = r / gsz;
+    }
     g = 0;
     m0 = mt * p.m_step;
     row0 = ch * BN;
