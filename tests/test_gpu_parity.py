@@ -470,3 +470,41 @@ def test_full_size_prefill_every_token(name, full_weights):
         target = W.zipf_target_loads(w.T, w.E, w.k).numpy()
         assert loads[0] >= 0.99 * w.T and loads[1] >= 0.99 * w.T   # water-filled ranks 1-2 take ~every token
         assert np.abs(loads - target).sum() / (w.T * w.k) < 0.02
+
+
+# ------------------------------------------------------------------- shape-checked boundary
+def test_checked_entry_point_rejects_bad_tensors_and_matches_the_raw_one(mid):
+    """muse_latent_moe_forward_checked on real device tensors: a weight of the wrong shape, a
+    non-contiguous view and an output overlapping the input are each MUSE_ERR_INVALID_ARG with
+    nothing launched (the output keeps its contents); correct tensors give the raw entry
+    point's output bit for bit."""
+    w, inp = mid
+    model = moe.LatentMoE({k: v for k, v in inp.items() if k != "x"}, T_max=w.T, k=w.k, eps=w.eps)
+    cfg = model.config(w.T, model.workspace)
+    ws = [inp[n] for n in ("W_router", "W_pool", "W_gate", "W_up", "W_down", "gamma", "W_unpool")]
+    ref = torch.empty((w.T, w.D), dtype=torch.bfloat16, device="cuda")
+    moe.forward(cfg, inp["x"], *ws, ref)
+    out = torch.empty_like(ref)
+    moe.forward_checked(cfg, inp["x"], *ws, out)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
+    sentinel = torch.full_like(ref, 7.0)
+    bad_down = inp["W_down"][:, :, : w.I // 2]                      # [E, L, I/2] view: wrong shape
+    bad_pool = inp["W_pool"].t()                                     # transposed view: strides
+    cases = {
+        "W_down shape": (inp["x"], *ws[:4], bad_down.contiguous(), *ws[5:]),
+        "W_pool strides": (inp["x"], ws[0], bad_pool, *ws[2:]),
+        "x rows": (inp["x"][: w.T // 2], *ws),
+    }
+    for name, args in cases.items():
+        o = sentinel.clone()
+        with pytest.raises(moe.MuseError) as e:
+            moe.forward_checked(cfg, *args, o)
+        assert e.value.code == 1, name
+        torch.cuda.synchronize()
+        assert torch.equal(o, sentinel), f"{name}: something was written"
+    # out overlapping x
+    x2 = inp["x"].clone()
+    with pytest.raises(moe.MuseError) as e:
+        moe.forward_checked(cfg, x2, *ws, x2)
+    assert e.value.code == 1
