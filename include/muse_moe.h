@@ -395,6 +395,13 @@ MUSE_API muse_status muse_ep_combine(const muse_moe_config* cfg, int32_t ep_size
 /* Static string for a status code. */
 MUSE_API const char* muse_status_string(muse_status s);
 
+/* The CUDA runtime's description (a static string) of the last CUDA error behind a
+ * MUSE_ERR_CUDA that a call on the calling host thread returned -- e.g. a launch the device
+ * cannot schedule, or an error left by an earlier kernel. "no error" when no CUDA call has
+ * failed on this thread (a tensor-map encoding refused by the driver also returns
+ * MUSE_ERR_CUDA without a CUDA error). */
+MUSE_API const char* muse_last_cuda_error(void);
+
 /* Number of stages one forward call runs for cfg -- the positions of stage_events -- and
  * the name of stage i (a static string; NULL past the last). In order: [ffn_pre_norm],
  * router, topk, expert_hist, tiles, assign_rows, pooler, [pre_expert_norm], gather (with

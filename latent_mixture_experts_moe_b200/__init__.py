@@ -29,7 +29,7 @@ EXPORTS = ("muse_moe_config_init", "muse_latent_moe_workspace_size", "muse_laten
            "muse_status_string", "muse_latent_moe_launch_count", "muse_latent_moe_forward_static_scratch",
            "muse_selftest_bounded_wait", "muse_quantize_nvfp4_rows", "muse_latent_moe_forward_host_batches",
            "muse_ep_workspace_layout", "muse_ep_dispatch", "muse_ep_experts", "muse_ep_combine",
-           "muse_latent_moe_forward_checked", "muse_latent_moe_stage_name")
+           "muse_latent_moe_forward_checked", "muse_latent_moe_stage_name", "muse_last_cuda_error")
 
 # roles of an expert-parallel workspace (muse_ep_role)
 EP_HOME, EP_EXPERTS = 1, 2
@@ -41,7 +41,10 @@ STATIC_SCRATCH_BYTES = 16 << 20
 class MuseError(RuntimeError):
     def __init__(self, code: int, where: str):
         self.code = code
-        super().__init__(f"{where}: {STATUS.get(code, code)} ({status_string(code)})")
+        msg = f"{where}: {STATUS.get(code, code)} ({status_string(code)})"
+        if code == 4:  # MUSE_ERR_CUDA
+            msg += f": {last_cuda_error()}"
+        super().__init__(msg)
 
 
 class Config(ctypes.Structure):
@@ -117,6 +120,8 @@ def lib() -> ctypes.CDLL:
         L.muse_latent_moe_last_device_status.restype = ctypes.c_int
         L.muse_status_string.argtypes = [ctypes.c_int]
         L.muse_status_string.restype = ctypes.c_char_p
+        L.muse_last_cuda_error.argtypes = []
+        L.muse_last_cuda_error.restype = ctypes.c_char_p
         L.muse_latent_moe_forward_static_scratch.argtypes = [cp] + [vp] * 10
         L.muse_latent_moe_forward_static_scratch.restype = ctypes.c_int
         L.muse_selftest_bounded_wait.argtypes = [ctypes.c_uint64, vp, vp]
@@ -146,6 +151,12 @@ def lib() -> ctypes.CDLL:
 
 def status_string(code: int) -> str:
     return lib().muse_status_string(code).decode()
+
+
+def last_cuda_error() -> str:
+    """The CUDA runtime's description of the last CUDA error behind a MUSE_ERR_CUDA on this
+    thread ("no error" when none)."""
+    return lib().muse_last_cuda_error().decode()
 
 
 def _check(code: int, where: str) -> None:

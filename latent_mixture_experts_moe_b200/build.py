@@ -14,7 +14,7 @@ ROOT = os.path.dirname(PKG)
 SRC = os.path.join(PKG, "csrc", "muse_moe.cu")
 LIB = os.path.join(PKG, "libmuse_moe.so")
 KERNEL_SOURCES = ("muse_moe.cu", "gemm_umma.cuh", "gemm_umma_2sm.cuh", "gemm_umma_fp4.cuh", "gemm_umma_w4a4.cuh",
-                  "nvfp4_act.cuh", "route_kernels.cuh", "ptx.cuh")
+                  "gemv_fp4.cuh", "nvfp4_act.cuh", "route_kernels.cuh", "ptx.cuh")
 DEPS = [os.path.join(PKG, "csrc", f) for f in KERNEL_SOURCES] + [os.path.join(ROOT, "include", "muse_moe.h")]
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

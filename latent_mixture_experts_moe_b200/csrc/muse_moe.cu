@@ -23,6 +23,7 @@
 #include "gemm_umma_2sm.cuh"
 #include "gemm_umma_fp4.cuh"
 #include "gemm_umma_w4a4.cuh"
+#include "gemv_fp4.cuh"
 #include "nvfp4_act.cuh"
 #include "route_kernels.cuh"
 
@@ -40,7 +41,15 @@ bool w4a4(const muse_moe_config& c) { return c.act_format == MUSE_ACT_NVFP4; }
 #ifndef MUSE_NVFP4_TILE_TOKENS
 #define MUSE_NVFP4_TILE_TOKENS 192  // W4A16 prefill tiles: 128 or 192 tokens
 #endif
+// NVFP4 weights with 16-bit activations and a few rows per expert (decode): both expert GEMMs
+// run on the register-fed MMA kernel (gemv_fp4.cuh) -- 128 features and at most 16 token
+// rows per tile; K a multiple of its 256-element stage
+bool fp4_gemv(const muse_moe_config& c) {
+  return c.expert_weights == MUSE_EXPERTS_NVFP4 && !w4a4(c) && c.T * c.top_k <= 4 * c.E && c.L % 256 == 0 &&
+         c.I % 256 == 0;
+}
 int grouped_bn(const muse_moe_config& c) {
+  if (fp4_gemv(c)) return 16;
   if ((c.T * c.top_k) <= 32 * c.E) return 32;
   if (w4a4(c)) return 128;  // W4A4: accumulators leave TMEM room for scales
   // NVFP4 weights: accumulators leave TMEM room for converted weight slots
@@ -298,6 +307,27 @@ cudaError_t launch_gemm_fp4(int bn, int mt, const TmaMaps& maps, const GemmArgs&
   return launch_gemm_fp4_bn<192, EPI>(mt, maps, args, q4, grid, st);
 }
 
+// NVFP4 weights, 16-bit activations, decode-sized tiles: the register-fed MMA kernel. Maps:
+// the codes and block scales of one or two weight matrices [rows_w, K] and the activation rows.
+bool make_gemv_maps(GemvMaps* m, const muse_nvfp4_weight* w, const muse_nvfp4_weight* w2, int64_t rows_w,
+                    const void* x, int64_t R, int64_t K) {
+  std::memset(m, 0, sizeof(*m));
+  return make_code_map(&m->codes[0], w->codes, rows_w, K) && make_code_map(&m->codes[1], w2->codes, rows_w, K) &&
+         make_u8_map(&m->scales[0], w->block_scales, rows_w, K / 16, 16, 128, false) &&
+         make_u8_map(&m->scales[1], w2->block_scales, rows_w, K / 16, 16, 128, false) &&
+         make_map(&m->x, x, true, K, R, 16);
+}
+
+template <int EPI>
+cudaError_t launch_gemv_fp4(const GemvMaps& maps, const GemvArgs& args, int grid, cudaStream_t st) {
+  auto kern = k_fp4_gemv<EPI>;
+  const size_t smem = GemvShape<EPI == EPI_SWIGLU ? 2 : 1>::kSmemBytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kGemvThreads, smem, st>>>(maps, args);
+  return cudaGetLastError();
+}
+
 template <int BN, int EPI>
 cudaError_t launch_gemm_w4a4_t(const W4A4Maps& maps, const GemmArgs& args, const W4A4Args& q, int grid,
                                cudaStream_t st) {
@@ -466,6 +496,7 @@ GemmPlan plan_gate_up(const muse_moe_config& c, int bn_g) {
 }
 GemmPlan plan_down(const muse_moe_config& c, int bn_g) {
   if (w4a4(c)) return {false, 2, 256};
+  if (fp4_gemv(c)) return {false, 1, 128};
   if (c.expert_weights == MUSE_EXPERTS_NVFP4) return c.L % 256 == 0 ? GemmPlan{false, 2, 256} : GemmPlan{false, 1, 128};
   if (c.dtype == MUSE_BF16 && bn_g == 256 && c.L % 512 == 0) return {true, 2, 512};
   if (c.dtype == MUSE_BF16 && bn_g == 256 && c.L % 256 == 0) return {true, 1, 256};
@@ -473,9 +504,16 @@ GemmPlan plan_down(const muse_moe_config& c, int bn_g) {
   return {false, 1, 128};
 }
 
-#define MUSE_CK(x)                                 \
-  do {                                             \
-    if ((x) != cudaSuccess) return MUSE_ERR_CUDA;  \
+// the last CUDA error a call of this thread returned MUSE_ERR_CUDA for
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+#define MUSE_CK(x)                          \
+  do {                                      \
+    const cudaError_t muse_e_ = (x);        \
+    if (muse_e_ != cudaSuccess) {           \
+      g_last_cuda_error = muse_e_;          \
+      return MUSE_ERR_CUDA;                 \
+    }                                       \
   } while (0)
 
 #define MUSE_TRY(x)                     \
@@ -718,6 +756,22 @@ muse_status experts(Pass<T>& p, const T* zsrc, int64_t nsrc, const void* W_gate,
       const W4A4Args wq{wg->matrix_scale, wu->matrix_scale};
       g.k_blocks = static_cast<int>(L / 256);
       MUSE_CK(launch_gemm_w4a4<EPI_SWIGLU>(bn_g, wm, g, wq, nsm, st));
+    } else if (fp4_gemv(c)) {
+      const muse_nvfp4_weight* wg = static_cast<const muse_nvfp4_weight*>(W_gate);
+      const muse_nvfp4_weight* wu = static_cast<const muse_nvfp4_weight*>(W_up);
+      GemvMaps vm;
+      if (!make_gemv_maps(&vm, wg, wu, E * I, zp, R, L)) return MUSE_ERR_CUDA;
+      GemvArgs v{};
+      v.tiles = g.tiles;
+      v.num_tiles = g.num_tiles_dev;
+      v.mscale[0] = wg->matrix_scale;
+      v.mscale[1] = wu->matrix_scale;
+      v.rows_per_group = static_cast<int>(I);
+      v.K = static_cast<int>(L);
+      v.out = h;
+      v.ld_out = I;
+      v.status = p.status;
+      MUSE_CK(launch_gemv_fp4<EPI_SWIGLU>(vm, v, nsm, st));
     } else if (fp4) {
       MUSE_CK(launch_gemm_fp4<EPI_SWIGLU>(bn_g, 2, maps, g, q4, nsm, st));
     } else if (pgu.pair) {
@@ -776,6 +830,26 @@ muse_status experts(Pass<T>& p, const T* zsrc, int64_t nsrc, const void* W_gate,
       const W4A4Args wq{wd->matrix_scale, wd->matrix_scale};
       g.k_blocks = static_cast<int>(I / 256);
       MUSE_CK(launch_gemm_w4a4<EPI_STORE_SS>(bn_g, wm, g, wq, nsm, st));
+    } else if (fp4_gemv(c)) {
+      const muse_nvfp4_weight* wd = static_cast<const muse_nvfp4_weight*>(W_down);
+      GemvMaps vm;
+      if (!make_gemv_maps(&vm, wd, wd, E * L, h, R, I)) return MUSE_ERR_CUDA;
+      GemvArgs v{};
+      v.tiles = g.tiles;
+      v.num_tiles = g.num_tiles_dev;
+      v.mscale[0] = v.mscale[1] = wd->matrix_scale;
+      v.rows_per_group = static_cast<int>(L);
+      v.K = static_cast<int>(I);
+      v.out = y;
+      v.status = p.status;
+      v.ld_out = L;
+      v.ss = ss;
+      v.ss_ld = static_cast<int>(L / 32);
+      if (c.norm_mode == MUSE_NORM_INPUT_SCALED) {
+        v.ss_gain = static_cast<const __nv_bfloat16*>(gamma);
+        v.ss_gain_stride = c.gamma_shared ? 0 : L;
+      }
+      MUSE_CK(launch_gemv_fp4<EPI_STORE_SS>(vm, v, nsm, st));
     } else if (fp4) {
       MUSE_CK(launch_gemm_fp4<EPI_STORE_SS>(bn_g, pdn.mt, maps, g, q4, nsm, st));
     } else if (pdn.pair && pdn.mt == 2) {
@@ -1332,6 +1406,8 @@ muse_status muse_selftest_bounded_wait(uint64_t limit_ns, uint32_t* status_dev, 
   k_selftest_wait<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns, status_dev);
   return cudaGetLastError() == cudaSuccess ? MUSE_OK : MUSE_ERR_CUDA;
 }
+
+const char* muse_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda_error); }
 
 const char* muse_status_string(muse_status s) {
   switch (s) {

@@ -254,10 +254,19 @@ def check_every_token(w: W.Workload, inp: Dict[str, torch.Tensor], run: "Run", r
     # every assignment row of y and of its sum of squares (padding rows excluded)
     sel = torch.as_tensor(ginv.astype(np.int64), device=run.out.device)
     y = host(run.inter("y", act, (R, L))[sel]).reshape(T, k, L)
-    res["y"], _ = assert_close_stored(y, ref.pop("y"), f"{w.name} y (all {T * k} rows)", rel=rel, stored_bits=bits)
+    y_ref = ref.pop("y")
+    res["y"], _ = assert_close_stored(y, y_ref, f"{w.name} y (all {T * k} rows)", rel=rel, stored_bits=bits)
     del y
     ss = run.inter("ss", torch.float32, (R, L // 32))[sel].double().sum(1).cpu().numpy().reshape(T, k)
-    res["ss"], _ = assert_close(ss, ref.pop("ss"), f"{w.name} sum of squares", rel=2 * rel)
+    ss_ref = ref.pop("ss")
+    if oracle_modes.get("norm_mode") == "input_scaled":
+        # the input-scaled norm takes the squares of u = y * (1 + gain): the CUDA path's
+        # partials are of u, the oracle's stored sums of y
+        gam = host(inp["gamma"])
+        gam = gam[gidx] if gam.ndim == 2 else gam
+        ss_ref = np.sum((y_ref * (1.0 + gam)) ** 2, axis=-1)
+    del y_ref
+    res["ss"], _ = assert_close(ss, ss_ref, f"{w.name} sum of squares", rel=2 * rel)
     res["act_adopted"] = ref.get("act_adopted", 0)
     return res
 

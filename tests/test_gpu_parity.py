@@ -5,6 +5,8 @@ Zipf-skewed routing, T=4096 NVFP4 experts as W4A16 and W4A4) on every routing de
 the permutation, the pooler output, every expert-output row with its sum of squares, the
 combined latent and the block output.
 """
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -413,6 +415,45 @@ def test_nvfp4_experts(case):
         assert_close(y, ref["y"], f"{name} expert outputs", rel=NVFP4_REL_L2)
 
 
+NVFP4_GEMV = [
+    # name, T, D, L, I, E, k: a few rows per expert (T*k <= 4E), where both expert GEMMs run
+    # on the register-fed MMA kernel -- four rows per expert on average; up to ~10 rows per
+    # expert (one or two 8-token groups, ragged) with one 256-element stage past the first
+    # in the down projection; a latent of 4608 (18 stages in gate/up)
+    ("nvfp4_gemv", 64, 1024, 1024, 1024, 64, 4),
+    ("nvfp4_gemv_ragged", 32, 256, 512, 768, 8, 1),
+    ("nvfp4_gemv_wide", 6, 256, 4608, 256, 4, 2),
+]
+
+
+@pytest.mark.parametrize("released", [False, True], ids=["centred", "released"])
+@pytest.mark.parametrize("case", NVFP4_GEMV, ids=[c[0] for c in NVFP4_GEMV])
+def test_nvfp4_decode_sized_experts_every_row(case, released):
+    """NVFP4 experts with bf16 activations at decode-sized tiles: out, z, c, every
+    assignment row of y and of its sum of squares, and the permutation against the oracle
+    (2e-2). The released variant adds the sigmoid router, the pre-expert norm and one
+    shared input-scaled post-expert gain (the sums of squares then carry the gain)."""
+    name, T, D, L, I, E, k = case
+    w = W.Workload(name, T=T, D=D, L=L, I=I, E=E, k=k, dtype="bf16", seed=17, experts="nvfp4")
+    if released:
+        w = dataclasses.replace(w, eps=1e-8)
+    inp = W.make_inputs(w, "cuda")
+    if released:
+        inp["gamma"] = inp["gamma"][0].contiguous()
+        pre = torch.empty(L, dtype=torch.bfloat16, device="cuda")
+        inp["pre_norm_gain"] = W.fill(pre, w.seed, 11, 0.3)
+        inp["router_bias"] = (W.normal_f64(w.seed, 12, 0, E) * 0.05).to(torch.float32).cuda()
+        scale = 1.0 / np.sqrt(D / 256)
+        run = Run(w, inp, router_mode=moe.ROUTER_SIGMOID, router_logit_scale=scale, routed_scaling=1.0,
+                  norm_mode=moe.NORM_INPUT_SCALED, gamma_shared=True, pre_norm_eps=1e-5)
+        res = check_every_token(w, inp, run, rel=NVFP4_REL_L2, router_mode="sigmoid", logit_scale=scale,
+                                routed_scaling=1.0, norm_mode="input_scaled", pre_norm_eps=1e-5)
+    else:
+        run = Run(w, inp)
+        res = check_every_token(w, inp, run, rel=NVFP4_REL_L2)
+    print(f"{name} ({'released' if released else 'centred'}): {res}")
+
+
 @pytest.mark.slow
 def test_full_size_nvfp4_layer_every_token():
     """The T=4096 layer with NVFP4 expert weights and bf16 activations (W4A16): every token
@@ -422,6 +463,34 @@ def test_full_size_nvfp4_layer_every_token():
     run = Run(w, inp)
     res = check_every_token(w, inp, run, rel=NVFP4_REL_L2)
     print(f"nvfp4 full layer: {res}")
+
+
+def test_nvfp4_decode_sized_skewed_expert():
+    """One expert taking every token (a strong selection bias, sigmoid router): two full
+    16-row tiles (two 8-token groups per MMA step), beside experts with a row or two."""
+    T, D, L, I, E, k = 32, 256, 512, 512, 16, 2
+    w = W.Workload("nvfp4_gemv_skew", T=T, D=D, L=L, I=I, E=E, k=k, dtype="bf16", seed=23, experts="nvfp4")
+    inp = W.make_inputs(w, "cuda")
+    bias = W.normal_f64(w.seed, 12, 0, E) * 0.05
+    bias[3] += 8.0
+    inp["router_bias"] = bias.to(torch.float32).cuda()
+    run = Run(w, inp, router_mode=moe.ROUTER_SIGMOID, routed_scaling=1.0)
+    counts = run.inter("expert_count", torch.int32, (E,)).cpu().numpy()
+    assert counts[3] == T and counts.max() == T, counts
+    res = check_every_token(w, inp, run, rel=NVFP4_REL_L2, router_mode="sigmoid", routed_scaling=1.0)
+    print(f"nvfp4_gemv_skew: {res}")
+
+
+@pytest.mark.slow
+def test_full_size_nvfp4_decode_every_token():
+    """The T=64 decode layer with NVFP4 expert weights and bf16 activations (both expert
+    GEMMs on the CUDA-core NVFP4 kernel): every token and every assignment row against the
+    oracle on the dequantised codes."""
+    w = W.WORKLOADS["nvfp4_decode"]
+    inp = W.make_inputs(w, "cuda")
+    run = Run(w, inp)
+    res = check_every_token(w, inp, run, rel=NVFP4_REL_L2)
+    print(f"nvfp4 decode layer: {res}")
 
 
 # ------------------------------------------------------------------------- full size
