@@ -102,18 +102,24 @@ __device__ __forceinline__ bool gemv_consume(const GemvArgs& p, uint8_t* smem, u
   using S = GemvShape<MATS>;
   constexpr int kStages = S::kStages;
   const int g = lane >> 2, t = lane & 3;
-  float acc[MATS][NB8][4];
+  // with one 8-token group, two accumulator sets (even and odd k-blocks) halve the chain of
+  // dependent MMAs per accumulator; they are summed before the epilogue
+  constexpr int CH = NB8 == 1 ? 2 : 1;
+  float acc[MATS][NB8][CH][4];
 #pragma unroll
   for (int m = 0; m < MATS; ++m)
 #pragma unroll
     for (int j8 = 0; j8 < NB8; ++j8)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) acc[m][j8][i] = 0.0f;
+      for (int c = 0; c < CH; ++c)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[m][j8][c][i] = 0.0f;
   const uint32_t r_lo = static_cast<uint32_t>(16 * wc + g);  // this lane's rows in the 128-row boxes
   const uint32_t sel_t = static_cast<uint32_t>(t);
   bool ok = true;
   for (int s = 0; s < nstages; ++s) {
-    if (!mbar_wait(bar0 + 8u * stage, phase, abort_flag, p.status, 0xD00u + stage)) {
+    // (every lane waits; a failure in any lane fails the whole warp, which stays converged)
+    if (!__all_sync(0xffffffffu, mbar_wait(bar0 + 8u * stage, phase, abort_flag, p.status, 0xD00u + stage))) {
       ok = false;
       break;
     }
@@ -162,8 +168,8 @@ __device__ __forceinline__ bool gemv_consume(const GemvArgs& p, uint8_t* smem, u
         for (int q = 0; q < 4; ++q)
 #pragma unroll
           for (int j8 = 0; j8 < NB8; ++j8)
-            mma_f16_16816(acc[m][j8], a_lo[2 * q], a_hi[2 * q], a_lo[2 * q + 1], a_hi[2 * q + 1], xv[j8][2 * q],
-                          xv[j8][2 * q + 1]);
+            mma_f16_16816(acc[m][j8][j % CH], a_lo[2 * q], a_hi[2 * q], a_lo[2 * q + 1], a_hi[2 * q + 1],
+                          xv[j8][2 * q], xv[j8][2 * q + 1]);
       }
     }
     __syncwarp();
@@ -173,6 +179,14 @@ __device__ __forceinline__ bool gemv_consume(const GemvArgs& p, uint8_t* smem, u
       phase ^= 1u;
     }
   }
+#pragma unroll
+  for (int m = 0; m < MATS; ++m)
+#pragma unroll
+    for (int j8 = 0; j8 < NB8; ++j8)
+#pragma unroll
+      for (int c = 1; c < CH; ++c)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[m][j8][0][i] += acc[m][j8][c][i];
   // epilogue: lane (g, t) holds rows f_lo = m0 + 16 wc + g and f_lo + 8, tokens 8 j8 + 2 t, + 1
   const int f_lo = m0 + 16 * wc + g;
   if constexpr (EPI == EPI_SWIGLU) {
@@ -186,7 +200,7 @@ __device__ __forceinline__ bool gemv_consume(const GemvArgs& p, uint8_t* smem, u
         const int tok = 8 * j8 + 2 * t + (i & 1);
         const int f = f_lo + 8 * (i >> 1);
         if (tok < n) {
-          const float h = silu_tanh(acc[0][j8][i] * ms_g) * (acc[1][j8][i] * ms_u);
+          const float h = silu_tanh(acc[0][j8][0][i] * ms_g) * (acc[1][j8][0][i] * ms_u);
           hout[(static_cast<int64_t>(row0) + tok) * p.ld_out + f] = f32_to_f16_sat(h);
         }
       }
@@ -205,7 +219,7 @@ __device__ __forceinline__ bool gemv_consume(const GemvArgs& p, uint8_t* smem, u
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         const int tok = 8 * j8 + 2 * t + c;
-        const float y0 = acc[0][j8][c] * ms, y1 = acc[0][j8][2 + c] * ms;
+        const float y0 = acc[0][j8][0][c] * ms, y1 = acc[0][j8][0][2 + c] * ms;
         if (ok && tok < n) {
           yout[(static_cast<int64_t>(row0) + tok) * p.ld_out + f_lo] = __float2bfloat16_rn(y0);
           yout[(static_cast<int64_t>(row0) + tok) * p.ld_out + f_lo + 8] = __float2bfloat16_rn(y1);
