@@ -1,7 +1,8 @@
 """GPU parity: the CUDA path (through the C ABI) against the FP64 oracle on the same
 seeded inputs. Every workload is compared element by element on every token: small ones
-on every intermediate, the full-size layers (T=64 decode, T=8192 prefill with uniform and
-Zipf-skewed routing, T=4096 NVFP4 experts as W4A16 and W4A4) on every routing decision,
+on every intermediate, the full-size layers (T=64 decode with BF16 and NVFP4 experts, T=8192
+prefill with uniform and Zipf-skewed routing, T=4096 NVFP4 experts as W4A16 and W4A4) on
+every routing decision,
 the permutation, the pooler output, every expert-output row with its sum of squares, the
 combined latent and the block output.
 """
