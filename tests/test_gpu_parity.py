@@ -2,9 +2,8 @@
 seeded inputs. Every workload is compared element by element on every token: small ones
 on every intermediate, the full-size layers (T=64 decode with BF16 and NVFP4 experts, T=8192
 prefill with uniform and Zipf-skewed routing, T=4096 NVFP4 experts as W4A16 and W4A4) on
-every routing decision,
-the permutation, the pooler output, every expert-output row with its sum of squares, the
-combined latent and the block output.
+every routing decision, the permutation, the pooler output, every expert-output row with its
+sum of squares, the combined latent and the block output.
 """
 import dataclasses
 
