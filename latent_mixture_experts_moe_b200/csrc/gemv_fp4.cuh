@@ -14,10 +14,10 @@
 //
 // Roles (288 threads, one CTA per SM, persistent over the tile list): warp 0 lane 0 is the
 // TMA producer; consumer warp wc = 0..7 (warp 1 + wc) owns weight rows 16 wc .. 16 wc + 15
-// of the tile's 128 (of both gate and up for SwiGLU). A ring stage carries 256 K elements:
-// per weight matrix four 128-row x 32-byte code boxes and one 128-row x 16-byte box of the
-// 16 block scales, and the tile's token rows as one 16-row x 128-byte box per 64-element
-// k-block (128-byte swizzle).
+// of the tile's 128 (of both gate and up for SwiGLU). A ring stage carries 256 K elements of
+// two weight matrices (gate/up) or 512 of one (down): per matrix a 128-row x 32-byte code box
+// per 64-element k-block and a 128-row x 16-byte box of block scales per 256 elements, and
+// the tile's token rows as one 16-row x 128-byte box per k-block (128-byte swizzle).
 //
 // The MMA's K order is free as long as A and B agree, so lane (g, t) of a warp (g = lane / 4,
 // t = lane % 4) takes whole 16-weight blocks: block t of each 64-element k-block, rows g and
@@ -38,7 +38,7 @@ namespace muse {
 
 constexpr int kGemvThreads = 288;        // producer warp + 8 consumer warps
 constexpr int kGemvMaxTokens = 16;       // token rows per tile (one 16-row token box)
-constexpr int kGemvKStage = 256;         // K elements per ring stage
+constexpr int kGemvKGroup = 256;         // K elements per block-scale box (16 blocks)
 
 struct GemvMaps {
   CUtensorMap codes[2];   // [E * rows, K/2] u8, 128-row x 32-byte boxes (gate, up; or down twice)
@@ -51,7 +51,7 @@ struct GemvArgs {
   const int* num_tiles;        // device count
   const float* mscale[2];      // per-expert matrix scales
   int rows_per_group;          // weight rows per expert (I for gate/up, L for down)
-  int K;                       // input width (multiple of kGemvKStage)
+  int K;                       // input width (multiple of kGemvKGroup)
   void* out;                   // SwiGLU: __half h [rows, ld_out]; store: bf16 y [rows, ld_out]
   int64_t ld_out;
   float* ss;                   // store: sums of squares [rows, ss_ld], one per 32 features
@@ -63,13 +63,18 @@ struct GemvArgs {
 
 template <int MATS>
 struct GemvShape {
+  // a stage holds SG groups of 256 K elements: one for two weight matrices (gate/up), two for
+  // one (down), so that a consumer warp has the same work per stage either way
+  static constexpr int kSG = MATS == 2 ? 1 : 2;
+  static constexpr int kKB = 4 * kSG;                                  // 64-element k-blocks per stage
+  static constexpr int kKStage = kGemvKGroup * kSG;                    // K elements per stage
   static constexpr uint32_t kCodeBox = 128u * 32u;                    // one 64-element k-block
-  static constexpr uint32_t kScaleBox = 128u * 16u;                   // 16 blocks = the stage
+  static constexpr uint32_t kScaleBox = 128u * 16u;                   // 16 blocks = 256 K elements
   static constexpr uint32_t kXBox = 16u * 128u;                       // 16 tokens x 64 elements
   static constexpr uint32_t kCodeOff = 0;
-  static constexpr uint32_t kScaleOff = kCodeOff + 4u * kCodeBox * MATS;
-  static constexpr uint32_t kXOff = kScaleOff + kScaleBox * MATS;
-  static constexpr uint32_t kStageBytes = kXOff + 4u * kXBox;         // 4 k-blocks x 1 token box
+  static constexpr uint32_t kScaleOff = kCodeOff + kKB * kCodeBox * MATS;
+  static constexpr uint32_t kXOff = kScaleOff + kSG * kScaleBox * MATS;
+  static constexpr uint32_t kStageBytes = kXOff + kKB * kXBox;        // k-blocks x 1 token box
   static constexpr uint32_t kSsBytes = 8u * 16u * 4u;                 // store epilogue partials
   static constexpr int kSmemBudget = 227 * 1024 - 1024 - static_cast<int>(kSsBytes) - 256;
   static constexpr int kStagesFit = kSmemBudget / static_cast<int>(kStageBytes);
@@ -124,15 +129,18 @@ __device__ __forceinline__ bool gemv_consume(const GemvArgs& p, uint8_t* smem, u
       break;
     }
     const uint8_t* st = smem + static_cast<uint32_t>(stage) * S::kStageBytes;
-    // the 16 block scales of rows r_lo and r_lo + 8 for this stage, per matrix
-    uint4 sw[MATS][2];
+    // the block scales of rows r_lo and r_lo + 8 for this stage: 16 per group, per matrix
+    uint4 sw[MATS][S::kSG][2];
 #pragma unroll
-    for (int m = 0; m < MATS; ++m) {
-      sw[m][0] = *reinterpret_cast<const uint4*>(st + S::kScaleOff + m * S::kScaleBox + r_lo * 16u);
-      sw[m][1] = *reinterpret_cast<const uint4*>(st + S::kScaleOff + m * S::kScaleBox + (r_lo + 8u) * 16u);
-    }
+    for (int m = 0; m < MATS; ++m)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {   // k-block of 64 elements; this lane's block in it: t
+      for (int sg = 0; sg < S::kSG; ++sg) {
+        const uint8_t* sb = st + S::kScaleOff + (m * S::kSG + sg) * S::kScaleBox;
+        sw[m][sg][0] = *reinterpret_cast<const uint4*>(sb + r_lo * 16u);
+        sw[m][sg][1] = *reinterpret_cast<const uint4*>(sb + (r_lo + 8u) * 16u);
+      }
+#pragma unroll
+    for (int j = 0; j < S::kKB; ++j) {   // k-block of 64 elements; this lane's block in it: t
       // activations: token g of each 8-token group, elements 16 t .. 16 t + 15 of the k-block
       uint32_t xv[NB8][8];
 #pragma unroll
@@ -146,11 +154,13 @@ __device__ __forceinline__ bool gemv_consume(const GemvArgs& p, uint8_t* smem, u
       }
 #pragma unroll
       for (int m = 0; m < MATS; ++m) {
-        const uint8_t* cb = st + S::kCodeOff + (4u * m + j) * S::kCodeBox;
+        const uint8_t* cb = st + S::kCodeOff + (S::kKB * m + j) * S::kCodeBox;
         const uint2 c_lo = *reinterpret_cast<const uint2*>(cb + r_lo * 32u + 8u * t);
         const uint2 c_hi = *reinterpret_cast<const uint2*>(cb + (r_lo + 8u) * 32u + 8u * t);
-        const uint32_t w_lo = j == 0 ? sw[m][0].x : j == 1 ? sw[m][0].y : j == 2 ? sw[m][0].z : sw[m][0].w;
-        const uint32_t w_hi = j == 0 ? sw[m][1].x : j == 1 ? sw[m][1].y : j == 2 ? sw[m][1].z : sw[m][1].w;
+        const uint4& q_lo = sw[m][j / 4][0];
+        const uint4& q_hi = sw[m][j / 4][1];
+        const uint32_t w_lo = j % 4 == 0 ? q_lo.x : j % 4 == 1 ? q_lo.y : j % 4 == 2 ? q_lo.z : q_lo.w;
+        const uint32_t w_hi = j % 4 == 0 ? q_hi.x : j % 4 == 1 ? q_hi.y : j % 4 == 2 ? q_hi.z : q_hi.w;
         const uint32_t s_lo = e4m3_bcast_f16x2(w_lo, sel_t), s_hi = e4m3_bcast_f16x2(w_hi, sel_t);
         uint32_t a_lo[8], a_hi[8];   // byte b of the block -> weights 2b, 2b + 1
         e2m1x8_to_f16x2(c_lo.x, a_lo[0], a_lo[1], a_lo[2], a_lo[3]);
@@ -285,7 +295,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_fp4_gemv(const __grid_const
   }
   __syncthreads();
   const int num_tiles = *p.num_tiles;
-  const int nstages = p.K / kGemvKStage;
+  // (a last stage past K reads zeros: the tensor maps fill outside the matrices)
+  const int nstages = (p.K + S::kKStage - 1) / S::kKStage;
   if (warp == 0) {
     if (lane == 0) {
       const uint64_t evict_first = policy_evict_first();
@@ -297,7 +308,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_fp4_gemv(const __grid_const
         const int a_row = tile.x * p.rows_per_group + tile.y;
         // (tiles hold at most 16 rows; a longer one is recorded and cut, never overrun)
         if (tile.w > kGemvMaxTokens) record_status(p.status, kStatusDevice, 0x6E00u);
-        const uint32_t bytes = (4u * S::kCodeBox + S::kScaleBox) * MATS + 4u * S::kXBox;
+        const uint32_t bytes = (S::kKB * S::kCodeBox + S::kSG * S::kScaleBox) * MATS + S::kKB * S::kXBox;
         for (int s = 0; s < nstages; ++s) {
           if (!mbar_wait(bar0 + 8u * (kStages + stage), phase ^ 1u, abort_flag, p.status, 0xE00u + stage)) {
             ok = false;
@@ -309,14 +320,16 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_fp4_gemv(const __grid_const
 #pragma unroll
           for (int m = 0; m < MATS; ++m) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              tma_load_2d_hint(st + S::kCodeOff + (4u * m + j) * S::kCodeBox, &maps.codes[m], full,
-                               (kGemvKStage / 2) * s + 32 * j, a_row, evict_first);
-            tma_load_2d_hint(st + S::kScaleOff + m * S::kScaleBox, &maps.scales[m], full, (kGemvKStage / 16) * s,
-                             a_row, evict_first);
+            for (int j = 0; j < S::kKB; ++j)
+              tma_load_2d_hint(st + S::kCodeOff + (S::kKB * m + j) * S::kCodeBox, &maps.codes[m], full,
+                               (S::kKStage / 2) * s + 32 * j, a_row, evict_first);
+#pragma unroll
+            for (int sg = 0; sg < S::kSG; ++sg)
+              tma_load_2d_hint(st + S::kScaleOff + (m * S::kSG + sg) * S::kScaleBox, &maps.scales[m], full,
+                               (S::kKStage / 16) * s + 16 * sg, a_row, evict_first);
           }
-          for (int j = 0; j < 4; ++j)
-            tma_load_2d(st + S::kXOff + j * S::kXBox, &maps.x, full, kGemvKStage * s + 64 * j, tile.z);
+          for (int j = 0; j < S::kKB; ++j)
+            tma_load_2d(st + S::kXOff + j * S::kXBox, &maps.x, full, S::kKStage * s + 64 * j, tile.z);
           issued_mask |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
           if (++stage == kStages) {
