@@ -4,6 +4,7 @@ import ctypes
 import os
 import re
 import subprocess
+import sys
 
 import pytest
 
@@ -280,3 +281,13 @@ def test_checked_forward_rejects_every_shape_mismatch_before_any_launch(nvfp4):
     w = args["W_down"][0]
     args["out"].data = w.data + 4096
     assert _call_checked(cfg, args) == 1
+
+
+def test_last_cuda_error_names_no_error_before_any_failure():
+    """muse_last_cuda_error() is a host-side query: in a fresh process, before any CUDA call
+    has failed, it returns the runtime's "no error" text."""
+    code = "import latent_mixture_experts_moe_b200 as moe; print(moe.last_cuda_error())"
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300,
+                         cwd=os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    assert out.returncode == 0, out.stderr[-2000:]
+    assert out.stdout.strip().splitlines()[-1] == "no error"
