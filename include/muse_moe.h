@@ -84,7 +84,12 @@ typedef struct muse_nvfp4_weight {
 
 /* Format of the expert GEMMs' activation operands (with NVFP4 expert weights). */
 typedef enum muse_act_format {
-  MUSE_ACT_BF16 = 0,          /* W4A16: activations stay bf16                           */
+  MUSE_ACT_BF16 = 0,          /* W4A16: activations stay 16-bit: the expert GEMMs
+                                 multiply f16 operands -- the decoded weights (exact) and
+                                 the latent rows converted bf16 -> f16 (exact for
+                                 magnitudes 2^-14 .. 65504; smaller ones round to f16's
+                                 subnormal grid, larger ones saturate); h is kept as f16;
+                                 FP32 accumulation                                       */
   MUSE_ACT_NVFP4 = 1          /* W4A4 (deep dive §7.4): the latent rows and the SwiGLU
                                  output are quantised per 16 values: scale E4M3(amax / 6),
                                  codes the E2M1 values nearest to value / scale (ties to
